@@ -1,0 +1,172 @@
+"""fp64 CPU oracle for the selective scan -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline leg and its
+``--impl reference`` arm) may import this package.  The CUDA library never does, and this
+package imports nothing from it.
+
+The arithmetic lives in ``ssm_oracle.c`` (scalar fp64, libm ``exp``/``log1p``, ``-O2`` without
+fast-math).  This module only compiles it with gcc, loads it with ctypes and marshals numpy
+arrays.  Inputs are converted to float64 exactly (fp32 and bf16 values are representable), so
+the oracle sees precisely the values the GPU sees.
+
+Definitions followed (cited by page title and section; see ``ssm_oracle.c`` for the full list):
+  * ufo.work "会议长序列建模状态空间模型加速…" §1.1 -- h_t = exp(Δ_t A) h_{t-1} + Δ_t B_t x_t,
+    y_t = C_t h_t;
+  * discosf.com "企业官网建设流程全解析" §1.1 (skip term D x) and §1.3 (Δ = softplus(·));
+  * ufo.work §4.2 -- packed sequences restart from h = 0 at each cu_seqlens boundary;
+  * ufo.work §4.1 -- single-token update of a persistent per-request state.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssm_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "libssm_oracle.so")
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile ssm_oracle.c into a shared object (gcc -O2, no fast-math). Returns its path."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared",
+               "-o", tmp, _SRC, "-lm", "-lpthread"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I = ctypes.c_int64
+            lib.oracle_scan.argtypes = [I, I, I, I] + [P] * 13 + [ctypes.c_int]
+            lib.oracle_scan.restype = ctypes.c_int
+            lib.oracle_scan_varlen.argtypes = [I, I, I] + [P] * 8 + [P, I] + [P] * 4 + [ctypes.c_int]
+            lib.oracle_scan_varlen.restype = ctypes.c_int
+            lib.oracle_state_update.argtypes = [I, I, I, P, P, P, I] + [P] * 9
+            lib.oracle_state_update.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def scan(u, delta, B, C, A, Dskip=None, bias=None, z=None, h0=None, nthreads: int = 1):
+    """Fixed-length batch scan.
+
+    u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; A: [dim, N]; Dskip, bias: [dim];
+    h0: [batch, dim, N] or None (zero state).
+    Returns dict with y [batch, dim, L], h_last [batch, dim, N] and the magnitudes
+    y_mag, h_mag used to scale errors.
+    """
+    u, delta, B, C, A = (_f64(x) for x in (u, delta, B, C, A))
+    z, Dskip, bias, h0 = (_f64(x) for x in (z, Dskip, bias, h0))
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    assert delta.shape == u.shape and B.shape == (batch, N, L) and C.shape == B.shape
+    assert A.shape == (dim, N)
+    if z is not None:
+        assert z.shape == u.shape
+    if h0 is not None:
+        assert h0.shape == (batch, dim, N)
+    y = np.empty((batch, dim, L))
+    y_mag = np.empty_like(y)
+    h_last = np.empty((batch, dim, N))
+    h_mag = np.empty_like(h_last)
+    rc = _load().oracle_scan(batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C),
+                             _ptr(A), _ptr(Dskip), _ptr(bias), _ptr(h0), _ptr(y), _ptr(h_last),
+                             _ptr(y_mag), _ptr(h_mag), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_scan rejected its arguments (code {rc})")
+    return {"y": y, "h_last": h_last, "y_mag": y_mag, "h_mag": h_mag}
+
+
+def scan_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, bias=None, z=None, nthreads: int = 1):
+    """Packed varlen scan. u, delta, z: [dim, T]; B, C: [N, T]; cu_seqlens: [nseq+1].
+
+    Every sequence starts from h = 0.  Returns y [dim, T], h_last [nseq, dim, N] and magnitudes.
+    """
+    u, delta, B, C, A = (_f64(x) for x in (u, delta, B, C, A))
+    z, Dskip, bias = (_f64(x) for x in (z, Dskip, bias))
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    dim, T = u.shape
+    N = A.shape[1]
+    nseq = cu.shape[0] - 1
+    assert B.shape == (N, T) and C.shape == (N, T) and delta.shape == u.shape
+    y = np.empty((dim, T))
+    y_mag = np.empty_like(y)
+    h_last = np.empty((nseq, dim, N))
+    h_mag = np.empty_like(h_last)
+    rc = _load().oracle_scan_varlen(dim, N, T, _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C),
+                                    _ptr(A), _ptr(Dskip), _ptr(bias), _ptr(cu), nseq, _ptr(y),
+                                    _ptr(h_last), _ptr(y_mag), _ptr(h_mag), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_scan_varlen rejected its arguments (code {rc})")
+    return {"y": y, "h_last": h_last, "y_mag": y_mag, "h_mag": h_mag}
+
+
+def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, bias=None, z=None, pool_mag=None):
+    """One decode step, in place on ``pool`` (float64 array [S, dim, N]).
+
+    slot_ids: [R]; u, delta, z: [R, dim]; B, C: [R, N].  ``pool_mag`` (same shape as pool, or
+    None) carries the magnitude recursion across steps.  Returns dict with y [R, dim], y_mag.
+    """
+    assert pool.dtype == np.float64 and pool.flags.c_contiguous
+    if pool_mag is not None:
+        assert pool_mag.dtype == np.float64 and pool_mag.flags.c_contiguous and pool_mag.shape == pool.shape
+    u, delta, B, C, A = (_f64(x) for x in (u, delta, B, C, A))
+    z, Dskip, bias = (_f64(x) for x in (z, Dskip, bias))
+    ids = np.ascontiguousarray(np.asarray(slot_ids, dtype=np.int64))
+    S, dim, N = pool.shape
+    R = ids.shape[0]
+    assert u.shape == (R, dim) and B.shape == (R, N)
+    y = np.empty((R, dim))
+    y_mag = np.empty_like(y)
+    rc = _load().oracle_state_update(S, dim, N, _ptr(pool), _ptr(pool_mag), _ptr(ids), R, _ptr(u),
+                                     _ptr(delta), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(Dskip),
+                                     _ptr(bias), _ptr(y), _ptr(y_mag))
+    if rc != 0:
+        raise ValueError(f"oracle_state_update rejected its arguments (code {rc})")
+    return {"y": y, "y_mag": y_mag}
+
+
+def scaled_error(x, ref, mag) -> float:
+    """max_i |x_i - ref_i| / mag_i, where mag is the oracle's magnitude bound (|ref| <= mag).
+
+    Non-finite values in x give +inf.  Where mag == 0 the reference is exactly zero and any
+    nonzero x counts as an infinite error.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    mag = np.asarray(mag, dtype=np.float64)
+    if not np.all(np.isfinite(x)):
+        return float("inf")
+    diff = np.abs(x - ref)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(mag > 0, diff / np.where(mag > 0, mag, 1.0), np.where(diff > 0, np.inf, 0.0))
+    return float(r.max()) if r.size else 0.0

@@ -1,0 +1,276 @@
+"""Pins for the fp64 oracle, independent of the oracle's own code (CPU only).
+
+Each check compares the oracle with something the pages or plain mathematics fix, chosen so
+that a plausible slip (a dropped term, a sign, h_{t-1} instead of h_t, B and C swapped, A
+transposed, a wrong reset) fails at least one of them:
+  * a hand-derived worked example (tests/golden/worked_example.json);
+  * a 50-digit decimal brute force of the unrolled sum (oracle/brute.py);
+  * the time-invariant case equals a causal convolution (discosf.com §1.1: "train with the
+    convolution, infer with the recurrence"; kj168168.com §三.3 kernel of decaying powers);
+  * A = 0 reduces the state to a cumulative sum;
+  * chunk transfer operators compose to the sequential result (ufo.work §3.1);
+  * varlen equals independent scans; L decode steps equal one scan (ufo.work §4.1, §4.2);
+  * extreme step sizes (ufo.work §6 pitfall 1: Δ large must not overflow).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import brute
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_example.json")
+
+
+def _rand_problem(rng, b, D, N, L, gate=True, h0=True, A_range=(0.2, 3.0)):
+    u = rng.standard_normal((b, D, L))
+    delta = rng.standard_normal((b, D, L))
+    z = rng.standard_normal((b, D, L)) if gate else None
+    B = rng.standard_normal((b, N, L))
+    C = rng.standard_normal((b, N, L))
+    A = -rng.uniform(*A_range, size=(D, N))
+    Dskip = rng.standard_normal(D)
+    bias = rng.uniform(-3.0, 1.0, size=D)
+    h = rng.standard_normal((b, D, N)) if h0 else None
+    return dict(u=u, delta=delta, z=z, B=B, C=C, A=A, Dskip=Dskip, bias=bias, h0=h)
+
+
+def test_golden_worked_example():
+    g = json.load(open(GOLDEN))
+    c = g["common"]
+    ln2 = math.log(2.0)
+    shape = (1, 1, 4)
+    for case in g["cases"]:
+        u = np.array(c["u"]).reshape(shape)
+        z = None if case["z"] is None else np.array(case["z"]).reshape(shape)
+        h0 = None if case["h0"] is None else np.array(case["h0"]).reshape(1, 1, 2)
+        out = oracle.scan(u, np.array(c["delta"]).reshape(shape), np.array(c["B"])[None],
+                          np.array(c["C"])[None], np.array(c["A"]), Dskip=np.array(c["Dskip"]),
+                          bias=np.array(c["bias"]), z=z, h0=h0)
+        y_exp = np.array([a * ln2 + k for a, k in case["y"]])
+        if "silu" in case:
+            y_exp = y_exp * np.array(case["silu"])
+        h_exp = np.array([a * ln2 + k for a, k in case["h_last"]])
+        np.testing.assert_allclose(out["y"].ravel(), y_exp, rtol=1e-14, atol=1e-15, err_msg=case["name"])
+        np.testing.assert_allclose(out["h_last"].ravel(), h_exp, rtol=1e-14, atol=1e-15, err_msg=case["name"])
+        assert np.all(out["y_mag"] >= np.abs(out["y"]) * (1 - 1e-15))
+
+
+@pytest.mark.parametrize("shape,gate,h0,seed", [
+    ((1, 1, 1, 1), False, False, 0),
+    ((1, 2, 3, 7), True, True, 1),
+    ((2, 2, 4, 12), True, False, 2),
+    ((1, 2, 4, 10), False, True, 3),
+])
+def test_brute_force_tiny(shape, gate, h0, seed):
+    b, D, N, L = shape
+    p = _rand_problem(np.random.default_rng(seed), b, D, N, L, gate, h0)
+    out = oracle.scan(**p)
+    y_ref, h_ref = brute.scan(p["u"], p["delta"], p["B"], p["C"], p["A"], p["Dskip"], p["bias"], p["z"], p["h0"])
+    assert oracle.scaled_error(out["y"], y_ref, out["y_mag"]) < 1e-13
+    assert oracle.scaled_error(out["h_last"], h_ref, out["h_mag"]) < 1e-13
+
+
+def test_brute_force_catches_swapped_B_C():
+    # B and C play different roles; swapping them must change the result well beyond rounding.
+    p = _rand_problem(np.random.default_rng(11), 1, 2, 3, 6)
+    out = oracle.scan(**p)
+    y_swapped, _ = brute.scan(p["u"], p["delta"], p["C"], p["B"], p["A"], p["Dskip"], p["bias"], p["z"], p["h0"])
+    assert oracle.scaled_error(out["y"], y_swapped, out["y_mag"]) > 1e-3
+
+
+def _delta_for_steps(steps, bias):
+    """δ such that softplus(δ + bias) = steps exactly in real arithmetic (inverse softplus)."""
+    return np.log(np.expm1(steps)) - bias
+
+
+def test_time_invariant_equals_causal_convolution():
+    rng = np.random.default_rng(5)
+    D, N, L = 3, 5, 64
+    steps = np.array([0.01, 0.2, 1.3])               # constant Δ per channel
+    bias = rng.uniform(-2, 0, size=D)
+    delta = np.repeat(_delta_for_steps(steps, bias)[:, None], L, axis=1)[None]
+    beta = rng.standard_normal(N)
+    gamma = rng.standard_normal(N)
+    B = np.repeat(beta[:, None], L, axis=1)[None]
+    C = np.repeat(gamma[:, None], L, axis=1)[None]
+    A = -rng.uniform(0.1, 2.0, size=(D, N))
+    Dskip = rng.standard_normal(D)
+    u = rng.standard_normal((1, D, L))
+    out = oracle.scan(u, delta, B, C, A, Dskip=Dskip, bias=bias)
+    j = np.arange(L)
+    for d in range(D):
+        # K_j = sum_n C_n exp(j Δ A_n) Δ B_n, then y = K * u + D u (causal convolution).
+        K = (gamma[None, :] * np.exp(j[:, None] * steps[d] * A[d][None, :]) * steps[d] * beta[None, :]).sum(1)
+        y_conv = np.convolve(u[0, d], K)[:L] + Dskip[d] * u[0, d]
+        err = np.max(np.abs(out["y"][0, d] - y_conv) / out["y_mag"][0, d])
+        assert err < 1e-12, (d, err)
+
+
+def test_A_zero_is_cumulative_sum():
+    rng = np.random.default_rng(6)
+    D, N, L = 2, 4, 50
+    bias = np.zeros(D)
+    delta = np.zeros((1, D, L))                      # Δ = softplus(0) = ln 2
+    u = rng.standard_normal((1, D, L))
+    B = rng.standard_normal((1, N, L))
+    C = rng.standard_normal((1, N, L))
+    Dskip = rng.standard_normal(D)
+    out = oracle.scan(u, delta, B, C, np.zeros((D, N)), Dskip=Dskip, bias=bias)
+    for d in range(D):
+        h = np.cumsum(math.log(2.0) * B[0] * u[0, d][None, :], axis=1)   # [N, L]
+        y = (C[0] * h).sum(0) + Dskip[d] * u[0, d]
+        np.testing.assert_allclose(out["y"][0, d], y, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(out["h_last"][0, d], h[:, -1], rtol=1e-12, atol=1e-12)
+
+
+def test_chunk_operators_compose_to_sequential():
+    """h_end = Abar_chunk h_start + Bbar_chunk, composed over any chunking, equals the full scan."""
+    rng = np.random.default_rng(7)
+    D, N, L = 2, 3, 97
+    bias = rng.uniform(-3, 0, size=D)
+    steps = rng.uniform(1e-3, 0.5, size=(D, L))
+    delta = _delta_for_steps(steps, bias[:, None])[None]
+    u = rng.standard_normal((1, D, L))
+    B = rng.standard_normal((1, N, L))
+    C = rng.standard_normal((1, N, L))
+    A = -rng.uniform(0.1, 3.0, size=(D, N))
+    h0 = rng.standard_normal((1, D, N))
+    full = oracle.scan(u, delta, B, C, A, bias=bias, h0=h0)
+    for cuts in ([0, L], [0, 1, L], [0, 40, 41, 90, L], list(range(0, L, 8)) + [L], list(range(L + 1))):
+        h = h0[0].copy()
+        ys = []
+        for s, e in zip(cuts[:-1], cuts[1:]):
+            sl = slice(s, e)
+            # transfer operator of the chunk: Abar = exp(A * sum Δ), Bbar = scan from zero
+            zero = oracle.scan(u[..., sl], delta[..., sl], B[..., sl], C[..., sl], A, bias=bias)
+            Abar = np.exp(A * steps[:, sl].sum(1)[:, None])
+            h_next = Abar * h + zero["h_last"][0]
+            # chained run with the carried state reproduces the chunk's outputs
+            chained = oracle.scan(u[..., sl], delta[..., sl], B[..., sl], C[..., sl], A, bias=bias, h0=h[None])
+            ys.append(chained["y"][0])
+            np.testing.assert_allclose(chained["h_last"][0], h_next, rtol=1e-12, atol=1e-13)
+            h = chained["h_last"][0]
+        np.testing.assert_allclose(h, full["h_last"][0], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(np.concatenate(ys, axis=1), full["y"][0], rtol=1e-12, atol=1e-13)
+
+
+def test_varlen_equals_independent_scans():
+    rng = np.random.default_rng(8)
+    D, N = 3, 4
+    lens = [5, 1, 17, 9]
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    p = dict(u=rng.standard_normal((D, T)), delta=rng.standard_normal((D, T)),
+             z=rng.standard_normal((D, T)), B=rng.standard_normal((N, T)), C=rng.standard_normal((N, T)))
+    A = -rng.uniform(0.1, 2, size=(D, N))
+    Dskip = rng.standard_normal(D)
+    bias = rng.uniform(-3, 0, size=D)
+    out = oracle.scan_varlen(p["u"], p["delta"], p["B"], p["C"], A, cu, Dskip=Dskip, bias=bias, z=p["z"])
+    for s in range(len(lens)):
+        sl = slice(cu[s], cu[s + 1])
+        one = oracle.scan(p["u"][None, :, sl], p["delta"][None, :, sl], p["B"][None, :, sl],
+                          p["C"][None, :, sl], A, Dskip=Dskip, bias=bias, z=p["z"][None, :, sl])
+        np.testing.assert_array_equal(out["y"][:, sl], one["y"][0])
+        np.testing.assert_array_equal(out["h_last"][s], one["h_last"][0])
+
+
+def test_varlen_resets_state_at_boundaries():
+    # Two sequences: the second must not see the first's state; compare with a zero prefix.
+    rng = np.random.default_rng(9)
+    D, N, T1, T2 = 2, 3, 6, 5
+    u = rng.standard_normal((D, T1 + T2))
+    delta = rng.standard_normal((D, T1 + T2))
+    B = rng.standard_normal((N, T1 + T2))
+    C = rng.standard_normal((N, T1 + T2))
+    A = -np.ones((D, N)) * 0.01                       # slow decay: leakage would be visible
+    out = oracle.scan_varlen(u, delta, B, C, A, [0, T1, T1 + T2])
+    u2 = u.copy()
+    u2[:, :T1] = 0.0                                  # zero input before the boundary = zero state
+    ref = oracle.scan(u2[None], delta[None], B[None], C[None], A)
+    np.testing.assert_allclose(out["y"][:, T1:], ref["y"][0, :, T1:], rtol=1e-13, atol=1e-15)
+
+
+def test_decode_steps_equal_scan():
+    rng = np.random.default_rng(10)
+    S, D, N, L = 5, 3, 4, 9
+    slots = np.array([3, 0])
+    R = len(slots)
+    pool = rng.standard_normal((S, D, N))
+    pool_before = pool.copy()
+    A = -rng.uniform(0.1, 2, size=(D, N))
+    Dskip = rng.standard_normal(D)
+    bias = rng.uniform(-3, 0, size=D)
+    u = rng.standard_normal((L, R, D))
+    delta = rng.standard_normal((L, R, D))
+    z = rng.standard_normal((L, R, D))
+    B = rng.standard_normal((L, R, N))
+    C = rng.standard_normal((L, R, N))
+    ys = []
+    for t in range(L):
+        ys.append(oracle.state_update(pool, slots, u[t], delta[t], B[t], C[t], A, Dskip, bias, z[t])["y"])
+    ys = np.stack(ys)                                 # [L, R, D]
+    for r, s in enumerate(slots):
+        ref = oracle.scan(u[:, r].T[None], delta[:, r].T[None], B[:, r].T[None], C[:, r].T[None], A,
+                          Dskip=Dskip, bias=bias, z=z[:, r].T[None], h0=pool_before[s][None])
+        np.testing.assert_allclose(ys[:, r].T, ref["y"][0], rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(pool[s], ref["h_last"][0], rtol=1e-13, atol=1e-14)
+    untouched = [s for s in range(S) if s not in slots]
+    np.testing.assert_array_equal(pool[untouched], pool_before[untouched])
+
+
+def test_extreme_steps():
+    rng = np.random.default_rng(12)
+    D, N, L = 2, 3, 5
+    u = rng.standard_normal((1, D, L))
+    B = rng.standard_normal((1, N, L))
+    C = rng.standard_normal((1, N, L))
+    A = -np.ones((D, N))
+    h0 = rng.standard_normal((1, D, N))
+    # Δ ≈ 30: abar = e^-30 wipes the previous state, h_t ≈ Δ B_t u_t, no overflow
+    big = oracle.scan(u, np.full((1, D, L), 30.0), B, C, A, h0=h0)
+    assert np.all(np.isfinite(big["y"]))
+    np.testing.assert_allclose(big["h_last"][0], 30.0 * B[0, :, -1][None, :] * u[0, :, -1][:, None], rtol=1e-11, atol=1e-10)
+    # Δ ≈ e^-50: abar ≈ 1 and the input term vanishes, so the state stays h0
+    tiny = oracle.scan(u, np.full((1, D, L), -50.0), B, C, A, h0=h0)
+    np.testing.assert_allclose(tiny["h_last"], h0, rtol=1e-15, atol=1e-20)
+    np.testing.assert_allclose(tiny["y"][0], np.einsum("nl,dn->dl", C[0], h0[0]), rtol=1e-12, atol=1e-14)
+
+
+def test_softplus_of_generated_bias_recovers_step():
+    """The workload recipe sets bias = log(expm1(dt)); the oracle's Δ = softplus(bias) must
+    satisfy the defining identity e^Δ - 1 = e^bias."""
+    rng = np.random.default_rng(3)
+    _, _, bias = workloads.channel_params(rng, 64, 1)
+    bias = bias.astype(np.float64)
+    D = bias.shape[0]
+    one = np.ones((1, D, 1))
+    out = oracle.scan(one, np.zeros((1, D, 1)), np.ones((1, 1, 1)), np.ones((1, 1, 1)),
+                      np.zeros((D, 1)), bias=bias)              # y = h = Δ · 1 · 1
+    dt = out["y"][0, :, 0]
+    np.testing.assert_allclose(np.expm1(dt), np.exp(bias), rtol=1e-13)
+    assert dt.min() > 0.9e-3 and dt.max() < 1.1e-1
+
+
+def test_scaled_error_semantics():
+    ref = np.array([1.0, -2.0, 0.0])
+    mag = np.array([2.0, 4.0, 0.0])
+    assert oracle.scaled_error(ref, ref, mag) == 0.0
+    assert oracle.scaled_error(np.array([1.5, -2.0, 0.0]), ref, mag) == pytest.approx(0.25)
+    assert oracle.scaled_error(np.array([1.0, -2.0, 1e-30]), ref, mag) == float("inf")
+    assert oracle.scaled_error(np.array([np.nan, -2.0, 0.0]), ref, mag) == float("inf")
+
+
+def test_workload_generator_is_deterministic_and_bf16_exact():
+    a = workloads.batch_inputs(1, 4, 16, 64, "bf16", seed=3)
+    b = workloads.batch_inputs(1, 4, 16, 64, "bf16", seed=3)
+    np.testing.assert_array_equal(a.u, b.u)
+    bits = a.u.view(np.uint32)
+    assert np.all((bits & 0xFFFF) == 0)               # representable in bf16
+    # ties round to even: 1 + 2^-8 (exactly halfway between two bf16 values) rounds down to 1
+    x = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8], dtype=np.float32)
+    np.testing.assert_array_equal(workloads.round_to_bf16(x), np.array([1.0, 1.0 + 2.0 ** -6], dtype=np.float32))
