@@ -1,0 +1,460 @@
+"""Benchmark of the selective scan on B200: one JSON line on rank 0.
+
+Default workload (the metric's shape): packed varlen bf16 scan, 16 sequences with lengths
+drawn uniformly in [256, 4096], D = 2048 channels, N = 16 states, SiLU(z) gate.  A "step"
+is one ssm_scan_fwd_varlen call over one packed batch (all steps of the hot path: staging,
+softplus, discretisation, chunked scan, carry, contraction, gate, store, final states).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-secondary]
+
+Multi-GPU (torchrun, one rank per GPU): every rank scans its own packed batch (seed offset by
+rank), no collective on the data path ("scaling": "weak"); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+SFU_PER_CLK_PER_SM = 16          # ex2/lg2/rcp results per clock per SM (measured on B200)
+N_SM = 148
+METRIC = "selective-scan tokens/s at D=2048,N=16; achieved HBM GB/s & roofline frac"
+WORKLOAD = "varlen_bf16"
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", 1965.0)), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1965.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_15_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(key: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernels are unchanged."""
+    try:
+        with open(TRAFFIC_PATH) as f:
+            t = json.load(f)
+        e = t.get(key)
+        if e and e.get("kernel_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.6)
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------------------ inputs
+
+def varlen_device_inputs(rank: int, device):
+    import torch
+    c = workloads.CONFIGS[WORKLOAD]
+    seed = c["seed"] + 1000 * rank
+    lens = workloads.varlen_lengths(c["nseq"], c["len_lo"], c["len_hi"], seed)
+    inp = workloads.varlen_inputs(lens, c["dim"], c["dstate"], c["dtype"], seed)
+    T = inp.meta["total"]
+    pitch = (T + 7) // 8 * 8           # rows padded to a 16-byte pitch
+
+    def up(x, dt=torch.bfloat16):
+        t = torch.zeros(x.shape[:-1] + (pitch,), dtype=dt)
+        t[..., :T] = torch.from_numpy(x).to(dt)
+        return t
+    host = {k: up(getattr(inp, k)) for k in ("u", "delta", "z", "B", "C")}
+    dev = {k: v.to(device) for k, v in host.items()}
+    for k in ("A", "Dskip", "bias"):
+        dev[k] = torch.from_numpy(getattr(inp, k)).to(device)
+    dev["cu"] = torch.from_numpy(inp.cu_seqlens).to(device)
+    host["cu"] = torch.from_numpy(inp.cu_seqlens)
+    return inp, host, dev, T, pitch
+
+
+def scan_counts(T, D, N, in_bytes, out_bytes, nseq):
+    """Algorithmic bytes and exponentials of one scan launch."""
+    bytes_ = T * D * (3 * in_bytes + out_bytes) + 2 * T * N * in_bytes + nseq * D * N * 4 + D * (N + 2) * 4
+    exps = T * D * (N + 2)
+    return bytes_, exps
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+
+class CpuOracle:
+    """The fp64 oracle on all host cores over a bounded channel sample of the packed batch.
+
+    Channels are independent, so the sample's time scales to the full batch by D / channels."""
+
+    def __init__(self, inp, budget_s: float):
+        import oracle
+        oracle.build()
+        self.oracle, self.inp = oracle, inp
+        self.threads = oracle.default_threads()
+        self.D = inp.u.shape[0]
+        self.T = inp.meta["total"]
+        n0 = min(self.D, max(self.threads, 8))
+        t_small = self._run(n0)
+        self.nch = int(min(self.D, max(n0, n0 * budget_s / max(t_small, 1e-3))))
+
+    def _run(self, nch):
+        inp = self.inp
+        ch = np.linspace(0, self.D - 1, nch).astype(np.int64)
+        t0 = time.perf_counter()
+        self.oracle.scan_varlen(inp.u[ch], inp.delta[ch], inp.B, inp.C, inp.A[ch], inp.cu_seqlens, inp.Dskip[ch],
+                                inp.bias[ch], inp.z[ch], nthreads=self.threads)
+        return time.perf_counter() - t0
+
+    def measure(self):
+        t = self._run(self.nch)
+        return {"value": self.T * (self.nch / self.D) / t, "unit": "tokens/s", "cores": self.threads, "kind": "oracle",
+                "sample": f"all {self.inp.meta['nseq']} sequences ({self.T} tokens) on {self.nch} of {self.D} "
+                          f"channels, scaled by {self.D}/{self.nch}; {t:.2f} s wall"}
+
+
+def cpu_oracle_rate(inp, budget_s: float = 12.0):
+    return CpuOracle(inp, budget_s).measure()
+
+
+# ------------------------------------------------------------------------------ timing
+
+def time_kernel(fn, steps, warmup, stream, flush=None):
+    """Per-launch duration (ms) from CUDA events on the launching stream."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+    total = 0.0
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    return total / steps
+
+
+def secondary(steps, warmup, hbm_peak, sfu_peak):
+    """Kernel-only figures for the long-sequence and decode workloads (single GPU)."""
+    import torch
+    import selective_state_space_15_b200 as ssm
+    out = {}
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device="cuda")
+    for name in ("long_bf16", "long_n128_bf16"):
+        c = workloads.CONFIGS[name]
+        D, N, L = c["dim"], c["dstate"], c["seqlen"]
+        g.manual_seed(c["seed"])
+        mk = lambda *s: torch.randn(*s, generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)  # noqa: E731
+        u, dl, z, B, C = mk(1, D, L), mk(1, D, L), mk(1, D, L), mk(1, N, L), mk(1, N, L)
+        A, Dsk, bias = (torch.from_numpy(x).cuda() for x in workloads.channel_params(np.random.default_rng(c["seed"]), D, N))
+        y = torch.empty_like(u)
+        hl = torch.empty(1, D, N, device="cuda")
+        ms = time_kernel(lambda: ssm.scan_fwd(u, dl, B, C, A, Dsk, bias, z, y=y, h_last=hl), max(3, steps // 4),
+                         warmup, stream)
+        nb, ne = scan_counts(L, D, N, 2, 2, 1)
+        out[name] = {"ms": round(ms, 4), "tokens_per_s": L / (ms * 1e-3),
+                     "sfu_frac": round(ne / (ms * 1e-3) / sfu_peak, 4),
+                     "hbm_gbs": round(nb / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm_peak, 4)}
+        del u, dl, z, B, C, y
+    # decode: 256 of 1024 slots, D=5120, N=16; the state (84 MB) fits in L2, so L2 is flushed
+    c = workloads.CONFIGS["decode_bf16"]
+    prob = workloads.decode_problem(c["num_slots"], c["dim"], c["dstate"], c["R"], c["dtype"], c["seed"])
+    pool = torch.from_numpy(prob.pool0).cuda()
+    slots = torch.from_numpy(prob.slot_ids).cuda()
+    A, Dsk, bias = (torch.from_numpy(x).cuda() for x in (prob.A, prob.Dskip, prob.bias))
+    x = workloads.decode_step_inputs(prob, 0)
+    bf = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)  # noqa: E731
+    u, dl, z, B, C = bf(x["u"]), bf(x["delta"]), bf(x["z"]), bf(x["B"]), bf(x["C"])
+    y = torch.empty_like(u)
+    scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    ms = time_kernel(lambda: ssm.state_update(pool, slots, u, dl, B, C, A, Dsk, bias, z, y=y), steps, warmup, stream,
+                     flush=lambda: scratch.add_(1))
+    R, D, N = c["R"], c["dim"], c["dstate"]
+    nb = R * D * N * 4 * 2 + R * D * 2 * 4 + R * N * 2 * 2 + D * (N + 2) * 4
+    out["decode_bf16"] = {"ms_per_step": round(ms, 5), "tokens_per_s": R / (ms * 1e-3),
+                          "hbm_gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                          "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm_peak, 4), "l2": "flushed before each step"}
+    return out
+
+
+# ------------------------------------------------------------------------------ arms
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    c = workloads.CONFIGS[WORKLOAD]
+    lens = workloads.varlen_lengths(c["nseq"], c["len_lo"], c["len_hi"], c["seed"])
+    inp = workloads.varlen_inputs(lens, c["dim"], c["dstate"], c["dtype"], c["seed"])
+    # each step: the oracle over a channel sample sized so that the whole run takes ~2 minutes
+    cpu = CpuOracle(inp, budget_s=min(10.0, max(0.05, 120.0 / max(1, args.steps + args.warmup))))
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        r = cpu.measure()
+        if i >= args.warmup:
+            per_step.append(r)
+    value = statistics.median(r["value"] for r in per_step)
+    T = inp.meta["total"]
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": T / value * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_desc(T)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": per_step[-1]["cores"], "kind": "oracle",
+                             "sample": per_step[-1]["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def workload_desc(T):
+    return (f"varlen_bf16: 16 packed sequences, lengths U[256,4096] ({T} tokens on rank 0), D=2048, N=16, "
+            "bf16 in/out, fp32 state, SiLU(z) gate")
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import selective_state_space_15_b200 as ssm
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    ssm.load()
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    hbm_peak, sm_max, peak_kind = peaks()
+    sfu_peak = N_SM * SFU_PER_CLK_PER_SM * sm_max * 1e6
+
+    inp, host, dev, T, pitch = varlen_device_inputs(rank, device)
+    D, N, nseq = inp.u.shape[0], inp.A.shape[1], inp.meta["nseq"]
+    y = torch.empty((D, pitch), dtype=torch.bfloat16, device=device)
+    hl = torch.empty((nseq, D, N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ssm.scan_fwd_varlen(dev["u"], dev["delta"], dev["B"], dev["C"], dev["A"], dev["cu"], dev["Dskip"],
+                            dev["bias"], dev["z"], y=y, h_last=hl, total=T, stream=stream)
+
+    # ---- kernel-resident timing (inputs in HBM; 0.58 GB of inputs per step > 126 MB L2)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_local = e0.elapsed_time(e1)
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    tokens_local = T * args.steps
+    ms_max, tokens_all = ms_local, tokens_local
+    if dist:
+        t = torch.tensor([ms_local, float(tokens_local)], dtype=torch.float64, device=device)
+        m = t.clone()
+        dist.all_reduce(m[0:1], op=dist.ReduceOp.MAX)
+        dist.all_reduce(m[1:2], op=dist.ReduceOp.SUM)
+        ms_max, tokens_all = float(m[0]), float(m[1])
+    value = tokens_all / (ms_max * 1e-3)
+    ms_per_step = ms_max / args.steps
+
+    if args.kernel_only:
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                              "mode": "kernel-only (ncu capture; e2e, CPU and secondary legs not run)"}))
+        return 0
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    y_host = torch.empty((D, pitch), dtype=torch.bfloat16).pin_memory()
+    hl_host = torch.empty((nseq, D, N), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y_host.numel() * y_host.element_size() + hl_host.numel() * hl_host.element_size()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev[k].copy_(v, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        hl_host.copy_(hl, non_blocking=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(min(args.warmup, 3)):
+        e2e_step()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    e2e_tokens = T * e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms, float(e2e_tokens)], dtype=torch.float64, device=device)
+        dist.all_reduce(t[0:1], op=dist.ReduceOp.MAX)
+        dist.all_reduce(t[1:2], op=dist.ReduceOp.SUM)
+        e2e_ms, e2e_tokens = float(t[0]), float(t[1])
+    e2e_value = e2e_tokens / (e2e_ms * 1e-3)
+
+    extra = None
+    if rank == 0 and world == 1 and not args.no_secondary:
+        extra = secondary(args.steps, args.warmup, hbm_peak, sfu_peak)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    # roofline of the (single) kernel on rank 0's batch, per launch
+    launch_s = ms_local / args.steps * 1e-3
+    nbytes, nexps = scan_counts(T, D, N, 2, 2, nseq)
+    traffic = ncu_traffic(WORKLOAD)
+    cpu = cpu_oracle_rate(inp) if world == 1 else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(T), "tokens_per_step_rank0": T, "global_batch_tokens": tokens_all / args.steps,
+                   "l2": "inputs 0.58 GB per step > 126 MB L2; no flush", "parallelism": f"dp{world} (independent batches)"},
+        "roofline": {"bound": "alu", "unit": "Gexp/s", "achieved": nexps / launch_s / 1e9, "peak": sfu_peak / 1e9,
+                     "frac": nexps / launch_s / sfu_peak, "traffic": traffic,
+                     "peak_note": f"MUFU: {N_SM} SMs x {SFU_PER_CLK_PER_SM} ex2/clk x {sm_max:.0f} MHz; exps/token = D(N+2)"},
+        "roofline_hbm": {"bound": "hbm", "unit": "GB/s", "achieved": nbytes / launch_s / 1e9, "peak": hbm_peak,
+                         "frac": nbytes / launch_s / 1e9 / hbm_peak, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": nbytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if extra:
+        line["secondary"] = extra
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-secondary", action="store_true", help="skip the long-sequence/decode figures")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="only the warm-up and timed kernel steps (for ncu captures); prints a short line")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,159 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 (sm_100a) selective-scan library (libssm_scan.so).
+ *
+ * The operation (Mamba selective scan).  For every sequence b, channel d and state n:
+ *
+ *     Delta_t = softplus(delta[b,d,t] + delta_bias[d])
+ *     h_t[n]  = exp(Delta_t * A[d,n]) * h_{t-1}[n] + Delta_t * B[b,n,t] * u[b,d,t]
+ *     y[b,d,t] = (sum_n C[b,n,t] * h_t[n] + Dskip[d] * u[b,d,t]) * silu(z[b,d,t])
+ *
+ * Sources (web pages on the subject, cited by title and section):
+ *   - "会议长序列建模状态空间模型加速：深度剖析Mamba硬件感知算子融合与选择性扫描并行化策略"
+ *     (ufo.work) §1.1: the recurrence with Abar = exp(Delta A), Bbar = Delta B, y = C h and
+ *     input-dependent Delta, B, C; §3.1: chunk transfer operators composed across chunks;
+ *     §4.1: a persistent state pool and a one-token update kernel; §4.2: packed sequences with
+ *     cu_seqlens and a state reset at each boundary.
+ *   - "企业官网建设流程全解析" (discosf.com) §1.1: the skip term y = C h + D x; §1.3:
+ *     Delta = softplus of a per-token linear map (here: delta + per-channel bias).
+ *   The pages do not fix the bias placement or the output gate; this library puts the bias
+ *   inside the softplus and multiplies the whole output by silu(z) = z * sigmoid(z) when z is
+ *   given.  The gated value never feeds back into the state.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates device memory and never synchronises the stream (except
+ *     ssm_get_device_status, which must read a device word back).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Errors are returned as ssm_status_t; nothing is thrown.  Argument checks on the host
+ *     happen before any launch: on error nothing is launched and outputs are untouched.
+ *     Problems found by a kernel (e.g. an out-of-range slot id) are recorded in a device
+ *     status word read by ssm_get_device_status.
+ *   - Element strides are in elements; the time axis always has stride 1.  A stride of 0
+ *     means "contiguous" (the natural value for the documented layout).
+ *   - Inputs u, delta, z, B, C have the dtype `dtype`; y has it too unless y_fp32 is set
+ *     (then y is float32).  A, Dskip, delta_bias and all states (h0, h_last, the decode pool)
+ *     are float32.  Arithmetic is float32; a bf16 y is rounded to nearest-even once, at the
+ *     store.
+ *   - Supported state sizes: dstate in {16, 32, 64, 128} for the scans, any multiple of 4
+ *     up to 128 for the decode update.  Other values return SSM_ERR_UNSUPPORTED.
+ *   - Fast path: when every tensor base is 16-byte aligned and every row stride is a
+ *     multiple of 16 bytes, inputs are staged with 16-byte asynchronous copies.  Other
+ *     layouts are accepted and take a slower element-wise staging path.
+ */
+#ifndef SSM_SCAN_H_
+#define SSM_SCAN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSM_ABI_VERSION 1
+
+typedef enum {
+  SSM_OK = 0,
+  SSM_ERR_INVALID_ARG = 1, /* null pointer where one is required, bad size/stride/alignment  */
+  SSM_ERR_UNSUPPORTED = 2, /* a valid request this build has no kernel for (e.g. dstate = 24) */
+  SSM_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch error, no device, ...)      */
+  SSM_ERR_BAD_SLOT = 4,    /* device-detected: a decode slot id outside [0, num_slots)       */
+  SSM_ERR_TIMEOUT = 5,     /* device-detected: a bounded wait on another CTA gave up          */
+  SSM_ERR_WORKSPACE = 6    /* workspace pointer/size smaller than ssm_scan_workspace_size()   */
+} ssm_status_t;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
+
+/* Opaque CUDA stream handle; pass a cudaStream_t (they are the same pointer type). */
+typedef struct CUstream_st *ssm_stream_t;
+
+/*
+ * Problem description shared by all entry points.
+ *
+ * Fixed-length batch (ssm_scan_fwd):
+ *   u, delta, z, y : [batch][dim][seqlen]   element (b,d,t) at b*x_batch_stride + d*x_dim_stride + t
+ *   B, C           : [batch][dstate][seqlen] element (b,n,t) at b*bc_batch_stride + n*bc_state_stride + t
+ *   A              : [dim][dstate] contiguous; Dskip, delta_bias : [dim]
+ *   h0, h_last     : [batch][dim][dstate] contiguous
+ * Packed varlen (ssm_scan_fwd_varlen): batch = 1 and seqlen = total tokens T; sequences are
+ *   the column ranges [cu_seqlens[i], cu_seqlens[i+1]) of u, delta, z, y ([dim][T], row
+ *   stride x_dim_stride >= T) and of B, C ([dstate][T], row stride bc_state_stride >= T);
+ *   h0, h_last : [nseq][dim][dstate].
+ * Decode (ssm_state_update): batch = R requests, seqlen = 1; u, delta, z, y : [R][dim] with row
+ *   stride x_batch_stride (>= dim); B, C : [R][dstate] with row stride bc_batch_stride.
+ *
+ * Optional pointers (may be NULL): z (no gate), Dskip (= 0), delta_bias (= 0), h0 (zero
+ * state), h_last (final state not written).  Required: u, delta, B, C, A, y.
+ */
+typedef struct ssm_scan_params {
+  ssm_dtype_t dtype;       /* dtype of u, delta, z, B, C (and of y unless y_fp32 is set)       */
+  int32_t y_fp32;          /* nonzero: y is written as float32 whatever `dtype` is             */
+  int64_t batch;
+  int64_t dim;
+  int64_t dstate;
+  int64_t seqlen;
+  int64_t x_batch_stride;  /* 0 -> dim * x_dim_stride (batch mode); dim (decode)            */
+  int64_t x_dim_stride;    /* 0 -> seqlen                                                    */
+  int64_t bc_batch_stride; /* 0 -> dstate * bc_state_stride (batch mode); dstate (decode)    */
+  int64_t bc_state_stride; /* 0 -> seqlen                                                    */
+  const void *u;
+  const void *delta;
+  const void *z;
+  const void *B;
+  const void *C;
+  const float *A;
+  const float *Dskip;
+  const float *delta_bias;
+  const float *h0;
+  void *y;
+  float *h_last;
+} ssm_scan_params;
+
+/*
+ * Fixed-length batched prefill scan (ufo.work page §1.1 recurrence, §3.1 chunked carry).
+ * `workspace` may be NULL when ssm_scan_workspace_size() returns 0; otherwise it must point
+ * to that many bytes of device memory that no concurrent call uses.  Its contents on entry
+ * do not matter.
+ */
+ssm_status_t ssm_scan_fwd(const ssm_scan_params *p, void *workspace, size_t workspace_bytes,
+                          ssm_stream_t stream);
+
+/*
+ * Packed variable-length scan (ufo.work page §4.2): `cu_seqlens` is a DEVICE int32 array of
+ * nseq+1 non-decreasing offsets with cu_seqlens[0] = 0 and cu_seqlens[nseq] = p->seqlen.
+ * Each sequence starts from h0[i] (or zero) and h_last[i] receives its final state; empty
+ * sequences produce h_last[i] = h0[i] (or zero).  The offsets are read on the device only.
+ */
+ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seqlens, int64_t nseq,
+                                 void *workspace, size_t workspace_bytes, ssm_stream_t stream);
+
+/*
+ * One decode step over a slot-indexed state pool (ufo.work page §4.1 and its second
+ * article §4.1): for each request r, h = pool[slot_ids[r]] ([dim][dstate] float32) advances
+ * by one token in place and y[r] is written.  `slot_ids` is a DEVICE int32 array of R ids;
+ * ids must be distinct (duplicates race).  An id outside [0, num_slots) is skipped (its y row
+ * is not written) and SSM_ERR_BAD_SLOT is recorded in the device status word.
+ * p->batch must equal R and p->seqlen must be 1; p->h0 and p->h_last are ignored.
+ */
+ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slot_ids, int64_t R,
+                              const ssm_scan_params *p, ssm_stream_t stream);
+
+/* Bytes of device workspace the scan entry points need for this problem (0 if none).
+ * For the fixed-length scan pass nseq = 0. */
+size_t ssm_scan_workspace_size(const ssm_scan_params *p, int64_t nseq);
+
+/* Synchronises `stream`, then reads and clears the device status word (SSM_OK if no kernel
+ * reported a problem since the last call). */
+ssm_status_t ssm_get_device_status(ssm_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *ssm_status_string(ssm_status_t s);
+
+/* SSM_ABI_VERSION of the built library. */
+int ssm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H_ */

@@ -1,0 +1,256 @@
+"""Thin Python binding over libssm_scan.so (the C ABI declared in include/ssm_scan.h).
+
+Argument marshalling only: every step of the selective scan runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current CUDA stream.  If the shared
+library has not been built, loading raises -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB_PATH, build  # noqa: F401  (build is re-exported for convenience)
+
+SSM_OK = 0
+_STATUS = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED", 3: "SSM_ERR_CUDA",
+           4: "SSM_ERR_BAD_SLOT", 5: "SSM_ERR_TIMEOUT", 6: "SSM_ERR_WORKSPACE"}
+SSM_F32, SSM_BF16 = 0, 1
+ABI_VERSION = 1
+
+# Every function the header declares; tests check the library exports all of them.
+EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
+            "ssm_get_device_status", "ssm_status_string", "ssm_abi_version")
+
+
+class SSMError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_STATUS.get(code, code)}")
+
+
+class ScanParams(ctypes.Structure):
+    """Mirror of ssm_scan_params."""
+    _fields_ = [
+        ("dtype", ctypes.c_int), ("y_fp32", ctypes.c_int32),
+        ("batch", ctypes.c_int64), ("dim", ctypes.c_int64), ("dstate", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64),
+        ("x_batch_stride", ctypes.c_int64), ("x_dim_stride", ctypes.c_int64),
+        ("bc_batch_stride", ctypes.c_int64), ("bc_state_stride", ctypes.c_int64),
+        ("u", ctypes.c_void_p), ("delta", ctypes.c_void_p), ("z", ctypes.c_void_p),
+        ("B", ctypes.c_void_p), ("C", ctypes.c_void_p),
+        ("A", ctypes.c_void_p), ("Dskip", ctypes.c_void_p), ("delta_bias", ctypes.c_void_p),
+        ("h0", ctypes.c_void_p), ("y", ctypes.c_void_p), ("h_last", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the built library.  Raises FileNotFoundError if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise FileNotFoundError(
+            f"{p} is missing: build the CUDA library first (python -m selective_state_space_15_b200.build)")
+    lib = ctypes.CDLL(p)
+    P, I64, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+    pp = ctypes.POINTER(ScanParams)
+    lib.ssm_scan_fwd.argtypes = [pp, P, S, P]
+    lib.ssm_scan_fwd_varlen.argtypes = [pp, P, I64, P, S, P]
+    lib.ssm_state_update.argtypes = [P, I64, P, I64, pp, P]
+    lib.ssm_scan_workspace_size.argtypes = [pp, I64]
+    lib.ssm_scan_workspace_size.restype = S
+    lib.ssm_get_device_status.argtypes = [P]
+    lib.ssm_status_string.argtypes = [ctypes.c_int]
+    lib.ssm_status_string.restype = ctypes.c_char_p
+    lib.ssm_abi_version.argtypes = []
+    for f in ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_get_device_status"):
+        getattr(lib, f).restype = ctypes.c_int
+    if lib.ssm_abi_version() != ABI_VERSION:
+        raise RuntimeError(f"libssm_scan ABI {lib.ssm_abi_version()} != binding ABI {ABI_VERSION}")
+    if path is None:
+        _lib = lib
+    return lib
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    if t.dtype == torch.float32:
+        return SSM_F32
+    raise TypeError(f"unsupported input dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _check(code: int, where: str):
+    if code != SSM_OK:
+        raise SSMError(code, where)
+
+
+def _y_fp32(u, y):
+    """1 when y is float32 while the inputs are bf16 (the float32-output option)."""
+    import torch
+    if y is None or y.dtype == u.dtype:
+        return 0
+    if y.dtype == torch.float32:
+        return 1
+    raise TypeError("y must have the input dtype or float32")
+
+
+def _time_contig(*ts):
+    for t in ts:
+        if t is not None and t.stride(-1) != 1:
+            raise ValueError("the time (last) axis must have stride 1")
+
+
+def _f32(t):
+    import torch
+    if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+        raise ValueError("A, Dskip, delta_bias and states must be contiguous float32")
+    return t
+
+
+# ----------------------------------------------------------------------------- scans
+
+def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None):
+    """Fill ScanParams for the fixed-length layout u/delta/z/y [b, D, L], B/C [b, N, L]."""
+    bsz, dim, L = u.shape
+    N = A.shape[1]
+    _time_contig(u, delta, z, B, C, y)
+    for t in (delta, z, y):
+        if t is not None and (t.shape != u.shape or t.stride() != u.stride()):
+            raise ValueError("delta, z and y must match u's shape and strides")
+    if B.shape != (bsz, N, L) or C.shape != B.shape or C.stride() != B.stride():
+        raise ValueError("B and C must be [batch, dstate, seqlen] with equal strides")
+    for t in (A, Dskip, delta_bias, h0, h_last):
+        _f32(t)
+    p = ScanParams()
+    p.dtype = _dtype_code(u)
+    p.y_fp32 = _y_fp32(u, y)
+    p.batch, p.dim, p.dstate, p.seqlen = bsz, dim, N, L
+    p.x_batch_stride, p.x_dim_stride = u.stride(0), u.stride(1)
+    p.bc_batch_stride, p.bc_state_stride = B.stride(0), B.stride(1)
+    p.u, p.delta, p.z, p.B, p.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
+    p.A, p.Dskip, p.delta_bias, p.h0 = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(h0)
+    p.y, p.h_last = _ptr(y), _ptr(h_last)
+    return p
+
+
+def scan_fwd(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None,
+             return_last_state=True, stream=None, y_dtype=None):
+    """Selective scan over a fixed-length batch.  Returns (y, h_last).
+
+    y is allocated in ``y_dtype`` (default: the input dtype; float32 is also accepted)."""
+    import torch
+    y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
+    if h_last is None and return_last_state:
+        h_last = torch.empty((u.shape[0], u.shape[1], A.shape[1]), device=u.device, dtype=torch.float32)
+    p = scan_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last)
+    lib = load()
+    ws = lib.ssm_scan_workspace_size(ctypes.byref(p), 0)
+    wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
+    _check(lib.ssm_scan_fwd(ctypes.byref(p), _ptr(wbuf), ws, _stream(stream)), "ssm_scan_fwd")
+    return y, h_last
+
+
+def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None,
+                  total=None):
+    """ScanParams for the packed layout u/delta/z/y [D, T(+pad)], B/C [N, T(+pad)].
+
+    ``total`` is the number of packed tokens T when the rows are padded beyond it.
+    """
+    dim, width = u.shape
+    T = width if total is None else int(total)
+    N = A.shape[1]
+    _time_contig(u, delta, z, B, C, y)
+    for t in (delta, z, y):
+        if t is not None and (t.shape != u.shape or t.stride() != u.stride()):
+            raise ValueError("delta, z and y must match u's shape and strides")
+    if B.shape[0] != N or C.shape != B.shape or C.stride() != B.stride() or B.shape[1] < T:
+        raise ValueError("B and C must be [dstate, >=T] with equal strides")
+    for t in (A, Dskip, delta_bias, h0, h_last):
+        _f32(t)
+    p = ScanParams()
+    p.dtype = _dtype_code(u)
+    p.y_fp32 = _y_fp32(u, y)
+    p.batch, p.dim, p.dstate, p.seqlen = 1, dim, N, T
+    p.x_batch_stride, p.x_dim_stride = 0, u.stride(0)
+    p.bc_batch_stride, p.bc_state_stride = 0, B.stride(0)
+    p.u, p.delta, p.z, p.B, p.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
+    p.A, p.Dskip, p.delta_bias, p.h0 = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(h0)
+    p.y, p.h_last = _ptr(y), _ptr(h_last)
+    return p
+
+
+def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, z=None, h0=None, y=None,
+                    h_last=None, total=None, return_last_state=True, stream=None, y_dtype=None):
+    """Packed variable-length scan.  cu_seqlens: int32 device tensor [nseq+1].  Returns (y, h_last)."""
+    import torch
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 tensor")
+    nseq = cu_seqlens.shape[0] - 1
+    y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
+    if h_last is None and return_last_state:
+        h_last = torch.empty((nseq, u.shape[0], A.shape[1]), device=u.device, dtype=torch.float32)
+    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last, total)
+    lib = load()
+    ws = lib.ssm_scan_workspace_size(ctypes.byref(p), nseq)
+    wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
+    _check(lib.ssm_scan_fwd_varlen(ctypes.byref(p), _ptr(cu_seqlens), nseq, _ptr(wbuf), ws, _stream(stream)),
+           "ssm_scan_fwd_varlen")
+    return y, h_last
+
+
+def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, y=None, stream=None,
+                 y_dtype=None):
+    """One decode step in place on ``pool`` [S, D, N] float32.  u/delta/z [R, D]; B/C [R, N]."""
+    import torch
+    if slot_ids.dtype != torch.int32 or not slot_ids.is_contiguous():
+        raise ValueError("slot_ids must be a contiguous int32 tensor")
+    S, dim, N = pool.shape
+    R = slot_ids.shape[0]
+    _f32(pool)
+    for t in (A, Dskip, delta_bias):
+        _f32(t)
+    _time_contig(u, delta, z, B, C)
+    y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
+    p = ScanParams()
+    p.dtype = _dtype_code(u)
+    p.y_fp32 = _y_fp32(u, y)
+    p.batch, p.dim, p.dstate, p.seqlen = R, dim, N, 1
+    p.x_batch_stride, p.x_dim_stride = u.stride(0), 0
+    p.bc_batch_stride, p.bc_state_stride = B.stride(0), 0
+    for t in (delta, z, y):
+        if t is not None and t.stride(0) != u.stride(0):
+            raise ValueError("u, delta, z and y must share the row stride")
+    if C.stride(0) != B.stride(0):
+        raise ValueError("B and C must share the row stride")
+    p.u, p.delta, p.z, p.B, p.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
+    p.A, p.Dskip, p.delta_bias, p.y = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(y)
+    _check(load().ssm_state_update(_ptr(pool), S, _ptr(slot_ids), R, ctypes.byref(p), _stream(stream)),
+           "ssm_state_update")
+    return y
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream, then read-and-clear the library's device status word."""
+    return load().ssm_get_device_status(_stream(stream))
+
+
+def status_string(code: int) -> str:
+    return load().ssm_status_string(code).decode()

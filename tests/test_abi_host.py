@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel is launched).
+
+The library must build for sm_100a, load, export every function include/ssm_scan.h declares,
+and reject bad arguments on the host before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import selective_state_space_15_b200 as ssm
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "ssm_scan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssm.build()
+    return ssm.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssm_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_list():
+    assert declared_functions() == sorted(ssm.EXPORTED)
+
+
+def test_library_exports_every_declared_function(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.ssm_abi_version() == ssm.ABI_VERSION
+    for code, name in ssm._STATUS.items():
+        assert lib.ssm_status_string(code).decode() == name
+    assert lib.ssm_status_string(99).decode() == "SSM_ERR_UNKNOWN"
+
+
+def _params(**kw):
+    p = ssm.ScanParams()
+    p.dtype = ssm.SSM_BF16
+    p.batch, p.dim, p.dstate, p.seqlen = 1, 64, 16, 128
+    fake = 0x10000  # never dereferenced: every call below fails a host check first
+    p.u = p.delta = p.B = p.C = p.A = p.y = fake
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("u", None, 1), ("delta", None, 1), ("B", None, 1), ("C", None, 1), ("A", None, 1), ("y", None, 1),
+    ("dim", 0, 1), ("dstate", 0, 1), ("seqlen", -1, 1), ("batch", -1, 1), ("dtype", 7, 1),
+    ("dstate", 24, 2), ("dstate", 256, 2),
+    ("x_dim_stride", 100, 1),           # row stride shorter than the sequence
+    ("bc_state_stride", 100, 1),
+])
+def test_scan_rejects_bad_arguments_on_host(lib, field, value, code):
+    p = _params(**{field: value})
+    assert lib.ssm_scan_fwd(ctypes.byref(p), None, 0, None) == code
+
+
+def test_null_params_and_varlen_checks(lib):
+    assert lib.ssm_scan_fwd(None, None, 0, None) == 1
+    p = _params()
+    assert lib.ssm_scan_fwd_varlen(ctypes.byref(p), None, 4, None, 0, None) == 1   # no cu_seqlens
+    assert lib.ssm_scan_fwd_varlen(ctypes.byref(p), 0x10000, -1, None, 0, None) == 1
+    p2 = _params(batch=2)
+    assert lib.ssm_scan_fwd_varlen(ctypes.byref(p2), 0x10000, 4, None, 0, None) == 1  # varlen needs batch 1
+
+
+def test_state_update_host_checks(lib):
+    p = _params(batch=8, seqlen=1, dim=32, dstate=16)
+    fake = 0x10000
+    assert lib.ssm_state_update(None, 4, fake, 8, ctypes.byref(p), None) == 1
+    assert lib.ssm_state_update(fake, 4, None, 8, ctypes.byref(p), None) == 1
+    assert lib.ssm_state_update(fake, 0, fake, 8, ctypes.byref(p), None) == 1
+    assert lib.ssm_state_update(fake, 4, fake, 7, ctypes.byref(p), None) == 1      # batch != R
+    p2 = _params(batch=8, seqlen=1, dim=32, dstate=12)
+    assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p2), None) == 2     # 12/4 not a power of 2
+    p3 = _params(batch=8, seqlen=2, dim=32, dstate=16)
+    assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p3), None) == 1     # one token only
+    assert lib.ssm_state_update(fake + 4, 4, fake, 8, ctypes.byref(p), None) == 1  # pool not 16-byte aligned
+
+
+def test_workspace_size_query_is_host_only(lib):
+    p = _params()
+    assert lib.ssm_scan_workspace_size(ctypes.byref(p), 0) >= 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(FileNotFoundError):
+        ssm.load(str(tmp_path / "nope.so"))
