@@ -70,7 +70,7 @@ def test_decode_workload_1000_steps_channel_subset():
     slots_t = torch.from_numpy(prob.slot_ids).cuda()
     A, D, bias = (torch.from_numpy(x).cuda() for x in (prob.A, prob.Dskip, prob.bias))
     ch = np.arange(0, prob.dim, 64)
-    sub = prob.pool0[prob.slot_ids][:, ch].astype(np.float64)
+    sub = np.ascontiguousarray(prob.pool0[prob.slot_ids][:, ch], dtype=np.float64)
     mag = np.abs(sub)
     ids = np.arange(prob.R)
     worst = 0.0
