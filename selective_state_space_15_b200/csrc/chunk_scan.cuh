@@ -14,16 +14,20 @@
 // No h_t ever leaves registers; only y and the final state are written.  Each exponential
 // exp(Delta A) is evaluated once.
 //
-// Staging.  u, delta, z rows of the tile and the B, C rows of the chunk window are copied
-// into shared memory with 16-byte cp.async (double-buffered: chunk c+1 streams in while
-// chunk c is computed).  B and C are then converted to float32 in an interleaved layout
-// [n][KI/4][SPW] of float4 so that the SPW segment lanes read consecutive 16-byte words
-// (no bank conflicts) and the CPW channel groups of a warp read the same words (broadcast).
+// Staging.  u, delta, z rows of the tile (double-buffered) and the B, C rows of the chunk
+// window (single buffer, consumed right after arrival) are copied into shared memory while
+// the previous chunk is computed: one TMA bulk copy per row (cp.async.bulk completing on an
+// mbarrier) when every row is 16-byte aligned, element-wise loads otherwise.  B and C are
+// converted once per chunk to float32 in an interleaved [n][KI/4][SPW] float4 layout: the
+// SPW segment lanes read consecutive 16-byte words and the CPW channel groups of a warp
+// read the same words.  Chunks that lie entirely inside the sequence skip all masking.
 //
 // Windows start at the sequence start rounded down to a 16-byte boundary; steps outside
 // [seq_start, seq_end) are made identities (Delta = 0, Delta*u = 0, B = C = 0) and are not
 // stored, which also resets the state at packed-sequence boundaries ("ufo.work" §4.2).
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -41,47 +45,69 @@ struct ScanArgs {
   int ntiles;  // channel tiles per sequence
 };
 
+// Packed sequences are visited longest first (CTAs with low indices start first), which
+// keeps the tail short when lengths differ; the ordering is computed in each CTA, so it is
+// only done for modest sequence counts.
+constexpr int kMaxSortedSeqs = 64;
+
 template <typename T, int N, int KI, int SPW, int CPW, int WARPS>
 struct ChunkCfg {
   static constexpr int kTC = SPW * KI;     // chunk length (time steps)
   static constexpr int kCT = CPW * WARPS;  // channels per CTA
   static constexpr int kVec = Elem<T>::kVec;
   static constexpr int kThreads = WARPS * 32;
+  static constexpr int kVPR = kTC / kVec;  // 16-byte vectors per staged row
   // shared memory layout (bytes)
-  static constexpr size_t kXBytes = size_t(3) * kCT * kTC * sizeof(T);  // u, delta, z
+  static constexpr size_t kXBytes = size_t(3) * kCT * kTC * sizeof(T);  // u, delta, z of one chunk
   static constexpr size_t kBCRawBytes = size_t(2) * N * kTC * sizeof(T);
-  static constexpr size_t kStageBytes = kXBytes + kBCRawBytes;
   static constexpr size_t kConvBytes = size_t(2) * N * kTC * sizeof(float);
-  static constexpr size_t kParamBytes = size_t(2) * kCT * N * sizeof(float) + size_t(2) * kCT * sizeof(float);
-  static constexpr size_t kSmemBytes = 2 * kStageBytes + kConvBytes + kParamBytes;
+  static constexpr size_t kParamBytes =
+      size_t(2) * kCT * N * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
+  static constexpr size_t kSmemBytes = 2 * kXBytes + kBCRawBytes + kConvBytes + kParamBytes;
   static_assert(KI % 4 == 0 && KI % kVec == 0, "a lane's steps must be whole float4 and 16-byte vectors");
-  static_assert(kTC % kVec == 0, "chunk must be whole vectors");
   static_assert(32 % SPW == 0 && CPW * SPW == 32, "lane split");
 };
 
+
 template <typename T, typename TO, int N, int KI, int SPW, int CPW, int WARPS, bool HAS_Z, bool VEC>
-__global__ void __launch_bounds__(WARPS * 32)
+__global__ void __launch_bounds__(WARPS * 32, (WARPS <= 8 ? 16 / WARPS : 1))
 chunk_scan_kernel(const ScanArgs args) {
   using Cfg = ChunkCfg<T, N, KI, SPW, CPW, WARPS>;
-  constexpr int TC = Cfg::kTC, CT = Cfg::kCT, V = Cfg::kVec, NT = Cfg::kThreads;
+  constexpr int TC = Cfg::kTC, CT = Cfg::kCT, V = Cfg::kVec, NT = Cfg::kThreads, VPR = Cfg::kVPR;
+  constexpr int LV = KI / V;  // 16-byte vectors per lane
   constexpr bool kFast = Elem<T>::kFast;
 
   extern __shared__ __align__(16) unsigned char smem[];
-  T *stage[2];
-  stage[0] = reinterpret_cast<T *>(smem);
-  stage[1] = reinterpret_cast<T *>(smem + Cfg::kStageBytes);
-  float4 *Bs4 = reinterpret_cast<float4 *>(smem + 2 * Cfg::kStageBytes);  // [N][KI/4][SPW]
+  T *const xs0 = reinterpret_cast<T *>(smem);  // u, delta, z rows; buffer b at xs0 + b * kXElems
+  constexpr size_t kXElems = Cfg::kXBytes / sizeof(T);
+  T *bcraw = reinterpret_cast<T *>(smem + 2 * Cfg::kXBytes);
+  float4 *Bs4 = reinterpret_cast<float4 *>(smem + 2 * Cfg::kXBytes + Cfg::kBCRawBytes);  // [N][KI/4][SPW]
   float4 *Cs4 = Bs4 + N * (TC / 4);
   float *A2s = reinterpret_cast<float *>(Cs4 + N * (TC / 4));  // [CT][N]  A * log2(e)
   float *carry_s = A2s + CT * N;                                // [CT][N]
   float *Dsk = carry_s + CT * N;                                // [CT]
   float *bias_s = Dsk + CT;                                     // [CT]
+  int *order = reinterpret_cast<int *>(bias_s + CT);            // [kMaxSortedSeqs]
 
   const int tile = blockIdx.x % args.ntiles;
-  const int s = blockIdx.x / args.ntiles;
+  int s = blockIdx.x / args.ntiles;
   const int d0 = tile * CT;
   int64_t t_lo, t_hi, xbase, bcbase;
   if (args.cu_seqlens) {
+    if (args.nseq <= kMaxSortedSeqs) {
+      // rank sequences by length (descending, ties by index); order[rank] = sequence
+      for (int i = threadIdx.x; i < args.nseq; i += NT) {
+        const int li = args.cu_seqlens[i + 1] - args.cu_seqlens[i];
+        int rank = 0;
+        for (int j = 0; j < args.nseq; ++j) {
+          const int lj = args.cu_seqlens[j + 1] - args.cu_seqlens[j];
+          rank += (lj > li) || (lj == li && j < i);
+        }
+        order[rank] = i;
+      }
+      __syncthreads();
+      s = order[s];
+    }
     t_lo = args.cu_seqlens[s];
     t_hi = args.cu_seqlens[s + 1];
     xbase = 0;
@@ -110,65 +136,65 @@ chunk_scan_kernel(const ScanArgs args) {
     bias_s[i] = (ok && args.bias) ? args.bias[d] : 0.f;
   }
 
-  const T *gu = static_cast<const T *>(args.u);
-  const T *gdl = static_cast<const T *>(args.delta);
-  const T *gz = static_cast<const T *>(args.z);
-  const T *gB = static_cast<const T *>(args.B);
-  const T *gC = static_cast<const T *>(args.C);
+  // tensor bases are read from the kernel parameters where used (no registers held across
+  // the chunk loop)
+#define SSM_GU static_cast<const T *>(args.u)
+#define SSM_GDL static_cast<const T *>(args.delta)
+#define SSM_GZ static_cast<const T *>(args.z)
+#define SSM_GB static_cast<const T *>(args.B)
+#define SSM_GC static_cast<const T *>(args.C)
+  constexpr int nx = HAS_Z ? 3 : 2;
 
-  // Stage chunk `c` into buffer `buf`: rows [x: 3*CT][bc: 2*N], TC elements each.
-  auto stage_chunk = [&](int buf, int c) {
-    T *dst = stage[buf];
+  __shared__ __align__(8) uint64_t bars[2];  // chunk-arrival barriers of the two X buffers
+  const int nvalid_ch = int(min64(CT, args.dim - d0));
+  // rows are readable up to the seqlen rounded up to a 16-byte vector (row strides are
+  // multiples of 16 bytes on this path)
+  const int64_t seqlen_r = (args.seqlen + V - 1) / V * V;
+
+  // TMA: chunk c's u/delta/z rows into X buffer `buf` and its B/C rows into bcraw.
+  auto issue_chunk = [&](int buf, int c) {
     const int64_t wstart = w0 + int64_t(c) * TC;
-    constexpr int nx = HAS_Z ? 3 : 2;
-    constexpr int rows = nx * CT + 2 * N;
-    if constexpr (VEC) {
-      constexpr int vpr = TC / V;  // vectors per row
-      for (int i = threadIdx.x; i < rows * vpr; i += NT) {
-        const int row = i / vpr, v = i % vpr;
-        const int64_t t = wstart + int64_t(v) * V;
-        const T *base, *src;
-        int64_t lim;
-        T *sdst;
-        if (row < nx * CT) {
-          const int which = row / CT, ch = row % CT;
-          const int64_t d = d0 + ch;
-          base = which == 0 ? gu : (which == 1 ? gdl : gz);
-          lim = d < args.dim ? args.seqlen : 0;
-          src = base + (d < args.dim ? xbase + d * args.x_dim_stride + t : 0);
-          sdst = dst + (size_t(which) * CT + ch) * TC + v * V;
-        } else {
-          const int r2 = row - nx * CT, which = r2 / N, n = r2 % N;
-          base = which == 0 ? gB : gC;
-          lim = args.seqlen;
-          src = base + bcbase + int64_t(n) * args.bc_state_stride + t;
-          sdst = dst + size_t(3) * CT * TC + (size_t(which) * N + n) * TC + v * V;
-        }
-        int64_t avail = lim - t;
-        avail = avail < 0 ? 0 : (avail > V ? V : avail);
-        // a zero-byte copy reads nothing; point it at the tensor base all the same
-        cp_async_16(sdst, avail > 0 ? (const void *)src : (const void *)base, int(avail * sizeof(T)));
+    const int64_t wend = min64(wstart + TC, seqlen_r);
+    const uint32_t row_bytes = uint32_t((wend - wstart) * int64_t(sizeof(T)));
+    T *xdst = xs0 + buf * kXElems;
+    fence_proxy_async_smem();
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(&bars[buf], row_bytes * uint32_t(nx * nvalid_ch + 2 * N));
+    for (int r = threadIdx.x; r < nx * CT + 2 * N; r += NT) {
+      if (r < nx * CT) {
+        const int which = r / CT, ch = r % CT;
+        if (ch >= nvalid_ch) continue;
+        const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
+        bulk_g2s(xdst + size_t(r) * TC, base + xbase + (d0 + ch) * args.x_dim_stride + wstart, row_bytes,
+                 &bars[buf]);
+      } else {
+        const int r2 = r - nx * CT, which = r2 / N, n = r2 % N;
+        const T *base = which == 0 ? SSM_GB : SSM_GC;
+        bulk_g2s(bcraw + size_t(r2) * TC, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, row_bytes,
+                 &bars[buf]);
       }
-    } else {
-      for (int i = threadIdx.x; i < rows * TC; i += NT) {
-        const int row = i / TC, j = i % TC;
-        const int64_t t = wstart + j;
-        T val = Elem<T>::from_f32(0.f);
-        T *sdst;
-        if (row < nx * CT) {
-          const int which = row / CT, ch = row % CT;
-          const int64_t d = d0 + ch;
-          const T *base = which == 0 ? gu : (which == 1 ? gdl : gz);
-          if (d < args.dim && t < args.seqlen) val = base[xbase + d * args.x_dim_stride + t];
-          sdst = dst + (size_t(which) * CT + ch) * TC + j;
-        } else {
-          const int r2 = row - nx * CT, which = r2 / N, n = r2 % N;
-          const T *base = which == 0 ? gB : gC;
-          if (t < args.seqlen) val = base[bcbase + int64_t(n) * args.bc_state_stride + t];
-          sdst = dst + size_t(3) * CT * TC + (size_t(which) * N + n) * TC + j;
-        }
-        *sdst = val;
-      }
+    }
+  };
+  // Element-wise staging (rows not 16-byte aligned): u/delta/z rows into xs[buf], B/C into bcraw.
+  auto stage_scalar = [&](int buf, int c) {
+    T *dst = xs0 + buf * kXElems;
+    const int64_t wstart = w0 + int64_t(c) * TC;
+    for (int i = threadIdx.x; i < nx * CT * TC; i += NT) {
+      const int row = i / TC, j = i % TC;
+      const int which = row / CT, ch = row % CT;
+      const int64_t d = d0 + ch, t = wstart + j;
+      const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
+      T val = Elem<T>::from_f32(0.f);
+      if (d < args.dim && t < args.seqlen) val = base[xbase + d * args.x_dim_stride + t];
+      dst[size_t(row) * TC + j] = val;
+    }
+    for (int i = threadIdx.x; i < 2 * N * TC; i += NT) {
+      const int row = i / TC, j = i % TC;
+      const int which = row / N, n = row % N;
+      const int64_t t = wstart + j;
+      const T *base = which == 0 ? SSM_GB : SSM_GC;
+      T val = Elem<T>::from_f32(0.f);
+      if (t < args.seqlen) val = base[bcbase + int64_t(n) * args.bc_state_stride + t];
+      bcraw[size_t(row) * TC + j] = val;
     }
   };
 
@@ -179,63 +205,100 @@ chunk_scan_kernel(const ScanArgs args) {
   const bool ch_ok = d < args.dim;
 
   if constexpr (VEC) {
-    if (nchunks > 0) stage_chunk(0, 0);
-    cp_async_commit();
+    if (threadIdx.x == 0) {
+      mbar_init(&bars[0], 1);
+      mbar_init(&bars[1], 1);
+      mbar_init_fence();
+    }
+    __syncthreads();
+    if (nchunks > 0) issue_chunk(0, 0);
   }
 
   for (int c = 0; c < nchunks; ++c) {
     const int buf = c & 1;
     const int64_t wstart = w0 + int64_t(c) * TC;
     if constexpr (VEC) {
-      cp_async_wait_all();
-      __syncthreads();  // chunk c visible; everyone is done with chunk c-1
-      if (c + 1 < nchunks) stage_chunk(buf ^ 1, c + 1);
-      cp_async_commit();
+      mbar_wait_bounded(&bars[buf], uint32_t(c >> 1) & 1u);
     } else {
-      __syncthreads();  // everyone is done with chunk c-1's buffers
-      stage_chunk(buf, c);
-      __syncthreads();
+      stage_scalar(buf, c);
     }
-    const T *X = stage[buf];
-    const T *Braw = X + size_t(3) * CT * TC;
-    const T *Craw = Braw + size_t(N) * TC;
+    __syncthreads();  // chunk c visible to all; everyone is done with chunk c-1
+    // chunk-relative sequence bounds; a chunk strictly inside the sequence needs no masks
+    const int rel_lo = int(max64(t_lo - wstart, -1));
+    const int rel_hi = int(min64(t_hi - wstart, TC + 1));
+    const bool full = rel_lo <= 0 && rel_hi >= TC;
 
-    // B, C -> float32 interleaved layout, steps outside the sequence zeroed.
-    for (int i = threadIdx.x; i < N * (TC / 4); i += NT) {
-      const int sg = i % SPW, q = (i / SPW) % (KI / 4), n = i / (SPW * (KI / 4));
-      const int tl = sg * KI + q * 4;
-      float bv[4], cv[4];
+    // B, C -> float32 interleaved layout (steps outside the sequence zeroed).
+    auto convert = [&](auto masked_tag) {
+      constexpr bool kMasked = decltype(masked_tag)::value;
+      for (int i = threadIdx.x; i < 2 * N * VPR; i += NT) {
+        const int row = i / VPR, v = i % VPR;  // row < N: B, else C
+        const int n = row % N;
+        float4 *dstv = row < N ? Bs4 : Cs4;
+        float raw[V];
+        unpack16<T>(*reinterpret_cast<const uint4 *>(bcraw + size_t(row) * TC + v * V), raw);
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int64_t tg = wstart + tl + r;
-        const bool in = tg >= t_lo && tg < t_hi;
-        bv[r] = in ? Elem<T>::to_f32(Braw[size_t(n) * TC + tl + r]) : 0.f;
-        cv[r] = in ? Elem<T>::to_f32(Craw[size_t(n) * TC + tl + r]) : 0.f;
+        for (int g = 0; g < V / 4; ++g) {
+          const int tl = v * V + g * 4;  // chunk-local step of the first of 4
+          const int sg = tl / KI, q = (tl % KI) / 4;
+          float f[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) f[r] = (!kMasked || (tl + r >= rel_lo && tl + r < rel_hi)) ? raw[g * 4 + r] : 0.f;
+          dstv[(n * (KI / 4) + q) * SPW + sg] = make_float4(f[0], f[1], f[2], f[3]);
+        }
       }
-      Bs4[i] = make_float4(bv[0], bv[1], bv[2], bv[3]);
-      Cs4[i] = make_float4(cv[0], cv[1], cv[2], cv[3]);
-    }
-    __syncthreads();
+    };
+    if (full) convert(std::false_type{});
+    else convert(std::true_type{});
+    __syncthreads();  // conversions visible; bcraw free again
 
+    // stream chunk c+1 in while chunk c is computed
+    if constexpr (VEC) {
+      if (c + 1 < nchunks) issue_chunk(buf ^ 1, c + 1);
+    }
+
+    const T *X = xs0 + buf * kXElems;
     // ---- per-lane prologue: Delta and Delta*u for the lane's KI steps ----
-    const T *xu = X + size_t(ch) * TC + seg * KI;
-    const T *xd = X + size_t(CT + ch) * TC + seg * KI;
-    const float bias = bias_s[ch];
     float dl[KI], du[KI], y[KI];
     float dsum = 0.f;
+    {
+      const T *ru = X + size_t(ch) * TC;
+      const T *rd = X + size_t(CT + ch) * TC;
+      const float bias = bias_s[ch];
 #pragma unroll
-    for (int i = 0; i < KI; ++i) {
-      const int64_t tg = wstart + seg * KI + i;
-      const bool in = tg >= t_lo && tg < t_hi;
-      const float dt = softplus_t<kFast>(Elem<T>::to_f32(xd[i]) + bias);
-      dl[i] = in ? dt : 0.f;
-      du[i] = in ? dt * Elem<T>::to_f32(xu[i]) : 0.f;
-      dsum += dl[i];
-      y[i] = 0.f;
+      for (int lv = 0; lv < LV; ++lv) {
+        const int pv = (seg * LV + lv) * V;
+        float vu[V], vd[V];
+        unpack16<T>(*reinterpret_cast<const uint4 *>(ru + pv), vu);
+        unpack16<T>(*reinterpret_cast<const uint4 *>(rd + pv), vd);
+        if (full) {
+#pragma unroll
+          for (int e = 0; e < V; ++e) {
+            const int i = lv * V + e;
+            dl[i] = softplus_t<kFast>(vd[e] + bias);
+            du[i] = dl[i] * vu[e];
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < V; ++e) {
+            const int i = lv * V + e;
+            const int tl = seg * KI + i;
+            const bool in = tl >= rel_lo && tl < rel_hi;
+            const float dt = softplus_t<kFast>(vd[e] + bias);
+            dl[i] = in ? dt : 0.f;
+            du[i] = in ? dt * vu[e] : 0.f;  // select, so a non-finite u outside the sequence stays out
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          dsum += dl[lv * V + e];
+          y[lv * V + e] = 0.f;
+        }
+      }
     }
 
     // ---- state loop ----
-#pragma unroll 2
+#pragma unroll 1
     for (int n = 0; n < N; ++n) {
       const float A2 = A2s[ch * N + n];
       const float carry = carry_s[ch * N + n];
@@ -289,28 +352,42 @@ chunk_scan_kernel(const ScanArgs args) {
     // ---- epilogue: skip term, gate, store ----
     if (ch_ok) {
       const float Dd = Dsk[ch];
-      const T *xz = X + size_t(2 * CT + ch) * TC + seg * KI;
+      const T *ru = X + size_t(ch) * TC;
+      const T *rz = X + size_t(2 * CT + ch) * TC;
       const int64_t t0 = wstart + seg * KI;
       constexpr int VO = Elem<TO>::kVec;  // output elements per 16-byte store
-      alignas(16) TO out[KI];
 #pragma unroll
-      for (int i = 0; i < KI; ++i) {
-        float v = fmaf(Dd, Elem<T>::to_f32(xu[i]), y[i]);
-        if constexpr (HAS_Z) v *= silu_t<kFast>(Elem<T>::to_f32(xz[i]));
-        out[i] = Elem<TO>::from_f32(v);
+      for (int lv = 0; lv < LV; ++lv) {
+        const int pv = (seg * LV + lv) * V;
+        float vu[V], vz[V];
+        unpack16<T>(*reinterpret_cast<const uint4 *>(ru + pv), vu);
+        if constexpr (HAS_Z) unpack16<T>(*reinterpret_cast<const uint4 *>(rz + pv), vz);
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          const int i = lv * V + e;
+          float v = fmaf(Dd, vu[e], y[i]);
+          if constexpr (HAS_Z) v *= silu_t<kFast>(vz[e]);
+          y[i] = v;
+        }
       }
       TO *gy = static_cast<TO *>(args.y) + xbase + d * args.x_dim_stride + t0;
-      if (VEC && t0 >= t_lo && t0 + KI <= t_hi) {
+      const int tl0 = seg * KI;
+      if (VEC && tl0 >= rel_lo && tl0 + KI <= rel_hi) {
 #pragma unroll
-        for (int v = 0; v < KI / VO; ++v)
-          *reinterpret_cast<uint4 *>(gy + v * VO) = *reinterpret_cast<const uint4 *>(out + v * VO);
+        for (int v = 0; v < KI / VO; ++v) *reinterpret_cast<uint4 *>(gy + v * VO) = pack16<TO>(y + v * VO);
       } else {
 #pragma unroll
         for (int i = 0; i < KI; ++i)
-          if (t0 + i >= t_lo && t0 + i < t_hi) gy[i] = out[i];
+          if (tl0 + i >= rel_lo && tl0 + i < rel_hi) gy[i] = Elem<TO>::from_f32(y[i]);
       }
     }
   }
+
+#undef SSM_GU
+#undef SSM_GDL
+#undef SSM_GZ
+#undef SSM_GB
+#undef SSM_GC
 
   // final state of each channel of the tile
   __syncthreads();

@@ -10,6 +10,9 @@ namespace ssm {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
 // MUFU approximations (PTX ISA: ex2/lg2/rcp .approx).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -37,20 +40,20 @@ __device__ __forceinline__ float softplus_precise(float x) {
 // w - w^2/2 + ... + w^7/7 when w < 1/8 (truncation error below w^8/8, i.e. relative
 // error < 3e-7), else ln2 * log2(1 + w) through lg2, whose absolute error (~1e-7) is small
 // against a result of at least log(1.125) = 0.118 there.
+// Both branches are evaluated and selected (no divergence); the unselected one may be
+// inf/nan for large x, which a select does not propagate.
 __device__ __forceinline__ float softplus_fast(float x) {
-  if (x > 15.f) return x;
   const float w = ex2_approx(x * kLog2e);
-  if (w < 0.125f) {
-    float p = fmaf(w, -1.f / 7.f, 1.f / 6.f);
-    p = fmaf(w, p, -1.f / 5.f);
-    p = fmaf(w, p, 1.f / 4.f);
-    p = fmaf(w, p, -1.f / 3.f);
-    p = fmaf(w, p, 1.f / 2.f);
-    // log1p(w) = w - w^2 (1/2 - w/3 + w^2/4 - ...) = w * (1 - w * p)
-    p = fmaf(-w, p, 1.f);
-    return w * p;
-  }
-  return kLn2 * lg2_approx(1.f + w);
+  float p = fmaf(w, -1.f / 7.f, 1.f / 6.f);
+  p = fmaf(w, p, -1.f / 5.f);
+  p = fmaf(w, p, 1.f / 4.f);
+  p = fmaf(w, p, -1.f / 3.f);
+  p = fmaf(w, p, 1.f / 2.f);
+  // log1p(w) = w - w^2 (1/2 - w/3 + w^2/4 - ...) = w * (1 - w * p)
+  const float series = w * fmaf(-w, p, 1.f);
+  const float viaLog = kLn2 * lg2_approx(1.f + w);
+  const float r = w < 0.125f ? series : viaLog;
+  return x > 15.f ? x : r;
 }
 
 // silu(z) = z * sigmoid(z) = z / (1 + e^-z).
@@ -71,6 +74,33 @@ template <> struct Elem<__nv_bfloat16> {
   static constexpr bool kFast = true;
 };
 
+// 16-byte vector <-> float32 lanes, in registers (bf16 -> f32 is a 16-bit shift).
+template <typename T> __device__ __forceinline__ void unpack16(const uint4 v, float *f);
+template <> __device__ __forceinline__ void unpack16<float>(const uint4 v, float *f) {
+  f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+}
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4 v, float *f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    f[2 * k] = __uint_as_float(w[k] << 16);
+    f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+  }
+}
+template <typename T> __device__ __forceinline__ uint4 pack16(const float *f);
+template <> __device__ __forceinline__ uint4 pack16<float>(const float *f) {
+  return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return (uint32_t(__bfloat16_as_ushort(p.y)) << 16) | uint32_t(__bfloat16_as_ushort(p.x));
+}
+template <> __device__ __forceinline__ uint4 pack16<__nv_bfloat16>(const float *f) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
 template <bool kFast> __device__ __forceinline__ float softplus_t(float x) {
   return kFast ? softplus_fast(x) : softplus_precise(x);
 }
@@ -88,9 +118,57 @@ __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gmem_src
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
+// ---- TMA bulk copies completing on an mbarrier (PTX ISA: cp.async.bulk, mbarrier) ----
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Orders this thread's earlier generic-proxy shared-memory accesses before later async-proxy
+// (TMA) writes to the same buffers.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// 1-D bulk copy global -> shared (no multicast).  dst, src 16-byte aligned; bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Device status word (read and cleared by ssm_get_device_status on the host).  The library
 // is a single translation unit, so this is the only definition.
 __device__ int g_status = 0;
 __device__ __forceinline__ void report_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// Bounded wait for an mbarrier phase: every try_wait suspends for a hardware-defined time;
+// after kMaxTries failed tries the wait gives up, records SSM_ERR_TIMEOUT and returns false
+// so that the caller carries on (with unusable data) instead of hanging the GPU.
+constexpr uint32_t kMaxTries = 1u << 22;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kMaxTries; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  report_status(5 /* SSM_ERR_TIMEOUT */);
+  return false;
+}
 
 }  // namespace ssm

@@ -16,10 +16,10 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 // Tile shapes per state size: KI steps per lane, SPW segment lanes per channel, CPW channels
 // per warp, WARPS warps per CTA.  Larger states get shorter chunks to bound shared memory.
 template <int N> struct Shape;
-template <> struct Shape<16> { static constexpr int KI = 16, SPW = 16, CPW = 2, WARPS = 4; };
-template <> struct Shape<32> { static constexpr int KI = 16, SPW = 8, CPW = 4, WARPS = 2; };
-template <> struct Shape<64> { static constexpr int KI = 8, SPW = 8, CPW = 4, WARPS = 2; };
-template <> struct Shape<128> { static constexpr int KI = 8, SPW = 8, CPW = 4, WARPS = 2; };
+template <> struct Shape<16> { static constexpr int KI = 16, SPW = 16, CPW = 2, WARPS = 8; };
+template <> struct Shape<32> { static constexpr int KI = 16, SPW = 8, CPW = 4, WARPS = 8; };
+template <> struct Shape<64> { static constexpr int KI = 8, SPW = 8, CPW = 4, WARPS = 8; };
+template <> struct Shape<128> { static constexpr int KI = 8, SPW = 4, CPW = 8, WARPS = 4; };
 
 template <typename T, typename TO, int N, bool HAS_Z, bool VEC>
 ssm_status_t launch_chunk(const ScanArgs &a, cudaStream_t stream) {
