@@ -26,6 +26,15 @@
 // u/delta/z rows are padded by 16 bytes so that the channel groups of a phase read
 // different banks.  Chunks that lie entirely inside the sequence skip all masking.
 //
+// Scheduling.  Packed sequences: one CTA per (sequence, channel tile), sequences longest
+// first.  Fixed-length batches: a persistent grid takes work units -- (channel-tile chain,
+// group of consecutive chunks) -- from an atomic ticket in chunk-major order, so every
+// chain advances and all SMs stay busy even when the batch has few channel tiles; the
+// state crosses unit boundaries through a device workspace (release/acquire flag per
+// chain, bounded wait).  With NG > 1 the N states are split across NG warps that share the
+// same channels and steps (more parallelism for narrow problems); their partial outputs
+// are summed through shared memory.
+//
 // Windows start at the sequence start rounded down to a 16-byte boundary; steps outside
 // [seq_start, seq_end) are made identities (Delta = 0, Delta*u = 0, B = 0) and are not
 // stored, which also resets the state at packed-sequence boundaries ("ufo.work" §4.2).
@@ -47,96 +56,73 @@ struct ScanArgs {
   int64_t x_batch_stride, x_dim_stride, bc_batch_stride, bc_state_stride;
   int nseq;    // sequences (batch size or number of packed sequences)
   int ntiles;  // channel tiles per sequence
+  // persistent scheduling (fixed-length batches only)
+  uint32_t *ticket;  // work counter, zero at launch
+  uint32_t *flags;   // [nchains] chunk groups completed per chain, zero at launch
+  float *carries;    // [nchains][CT][N] state at the end of the last completed group
+  int nchains;       // nseq * ntiles
+  int group;         // chunks per work unit
+  int total_units;   // nchains * ceil(nchunks / group)
 };
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
 // Packed sequences are visited longest first (CTAs with low indices start first), which
 // keeps the tail short when lengths differ; the ordering is computed in each CTA, so it is
 // only done for modest sequence counts.
 constexpr int kMaxSortedSeqs = 64;
 
-template <typename T, int N, int KI, int SPW, int CPW, int WARPS>
+// CW warps hold distinct channel groups; NG warps share them and split the N states.
+template <typename T, int N, int KI, int SPW, int CPW, int CW, int NG>
 struct ChunkCfg {
-  static constexpr int kTC = SPW * KI;     // chunk length (time steps)
-  static constexpr int kCT = CPW * WARPS;  // channels per CTA
+  static constexpr int kTC = SPW * KI;      // chunk length (time steps)
+  static constexpr int kCT = CPW * CW;      // channels per CTA
+  static constexpr int kWarps = CW * NG;
+  static constexpr int kNS = N / NG;        // states per warp
   static constexpr int kVec = Elem<T>::kVec;
-  static constexpr int kThreads = WARPS * 32;
+  static constexpr int kThreads = kWarps * 32;
   static constexpr int kXPitch = kTC + kVec;  // u/delta/z row pitch (elements): +16 bytes
-  // shared memory layout (bytes), everything double-buffered except the parameters
+  // shared memory layout (bytes), staging double-buffered
   static constexpr size_t kXBytes = size_t(3) * kCT * kXPitch * sizeof(T);  // u, delta, z
   static constexpr size_t kBCBytes = size_t(2) * N * kTC * sizeof(T);       // B, C
+  static constexpr size_t kYBytes = NG > 1 ? size_t(NG) * kCT * kTC * sizeof(float) : 0;  // partial y
   static constexpr size_t kParamBytes =
       size_t(2) * kCT * N * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
-  static constexpr size_t kSmemBytes = 2 * kXBytes + 2 * kBCBytes + kParamBytes;
+  static constexpr size_t kSmemBytes = 2 * kXBytes + 2 * kBCBytes + kYBytes + kParamBytes;
   static_assert(KI % 4 == 0 && KI % kVec == 0, "a lane's steps must be whole 16-byte vectors");
   static_assert(32 % SPW == 0 && CPW * SPW == 32, "lane split");
+  static_assert(N % NG == 0 && (KI / NG) % 2 == 0, "state / step split");
   static_assert(kXBytes % 16 == 0 && kBCBytes % 16 == 0, "16-byte aligned buffers");
 };
 
-template <typename T, typename TO, int N, int KI, int SPW, int CPW, int WARPS, bool HAS_Z, bool VEC>
-__global__ void __launch_bounds__(WARPS * 32, (WARPS <= 8 ? 16 / WARPS : 1))
+template <typename T, typename TO, int N, int KI, int SPW, int CPW, int CW, int NG, bool HAS_Z, bool VEC,
+          bool PERSIST>
+__global__ void __launch_bounds__(CW * NG * 32, (CW * NG <= 8 ? 16 / (CW * NG) : 1))
 chunk_scan_kernel(const ScanArgs args) {
-  using Cfg = ChunkCfg<T, N, KI, SPW, CPW, WARPS>;
+  using Cfg = ChunkCfg<T, N, KI, SPW, CPW, CW, NG>;
   constexpr int TC = Cfg::kTC, CT = Cfg::kCT, V = Cfg::kVec, NT = Cfg::kThreads, XP = Cfg::kXPitch;
+  constexpr int NS = Cfg::kNS;
   constexpr int LV = KI / V;  // 16-byte vectors per lane
+  constexpr int KP = KI / 2;  // step pairs per lane
   constexpr bool kFast = Elem<T>::kFast;
   constexpr size_t kXElems = Cfg::kXBytes / sizeof(T), kBCElems = Cfg::kBCBytes / sizeof(T);
+  static_assert(!PERSIST || VEC, "persistent scheduling uses the TMA staging path");
 
   extern __shared__ __align__(16) unsigned char smem[];
-  T *const xs0 = reinterpret_cast<T *>(smem);                          // [2][3][CT][XP]
-  T *const bc0 = reinterpret_cast<T *>(smem + 2 * Cfg::kXBytes);       // [2][2][N][TC]
-  float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes);  // [CT][N]
-  float *carry_s = A2s + CT * N;                                       // [CT][N]
-  float *Dsk = carry_s + CT * N;                                       // [CT]
-  float *bias_s = Dsk + CT;                                            // [CT]
-  int *order = reinterpret_cast<int *>(bias_s + CT);                   // [kMaxSortedSeqs]
-  __shared__ __align__(8) uint64_t bars[2];                           // chunk-arrival barriers
-
-  const int tile = blockIdx.x % args.ntiles;
-  int s = blockIdx.x / args.ntiles;
-  const int d0 = tile * CT;
-  int64_t t_lo, t_hi, xbase, bcbase;
-  if (args.cu_seqlens) {
-    if (args.nseq <= kMaxSortedSeqs) {
-      // rank sequences by length (descending, ties by index); order[rank] = sequence
-      for (int i = threadIdx.x; i < args.nseq; i += NT) {
-        const int li = args.cu_seqlens[i + 1] - args.cu_seqlens[i];
-        int rank = 0;
-        for (int j = 0; j < args.nseq; ++j) {
-          const int lj = args.cu_seqlens[j + 1] - args.cu_seqlens[j];
-          rank += (lj > li) || (lj == li && j < i);
-        }
-        order[rank] = i;
-      }
-      __syncthreads();
-      s = order[s];
-    }
-    t_lo = args.cu_seqlens[s];
-    t_hi = args.cu_seqlens[s + 1];
-    xbase = 0;
-    bcbase = 0;
-  } else {
-    t_lo = 0;
-    t_hi = args.seqlen;
-    xbase = int64_t(s) * args.x_batch_stride;
-    bcbase = int64_t(s) * args.bc_batch_stride;
-  }
-  const int64_t w0 = t_lo & ~int64_t(V - 1);
-  const int nchunks = t_hi > t_lo ? int((t_hi - w0 + TC - 1) / TC) : 0;
-
-  // per-tile constants and initial state
-  for (int i = threadIdx.x; i < CT * N; i += NT) {
-    const int ch = i / N, n = i % N;
-    const int64_t d = d0 + ch;
-    const bool ok = d < args.dim;
-    A2s[i] = ok ? args.A[d * N + n] * kLog2e : 0.f;
-    carry_s[i] = (ok && args.h0) ? args.h0[(int64_t(s) * args.dim + d) * N + n] : 0.f;
-  }
-  for (int i = threadIdx.x; i < CT; i += NT) {
-    const int64_t d = d0 + i;
-    const bool ok = d < args.dim;
-    Dsk[i] = (ok && args.Dskip) ? args.Dskip[d] : 0.f;
-    bias_s[i] = (ok && args.bias) ? args.bias[d] : 0.f;
-  }
+  T *const xs0 = reinterpret_cast<T *>(smem);                     // [2][3][CT][XP]
+  T *const bc0 = reinterpret_cast<T *>(smem + 2 * Cfg::kXBytes);  // [2][2][N][TC]
+  float *ypart = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes);  // [NG][CT][TC]
+  float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes);  // [CT][N]
+  float *carry_s = A2s + CT * N;                                  // [CT][N]
+  float *Dsk = carry_s + CT * N;                                  // [CT]
+  float *bias_s = Dsk + CT;                                       // [CT]
+  int *order = reinterpret_cast<int *>(bias_s + CT);              // [kMaxSortedSeqs]
+  __shared__ __align__(8) uint64_t bars[2];                      // chunk-arrival barriers
+  __shared__ int unit_sh;
 
   // tensor bases are read from the kernel parameters where used
 #define SSM_GU static_cast<const T *>(args.u)
@@ -145,65 +131,15 @@ chunk_scan_kernel(const ScanArgs args) {
 #define SSM_GB static_cast<const T *>(args.B)
 #define SSM_GC static_cast<const T *>(args.C)
   constexpr int nx = HAS_Z ? 3 : 2;
-  const int nvalid_ch = int(min64(CT, args.dim - d0));
   // rows are readable up to the seqlen rounded up to a 16-byte vector (row strides are
-  // multiples of 16 bytes on this path)
+  // multiples of 16 bytes on the TMA path)
   const int64_t seqlen_r = (args.seqlen + V - 1) / V * V;
 
-  // TMA: chunk c's u/delta/z and B/C rows into buffer `buf`.
-  auto issue_chunk = [&](int buf, int c) {
-    const int64_t wstart = w0 + int64_t(c) * TC;
-    const int64_t wend = min64(wstart + TC, seqlen_r);
-    const uint32_t row_bytes = uint32_t((wend - wstart) * int64_t(sizeof(T)));
-    T *xdst = xs0 + buf * kXElems;
-    T *bdst = bc0 + buf * kBCElems;
-    fence_proxy_async_smem();
-    if (threadIdx.x == 0) mbar_arrive_expect_tx(&bars[buf], row_bytes * uint32_t(nx * nvalid_ch + 2 * N));
-    for (int r = threadIdx.x; r < nx * CT + 2 * N; r += NT) {
-      if (r < nx * CT) {
-        const int which = r / CT, ch = r % CT;
-        if (ch >= nvalid_ch) continue;
-        const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
-        bulk_g2s(xdst + size_t(r) * XP, base + xbase + (d0 + ch) * args.x_dim_stride + wstart, row_bytes,
-                 &bars[buf]);
-      } else {
-        const int r2 = r - nx * CT, which = r2 / N, n = r2 % N;
-        const T *base = which == 0 ? SSM_GB : SSM_GC;
-        bulk_g2s(bdst + size_t(r2) * TC, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, row_bytes,
-                 &bars[buf]);
-      }
-    }
-  };
-  // Element-wise staging for rows that are not 16-byte aligned (zero outside the tensor).
-  auto stage_scalar = [&](int buf, int c) {
-    T *xdst = xs0 + buf * kXElems;
-    T *bdst = bc0 + buf * kBCElems;
-    const int64_t wstart = w0 + int64_t(c) * TC;
-    for (int i = threadIdx.x; i < nx * CT * TC; i += NT) {
-      const int row = i / TC, j = i % TC;
-      const int which = row / CT, ch = row % CT;
-      const int64_t d = d0 + ch, t = wstart + j;
-      const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
-      T val = Elem<T>::from_f32(0.f);
-      if (d < args.dim && t < args.seqlen) val = base[xbase + d * args.x_dim_stride + t];
-      xdst[size_t(row) * XP + j] = val;
-    }
-    for (int i = threadIdx.x; i < 2 * N * TC; i += NT) {
-      const int row = i / TC, j = i % TC;
-      const int which = row / N, n = row % N;
-      const int64_t t = wstart + j;
-      const T *base = which == 0 ? SSM_GB : SSM_GC;
-      T val = Elem<T>::from_f32(0.f);
-      if (t < args.seqlen) val = base[bcbase + int64_t(n) * args.bc_state_stride + t];
-      bdst[size_t(row) * TC + j] = val;
-    }
-  };
-
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int cg = lane % CPW, seg = lane / CPW;  // interleaved channel groups
-  const int ch = warp * CPW + cg;
-  const int64_t d = d0 + ch;
-  const bool ch_ok = d < args.dim;
+  const int cw = warp % CW, g = warp / CW;        // channel warp, state group
+  const int cg = lane % CPW, seg = lane / CPW;    // interleaved channel groups
+  const int ch = cw * CPW + cg;
+  const int n0 = g * NS;
 
   if constexpr (VEC) {
     if (threadIdx.x == 0) {
@@ -212,187 +148,376 @@ chunk_scan_kernel(const ScanArgs args) {
       mbar_init_fence();
     }
     __syncthreads();
-    if (nchunks > 0) issue_chunk(0, 0);
   }
+  uint32_t gc = 0;  // chunks staged by this CTA so far: selects buffer and barrier parity
 
-  // One chunk of the lane's work; the masked instance handles chunks that straddle a
-  // sequence end.
-  auto compute_chunk = [&](auto masked_tag, const T *X, const T *Bsm, const T *Csm, int64_t wstart, int rel_lo,
-                           int rel_hi) {
-    constexpr bool kMasked = decltype(masked_tag)::value;
-    const int tl0 = seg * KI;  // chunk-local first step of this lane
-    // ---- prologue: Delta and Delta*u for the lane's KI steps (as pairs of steps) ----
-    constexpr int KP = KI / 2;
-    float2 dl[KP], du[KP], y[KP];
-    float dsum = 0.f;
-    {
-      const T *ru = X + size_t(ch) * XP + tl0;
-      const T *rd = X + size_t(CT + ch) * XP + tl0;
-      const float bias = bias_s[ch];
-#pragma unroll
-      for (int lv = 0; lv < LV; ++lv) {
-        float2 vu[V / 2], vd[V / 2];
-        unpack16x2<T>(*reinterpret_cast<const uint4 *>(ru + lv * V), vu);
-        unpack16x2<T>(*reinterpret_cast<const uint4 *>(rd + lv * V), vd);
-#pragma unroll
-        for (int e = 0; e < V / 2; ++e) {
-          const int p = lv * (V / 2) + e;
-          float2 dt = make_float2(softplus_t<kFast>(vd[e].x + bias), softplus_t<kFast>(vd[e].y + bias));
-          if constexpr (kMasked) {
-            const int i = tl0 + 2 * p;
-            dt.x = (i >= rel_lo && i < rel_hi) ? dt.x : 0.f;
-            dt.y = (i + 1 >= rel_lo && i + 1 < rel_hi) ? dt.y : 0.f;
-            // select, so a non-finite u outside the sequence stays out
-            du[p] = make_float2(dt.x != 0.f ? dt.x * vu[e].x : 0.f, dt.y != 0.f ? dt.y * vu[e].y : 0.f);
-          } else {
-            du[p] = __fmul2_rn(dt, vu[e]);
-          }
-          dl[p] = dt;
-          dsum += dt.x + dt.y;
-          y[p] = make_float2(0.f, 0.f);
-        }
-      }
-    }
-
-    // ---- state loop ----
-#pragma unroll 1
-    for (int n = 0; n < N; ++n) {
-      const float A2 = A2s[ch * N + n];
-      const float2 A22 = make_float2(A2, A2);
-      const float carry = carry_s[ch * N + n];
-      float a[KI];
-      float2 b[KP];
-      float G = 0.f;
-      const T *rb = Bsm + size_t(n) * TC + tl0;
-#pragma unroll
-      for (int lv = 0; lv < LV; ++lv) {
-        float2 bb[V / 2];
-        unpack16x2<T>(*reinterpret_cast<const uint4 *>(rb + lv * V), bb);
-#pragma unroll
-        for (int e = 0; e < V / 2; ++e) {
-          const int p = lv * (V / 2) + e;
-          const float2 x = __fmul2_rn(dl[p], A22);
-          a[2 * p] = ex2_approx(x.x);
-          a[2 * p + 1] = ex2_approx(x.y);
-          if constexpr (kMasked) {
-            // stale B outside the window never reaches h (du is 0 there, B may be non-finite)
-            b[p] = make_float2(du[p].x != 0.f ? du[p].x * bb[e].x : 0.f, du[p].y != 0.f ? du[p].y * bb[e].y : 0.f);
-          } else {
-            b[p] = __fmul2_rn(du[p], bb[e]);
-          }
-          G = fmaf(a[2 * p], G, b[p].x);
-          G = fmaf(a[2 * p + 1], G, b[p].y);
-        }
-      }
-      float P = ex2_approx(dsum * A2);  // product of the lane's a_i
-      // inclusive scan of segment operators across the SPW segment lanes of this channel
-#pragma unroll
-      for (int off = 1; off < SPW; off *= 2) {
-        const float Pu = __shfl_up_sync(0xffffffffu, P, off * CPW);
-        const float Gu = __shfl_up_sync(0xffffffffu, G, off * CPW);
-        if (seg >= off) {
-          G = fmaf(P, Gu, G);
-          P *= Pu;
-        }
-      }
-      float Pe = __shfl_up_sync(0xffffffffu, P, CPW);
-      float Ge = __shfl_up_sync(0xffffffffu, G, CPW);
-      if (seg == 0) {
-        Pe = 1.f;
-        Ge = 0.f;
-      }
-      float h = fmaf(Pe, carry, Ge);  // state entering this lane's first step
-      __syncwarp();
-      if (seg == SPW - 1) carry_s[ch * N + n] = fmaf(P, carry, G);  // state leaving the chunk
-      const T *rc = Csm + size_t(n) * TC + tl0;
-#pragma unroll
-      for (int lv = 0; lv < LV; ++lv) {
-        float2 cc[V / 2];
-        unpack16x2<T>(*reinterpret_cast<const uint4 *>(rc + lv * V), cc);
-#pragma unroll
-        for (int e = 0; e < V / 2; ++e) {
-          const int p = lv * (V / 2) + e;
-          float2 hh;
-          h = fmaf(a[2 * p], h, b[p].x);
-          hh.x = h;
-          h = fmaf(a[2 * p + 1], h, b[p].y);
-          hh.y = h;
-          y[p] = __ffma2_rn(cc[e], hh, y[p]);
-        }
-      }
-    }
-
-    // ---- epilogue: skip term, gate, store ----
-    if (ch_ok) {
-      const float Dd = Dsk[ch];
-      const T *ru = X + size_t(ch) * XP + tl0;
-      [[maybe_unused]] const T *rz = X + size_t(2 * CT + ch) * XP + tl0;
-      constexpr int VO = Elem<TO>::kVec;  // output elements per 16-byte store
-      float yo[KI];
-#pragma unroll
-      for (int lv = 0; lv < LV; ++lv) {
-        float vu[V];
-        [[maybe_unused]] float vz[V];
-        unpack16<T>(*reinterpret_cast<const uint4 *>(ru + lv * V), vu);
-        if constexpr (HAS_Z) unpack16<T>(*reinterpret_cast<const uint4 *>(rz + lv * V), vz);
-#pragma unroll
-        for (int e = 0; e < V; ++e) {
-          const int i = lv * V + e;
-          float v = fmaf(Dd, vu[e], (i & 1) ? y[i / 2].y : y[i / 2].x);
-          if constexpr (HAS_Z) v *= silu_t<kFast>(vz[e]);
-          yo[i] = v;
-        }
-      }
-      TO *gy = static_cast<TO *>(args.y) + xbase + d * args.x_dim_stride + wstart + tl0;
-      if (VEC && (!kMasked || (tl0 >= rel_lo && tl0 + KI <= rel_hi))) {
-#pragma unroll
-        for (int v = 0; v < KI / VO; ++v) *reinterpret_cast<uint4 *>(gy + v * VO) = pack16<TO>(yo + v * VO);
-      } else {
-#pragma unroll
-        for (int i = 0; i < KI; ++i)
-          if (!kMasked || (tl0 + i >= rel_lo && tl0 + i < rel_hi)) gy[i] = Elem<TO>::from_f32(yo[i]);
-      }
-    }
-  };
-
-  for (int c = 0; c < nchunks; ++c) {
-    const int buf = c & 1;
-    const int64_t wstart = w0 + int64_t(c) * TC;
-    if constexpr (VEC) {
-      mbar_wait_bounded(&bars[buf], uint32_t(c >> 1) & 1u);
+  for (int iter = 0;; ++iter) {
+    // ------------------------------------------------------------- pick a work unit
+    int unit;
+    if constexpr (PERSIST) {
+      if (threadIdx.x == 0) unit_sh = int(atomicAdd(args.ticket, 1u));
+      __syncthreads();
+      unit = unit_sh;
+      if (unit >= args.total_units) break;
     } else {
-      stage_scalar(buf, c);
+      if (iter > 0) break;
+      unit = blockIdx.x;
     }
-    __syncthreads();  // chunk c visible to all; everyone is done with chunk c-1's buffers
+    int chain, kgrp;
+    if constexpr (PERSIST) {
+      chain = unit % args.nchains;  // chunk-major order: all chains' group k before group k+1
+      kgrp = unit / args.nchains;
+    } else {
+      chain = unit;
+      kgrp = 0;
+    }
+    const int tile = chain % args.ntiles;
+    int s = chain / args.ntiles;
+    const int d0 = tile * CT;
+    int64_t t_lo, t_hi, xbase, bcbase;
+    if (args.cu_seqlens) {
+      if (args.nseq <= kMaxSortedSeqs) {
+        // rank sequences by length (descending, ties by index); order[rank] = sequence
+        for (int i = threadIdx.x; i < args.nseq; i += NT) {
+          const int li = args.cu_seqlens[i + 1] - args.cu_seqlens[i];
+          int rank = 0;
+          for (int j = 0; j < args.nseq; ++j) {
+            const int lj = args.cu_seqlens[j + 1] - args.cu_seqlens[j];
+            rank += (lj > li) || (lj == li && j < i);
+          }
+          order[rank] = i;
+        }
+        __syncthreads();
+        s = order[s];
+      }
+      t_lo = args.cu_seqlens[s];
+      t_hi = args.cu_seqlens[s + 1];
+      xbase = 0;
+      bcbase = 0;
+    } else {
+      t_lo = 0;
+      t_hi = args.seqlen;
+      xbase = int64_t(s) * args.x_batch_stride;
+      bcbase = int64_t(s) * args.bc_batch_stride;
+    }
+    const int64_t w0 = t_lo & ~int64_t(V - 1);
+    const int nchunks = t_hi > t_lo ? int((t_hi - w0 + TC - 1) / TC) : 0;
+    const int c_begin = PERSIST ? kgrp * args.group : 0;
+    const int c_end = PERSIST ? min(c_begin + args.group, nchunks) : nchunks;
+    const int nvalid_ch = int(min64(CT, args.dim - d0));
+    const int64_t d = d0 + ch;
+    const bool ch_ok = d < args.dim;
+
+    // per-tile constants
+    for (int i = threadIdx.x; i < CT * N; i += NT) {
+      const int c2 = i / N, n = i % N;
+      const int64_t dd = d0 + c2;
+      A2s[i] = dd < args.dim ? args.A[dd * N + n] * kLog2e : 0.f;
+    }
+    for (int i = threadIdx.x; i < CT; i += NT) {
+      const int64_t dd = d0 + i;
+      const bool ok = dd < args.dim;
+      Dsk[i] = (ok && args.Dskip) ? args.Dskip[dd] : 0.f;
+      bias_s[i] = (ok && args.bias) ? args.bias[dd] : 0.f;
+    }
+    // state entering the unit: h0 (or zero) for a chain's first unit, otherwise the state
+    // the previous unit of the chain published
+    if (!PERSIST || kgrp == 0) {
+      for (int i = threadIdx.x; i < CT * N; i += NT) {
+        const int c2 = i / N, n = i % N;
+        const int64_t dd = d0 + c2;
+        carry_s[i] = (dd < args.dim && args.h0) ? args.h0[(int64_t(s) * args.dim + dd) * N + n] : 0.f;
+      }
+    } else {
+      if (threadIdx.x == 0) {
+        uint32_t tries = 0;
+        while (ld_acquire_u32(args.flags + chain) < uint32_t(kgrp)) {
+          if (++tries > kMaxTries) {
+            report_status(5 /* SSM_ERR_TIMEOUT */);
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      __syncthreads();
+      const float *src = args.carries + size_t(chain) * CT * N;
+      for (int i = threadIdx.x; i < CT * N; i += NT) carry_s[i] = __ldcg(src + i);
+    }
+
+    // TMA: chunk c's u/delta/z and B/C rows into buffer `buf`.
+    auto issue_chunk = [&](int buf, int c) {
+      const int64_t wstart = w0 + int64_t(c) * TC;
+      const int64_t wend = min64(wstart + TC, seqlen_r);
+      const uint32_t row_bytes = uint32_t((wend - wstart) * int64_t(sizeof(T)));
+      T *xdst = xs0 + buf * kXElems;
+      T *bdst = bc0 + buf * kBCElems;
+      fence_proxy_async_smem();
+      if (threadIdx.x == 0) mbar_arrive_expect_tx(&bars[buf], row_bytes * uint32_t(nx * nvalid_ch + 2 * N));
+      for (int r = threadIdx.x; r < nx * CT + 2 * N; r += NT) {
+        if (r < nx * CT) {
+          const int which = r / CT, c2 = r % CT;
+          if (c2 >= nvalid_ch) continue;
+          const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
+          bulk_g2s(xdst + size_t(r) * XP, base + xbase + (d0 + c2) * args.x_dim_stride + wstart, row_bytes,
+                   &bars[buf]);
+        } else {
+          const int r2 = r - nx * CT, which = r2 / N, n = r2 % N;
+          const T *base = which == 0 ? SSM_GB : SSM_GC;
+          bulk_g2s(bdst + size_t(r2) * TC, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, row_bytes,
+                   &bars[buf]);
+        }
+      }
+    };
+    // Element-wise staging for rows that are not 16-byte aligned (zero outside the tensor).
+    auto stage_scalar = [&](int buf, int c) {
+      T *xdst = xs0 + buf * kXElems;
+      T *bdst = bc0 + buf * kBCElems;
+      const int64_t wstart = w0 + int64_t(c) * TC;
+      for (int i = threadIdx.x; i < nx * CT * TC; i += NT) {
+        const int row = i / TC, j = i % TC;
+        const int which = row / CT, c2 = row % CT;
+        const int64_t dd = d0 + c2, t = wstart + j;
+        const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
+        T val = Elem<T>::from_f32(0.f);
+        if (dd < args.dim && t < args.seqlen) val = base[xbase + dd * args.x_dim_stride + t];
+        xdst[size_t(row) * XP + j] = val;
+      }
+      for (int i = threadIdx.x; i < 2 * N * TC; i += NT) {
+        const int row = i / TC, j = i % TC;
+        const int which = row / N, n = row % N;
+        const int64_t t = wstart + j;
+        const T *base = which == 0 ? SSM_GB : SSM_GC;
+        T val = Elem<T>::from_f32(0.f);
+        if (t < args.seqlen) val = base[bcbase + int64_t(n) * args.bc_state_stride + t];
+        bdst[size_t(row) * TC + j] = val;
+      }
+    };
+
+    // One chunk of the lane's work; the masked instance handles chunks that straddle a
+    // sequence end.
+    auto compute_chunk = [&](auto masked_tag, const T *X, const T *Bsm, const T *Csm, int64_t wstart, int rel_lo,
+                             int rel_hi) {
+      constexpr bool kMasked = decltype(masked_tag)::value;
+      const int tl0 = seg * KI;  // chunk-local first step of this lane
+      // ---- prologue: Delta and Delta*u for the lane's KI steps (as pairs of steps) ----
+      float2 dl[KP], du[KP], y[KP];
+      float dsum = 0.f;
+      {
+        const T *ru = X + size_t(ch) * XP + tl0;
+        const T *rd = X + size_t(CT + ch) * XP + tl0;
+        const float bias = bias_s[ch];
+#pragma unroll
+        for (int lv = 0; lv < LV; ++lv) {
+          float2 vu[V / 2], vd[V / 2];
+          unpack16x2<T>(*reinterpret_cast<const uint4 *>(ru + lv * V), vu);
+          unpack16x2<T>(*reinterpret_cast<const uint4 *>(rd + lv * V), vd);
+#pragma unroll
+          for (int e = 0; e < V / 2; ++e) {
+            const int p = lv * (V / 2) + e;
+            float2 dt = make_float2(softplus_t<kFast>(vd[e].x + bias), softplus_t<kFast>(vd[e].y + bias));
+            if constexpr (kMasked) {
+              const int i = tl0 + 2 * p;
+              dt.x = (i >= rel_lo && i < rel_hi) ? dt.x : 0.f;
+              dt.y = (i + 1 >= rel_lo && i + 1 < rel_hi) ? dt.y : 0.f;
+              // select, so a non-finite u outside the sequence stays out
+              du[p] = make_float2(dt.x != 0.f ? dt.x * vu[e].x : 0.f, dt.y != 0.f ? dt.y * vu[e].y : 0.f);
+            } else {
+              du[p] = __fmul2_rn(dt, vu[e]);
+            }
+            dl[p] = dt;
+            dsum += dt.x + dt.y;
+            y[p] = make_float2(0.f, 0.f);
+          }
+        }
+      }
+
+      // ---- state loop over this warp's NS states ----
+#pragma unroll 1
+      for (int n = n0; n < n0 + NS; ++n) {
+        const float A2 = A2s[ch * N + n];
+        const float2 A22 = make_float2(A2, A2);
+        const float carry = carry_s[ch * N + n];
+        float a[KI];
+        float2 b[KP];
+        float G = 0.f;
+        const T *rb = Bsm + size_t(n) * TC + tl0;
+#pragma unroll
+        for (int lv = 0; lv < LV; ++lv) {
+          float2 bb[V / 2];
+          unpack16x2<T>(*reinterpret_cast<const uint4 *>(rb + lv * V), bb);
+#pragma unroll
+          for (int e = 0; e < V / 2; ++e) {
+            const int p = lv * (V / 2) + e;
+            const float2 x = __fmul2_rn(dl[p], A22);
+            a[2 * p] = ex2_approx(x.x);
+            a[2 * p + 1] = ex2_approx(x.y);
+            if constexpr (kMasked) {
+              // stale B outside the window never reaches h (du is 0 there, B may be non-finite)
+              b[p] = make_float2(du[p].x != 0.f ? du[p].x * bb[e].x : 0.f,
+                                 du[p].y != 0.f ? du[p].y * bb[e].y : 0.f);
+            } else {
+              b[p] = __fmul2_rn(du[p], bb[e]);
+            }
+            G = fmaf(a[2 * p], G, b[p].x);
+            G = fmaf(a[2 * p + 1], G, b[p].y);
+          }
+        }
+        float P = ex2_approx(dsum * A2);  // product of the lane's a_i
+        // inclusive scan of segment operators across the SPW segment lanes of this channel
+#pragma unroll
+        for (int off = 1; off < SPW; off *= 2) {
+          const float Pu = __shfl_up_sync(0xffffffffu, P, off * CPW);
+          const float Gu = __shfl_up_sync(0xffffffffu, G, off * CPW);
+          if (seg >= off) {
+            G = fmaf(P, Gu, G);
+            P *= Pu;
+          }
+        }
+        float Pe = __shfl_up_sync(0xffffffffu, P, CPW);
+        float Ge = __shfl_up_sync(0xffffffffu, G, CPW);
+        if (seg == 0) {
+          Pe = 1.f;
+          Ge = 0.f;
+        }
+        float h = fmaf(Pe, carry, Ge);  // state entering this lane's first step
+        __syncwarp();
+        if (seg == SPW - 1) carry_s[ch * N + n] = fmaf(P, carry, G);  // state leaving the chunk
+        const T *rc = Csm + size_t(n) * TC + tl0;
+#pragma unroll
+        for (int lv = 0; lv < LV; ++lv) {
+          float2 cc[V / 2];
+          unpack16x2<T>(*reinterpret_cast<const uint4 *>(rc + lv * V), cc);
+#pragma unroll
+          for (int e = 0; e < V / 2; ++e) {
+            const int p = lv * (V / 2) + e;
+            float2 hh;
+            h = fmaf(a[2 * p], h, b[p].x);
+            hh.x = h;
+            h = fmaf(a[2 * p + 1], h, b[p].y);
+            hh.y = h;
+            y[p] = __ffma2_rn(cc[e], hh, y[p]);
+          }
+        }
+      }
+
+      // ---- epilogue: sum of the state groups, skip term, gate, store ----
+      // A lane finishes steps [e0, e0 + KE) of its segment: all KI steps when NG == 1,
+      // otherwise the g-th slice, after the partial sums went through shared memory.
+      constexpr int KE = KI / NG;
+      const int e0 = g * KE;
+      float yo[KE];
+      if constexpr (NG == 1) {
+#pragma unroll
+        for (int i = 0; i < KI; ++i) yo[i] = (i & 1) ? y[i / 2].y : y[i / 2].x;
+      } else {
+        float2 *mine = reinterpret_cast<float2 *>(ypart + (size_t(g) * CT + ch) * TC + tl0);
+#pragma unroll
+        for (int p = 0; p < KP; ++p) mine[p] = y[p];
+        __syncthreads();  // every state group's partial sums visible
+#pragma unroll
+        for (int i = 0; i < KE; ++i) yo[i] = 0.f;
+#pragma unroll
+        for (int gg = 0; gg < NG; ++gg) {
+          const float2 *src = reinterpret_cast<const float2 *>(ypart + (size_t(gg) * CT + ch) * TC + tl0 + e0);
+#pragma unroll
+          for (int p = 0; p < KE / 2; ++p) {
+            const float2 v = src[p];
+            yo[2 * p] += v.x;
+            yo[2 * p + 1] += v.y;
+          }
+        }
+      }
+      if (ch_ok) {
+        const float Dd = Dsk[ch];
+        const T *ru = X + size_t(ch) * XP + tl0 + e0;
+        [[maybe_unused]] const T *rz = X + size_t(2 * CT + ch) * XP + tl0 + e0;
+        constexpr int VE = KE < V ? KE : V;  // elements per input vector read
+        constexpr int VO = Elem<TO>::kVec;   // output elements per 16-byte store
+#pragma unroll
+        for (int lv = 0; lv < KE / VE; ++lv) {
+          float vu[V];
+          [[maybe_unused]] float vz[V];
+          if constexpr (VE == V) {
+            unpack16<T>(*reinterpret_cast<const uint4 *>(ru + lv * V), vu);
+            if constexpr (HAS_Z) unpack16<T>(*reinterpret_cast<const uint4 *>(rz + lv * V), vz);
+          } else {
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+              vu[e] = Elem<T>::to_f32(ru[e]);
+              if constexpr (HAS_Z) vz[e] = Elem<T>::to_f32(rz[e]);
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < VE; ++e) {
+            const int i = lv * VE + e;
+            float v = fmaf(Dd, vu[e], yo[i]);
+            if constexpr (HAS_Z) v *= silu_t<kFast>(vz[e]);
+            yo[i] = v;
+          }
+        }
+        const int te = tl0 + e0;
+        TO *gy = static_cast<TO *>(args.y) + xbase + d * args.x_dim_stride + wstart + te;
+        if (VEC && KE % VO == 0 && (!kMasked || (te >= rel_lo && te + KE <= rel_hi))) {
+#pragma unroll
+          for (int v = 0; v < KE / VO; ++v) *reinterpret_cast<uint4 *>(gy + v * VO) = pack16<TO>(yo + v * VO);
+        } else {
+#pragma unroll
+          for (int i = 0; i < KE; ++i)
+            if (!kMasked || (te + i >= rel_lo && te + i < rel_hi)) gy[i] = Elem<TO>::from_f32(yo[i]);
+        }
+      }
+    };
+
+    // ------------------------------------------------------------- the unit's chunks
     if constexpr (VEC) {
-      if (c + 1 < nchunks) issue_chunk(buf ^ 1, c + 1);  // streams in while chunk c is computed
+      if (c_begin < c_end) issue_chunk(int(gc & 1u), c_begin);
     }
-    // chunk-relative sequence bounds; a chunk strictly inside the sequence needs no masks
-    const int rel_lo = int(max64(t_lo - wstart, -1));
-    const int rel_hi = int(min64(t_hi - wstart, TC + 1));
-    const T *X = xs0 + buf * kXElems;
-    const T *Bsm = bc0 + buf * kBCElems;
-    const T *Csm = Bsm + size_t(N) * TC;
-    if (rel_lo <= 0 && rel_hi >= TC)
-      compute_chunk(std::false_type{}, X, Bsm, Csm, wstart, rel_lo, rel_hi);
-    else
-      compute_chunk(std::true_type{}, X, Bsm, Csm, wstart, rel_lo, rel_hi);
+    for (int c = c_begin; c < c_end; ++c, ++gc) {
+      const int buf = int(gc & 1u);
+      const int64_t wstart = w0 + int64_t(c) * TC;
+      if constexpr (VEC) {
+        mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
+      } else {
+        stage_scalar(buf, c);
+      }
+      __syncthreads();  // chunk c visible to all; everyone is done with chunk c-1's buffers
+      if constexpr (VEC) {
+        if (c + 1 < c_end) issue_chunk(buf ^ 1, c + 1);  // streams in while chunk c is computed
+      }
+      // chunk-relative sequence bounds; a chunk strictly inside the sequence needs no masks
+      const int rel_lo = int(max64(t_lo - wstart, -1));
+      const int rel_hi = int(min64(t_hi - wstart, TC + 1));
+      const T *X = xs0 + buf * kXElems;
+      const T *Bsm = bc0 + buf * kBCElems;
+      const T *Csm = Bsm + size_t(N) * TC;
+      if (rel_lo <= 0 && rel_hi >= TC)
+        compute_chunk(std::false_type{}, X, Bsm, Csm, wstart, rel_lo, rel_hi);
+      else
+        compute_chunk(std::true_type{}, X, Bsm, Csm, wstart, rel_lo, rel_hi);
+    }
+
+    // ------------------------------------------------------------- hand the state on
+    __syncthreads();
+    if (PERSIST && c_end < nchunks) {
+      float *dst = args.carries + size_t(chain) * CT * N;
+      for (int i = threadIdx.x; i < CT * N; i += NT) __stcg(dst + i, carry_s[i]);
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) atomicExch(args.flags + chain, uint32_t(kgrp + 1));
+    } else if (args.h_last) {
+      for (int i = threadIdx.x; i < CT * N; i += NT) {
+        const int c2 = i / N, n = i % N;
+        const int64_t dd = d0 + c2;
+        if (dd < args.dim) args.h_last[(int64_t(s) * args.dim + dd) * N + n] = carry_s[i];
+      }
+    }
+    __syncthreads();  // shared state of this unit is dead before the next unit overwrites it
   }
 #undef SSM_GU
 #undef SSM_GDL
 #undef SSM_GZ
 #undef SSM_GB
 #undef SSM_GC
-
-  // final state of each channel of the tile
-  __syncthreads();
-  if (args.h_last) {
-    for (int i = threadIdx.x; i < CT * N; i += NT) {
-      const int c2 = i / N, n = i % N;
-      const int64_t dd = d0 + c2;
-      if (dd < args.dim) args.h_last[(int64_t(s) * args.dim + dd) * N + n] = carry_s[i];
-    }
-  }
 }
 
 }  // namespace ssm

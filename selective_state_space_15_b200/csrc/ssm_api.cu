@@ -13,57 +13,131 @@ using ssm::ScanArgs;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// Tile shapes per state size: KI steps per lane, SPW segment lanes per channel, CPW channels
-// per warp, WARPS warps per CTA.  Larger states get shorter chunks to bound shared memory.
-template <int N> struct Shape;
-template <> struct Shape<16> { static constexpr int KI = 16, SPW = 16, CPW = 2, WARPS = 8; };
-template <> struct Shape<32> { static constexpr int KI = 16, SPW = 8, CPW = 4, WARPS = 8; };
-template <> struct Shape<64> { static constexpr int KI = 8, SPW = 8, CPW = 4, WARPS = 8; };
-template <> struct Shape<128> { static constexpr int KI = 8, SPW = 4, CPW = 8, WARPS = 4; };
+// Tile shapes: KI steps per lane, SPW segment lanes per channel, CPW channels per warp, CW
+// channel warps and NG state groups per CTA.  Larger states get shorter chunks to bound
+// shared memory; the N=16 narrow shape splits the states over two warps for parallelism.
+struct ShapeInfo {
+  int KI, SPW, CPW, CW, NG;
+  int ct() const { return CPW * CW; }
+  int tc() const { return SPW * KI; }
+};
+template <int N, bool NARROW> struct Shape;
+template <> struct Shape<16, false> { static constexpr int KI = 16, SPW = 16, CPW = 2, CW = 8, NG = 1; };
+template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW = 2, CW = 4, NG = 2; };
+template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 8, NG = 1; };
+template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
+template <> struct Shape<128, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 4, NG = 1; };
+template <int N, bool NARROW> ShapeInfo shape_of() {
+  using S = Shape<N, NARROW>;
+  return ShapeInfo{S::KI, S::SPW, S::CPW, S::CW, S::NG};
+}
+bool shape_for(int N, bool narrow, ShapeInfo &si) {
+  switch (N) {
+    case 16: si = narrow ? shape_of<16, true>() : shape_of<16, false>(); return true;
+    case 32: si = shape_of<32, false>(); return true;
+    case 64: si = shape_of<64, false>(); return true;
+    case 128: si = shape_of<128, false>(); return true;
+    default: return false;
+  }
+}
 
-template <typename T, typename TO, int N, bool HAS_Z, bool VEC>
-ssm_status_t launch_chunk(const ScanArgs &a, cudaStream_t stream) {
-  using S = Shape<N>;
-  using Cfg = ssm::ChunkCfg<T, N, S::KI, S::SPW, S::CPW, S::WARPS>;
-  auto kern = ssm::chunk_scan_kernel<T, TO, N, S::KI, S::SPW, S::CPW, S::WARPS, HAS_Z, VEC>;
-  static bool configured = false;  // per instantiation; the attribute is per device function
-  if (!configured) {
+// How a scan is run: persistent ticketed units for 16-byte aligned fixed-length batches,
+// one CTA per (sequence, tile) otherwise.
+struct Plan {
+  bool persist = false, narrow = false;
+  ShapeInfo si{};
+  int64_t ntiles = 0, nchains = 0, nchunks = 0;
+  size_t flags_off = 0, carries_off = 0, ws_bytes = 0;
+};
+constexpr int64_t kNarrowChannels = 8192;  // batch * dim below this: split states over 2 warps
+
+bool make_plan(int N, int64_t nseq, int64_t dim, int64_t seqlen, bool varlen, bool vec, Plan &pl) {
+  pl = Plan{};
+  pl.persist = !varlen && vec && seqlen > 0;
+  pl.narrow = pl.persist && N == 16 && nseq * dim < kNarrowChannels;
+  if (!shape_for(N, pl.narrow, pl.si)) return false;
+  pl.ntiles = (dim + pl.si.ct() - 1) / pl.si.ct();
+  pl.nchains = nseq * pl.ntiles;
+  pl.nchunks = pl.persist ? (seqlen + pl.si.tc() - 1) / pl.si.tc() : 0;
+  if (pl.persist) {
+    pl.flags_off = 16;  // the ticket counter lives in the first 16 bytes
+    pl.carries_off = (pl.flags_off + size_t(pl.nchains) * 4 + 15) / 16 * 16;
+    pl.ws_bytes = pl.carries_off + size_t(pl.nchains) * pl.si.ct() * N * sizeof(float);
+  }
+  return true;
+}
+
+template <typename T, typename TO, int N, bool NARROW, bool HAS_Z, bool VEC, bool PERSIST>
+ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t stream) {
+  using S = Shape<N, NARROW>;
+  using Cfg = ssm::ChunkCfg<T, N, S::KI, S::SPW, S::CPW, S::CW, S::NG>;
+  auto kern = ssm::chunk_scan_kernel<T, TO, N, S::KI, S::SPW, S::CPW, S::CW, S::NG, HAS_Z, VEC, PERSIST>;
+  static int configured_device = -1;  // the attribute is set once per device function per device
+  static int max_blocks_per_sm = 0;
+  static int num_sms = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
+  if (configured_device != dev) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) !=
         cudaSuccess)
       return SSM_ERR_CUDA;
-    configured = true;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&max_blocks_per_sm, kern, Cfg::kThreads, Cfg::kSmemBytes) !=
+        cudaSuccess)
+      return SSM_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SSM_ERR_CUDA;
+    configured_device = dev;
   }
-  const int64_t blocks = int64_t(a.nseq) * a.ntiles;
-  if (blocks == 0) return SSM_OK;
+  if (pl.nchains == 0) return SSM_OK;
+  int64_t blocks = pl.nchains;
+  if constexpr (PERSIST) {
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    if (cudaMemsetAsync(w, 0, pl.carries_off, stream) != cudaSuccess) return SSM_ERR_CUDA;
+    const int64_t resident = int64_t(num_sms) * (max_blocks_per_sm > 0 ? max_blocks_per_sm : 1);
+    // enough units per CTA for an even spread, as few as possible for low per-unit overhead
+    int64_t group = (pl.nchunks * pl.nchains) / (8 * resident);
+    group = group < 1 ? 1 : (group > pl.nchunks ? pl.nchunks : group);
+    const int64_t ngroups = (pl.nchunks + group - 1) / group;
+    if (pl.nchains * ngroups > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    a.ticket = reinterpret_cast<uint32_t *>(w);
+    a.flags = reinterpret_cast<uint32_t *>(w + pl.flags_off);
+    a.carries = reinterpret_cast<float *>(w + pl.carries_off);
+    a.nchains = int(pl.nchains);
+    a.group = int(group);
+    a.total_units = int(pl.nchains * ngroups);
+    blocks = a.total_units < resident ? a.total_units : resident;
+  }
   if (blocks > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
   kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
-template <typename T, typename TO, int N>
-ssm_status_t dispatch_zv(const ScanArgs &a, bool has_z, bool vec, cudaStream_t st) {
-  if (has_z) return vec ? launch_chunk<T, TO, N, true, true>(a, st) : launch_chunk<T, TO, N, true, false>(a, st);
-  return vec ? launch_chunk<T, TO, N, false, true>(a, st) : launch_chunk<T, TO, N, false, false>(a, st);
-}
-
-template <typename T, typename TO>
-ssm_status_t dispatch_n(const ScanArgs &a, int N, bool has_z, bool vec, cudaStream_t st) {
-  switch (N) {
-    case 16: return dispatch_zv<T, TO, 16>(a, has_z, vec, st);
-    case 32: return dispatch_zv<T, TO, 32>(a, has_z, vec, st);
-    case 64: return dispatch_zv<T, TO, 64>(a, has_z, vec, st);
-    case 128: return dispatch_zv<T, TO, 128>(a, has_z, vec, st);
-    default: return SSM_ERR_UNSUPPORTED;
+template <typename T, typename TO, int N, bool NARROW>
+ssm_status_t dispatch_zvp(const ScanArgs &a, const Plan &pl, bool has_z, bool vec, void *ws, cudaStream_t st) {
+  if (pl.persist) {
+    if (has_z) return launch_chunk<T, TO, N, NARROW, true, true, true>(a, pl, ws, st);
+    return launch_chunk<T, TO, N, NARROW, false, true, true>(a, pl, ws, st);
+  }
+  if constexpr (NARROW) {
+    return SSM_ERR_UNSUPPORTED;  // the narrow shape is only planned for persistent launches
+  } else {
+    if (has_z)
+      return vec ? launch_chunk<T, TO, N, false, true, true, false>(a, pl, ws, st)
+                 : launch_chunk<T, TO, N, false, true, false, false>(a, pl, ws, st);
+    return vec ? launch_chunk<T, TO, N, false, false, true, false>(a, pl, ws, st)
+               : launch_chunk<T, TO, N, false, false, false, false>(a, pl, ws, st);
   }
 }
 
-int tile_channels(int N) {
+template <typename T, typename TO>
+ssm_status_t dispatch_n(const ScanArgs &a, const Plan &pl, int N, bool has_z, bool vec, void *ws,
+                        cudaStream_t st) {
   switch (N) {
-    case 16: return Shape<16>::CPW * Shape<16>::WARPS;
-    case 32: return Shape<32>::CPW * Shape<32>::WARPS;
-    case 64: return Shape<64>::CPW * Shape<64>::WARPS;
-    case 128: return Shape<128>::CPW * Shape<128>::WARPS;
-    default: return 0;
+    case 16: return pl.narrow ? dispatch_zvp<T, TO, 16, true>(a, pl, has_z, vec, ws, st)
+                              : dispatch_zvp<T, TO, 16, false>(a, pl, has_z, vec, ws, st);
+    case 32: return dispatch_zvp<T, TO, 32, false>(a, pl, has_z, vec, ws, st);
+    case 64: return dispatch_zvp<T, TO, 64, false>(a, pl, has_z, vec, ws, st);
+    case 128: return dispatch_zvp<T, TO, 128, false>(a, pl, has_z, vec, ws, st);
+    default: return SSM_ERR_UNSUPPORTED;
   }
 }
 
@@ -76,7 +150,8 @@ ssm_status_t prepare_scan(const ssm_scan_params *p, bool varlen, ScanArgs &a, bo
   if (p->dim <= 0 || p->dstate <= 0 || p->seqlen < 0 || p->batch < 0) return SSM_ERR_INVALID_ARG;
   if (varlen && p->batch != 1) return SSM_ERR_INVALID_ARG;
   if (!p->u || !p->delta || !p->B || !p->C || !p->A || !p->y) return SSM_ERR_INVALID_ARG;
-  if (tile_channels(int(p->dstate)) == 0 || p->dstate != int64_t(int(p->dstate))) return SSM_ERR_UNSUPPORTED;
+  ShapeInfo probe;
+  if (p->dstate > 128 || !shape_for(int(p->dstate), false, probe)) return SSM_ERR_UNSUPPORTED;
   if (p->dim > (int64_t(1) << 31) || p->seqlen > (int64_t(1) << 40)) return SSM_ERR_UNSUPPORTED;
   a = ScanArgs{};
   a.u = p->u; a.delta = p->delta; a.z = p->z; a.B = p->B; a.C = p->C;
@@ -96,17 +171,21 @@ ssm_status_t prepare_scan(const ssm_scan_params *p, bool varlen, ScanArgs &a, bo
   vec = aligned16(p->u) && aligned16(p->delta) && aligned16(p->B) && aligned16(p->C) && aligned16(p->y) &&
         (!p->z || aligned16(p->z)) && a.x_dim_stride % V == 0 && a.bc_state_stride % V == 0 &&
         (varlen || (a.x_batch_stride % V == 0 && a.bc_batch_stride % V == 0));
-  a.ntiles = int((p->dim + tile_channels(int(p->dstate)) - 1) / tile_channels(int(p->dstate)));
   return SSM_OK;
 }
 
-ssm_status_t run_scan(const ScanArgs &a, ssm_dtype_t dt, bool y_fp32, int N, bool vec, cudaStream_t st) {
+ssm_status_t run_scan(ScanArgs a, const Plan &pl, ssm_dtype_t dt, bool y_fp32, int N, bool vec, void *ws,
+                      size_t ws_bytes, cudaStream_t st) {
+  if (pl.ws_bytes > 0 && (ws == nullptr || ws_bytes < pl.ws_bytes || (reinterpret_cast<uintptr_t>(ws) & 15)))
+    return SSM_ERR_WORKSPACE;
+  if (pl.ntiles > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+  a.ntiles = int(pl.ntiles);
   const bool has_z = a.z != nullptr;
   if (dt == SSM_BF16) {
-    if (y_fp32) return dispatch_n<__nv_bfloat16, float>(a, N, has_z, vec, st);
-    return dispatch_n<__nv_bfloat16, __nv_bfloat16>(a, N, has_z, vec, st);
+    if (y_fp32) return dispatch_n<__nv_bfloat16, float>(a, pl, N, has_z, vec, ws, st);
+    return dispatch_n<__nv_bfloat16, __nv_bfloat16>(a, pl, N, has_z, vec, ws, st);
   }
-  return dispatch_n<float, float>(a, N, has_z, vec, st);
+  return dispatch_n<float, float>(a, pl, N, has_z, vec, ws, st);
 }
 
 }  // namespace
@@ -115,23 +194,22 @@ extern "C" {
 
 ssm_status_t ssm_scan_fwd(const ssm_scan_params *p, void *workspace, size_t workspace_bytes,
                           ssm_stream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   ScanArgs a;
   bool vec = false;
   ssm_status_t st = prepare_scan(p, false, a, vec);
   if (st != SSM_OK) return st;
   if (p->batch == 0) return SSM_OK;
   if (p->batch > (int64_t(1) << 30)) return SSM_ERR_UNSUPPORTED;
+  Plan pl;
+  if (!make_plan(int(p->dstate), p->batch, p->dim, p->seqlen, false, vec, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = nullptr;
   a.nseq = int(p->batch);
-  return run_scan(a, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, reinterpret_cast<cudaStream_t>(stream));
+  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seqlens, int64_t nseq,
                                  void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (!cu_seqlens || nseq < 0) return SSM_ERR_INVALID_ARG;
   if (nseq > (int64_t(1) << 30)) return SSM_ERR_UNSUPPORTED;
   if (p && p->seqlen > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;  // int32 offsets
@@ -140,9 +218,12 @@ ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seq
   ssm_status_t st = prepare_scan(p, true, a, vec);
   if (st != SSM_OK) return st;
   if (nseq == 0) return SSM_OK;
+  Plan pl;
+  if (!make_plan(int(p->dstate), nseq, p->dim, p->seqlen, true, vec, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = cu_seqlens;
   a.nseq = int(nseq);
-  return run_scan(a, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, reinterpret_cast<cudaStream_t>(stream));
+  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slot_ids, int64_t R,
@@ -188,9 +269,13 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
 }
 
 size_t ssm_scan_workspace_size(const ssm_scan_params *p, int64_t nseq) {
-  (void)p;
-  (void)nseq;
-  return 0;
+  ScanArgs a;
+  bool vec = false;
+  const bool varlen = nseq > 0;
+  if (prepare_scan(p, varlen, a, vec) != SSM_OK) return 0;
+  Plan pl;
+  if (!make_plan(int(p->dstate), varlen ? nseq : p->batch, p->dim, p->seqlen, varlen, vec, pl)) return 0;
+  return pl.ws_bytes;
 }
 
 ssm_status_t ssm_get_device_status(ssm_stream_t stream) {

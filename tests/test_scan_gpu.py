@@ -199,3 +199,36 @@ def test_varlen_workload_float32_output_strict():
     ref = oracle.scan_varlen(inp.u[ch], inp.delta[ch], inp.B, inp.C, inp.A[ch], inp.cu_seqlens, inp.Dskip[ch],
                              inp.bias[ch], inp.z[ch], nthreads=NTHREADS)
     check("y", y[ch], ref["y"], ref["y_mag"], TOL["bf16"], "f32")
+
+
+def test_persistent_paths_and_workspace():
+    """Aligned fixed-length batches run on the persistent ticketed grid (state handed between
+    units through the workspace); narrow problems split the states over two warps."""
+    import ctypes
+    lib = ssm.load()
+    for (b, D, L, seed) in [(1, 8, 4096, 21), (3, 40, 2304, 22), (2, 2048 + 8, 512, 23)]:
+        inp = workloads.batch_inputs(b, D, 16, L, "bf16", seed=seed)
+        y, hl = run_batch(inp, "bf16", y_dtype=torch.float32)
+        ch = np.arange(0, D, max(1, D // 24))
+        ref = oracle_batch(inp, channels=ch)
+        check("y", y[:, ch], ref["y"], ref["y_mag"], TOL["bf16"], "f32")
+        check("h_last", hl[:, ch], ref["h_last"], ref["h_mag"], TOL["bf16"])
+    # the workspace size is reported and enforced
+    inp = workloads.batch_inputs(1, 8, 16, 256, "bf16", seed=24)
+    u, dl, z, B, C = (dev(x, "bf16") for x in (inp.u, inp.delta, inp.z, inp.B, inp.C))
+    A = torch.from_numpy(inp.A).cuda()
+    y = torch.empty_like(u)
+    p = ssm.scan_params(u, dl, B, C, A, z=z, y=y)
+    need = lib.ssm_scan_workspace_size(ctypes.byref(p), 0)
+    assert need > 0
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.ssm_scan_fwd(ctypes.byref(p), None, 0, stream) == 6                    # SSM_ERR_WORKSPACE
+    small = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    assert lib.ssm_scan_fwd(ctypes.byref(p), ctypes.c_void_p(small.data_ptr()), need - 16, stream) == 6
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    for _ in range(2):                                                                # reuse of a workspace
+        assert lib.ssm_scan_fwd(ctypes.byref(p), ctypes.c_void_p(ws.data_ptr()), need, stream) == 0
+    torch.cuda.synchronize()
+    ref = oracle.scan(inp.u, inp.delta, inp.B, inp.C, inp.A, z=inp.z)
+    check("y", host(y), ref["y"], ref["y_mag"], TOL["bf16"], "bf16")
+    assert ssm.device_status() == 0
