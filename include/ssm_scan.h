@@ -138,6 +138,29 @@ ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seq
 ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slot_ids, int64_t R,
                               const ssm_scan_params *p, ssm_stream_t stream);
 
+/*
+ * Allocation-free variant of ssm_scan_fwd.  (The pages have no counterpart; this is a
+ * library convenience.)
+ *
+ * Some callers cannot allocate device memory while they run: a plugin inside an inference
+ * engine whose enqueue step must not allocate, or a serving loop that bans cudaMalloc after
+ * start-up because cudaMalloc can synchronise the device and stall other streams.  Such a
+ * caller cannot provide the workspace ssm_scan_fwd may ask for.  This entry point takes the
+ * same problem description and computes the same result, but its scratch is a static device
+ * array of SSM_NOALLOC_SCRATCH_BYTES inside the library (every GPU that loads the library
+ * holds it until the process exits).  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *   - The first call on a device looks up the array's device address for that device
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - A problem whose scratch need (ssm_scan_workspace_size) exceeds
+ *     SSM_NOALLOC_SCRATCH_BYTES is rejected with SSM_ERR_WORKSPACE before anything runs.
+ *   - All calls share the one array and it keeps the last call's contents; each call clears
+ *     the part that must start at zero (an asynchronous memset on `stream`).  Calls that can
+ *     overlap on the GPU (e.g. on two streams without ordering) race on the array: order them.
+ */
+#define SSM_NOALLOC_SCRATCH_BYTES (4u << 20)
+ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_params *p, ssm_stream_t stream);
+
 /* Bytes of device workspace the scan entry points need for this problem (0 if none).
  * For the fixed-length scan pass nseq = 0. */
 size_t ssm_scan_workspace_size(const ssm_scan_params *p, int64_t nseq);

@@ -19,7 +19,8 @@ ABI_VERSION = 1
 
 # Every function the header declares; tests check the library exports all of them.
 EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
-            "ssm_get_device_status", "ssm_status_string", "ssm_abi_version")
+            "ssm_get_device_status", "ssm_status_string", "ssm_abi_version", "ssm_scan_fwd_noalloc")
+NOALLOC_SCRATCH_BYTES = 4 << 20  # SSM_NOALLOC_SCRATCH_BYTES
 
 
 class SSMError(RuntimeError):
@@ -59,6 +60,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     P, I64, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
     pp = ctypes.POINTER(ScanParams)
     lib.ssm_scan_fwd.argtypes = [pp, P, S, P]
+    lib.ssm_scan_fwd_noalloc.argtypes = [pp, P]
+    lib.ssm_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssm_scan_fwd_varlen.argtypes = [pp, P, I64, P, S, P]
     lib.ssm_state_update.argtypes = [P, I64, P, I64, pp, P]
     lib.ssm_scan_workspace_size.argtypes = [pp, I64]

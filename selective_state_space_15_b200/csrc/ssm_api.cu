@@ -3,6 +3,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "ssm_scan.h"
 #include "chunk_scan.cuh"
 #include "state_update.cuh"
@@ -188,9 +190,52 @@ ssm_status_t run_scan(ScanArgs a, const Plan &pl, ssm_dtype_t dt, bool y_fp32, i
   return dispatch_n<float, float>(a, pl, N, has_z, vec, ws, st);
 }
 
+// Scratch for ssm_scan_fwd_noalloc: a static device array that every GPU loading the
+// library holds until the process exits.  In host code `g_noalloc_scratch` names a host-side
+// stand-in, not device memory, so its device address is looked up once per device.
+constexpr size_t kNoAllocScratchBytes = SSM_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device (looked up on first use).
+ssm_status_t noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return SSM_ERR_CUDA;
+  if (dev >= kMaxDevices) return SSM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return SSM_ERR_CUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return SSM_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_params *p, ssm_stream_t stream) {
+  ScanArgs a;
+  bool vec = false;
+  ssm_status_t st = prepare_scan(p, false, a, vec);
+  if (st != SSM_OK) return st;
+  if (p->batch == 0) return SSM_OK;
+  if (p->batch > (int64_t(1) << 30)) return SSM_ERR_UNSUPPORTED;
+  Plan pl;
+  if (!make_plan(int(p->dstate), p->batch, p->dim, p->seqlen, false, vec, pl)) return SSM_ERR_UNSUPPORTED;
+  if (pl.ws_bytes > kNoAllocScratchBytes) return SSM_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != SSM_OK) return st;
+  a.cu_seqlens = nullptr;
+  a.nseq = int(p->batch);
+  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, scratch, kNoAllocScratchBytes,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
 
 ssm_status_t ssm_scan_fwd(const ssm_scan_params *p, void *workspace, size_t workspace_bytes,
                           ssm_stream_t stream) {
