@@ -90,12 +90,13 @@ struct ChunkCfg {
   static constexpr size_t kXBytes = size_t(3) * kCT * kXPitch * sizeof(T);  // u, delta, z
   static constexpr size_t kBCBytes = size_t(2) * N * kTC * sizeof(T);       // B, C
   static constexpr size_t kYBytes = NG > 1 ? size_t(NG) * kCT * kTC * sizeof(float) : 0;  // partial y
+  static constexpr int kNP = N + 1;         // row pitch of the per-(channel, state) arrays
   static constexpr size_t kParamBytes =
-      size_t(2) * kCT * N * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
+      size_t(2) * kCT * kNP * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
   static constexpr size_t kSmemBytes = 2 * kXBytes + 2 * kBCBytes + kYBytes + kParamBytes;
   static_assert(KI % 4 == 0 && KI % kVec == 0, "a lane's steps must be whole 16-byte vectors");
   static_assert(32 % SPW == 0 && CPW * SPW == 32, "lane split");
-  static_assert(N % NG == 0 && (KI / NG) % 2 == 0, "state / step split");
+  static_assert(N % NG == 0 && KI % NG == 0, "state / step split");
   static_assert(kXBytes % 16 == 0 && kBCBytes % 16 == 0, "16-byte aligned buffers");
 };
 
@@ -116,9 +117,11 @@ chunk_scan_kernel(const ScanArgs args) {
   T *const xs0 = reinterpret_cast<T *>(smem);                     // [2][3][CT][XP]
   T *const bc0 = reinterpret_cast<T *>(smem + 2 * Cfg::kXBytes);  // [2][2][N][TC]
   float *ypart = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes);  // [NG][CT][TC]
-  float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes);  // [CT][N]
-  float *carry_s = A2s + CT * N;                                  // [CT][N]
-  float *Dsk = carry_s + CT * N;                                  // [CT]
+  // [CT][N] arrays use a row pitch of N + 1 words, so the channels of a warp hit distinct banks
+  constexpr int NP = Cfg::kNP;
+  float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes);  // [CT][NP]
+  float *carry_s = A2s + CT * NP;                                 // [CT][NP]
+  float *Dsk = carry_s + CT * NP;                                 // [CT]
   float *bias_s = Dsk + CT;                                       // [CT]
   int *order = reinterpret_cast<int *>(bias_s + CT);              // [kMaxSortedSeqs]
   __shared__ __align__(8) uint64_t bars[2];                      // chunk-arrival barriers
@@ -212,7 +215,7 @@ chunk_scan_kernel(const ScanArgs args) {
     for (int i = threadIdx.x; i < CT * N; i += NT) {
       const int c2 = i / N, n = i % N;
       const int64_t dd = d0 + c2;
-      A2s[i] = dd < args.dim ? args.A[dd * N + n] * kLog2e : 0.f;
+      A2s[c2 * NP + n] = dd < args.dim ? args.A[dd * N + n] * kLog2e : 0.f;
     }
     for (int i = threadIdx.x; i < CT; i += NT) {
       const int64_t dd = d0 + i;
@@ -226,7 +229,7 @@ chunk_scan_kernel(const ScanArgs args) {
       for (int i = threadIdx.x; i < CT * N; i += NT) {
         const int c2 = i / N, n = i % N;
         const int64_t dd = d0 + c2;
-        carry_s[i] = (dd < args.dim && args.h0) ? args.h0[(int64_t(s) * args.dim + dd) * N + n] : 0.f;
+        carry_s[c2 * NP + n] = (dd < args.dim && args.h0) ? args.h0[(int64_t(s) * args.dim + dd) * N + n] : 0.f;
       }
     } else {
       if (threadIdx.x == 0) {
@@ -241,7 +244,7 @@ chunk_scan_kernel(const ScanArgs args) {
       }
       __syncthreads();
       const float *src = args.carries + size_t(chain) * CT * N;
-      for (int i = threadIdx.x; i < CT * N; i += NT) carry_s[i] = __ldcg(src + i);
+      for (int i = threadIdx.x; i < CT * N; i += NT) carry_s[(i / N) * NP + i % N] = __ldcg(src + i);
     }
 
     // TMA: chunk c's u/delta/z and B/C rows into buffer `buf`.
@@ -302,6 +305,8 @@ chunk_scan_kernel(const ScanArgs args) {
       // ---- prologue: Delta and Delta*u for the lane's KI steps (as pairs of steps) ----
       float2 dl[KP], du[KP], y[KP];
       float dsum = 0.f;
+#pragma unroll
+      for (int p = 0; p < KP; ++p) y[p] = make_float2(0.f, 0.f);
       {
         const T *ru = X + size_t(ch) * XP + tl0;
         const T *rd = X + size_t(CT + ch) * XP + tl0;
@@ -326,44 +331,64 @@ chunk_scan_kernel(const ScanArgs args) {
             }
             dl[p] = dt;
             dsum += dt.x + dt.y;
-            y[p] = make_float2(0.f, 0.f);
           }
         }
       }
 
       // ---- state loop over this warp's NS states ----
-#pragma unroll 1
-      for (int n = n0; n < n0 + NS; ++n) {
-        const float A2 = A2s[ch * N + n];
+      // Software-pipelined: the forward pass of state n (exponentials, b_i, segment operator)
+      // runs in the same step loop as the output pass of state n - 1, which frees a[i], b[i]
+      // just before they are refilled.  Two independent recurrence chains are then in flight
+      // and the exponentials are spread over the whole loop.
+      float a[KI];
+      float2 b[KP];
+      // FWD: a, b and the segment operator G of state n1 from zero; OUT: h over the steps of
+      // state n2 (a, b as left by its forward pass) and y += C h.
+      auto steps = [&](auto fwd_tag, auto out_tag, int n1, int n2, float &G, float &h) {
+        constexpr bool FWD = decltype(fwd_tag)::value, OUT = decltype(out_tag)::value;
+        const float A2 = FWD ? A2s[ch * NP + n1] : 0.f;
         const float2 A22 = make_float2(A2, A2);
-        const float carry = carry_s[ch * N + n];
-        float a[KI];
-        float2 b[KP];
-        float G = 0.f;
-        const T *rb = Bsm + size_t(n) * TC + tl0;
+        const T *rb = Bsm + size_t(n1) * TC + tl0;
+        const T *rc = Csm + size_t(n2) * TC + tl0;
 #pragma unroll
         for (int lv = 0; lv < LV; ++lv) {
-          float2 bb[V / 2];
-          unpack16x2<T>(*reinterpret_cast<const uint4 *>(rb + lv * V), bb);
+          float2 bb[V / 2], cc[V / 2];
+          if constexpr (FWD) unpack16x2<T>(*reinterpret_cast<const uint4 *>(rb + lv * V), bb);
+          if constexpr (OUT) unpack16x2<T>(*reinterpret_cast<const uint4 *>(rc + lv * V), cc);
 #pragma unroll
           for (int e = 0; e < V / 2; ++e) {
             const int p = lv * (V / 2) + e;
-            const float2 x = __fmul2_rn(dl[p], A22);
-            a[2 * p] = ex2_approx(x.x);
-            a[2 * p + 1] = ex2_approx(x.y);
-            if constexpr (kMasked) {
-              // stale B outside the window never reaches h (du is 0 there, B may be non-finite)
-              b[p] = make_float2(du[p].x != 0.f ? du[p].x * bb[e].x : 0.f,
-                                 du[p].y != 0.f ? du[p].y * bb[e].y : 0.f);
-            } else {
-              b[p] = __fmul2_rn(du[p], bb[e]);
+            if constexpr (OUT) {
+              float2 hh;
+              h = fmaf(a[2 * p], h, b[p].x);
+              hh.x = h;
+              h = fmaf(a[2 * p + 1], h, b[p].y);
+              hh.y = h;
+              y[p] = __ffma2_rn(cc[e], hh, y[p]);
             }
-            G = fmaf(a[2 * p], G, b[p].x);
-            G = fmaf(a[2 * p + 1], G, b[p].y);
+            if constexpr (FWD) {
+              const float2 x = __fmul2_rn(dl[p], A22);
+              a[2 * p] = ex2_approx(x.x);
+              a[2 * p + 1] = ex2_approx(x.y);
+              if constexpr (kMasked) {
+                // stale B outside the window never reaches h (du is 0 there, B may be non-finite)
+                b[p] = make_float2(du[p].x != 0.f ? du[p].x * bb[e].x : 0.f,
+                                   du[p].y != 0.f ? du[p].y * bb[e].y : 0.f);
+              } else {
+                b[p] = __fmul2_rn(du[p], bb[e]);
+              }
+              G = fmaf(a[2 * p], G, b[p].x);
+              G = fmaf(a[2 * p + 1], G, b[p].y);
+            }
           }
         }
+      };
+      // Scan of the segment operators of state n across the SPW segment lanes of each
+      // channel; returns the state entering this lane's first step and advances the carry.
+      auto scan_state = [&](int n, float G) -> float {
+        const float A2 = A2s[ch * NP + n];
+        const float carry = carry_s[ch * NP + n];
         float P = ex2_approx(dsum * A2);  // product of the lane's a_i
-        // inclusive scan of segment operators across the SPW segment lanes of this channel
 #pragma unroll
         for (int off = 1; off < SPW; off *= 2) {
           const float Pu = __shfl_up_sync(0xffffffffu, P, off * CPW);
@@ -379,25 +404,23 @@ chunk_scan_kernel(const ScanArgs args) {
           Pe = 1.f;
           Ge = 0.f;
         }
-        float h = fmaf(Pe, carry, Ge);  // state entering this lane's first step
         __syncwarp();
-        if (seg == SPW - 1) carry_s[ch * N + n] = fmaf(P, carry, G);  // state leaving the chunk
-        const T *rc = Csm + size_t(n) * TC + tl0;
-#pragma unroll
-        for (int lv = 0; lv < LV; ++lv) {
-          float2 cc[V / 2];
-          unpack16x2<T>(*reinterpret_cast<const uint4 *>(rc + lv * V), cc);
-#pragma unroll
-          for (int e = 0; e < V / 2; ++e) {
-            const int p = lv * (V / 2) + e;
-            float2 hh;
-            h = fmaf(a[2 * p], h, b[p].x);
-            hh.x = h;
-            h = fmaf(a[2 * p + 1], h, b[p].y);
-            hh.y = h;
-            y[p] = __ffma2_rn(cc[e], hh, y[p]);
-          }
+        if (seg == SPW - 1) carry_s[ch * NP + n] = fmaf(P, carry, G);  // state leaving the chunk
+        return fmaf(Pe, carry, Ge);
+      };
+      {
+        using yes = std::true_type;
+        using no = std::false_type;
+        float G = 0.f, h = 0.f;
+        steps(yes{}, no{}, n0, n0, G, h);
+        h = scan_state(n0, G);
+#pragma unroll 1
+        for (int n = n0 + 1; n < n0 + NS; ++n) {
+          G = 0.f;
+          steps(yes{}, yes{}, n, n - 1, G, h);
+          h = scan_state(n, G);
         }
+        steps(no{}, yes{}, n0 + NS - 1, n0 + NS - 1, G, h);
       }
 
       // ---- epilogue: sum of the state groups, skip term, gate, store ----
@@ -418,12 +441,17 @@ chunk_scan_kernel(const ScanArgs args) {
         for (int i = 0; i < KE; ++i) yo[i] = 0.f;
 #pragma unroll
         for (int gg = 0; gg < NG; ++gg) {
-          const float2 *src = reinterpret_cast<const float2 *>(ypart + (size_t(gg) * CT + ch) * TC + tl0 + e0);
+          const float *src = ypart + (size_t(gg) * CT + ch) * TC + tl0 + e0;
+          if constexpr (KE % 2 == 0) {
 #pragma unroll
-          for (int p = 0; p < KE / 2; ++p) {
-            const float2 v = src[p];
-            yo[2 * p] += v.x;
-            yo[2 * p + 1] += v.y;
+            for (int p = 0; p < KE / 2; ++p) {
+              const float2 v = reinterpret_cast<const float2 *>(src)[p];
+              yo[2 * p] += v.x;
+              yo[2 * p + 1] += v.y;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < KE; ++i) yo[i] += src[i];
           }
         }
       }
@@ -500,7 +528,7 @@ chunk_scan_kernel(const ScanArgs args) {
     __syncthreads();
     if (PERSIST && c_end < nchunks) {
       float *dst = args.carries + size_t(chain) * CT * N;
-      for (int i = threadIdx.x; i < CT * N; i += NT) __stcg(dst + i, carry_s[i]);
+      for (int i = threadIdx.x; i < CT * N; i += NT) __stcg(dst + i, carry_s[(i / N) * NP + i % N]);
       __threadfence();
       __syncthreads();
       if (threadIdx.x == 0) atomicExch(args.flags + chain, uint32_t(kgrp + 1));
@@ -508,7 +536,7 @@ chunk_scan_kernel(const ScanArgs args) {
       for (int i = threadIdx.x; i < CT * N; i += NT) {
         const int c2 = i / N, n = i % N;
         const int64_t dd = d0 + c2;
-        if (dd < args.dim) args.h_last[(int64_t(s) * args.dim + dd) * N + n] = carry_s[i];
+        if (dd < args.dim) args.h_last[(int64_t(s) * args.dim + dd) * N + n] = carry_s[c2 * NP + n];
       }
     }
     __syncthreads();  // shared state of this unit is dead before the next unit overwrites it

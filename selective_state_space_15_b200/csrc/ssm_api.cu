@@ -17,18 +17,19 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 // Tile shapes: KI steps per lane, SPW segment lanes per channel, CPW channels per warp, CW
 // channel warps and NG state groups per CTA.  Larger states get shorter chunks to bound
-// shared memory; the N=16 narrow shape splits the states over two warps for parallelism.
+// shared memory; the narrow shapes split the states over several warps for parallelism.
 struct ShapeInfo {
   int KI, SPW, CPW, CW, NG;
   int ct() const { return CPW * CW; }
   int tc() const { return SPW * KI; }
 };
 template <int N, bool NARROW> struct Shape;
-template <> struct Shape<16, false> { static constexpr int KI = 16, SPW = 16, CPW = 2, CW = 8, NG = 1; };
+template <> struct Shape<16, false> { static constexpr int KI = 16, SPW = 4, CPW = 8, CW = 4, NG = 1; };
 template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW = 2, CW = 4, NG = 2; };
 template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<128, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 4, NG = 1; };
+template <> struct Shape<128, true> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 1, NG = 8; };
 template <int N, bool NARROW> ShapeInfo shape_of() {
   using S = Shape<N, NARROW>;
   return ShapeInfo{S::KI, S::SPW, S::CPW, S::CW, S::NG};
@@ -38,7 +39,7 @@ bool shape_for(int N, bool narrow, ShapeInfo &si) {
     case 16: si = narrow ? shape_of<16, true>() : shape_of<16, false>(); return true;
     case 32: si = shape_of<32, false>(); return true;
     case 64: si = shape_of<64, false>(); return true;
-    case 128: si = shape_of<128, false>(); return true;
+    case 128: si = narrow ? shape_of<128, true>() : shape_of<128, false>(); return true;
     default: return false;
   }
 }
@@ -51,12 +52,14 @@ struct Plan {
   int64_t ntiles = 0, nchains = 0, nchunks = 0;
   size_t flags_off = 0, carries_off = 0, ws_bytes = 0;
 };
-constexpr int64_t kNarrowChannels = 8192;  // batch * dim below this: split states over 2 warps
+// batch * dim below these: split the states over several warps (N=16: 2, N=128: 8)
+constexpr int64_t kNarrowChannels16 = 8192, kNarrowChannels128 = 32768;
 
 bool make_plan(int N, int64_t nseq, int64_t dim, int64_t seqlen, bool varlen, bool vec, Plan &pl) {
   pl = Plan{};
   pl.persist = !varlen && vec && seqlen > 0;
-  pl.narrow = pl.persist && N == 16 && nseq * dim < kNarrowChannels;
+  pl.narrow = pl.persist && ((N == 16 && nseq * dim < kNarrowChannels16) ||
+                             (N == 128 && nseq * dim < kNarrowChannels128));
   if (!shape_for(N, pl.narrow, pl.si)) return false;
   pl.ntiles = (dim + pl.si.ct() - 1) / pl.si.ct();
   pl.nchains = nseq * pl.ntiles;
@@ -138,7 +141,8 @@ ssm_status_t dispatch_n(const ScanArgs &a, const Plan &pl, int N, bool has_z, bo
                               : dispatch_zvp<T, TO, 16, false>(a, pl, has_z, vec, ws, st);
     case 32: return dispatch_zvp<T, TO, 32, false>(a, pl, has_z, vec, ws, st);
     case 64: return dispatch_zvp<T, TO, 64, false>(a, pl, has_z, vec, ws, st);
-    case 128: return dispatch_zvp<T, TO, 128, false>(a, pl, has_z, vec, ws, st);
+    case 128: return pl.narrow ? dispatch_zvp<T, TO, 128, true>(a, pl, has_z, vec, ws, st)
+                               : dispatch_zvp<T, TO, 128, false>(a, pl, has_z, vec, ws, st);
     default: return SSM_ERR_UNSUPPORTED;
   }
 }
@@ -294,21 +298,21 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
   if (a.x_stride < p->dim || a.bc_stride < N) return SSM_ERR_INVALID_ARG;
   a.dstate = int(N);
   a.qlog2 = qlog2;
-  const int64_t threads = R * p->dim * (N / 4);
-  const int64_t blocks = (threads + 255) / 256;
-  if (blocks > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+  const int64_t per_req = p->dim * (N / 4);  // threads per request
+  if (per_req > 0x7fffff00LL) return SSM_ERR_UNSUPPORTED;
+  const dim3 blocks(unsigned((per_req + 255) / 256), unsigned(R < 65535 ? R : 65535));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool has_z = p->z != nullptr;
   using bf16 = __nv_bfloat16;
   if (p->dtype == SSM_BF16 && !p->y_fp32) {
-    if (has_z) ssm::state_update_kernel<bf16, bf16, true><<<unsigned(blocks), 256, 0, st>>>(a);
-    else ssm::state_update_kernel<bf16, bf16, false><<<unsigned(blocks), 256, 0, st>>>(a);
+    if (has_z) ssm::state_update_kernel<bf16, bf16, true><<<blocks, 256, 0, st>>>(a);
+    else ssm::state_update_kernel<bf16, bf16, false><<<blocks, 256, 0, st>>>(a);
   } else if (p->dtype == SSM_BF16) {
-    if (has_z) ssm::state_update_kernel<bf16, float, true><<<unsigned(blocks), 256, 0, st>>>(a);
-    else ssm::state_update_kernel<bf16, float, false><<<unsigned(blocks), 256, 0, st>>>(a);
+    if (has_z) ssm::state_update_kernel<bf16, float, true><<<blocks, 256, 0, st>>>(a);
+    else ssm::state_update_kernel<bf16, float, false><<<blocks, 256, 0, st>>>(a);
   } else {
-    if (has_z) ssm::state_update_kernel<float, float, true><<<unsigned(blocks), 256, 0, st>>>(a);
-    else ssm::state_update_kernel<float, float, false><<<unsigned(blocks), 256, 0, st>>>(a);
+    if (has_z) ssm::state_update_kernel<float, float, true><<<blocks, 256, 0, st>>>(a);
+    else ssm::state_update_kernel<float, float, false><<<blocks, 256, 0, st>>>(a);
   }
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }

@@ -25,55 +25,54 @@ struct UpdateArgs {
   int qlog2;  // log2(dstate / 4): lanes per channel = 1 << qlog2
 };
 
+// Grid: x covers the dim * dstate/4 items of one request (256 per block), y strides over the
+// requests, so the (request, channel, quad) split needs no 64-bit division.
 template <typename T, typename TO, bool HAS_Z>
 __global__ void __launch_bounds__(256) state_update_kernel(const UpdateArgs args) {
   constexpr bool kFast = Elem<T>::kFast;
   const int Q = 1 << args.qlog2;
-  const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = args.R * args.dim * Q;
-  const bool valid = gid < total;
-  const int q = int(gid & (Q - 1));
-  const int64_t rd = gid >> args.qlog2;
-  const int64_t r = valid ? rd / args.dim : 0;
-  const int64_t d = valid ? rd % args.dim : 0;
   const int N = args.dstate;
-
-  int64_t slot = valid ? args.slot_ids[r] : 0;
-  const bool bad = valid && (slot < 0 || slot >= args.num_slots);
-  if (bad && d == 0 && q == 0) report_status(4 /* SSM_ERR_BAD_SLOT */);
-  const bool active = valid && !bad;
-
-  float part = 0.f, uval = 0.f;
-  if (active) {
-    const T *xu = static_cast<const T *>(args.u) + r * args.x_stride + d;
-    const T *xd = static_cast<const T *>(args.delta) + r * args.x_stride + d;
-    uval = Elem<T>::to_f32(*xu);
-    const float dt = softplus_t<kFast>(Elem<T>::to_f32(*xd) + (args.bias ? args.bias[d] : 0.f));
-    const float dtu = dt * uval;
-    float4 *hp = reinterpret_cast<float4 *>(args.pool + (slot * args.dim + d) * N + 4 * q);
-    const float4 a4 = *reinterpret_cast<const float4 *>(args.A + d * N + 4 * q);
-    const T *Bv = static_cast<const T *>(args.B) + r * args.bc_stride + 4 * q;
-    const T *Cv = static_cast<const T *>(args.C) + r * args.bc_stride + 4 * q;
-    float4 h = *hp;
-    float hv[4] = {h.x, h.y, h.z, h.w};
-    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+  const int item = blockIdx.x * 256 + threadIdx.x;  // < dim * Q, checked on the host
+  const bool valid = item < int(args.dim) * Q;
+  const int d = item >> args.qlog2, q = item & (Q - 1);
+  for (int64_t r = blockIdx.y; r < args.R; r += gridDim.y) {
+    const int64_t slot = args.slot_ids[r];
+    if (slot < 0 || slot >= args.num_slots) {  // uniform over the block: the row is skipped
+      if (blockIdx.x == 0 && threadIdx.x == 0) report_status(4 /* SSM_ERR_BAD_SLOT */);
+      continue;
+    }
+    float part = 0.f, uval = 0.f;
+    if (valid) {
+      const T *xu = static_cast<const T *>(args.u) + r * args.x_stride + d;
+      const T *xd = static_cast<const T *>(args.delta) + r * args.x_stride + d;
+      uval = Elem<T>::to_f32(*xu);
+      const float dt = softplus_t<kFast>(Elem<T>::to_f32(*xd) + (args.bias ? args.bias[d] : 0.f));
+      const float dtu = dt * uval;
+      float4 *hp = reinterpret_cast<float4 *>(args.pool + (slot * args.dim + d) * N + 4 * q);
+      const float4 a4 = *reinterpret_cast<const float4 *>(args.A + int64_t(d) * N + 4 * q);
+      const T *Bv = static_cast<const T *>(args.B) + r * args.bc_stride + 4 * q;
+      const T *Cv = static_cast<const T *>(args.C) + r * args.bc_stride + 4 * q;
+      const float4 h = *hp;
+      float hv[4] = {h.x, h.y, h.z, h.w};
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float abar = ex2_approx(dt * av[k] * kLog2e);
-      hv[k] = fmaf(abar, hv[k], dtu * Elem<T>::to_f32(Bv[k]));
-      part = fmaf(Elem<T>::to_f32(Cv[k]), hv[k], part);
+      for (int k = 0; k < 4; ++k) {
+        const float abar = ex2_approx(dt * av[k] * kLog2e);
+        hv[k] = fmaf(abar, hv[k], dtu * Elem<T>::to_f32(Bv[k]));
+        part = fmaf(Elem<T>::to_f32(Cv[k]), hv[k], part);
+      }
+      *hp = make_float4(hv[0], hv[1], hv[2], hv[3]);
     }
-    *hp = make_float4(hv[0], hv[1], hv[2], hv[3]);
-  }
-  // reduce over the Q lanes of this channel (aligned groups inside one warp)
-  for (int off = 1; off < Q; off *= 2) part += __shfl_xor_sync(0xffffffffu, part, off);
-  if (active && q == 0) {
-    float v = fmaf(args.Dskip ? args.Dskip[d] : 0.f, uval, part);
-    if constexpr (HAS_Z) {
-      const T *xz = static_cast<const T *>(args.z) + r * args.x_stride + d;
-      v *= silu_t<kFast>(Elem<T>::to_f32(*xz));
+    // reduce over the Q lanes of this channel (aligned groups inside one warp)
+    for (int off = 1; off < Q; off *= 2) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (valid && q == 0) {
+      float v = fmaf(args.Dskip ? args.Dskip[d] : 0.f, uval, part);
+      if constexpr (HAS_Z) {
+        const T *xz = static_cast<const T *>(args.z) + r * args.x_stride + d;
+        v *= silu_t<kFast>(Elem<T>::to_f32(*xz));
+      }
+      static_cast<TO *>(args.y)[r * args.x_stride + d] = Elem<TO>::from_f32(v);
     }
-    static_cast<TO *>(args.y)[r * args.x_stride + d] = Elem<TO>::from_f32(v);
   }
 }
 
