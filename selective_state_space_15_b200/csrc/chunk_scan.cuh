@@ -89,7 +89,10 @@ struct ChunkCfg {
   // shared memory layout (bytes), staging double-buffered
   static constexpr size_t kXBytes = size_t(3) * kCT * kXPitch * sizeof(T);  // u, delta, z
   static constexpr size_t kBCBytes = size_t(2) * N * kTC * sizeof(T);       // B, C
-  static constexpr size_t kYBytes = NG > 1 ? size_t(NG) * kCT * kTC * sizeof(float) : 0;  // partial y
+  // partial y of the state groups, [NG][CT] rows of kYPitch words: 4 words of padding after
+  // every 32 steps and 2 after the row put the lanes of a half-warp in distinct banks
+  static constexpr int kYPitch = kTC + kTC / 32 * 4 + 2;
+  static constexpr size_t kYBytes = NG > 1 ? size_t(NG) * kCT * kYPitch * sizeof(float) : 0;
   static constexpr int kNP = N + 1;         // row pitch of the per-(channel, state) arrays
   static constexpr size_t kParamBytes =
       size_t(2) * kCT * kNP * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
@@ -116,7 +119,7 @@ chunk_scan_kernel(const ScanArgs args) {
   extern __shared__ __align__(16) unsigned char smem[];
   T *const xs0 = reinterpret_cast<T *>(smem);                     // [2][3][CT][XP]
   T *const bc0 = reinterpret_cast<T *>(smem + 2 * Cfg::kXBytes);  // [2][2][N][TC]
-  float *ypart = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes);  // [NG][CT][TC]
+  float *ypart = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes);  // [NG][CT][YP]
   // [CT][N] arrays use a row pitch of N + 1 words, so the channels of a warp hit distinct banks
   constexpr int NP = Cfg::kNP;
   float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes);  // [CT][NP]
@@ -433,7 +436,10 @@ chunk_scan_kernel(const ScanArgs args) {
 #pragma unroll
         for (int i = 0; i < KI; ++i) yo[i] = (i & 1) ? y[i / 2].y : y[i / 2].x;
       } else {
-        float2 *mine = reinterpret_cast<float2 *>(ypart + (size_t(g) * CT + ch) * TC + tl0);
+        constexpr int YP = Cfg::kYPitch;
+        static_assert(32 % KI == 0 && TC % 32 == 0, "a lane's steps lie in one padded block");
+        const int yo0 = tl0 + (tl0 >> 5) * 4;  // padded position of the lane's first step
+        float2 *mine = reinterpret_cast<float2 *>(ypart + (size_t(g) * CT + ch) * YP + yo0);
 #pragma unroll
         for (int p = 0; p < KP; ++p) mine[p] = y[p];
         __syncthreads();  // every state group's partial sums visible
@@ -441,7 +447,7 @@ chunk_scan_kernel(const ScanArgs args) {
         for (int i = 0; i < KE; ++i) yo[i] = 0.f;
 #pragma unroll
         for (int gg = 0; gg < NG; ++gg) {
-          const float *src = ypart + (size_t(gg) * CT + ch) * TC + tl0 + e0;
+          const float *src = ypart + (size_t(gg) * CT + ch) * YP + yo0 + e0;
           if constexpr (KE % 2 == 0) {
 #pragma unroll
             for (int p = 0; p < KE / 2; ++p) {
