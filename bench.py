@@ -221,30 +221,33 @@ def time_kernel(fn, steps, warmup, stream, flush=None):
     return total / steps
 
 
-def secondary(steps, warmup, hbm_peak, sfu_peak):
-    """Kernel-only figures for the long-sequence and decode workloads (single GPU)."""
+def long_run(name, steps, warmup, hbm_peak, sfu_peak, seqlen=None):
+    """Kernel-only figures for one long single-sequence workload (inputs drawn on the device;
+    `seqlen` shortens the sequence for profiler captures)."""
     import torch
     import selective_state_space_15_b200 as ssm
-    out = {}
     stream = torch.cuda.current_stream()
     g = torch.Generator(device="cuda")
-    for name in ("long_bf16", "long_n128_bf16"):
-        c = workloads.CONFIGS[name]
-        D, N, L = c["dim"], c["dstate"], c["seqlen"]
-        g.manual_seed(c["seed"])
-        mk = lambda *s: torch.randn(*s, generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)  # noqa: E731
-        u, dl, z, B, C = mk(1, D, L), mk(1, D, L), mk(1, D, L), mk(1, N, L), mk(1, N, L)
-        A, Dsk, bias = (torch.from_numpy(x).cuda() for x in workloads.channel_params(np.random.default_rng(c["seed"]), D, N))
-        y = torch.empty_like(u)
-        hl = torch.empty(1, D, N, device="cuda")
-        ms = time_kernel(lambda: ssm.scan_fwd(u, dl, B, C, A, Dsk, bias, z, y=y, h_last=hl), max(3, steps // 4),
-                         warmup, stream)
-        nb, ne = scan_counts(L, D, N, 2, 2, 1)
-        out[name] = {"ms": round(ms, 4), "tokens_per_s": L / (ms * 1e-3),
-                     "sfu_frac": round(ne / (ms * 1e-3) / sfu_peak, 4),
-                     "hbm_gbs": round(nb / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm_peak, 4)}
-        del u, dl, z, B, C, y
-    # decode: 256 of 1024 slots, D=5120, N=16; the state (84 MB) fits in L2, so L2 is flushed
+    c = workloads.CONFIGS[name]
+    D, N, L = c["dim"], c["dstate"], seqlen or c["seqlen"]
+    g.manual_seed(c["seed"])
+    mk = lambda *s: torch.randn(*s, generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)  # noqa: E731
+    u, dl, z, B, C = mk(1, D, L), mk(1, D, L), mk(1, D, L), mk(1, N, L), mk(1, N, L)
+    A, Dsk, bias = (torch.from_numpy(x).cuda() for x in workloads.channel_params(np.random.default_rng(c["seed"]), D, N))
+    y = torch.empty_like(u)
+    hl = torch.empty(1, D, N, device="cuda")
+    ms = time_kernel(lambda: ssm.scan_fwd(u, dl, B, C, A, Dsk, bias, z, y=y, h_last=hl), steps, warmup, stream)
+    nb, ne = scan_counts(L, D, N, 2, 2, 1)
+    return {"ms": round(ms, 4), "tokens_per_s": L / (ms * 1e-3),
+            "sfu_frac": round(ne / (ms * 1e-3) / sfu_peak, 4),
+            "hbm_gbs": round(nb / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm_peak, 4)}
+
+
+def decode_run(steps, warmup, hbm_peak):
+    """Kernel-only figures for the decode workload: 256 of 1024 slots, D=5120, N=16."""
+    import torch
+    import selective_state_space_15_b200 as ssm
+    stream = torch.cuda.current_stream()
     c = workloads.CONFIGS["decode_bf16"]
     prob = workloads.decode_problem(c["num_slots"], c["dim"], c["dstate"], c["R"], c["dtype"], c["seed"])
     pool = torch.from_numpy(prob.pool0).cuda()
@@ -254,16 +257,35 @@ def secondary(steps, warmup, hbm_peak, sfu_peak):
     bf = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)  # noqa: E731
     u, dl, z, B, C = bf(x["u"]), bf(x["delta"]), bf(x["z"]), bf(x["B"]), bf(x["C"])
     y = torch.empty_like(u)
-    # read (not write) a 256 MB buffer between steps: L2 ends up holding clean lines, so no
-    # write-back of the flush lands inside the timed step
+    # the state (84 MB) fits in L2: read (not write) a 256 MB buffer between steps, so L2
+    # ends up holding clean lines and no write-back of the flush lands inside the timed step.
+    # The step is replayed from a CUDA graph: its kernel is shorter than a Python launch, and
+    # the replay is queued while the flush runs, so the events bracket the kernel alone.
     scratch = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
-    ms = time_kernel(lambda: ssm.state_update(pool, slots, u, dl, B, C, A, Dsk, bias, z, y=y), steps, warmup, stream,
-                     flush=lambda: scratch.sum())
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            ssm.state_update(pool, slots, u, dl, B, C, A, Dsk, bias, z, y=y)
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        ssm.state_update(pool, slots, u, dl, B, C, A, Dsk, bias, z, y=y)
+    ms = time_kernel(graph.replay, steps, warmup, stream, flush=lambda: scratch.sum())
+    del graph
     R, D, N = c["R"], c["dim"], c["dstate"]
     nb = R * D * N * 4 * 2 + R * D * 2 * 4 + R * N * 2 * 2 + D * (N + 2) * 4
-    out["decode_bf16"] = {"ms_per_step": round(ms, 5), "tokens_per_s": R / (ms * 1e-3),
-                          "hbm_gbs": round(nb / (ms * 1e-3) / 1e9, 1),
-                          "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm_peak, 4), "l2": "flushed (256 MB read) before each step"}
+    return {"ms_per_step": round(ms, 5), "tokens_per_s": R / (ms * 1e-3),
+            "hbm_gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+            "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm_peak, 4),
+            "l2": "flushed (256 MB read) before each step", "launch": "CUDA graph replay"}
+
+
+def secondary(steps, warmup, hbm_peak, sfu_peak):
+    """Kernel-only figures for the long-sequence and decode workloads (single GPU)."""
+    out = {name: long_run(name, max(3, steps // 4), warmup, hbm_peak, sfu_peak)
+           for name in ("long_bf16", "long_n128_bf16")}
+    out["decode_bf16"] = decode_run(steps, warmup, hbm_peak)
     return out
 
 
@@ -438,6 +460,25 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_other(args, rank, world, local_rank):
+    """--kernel-only --workload X: the kernel of a secondary workload alone, on one GPU."""
+    import torch
+    import selective_state_space_15_b200 as ssm
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local_rank)
+    ssm.load()
+    hbm_peak, sm_max, _ = peaks()
+    sfu_peak = N_SM * SFU_PER_CLK_PER_SM * sm_max * 1e6
+    if args.workload == "decode_bf16":
+        r = decode_run(args.steps, args.warmup, hbm_peak)
+    else:
+        r = long_run(args.workload, args.steps, args.warmup, hbm_peak, sfu_peak, args.seqlen)
+    print(json.dumps({"workload": args.workload, "seqlen": args.seqlen, "steps": args.steps, "warmup": args.warmup, **r,
+                      "mode": "kernel-only (ncu capture)"}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -445,16 +486,24 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-secondary", action="store_true", help="skip the long-sequence/decode figures")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "long_bf16", "long_n128_bf16", "decode_bf16"],
+                    help="with --kernel-only: time another workload's kernel alone (for ncu captures)")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="with --kernel-only and a long workload: a shorter sequence (profiler captures)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="only the warm-up and timed kernel steps (for ncu captures); prints a short line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.workload != WORKLOAD and not args.kernel_only:
+        ap.error("--workload other than the metric's needs --kernel-only")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload != WORKLOAD:
+        return run_other(args, rank, world, local_rank)
     return run_ours(args, rank, world, local_rank)
 
 

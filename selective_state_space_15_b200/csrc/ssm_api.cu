@@ -282,10 +282,7 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
   if (p->batch != R || p->seqlen != 1 || p->dim <= 0 || p->dstate <= 0) return SSM_ERR_INVALID_ARG;
   if (!p->u || !p->delta || !p->B || !p->C || !p->A || !p->y) return SSM_ERR_INVALID_ARG;
   const int64_t N = p->dstate;
-  if (N % 4 != 0 || N > 128) return SSM_ERR_UNSUPPORTED;
-  int qlog2 = 0;
-  while ((int64_t(4) << qlog2) < N) ++qlog2;
-  if ((int64_t(4) << qlog2) != N) return SSM_ERR_UNSUPPORTED;  // dstate/4 must be a power of two
+  if (N % 4 != 0 || N > ssm::kUpdateMaxState) return SSM_ERR_UNSUPPORTED;
   if (!aligned16(pool) || !aligned16(p->A)) return SSM_ERR_INVALID_ARG;
   if (R == 0) return SSM_OK;
   ssm::UpdateArgs a{};
@@ -297,23 +294,46 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
   a.bc_stride = p->bc_batch_stride ? p->bc_batch_stride : N;
   if (a.x_stride < p->dim || a.bc_stride < N) return SSM_ERR_INVALID_ARG;
   a.dstate = int(N);
-  a.qlog2 = qlog2;
-  const int64_t per_req = p->dim * (N / 4);  // threads per request
-  if (per_req > 0x7fffff00LL) return SSM_ERR_UNSUPPORTED;
-  const dim3 blocks(unsigned((per_req + 255) / 256), unsigned(R < 65535 ? R : 65535));
+  // states per thread: 16 when they divide dstate, else 8, else 4
+  const int G = N % 16 == 0 ? 16 : (N % 8 == 0 ? 8 : 4);
+  a.tpc = int(N / G);
+  const int64_t cpb = ssm::kUpdateThreads / a.tpc;  // channels per block
+  const int64_t gx = (p->dim + cpb - 1) / cpb;
+  if (gx > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+  const dim3 blocks(unsigned(gx), unsigned(R < 65535 ? R : 65535));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool has_z = p->z != nullptr;
   using bf16 = __nv_bfloat16;
-  if (p->dtype == SSM_BF16 && !p->y_fp32) {
-    if (has_z) ssm::state_update_kernel<bf16, bf16, true><<<blocks, 256, 0, st>>>(a);
-    else ssm::state_update_kernel<bf16, bf16, false><<<blocks, 256, 0, st>>>(a);
+#define SSM_UPDATE_LAUNCH(T, TO)                                                                          \
+  do {                                                                                                     \
+    if (G == 16) {                                                                                         \
+      if (has_z) ssm::state_update_kernel<T, TO, true, 16><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);      \
+      else ssm::state_update_kernel<T, TO, false, 16><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);           \
+    } else if (G == 8) {                                                                                   \
+      if (has_z) ssm::state_update_kernel<T, TO, true, 8><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);       \
+      else ssm::state_update_kernel<T, TO, false, 8><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);            \
+    } else {                                                                                               \
+      if (has_z) ssm::state_update_kernel<T, TO, true, 4><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);       \
+      else ssm::state_update_kernel<T, TO, false, 4><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);            \
+    }                                                                                                      \
+  } while (0)
+  if (N == 16) {  // one warp per 32 channels, coalesced quads
+    const dim3 b16(unsigned((p->dim + ssm::kUpdateThreads - 1) / ssm::kUpdateThreads), blocks.y);
+#define SSM_UPDATE16(T, TO)                                                                         \
+  (has_z ? ssm::state_update16_kernel<T, TO, true><<<b16, ssm::kUpdateThreads, 0, st>>>(a)          \
+         : ssm::state_update16_kernel<T, TO, false><<<b16, ssm::kUpdateThreads, 0, st>>>(a))
+    if (p->dtype == SSM_BF16 && !p->y_fp32) SSM_UPDATE16(bf16, bf16);
+    else if (p->dtype == SSM_BF16) SSM_UPDATE16(bf16, float);
+    else SSM_UPDATE16(float, float);
+#undef SSM_UPDATE16
+  } else if (p->dtype == SSM_BF16 && !p->y_fp32) {
+    SSM_UPDATE_LAUNCH(bf16, bf16);
   } else if (p->dtype == SSM_BF16) {
-    if (has_z) ssm::state_update_kernel<bf16, float, true><<<blocks, 256, 0, st>>>(a);
-    else ssm::state_update_kernel<bf16, float, false><<<blocks, 256, 0, st>>>(a);
+    SSM_UPDATE_LAUNCH(bf16, float);
   } else {
-    if (has_z) ssm::state_update_kernel<float, float, true><<<blocks, 256, 0, st>>>(a);
-    else ssm::state_update_kernel<float, float, false><<<blocks, 256, 0, st>>>(a);
+    SSM_UPDATE_LAUNCH(float, float);
   }
+#undef SSM_UPDATE_LAUNCH
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

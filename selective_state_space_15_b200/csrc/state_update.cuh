@@ -3,10 +3,14 @@
 // "ufo.work" page §4.1 and its second article §4.1: a persistent pool of per-request states
 // and a light kernel doing h_new = exp(Delta A) h_old + Delta B x for one token.  The
 // kernel is bound by HBM traffic on the pool (read + write of R x dim x dstate float32),
-// so the mapping is chosen for coalescing: a thread owns 4 consecutive states (one 16-byte
-// load and store) of one (request, channel); the dstate/4 threads of a channel are
-// adjacent lanes and reduce C.h with shuffles; consecutive channels of a request are
-// consecutive groups, so a warp streams one contiguous run of the pool row.
+// so the per-channel work is done once: a thread owns G consecutive states of one
+// (request, channel) -- a whole channel when dstate <= 16 -- loads them with 16-byte vectors
+// and keeps them in registers; Delta = softplus(delta + bias), the gate and the D term are
+// evaluated once per channel.  B and C of the request are staged in shared memory once per
+// block (every channel of the request reads the same values).  Consecutive threads take
+// consecutive channels, so a warp streams one contiguous run of the pool row.  When a
+// channel is split over several threads (dstate > 16) their partial C.h go through shared
+// memory.
 #pragma once
 
 #include "common.cuh"
@@ -22,56 +26,168 @@ struct UpdateArgs {
   int64_t num_slots, R, dim;
   int64_t x_stride, bc_stride;  // row strides of [R][dim] and [R][dstate] inputs
   int dstate;
-  int qlog2;  // log2(dstate / 4): lanes per channel = 1 << qlog2
+  int tpc;  // threads per channel = dstate / G
 };
 
-// Grid: x covers the dim * dstate/4 items of one request (256 per block), y strides over the
-// requests, so the (request, channel, quad) split needs no 64-bit division.
-template <typename T, typename TO, bool HAS_Z>
-__global__ void __launch_bounds__(256) state_update_kernel(const UpdateArgs args) {
+constexpr int kUpdateThreads = 256;
+constexpr int kUpdateMaxState = 128;
+
+// Grid: x over the channels of one request (kUpdateThreads / tpc per block), y strides over
+// the requests.  G states per thread (4, 8 or 16; G divides dstate).
+template <typename T, typename TO, bool HAS_Z, int G>
+__global__ void __launch_bounds__(kUpdateThreads) state_update_kernel(const UpdateArgs args) {
   constexpr bool kFast = Elem<T>::kFast;
-  const int Q = 1 << args.qlog2;
-  const int N = args.dstate;
-  const int item = blockIdx.x * 256 + threadIdx.x;  // < dim * Q, checked on the host
-  const bool valid = item < int(args.dim) * Q;
-  const int d = item >> args.qlog2, q = item & (Q - 1);
+  static_assert(G % 4 == 0 && G <= 16, "state group");
+  __shared__ __align__(16) float Bs[kUpdateMaxState], Cs[kUpdateMaxState];
+  __shared__ float red[kUpdateThreads];
+  const int N = args.dstate, tpc = args.tpc;
+  const int cpb = kUpdateThreads / tpc;  // channels per block
+  const int cl = threadIdx.x / tpc, part = threadIdx.x % tpc;
+  const int64_t d = int64_t(blockIdx.x) * cpb + cl;
+  const bool valid = cl < cpb && d < args.dim;
+  const int s0 = part * G;  // first state of this thread
   for (int64_t r = blockIdx.y; r < args.R; r += gridDim.y) {
     const int64_t slot = args.slot_ids[r];
     if (slot < 0 || slot >= args.num_slots) {  // uniform over the block: the row is skipped
       if (blockIdx.x == 0 && threadIdx.x == 0) report_status(4 /* SSM_ERR_BAD_SLOT */);
       continue;
     }
-    float part = 0.f, uval = 0.f;
-    if (valid) {
-      const T *xu = static_cast<const T *>(args.u) + r * args.x_stride + d;
-      const T *xd = static_cast<const T *>(args.delta) + r * args.x_stride + d;
-      uval = Elem<T>::to_f32(*xu);
-      const float dt = softplus_t<kFast>(Elem<T>::to_f32(*xd) + (args.bias ? args.bias[d] : 0.f));
-      const float dtu = dt * uval;
-      float4 *hp = reinterpret_cast<float4 *>(args.pool + (slot * args.dim + d) * N + 4 * q);
-      const float4 a4 = *reinterpret_cast<const float4 *>(args.A + int64_t(d) * N + 4 * q);
-      const T *Bv = static_cast<const T *>(args.B) + r * args.bc_stride + 4 * q;
-      const T *Cv = static_cast<const T *>(args.C) + r * args.bc_stride + 4 * q;
-      const float4 h = *hp;
-      float hv[4] = {h.x, h.y, h.z, h.w};
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float abar = ex2_approx(dt * av[k] * kLog2e);
-        hv[k] = fmaf(abar, hv[k], dtu * Elem<T>::to_f32(Bv[k]));
-        part = fmaf(Elem<T>::to_f32(Cv[k]), hv[k], part);
-      }
-      *hp = make_float4(hv[0], hv[1], hv[2], hv[3]);
+    __syncthreads();  // the previous request's B, C and partial sums are consumed
+    for (int i = threadIdx.x; i < N; i += kUpdateThreads) {
+      Bs[i] = Elem<T>::to_f32(static_cast<const T *>(args.B)[r * args.bc_stride + i]);
+      Cs[i] = Elem<T>::to_f32(static_cast<const T *>(args.C)[r * args.bc_stride + i]);
     }
-    // reduce over the Q lanes of this channel (aligned groups inside one warp)
-    for (int off = 1; off < Q; off *= 2) part += __shfl_xor_sync(0xffffffffu, part, off);
-    if (valid && q == 0) {
-      float v = fmaf(args.Dskip ? args.Dskip[d] : 0.f, uval, part);
-      if constexpr (HAS_Z) {
-        const T *xz = static_cast<const T *>(args.z) + r * args.x_stride + d;
-        v *= silu_t<kFast>(Elem<T>::to_f32(*xz));
+    __syncthreads();
+    float acc = 0.f, uval = 0.f;
+    if (valid) {
+      const int64_t xo = r * args.x_stride + d;
+      uval = Elem<T>::to_f32(static_cast<const T *>(args.u)[xo]);
+      const float dt = softplus_t<kFast>(Elem<T>::to_f32(static_cast<const T *>(args.delta)[xo]) +
+                                         (args.bias ? args.bias[d] : 0.f));
+      const float2 dtl = make_float2(dt * kLog2e, dt * kLog2e);
+      const float2 dtu = make_float2(dt * uval, dt * uval);
+      float4 *hp = reinterpret_cast<float4 *>(args.pool + (slot * args.dim + d) * N + s0);
+      const float4 *ap = reinterpret_cast<const float4 *>(args.A + d * N + s0);
+      float4 h[G / 4], av[G / 4];
+#pragma unroll
+      for (int k = 0; k < G / 4; ++k) {
+        h[k] = hp[k];
+        av[k] = ap[k];
       }
+      float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < G / 4; ++k) {
+        const float4 b4 = *reinterpret_cast<const float4 *>(Bs + s0 + 4 * k);
+        const float4 c4 = *reinterpret_cast<const float4 *>(Cs + s0 + 4 * k);
+        const float2 x01 = __fmul2_rn(dtl, make_float2(av[k].x, av[k].y));
+        const float2 x23 = __fmul2_rn(dtl, make_float2(av[k].z, av[k].w));
+        const float2 a01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+        const float2 a23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+        const float2 h01 = __ffma2_rn(a01, make_float2(h[k].x, h[k].y), __fmul2_rn(dtu, make_float2(b4.x, b4.y)));
+        const float2 h23 = __ffma2_rn(a23, make_float2(h[k].z, h[k].w), __fmul2_rn(dtu, make_float2(b4.z, b4.w)));
+        acc2 = __ffma2_rn(make_float2(c4.x, c4.y), h01, acc2);
+        acc2 = __ffma2_rn(make_float2(c4.z, c4.w), h23, acc2);
+        h[k] = make_float4(h01.x, h01.y, h23.x, h23.y);
+      }
+#pragma unroll
+      for (int k = 0; k < G / 4; ++k) hp[k] = h[k];
+      acc = acc2.x + acc2.y;
+    }
+    if (tpc > 1) {  // the channel's partial sums, in thread order
+      red[threadIdx.x] = acc;
+      __syncthreads();
+      if (valid && part == 0)
+        for (int p = 1; p < tpc; ++p) acc += red[threadIdx.x + p];
+    }
+    if (valid && part == 0) {
+      float v = fmaf(args.Dskip ? args.Dskip[d] : 0.f, uval, acc);
+      if constexpr (HAS_Z) v *= silu_t<kFast>(Elem<T>::to_f32(static_cast<const T *>(args.z)[r * args.x_stride + d]));
       static_cast<TO *>(args.y)[r * args.x_stride + d] = Elem<TO>::from_f32(v);
+    }
+  }
+}
+
+// dstate = 16: one warp updates 32 channels of a request with fully coalesced 16-byte
+// accesses.  Lane l = 4j + m holds state quad m of channels 8k + j (k = 0..3): the k-th load of
+// the warp covers 512 contiguous bytes of the pool row (and of A).  Each lane evaluates the
+// per-channel terms (softplus, Delta*u, gate) for one channel, 8m + j, and hands Delta to the
+// other three lanes of the channel with shuffles; C.h is reduced over the 4 lanes of a
+// channel, and lane l writes y for its own channel.
+template <typename T, typename TO, bool HAS_Z>
+__global__ void __launch_bounds__(kUpdateThreads) state_update16_kernel(const UpdateArgs args) {
+  constexpr bool kFast = Elem<T>::kFast;
+  constexpr int N = 16;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  const int j = lane >> 2, m = lane & 3;
+  const int64_t cb = int64_t(blockIdx.x) * kUpdateThreads + warp * 32;  // first channel of the warp
+  const int64_t c_own = cb + 8 * m + j;
+  const bool own_ok = c_own < args.dim;
+  for (int64_t r = blockIdx.y; r < args.R; r += gridDim.y) {
+    const int64_t slot = args.slot_ids[r];
+    if (slot < 0 || slot >= args.num_slots) {  // uniform over the block: the row is skipped
+      if (blockIdx.x == 0 && threadIdx.x == 0) report_status(4 /* SSM_ERR_BAD_SLOT */);
+      continue;
+    }
+    float *prow = args.pool + slot * args.dim * N;
+    // state quads: k-th vector = channel cb + 8k + j, states 4m..4m+3
+    float4 h[4], av[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t c = cb + 8 * k + j;
+      if (c < args.dim) {
+        h[k] = *reinterpret_cast<const float4 *>(prow + c * N + 4 * m);
+        av[k] = *reinterpret_cast<const float4 *>(args.A + c * N + 4 * m);
+      } else {
+        h[k] = av[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    const T *Br = static_cast<const T *>(args.B) + r * args.bc_stride + 4 * m;
+    const T *Cr = static_cast<const T *>(args.C) + r * args.bc_stride + 4 * m;
+    const float4 b4 = make_float4(Elem<T>::to_f32(Br[0]), Elem<T>::to_f32(Br[1]), Elem<T>::to_f32(Br[2]),
+                                  Elem<T>::to_f32(Br[3]));
+    const float4 c4 = make_float4(Elem<T>::to_f32(Cr[0]), Elem<T>::to_f32(Cr[1]), Elem<T>::to_f32(Cr[2]),
+                                  Elem<T>::to_f32(Cr[3]));
+    // this lane's own channel: Delta, Delta*u, u, gate
+    float dtl = 0.f, dtu = 0.f, uval = 0.f, zval = 0.f;
+    if (own_ok) {
+      const int64_t xo = r * args.x_stride + c_own;
+      uval = Elem<T>::to_f32(static_cast<const T *>(args.u)[xo]);
+      const float dt = softplus_t<kFast>(Elem<T>::to_f32(static_cast<const T *>(args.delta)[xo]) +
+                                         (args.bias ? args.bias[c_own] : 0.f));
+      dtl = dt * kLog2e;
+      dtu = dt * uval;
+      if constexpr (HAS_Z) zval = Elem<T>::to_f32(static_cast<const T *>(args.z)[xo]);
+    }
+    float own_sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      // channel cb + 8k + j belongs to lane 4j + k
+      const float l2 = __shfl_sync(0xffffffffu, dtl, 4 * j + k);
+      const float du = __shfl_sync(0xffffffffu, dtu, 4 * j + k);
+      const float2 L2 = make_float2(l2, l2), DU = make_float2(du, du);
+      const float2 x01 = __fmul2_rn(L2, make_float2(av[k].x, av[k].y));
+      const float2 x23 = __fmul2_rn(L2, make_float2(av[k].z, av[k].w));
+      const float2 a01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+      const float2 a23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+      const float2 h01 = __ffma2_rn(a01, make_float2(h[k].x, h[k].y), __fmul2_rn(DU, make_float2(b4.x, b4.y)));
+      const float2 h23 = __ffma2_rn(a23, make_float2(h[k].z, h[k].w), __fmul2_rn(DU, make_float2(b4.z, b4.w)));
+      h[k] = make_float4(h01.x, h01.y, h23.x, h23.y);
+      float2 p2 = __fmul2_rn(make_float2(c4.x, c4.y), h01);
+      p2 = __ffma2_rn(make_float2(c4.z, c4.w), h23, p2);
+      float part = p2.x + p2.y;
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      if (k == m) own_sum = part;  // channel cb + 8m + j is this lane's own
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t c = cb + 8 * k + j;
+      if (c < args.dim) *reinterpret_cast<float4 *>(prow + c * N + 4 * m) = h[k];
+    }
+    if (own_ok) {
+      float v = fmaf(args.Dskip ? args.Dskip[c_own] : 0.f, uval, own_sum);
+      if constexpr (HAS_Z) v *= silu_t<kFast>(zval);
+      static_cast<TO *>(args.y)[r * args.x_stride + c_own] = Elem<TO>::from_f32(v);
     }
   }
 }

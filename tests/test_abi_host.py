@@ -81,8 +81,10 @@ def test_state_update_host_checks(lib):
     assert lib.ssm_state_update(fake, 4, None, 8, ctypes.byref(p), None) == 1
     assert lib.ssm_state_update(fake, 0, fake, 8, ctypes.byref(p), None) == 1
     assert lib.ssm_state_update(fake, 4, fake, 7, ctypes.byref(p), None) == 1      # batch != R
-    p2 = _params(batch=8, seqlen=1, dim=32, dstate=12)
-    assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p2), None) == 2     # 12/4 not a power of 2
+    p2 = _params(batch=8, seqlen=1, dim=32, dstate=10)
+    assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p2), None) == 2     # not a multiple of 4
+    p2 = _params(batch=8, seqlen=1, dim=32, dstate=132)
+    assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p2), None) == 2     # above 128
     p3 = _params(batch=8, seqlen=2, dim=32, dstate=16)
     assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p3), None) == 1     # one token only
     assert lib.ssm_state_update(fake + 4, 4, fake, 8, ctypes.byref(p), None) == 1  # pool not 16-byte aligned
