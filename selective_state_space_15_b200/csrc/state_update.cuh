@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kUpdateThreads) state_update_kernel(const Upda
 // other three lanes of the channel with shuffles; C.h is reduced over the 4 lanes of a
 // channel, and lane l writes y for its own channel.
 template <typename T, typename TO, bool HAS_Z>
-__global__ void __launch_bounds__(kUpdateThreads) state_update16_kernel(const UpdateArgs args) {
+__global__ void __launch_bounds__(kUpdateThreads, 4) state_update16_kernel(const UpdateArgs args) {
   constexpr bool kFast = Elem<T>::kFast;
   constexpr int N = 16;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
