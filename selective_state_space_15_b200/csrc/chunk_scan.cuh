@@ -93,10 +93,16 @@ struct ChunkCfg {
   // every 32 steps and 2 after the row put the lanes of a half-warp in distinct banks
   static constexpr int kYPitch = kTC + kTC / 32 * 4 + 2;
   static constexpr size_t kYBytes = NG > 1 ? size_t(NG) * kCT * kYPitch * sizeof(float) : 0;
+  // With many state groups, Delta and Delta*u of the chunk are computed once per (channel,
+  // step) by the whole CTA and read by every group (rows padded by 4 words: a quarter-warp's
+  // channels hit distinct banks); with few groups each lane computes its own.
+  static constexpr bool kSharedDelta = NG >= 4;
+  static constexpr int kDPitch = kTC + 4;
+  static constexpr size_t kDBytes = kSharedDelta ? size_t(2) * kCT * kDPitch * sizeof(float) : 0;
   static constexpr int kNP = N + 1;         // row pitch of the per-(channel, state) arrays
   static constexpr size_t kParamBytes =
       size_t(2) * kCT * kNP * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
-  static constexpr size_t kSmemBytes = 2 * kXBytes + 2 * kBCBytes + kYBytes + kParamBytes;
+  static constexpr size_t kSmemBytes = 2 * kXBytes + 2 * kBCBytes + kYBytes + kDBytes + kParamBytes;
   static_assert(KI % 4 == 0 && KI % kVec == 0, "a lane's steps must be whole 16-byte vectors");
   static_assert(32 % SPW == 0 && CPW * SPW == 32, "lane split");
   static_assert(N % NG == 0 && KI % NG == 0, "state / step split");
@@ -122,7 +128,10 @@ chunk_scan_kernel(const ScanArgs args) {
   float *ypart = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes);  // [NG][CT][YP]
   // [CT][N] arrays use a row pitch of N + 1 words, so the channels of a warp hit distinct banks
   constexpr int NP = Cfg::kNP;
-  float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes);  // [CT][NP]
+  float *dls = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes);  // [2][CT][DP]
+  constexpr int DP = Cfg::kDPitch;
+  float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes +
+                                         Cfg::kDBytes);  // [CT][NP]
   float *carry_s = A2s + CT * NP;                                 // [CT][NP]
   float *Dsk = carry_s + CT * NP;                                 // [CT]
   float *bias_s = Dsk + CT;                                       // [CT]
@@ -310,7 +319,7 @@ chunk_scan_kernel(const ScanArgs args) {
       float dsum = 0.f;
 #pragma unroll
       for (int p = 0; p < KP; ++p) y[p] = make_float2(0.f, 0.f);
-      {
+      if constexpr (!Cfg::kSharedDelta) {
         const T *ru = X + size_t(ch) * XP + tl0;
         const T *rd = X + size_t(CT + ch) * XP + tl0;
         const float bias = bias_s[ch];
@@ -336,6 +345,36 @@ chunk_scan_kernel(const ScanArgs args) {
             dsum += dt.x + dt.y;
           }
         }
+      } else {
+        float *dus = dls + CT * DP;
+        for (int i = threadIdx.x; i < CT * TC; i += NT) {
+          const int c2 = i / TC, t = i % TC;
+          const float uv = Elem<T>::to_f32(X[size_t(c2) * XP + t]);
+          float dt = softplus_t<kFast>(Elem<T>::to_f32(X[size_t(CT + c2) * XP + t]) + bias_s[c2]);
+          float dtu = dt * uv;
+          if constexpr (kMasked) {
+            const bool in = t >= rel_lo && t < rel_hi;
+            dt = in ? dt : 0.f;
+            dtu = in ? dtu : 0.f;  // select: a non-finite u outside the sequence stays out
+          }
+          dls[c2 * DP + t] = dt;
+          dus[c2 * DP + t] = dtu;
+        }
+        __syncthreads();
+        const float4 *rl = reinterpret_cast<const float4 *>(dls + ch * DP + tl0);
+        const float4 *rv = reinterpret_cast<const float4 *>(dus + ch * DP + tl0);
+        float2 ds = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < KI / 4; ++q) {
+          const float4 l4 = rl[q], u4 = rv[q];
+          dl[2 * q] = make_float2(l4.x, l4.y);
+          dl[2 * q + 1] = make_float2(l4.z, l4.w);
+          du[2 * q] = make_float2(u4.x, u4.y);
+          du[2 * q + 1] = make_float2(u4.z, u4.w);
+          ds = __fadd2_rn(ds, dl[2 * q]);
+          ds = __fadd2_rn(ds, dl[2 * q + 1]);
+        }
+        dsum = ds.x + ds.y;
       }
 
       // ---- state loop over this warp's NS states ----

@@ -29,7 +29,7 @@ template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW
 template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<128, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 4, NG = 1; };
-template <> struct Shape<128, true> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 1, NG = 8; };
+template <> struct Shape<128, true> { static constexpr int KI = 16, SPW = 4, CPW = 8, CW = 1, NG = 16; };
 template <int N, bool NARROW> ShapeInfo shape_of() {
   using S = Shape<N, NARROW>;
   return ShapeInfo{S::KI, S::SPW, S::CPW, S::CW, S::NG};
