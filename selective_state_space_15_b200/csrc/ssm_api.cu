@@ -29,7 +29,7 @@ template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW
 template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<128, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 4, NG = 1; };
-template <> struct Shape<128, true> { static constexpr int KI = 16, SPW = 4, CPW = 8, CW = 1, NG = 16; };
+template <> struct Shape<128, true> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 1, NG = 16; };
 template <int N, bool NARROW> ShapeInfo shape_of() {
   using S = Shape<N, NARROW>;
   return ShapeInfo{S::KI, S::SPW, S::CPW, S::CW, S::NG};
@@ -52,14 +52,15 @@ struct Plan {
   int64_t ntiles = 0, nchains = 0, nchunks = 0;
   size_t flags_off = 0, carries_off = 0, ws_bytes = 0;
 };
-// batch * dim below these: split the states over several warps (N=16: 2, N=128: 8)
+// batch * dim below these: split the states over several warps (N=16: 2, N=128: 16; the
+// N=128 narrow tile is planned for 16-bit inputs only, whose B/C chunk fits in shared memory)
 constexpr int64_t kNarrowChannels16 = 8192, kNarrowChannels128 = 32768;
 
-bool make_plan(int N, int64_t nseq, int64_t dim, int64_t seqlen, bool varlen, bool vec, Plan &pl) {
+bool make_plan(int N, int64_t nseq, int64_t dim, int64_t seqlen, bool varlen, bool vec, bool bf16, Plan &pl) {
   pl = Plan{};
   pl.persist = !varlen && vec && seqlen > 0;
   pl.narrow = pl.persist && ((N == 16 && nseq * dim < kNarrowChannels16) ||
-                             (N == 128 && nseq * dim < kNarrowChannels128));
+                             (N == 128 && bf16 && nseq * dim < kNarrowChannels128));
   if (!shape_for(N, pl.narrow, pl.si)) return false;
   pl.ntiles = (dim + pl.si.ct() - 1) / pl.si.ct();
   pl.nchains = nseq * pl.ntiles;
@@ -141,8 +142,13 @@ ssm_status_t dispatch_n(const ScanArgs &a, const Plan &pl, int N, bool has_z, bo
                               : dispatch_zvp<T, TO, 16, false>(a, pl, has_z, vec, ws, st);
     case 32: return dispatch_zvp<T, TO, 32, false>(a, pl, has_z, vec, ws, st);
     case 64: return dispatch_zvp<T, TO, 64, false>(a, pl, has_z, vec, ws, st);
-    case 128: return pl.narrow ? dispatch_zvp<T, TO, 128, true>(a, pl, has_z, vec, ws, st)
-                               : dispatch_zvp<T, TO, 128, false>(a, pl, has_z, vec, ws, st);
+    case 128:
+      if constexpr (std::is_same<T, float>::value) {
+        return dispatch_zvp<T, TO, 128, false>(a, pl, has_z, vec, ws, st);  // no narrow plan for float32
+      } else {
+        return pl.narrow ? dispatch_zvp<T, TO, 128, true>(a, pl, has_z, vec, ws, st)
+                         : dispatch_zvp<T, TO, 128, false>(a, pl, has_z, vec, ws, st);
+      }
     default: return SSM_ERR_UNSUPPORTED;
   }
 }
@@ -230,7 +236,7 @@ ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_params *p, ssm_stream_t stream)
   if (p->batch == 0) return SSM_OK;
   if (p->batch > (int64_t(1) << 30)) return SSM_ERR_UNSUPPORTED;
   Plan pl;
-  if (!make_plan(int(p->dstate), p->batch, p->dim, p->seqlen, false, vec, pl)) return SSM_ERR_UNSUPPORTED;
+  if (!make_plan(int(p->dstate), p->batch, p->dim, p->seqlen, false, vec, p->dtype == SSM_BF16, pl)) return SSM_ERR_UNSUPPORTED;
   if (pl.ws_bytes > kNoAllocScratchBytes) return SSM_ERR_WORKSPACE;
   void *scratch = nullptr;
   st = noalloc_scratch(&scratch);
@@ -250,7 +256,7 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_params *p, void *workspace, size_t work
   if (p->batch == 0) return SSM_OK;
   if (p->batch > (int64_t(1) << 30)) return SSM_ERR_UNSUPPORTED;
   Plan pl;
-  if (!make_plan(int(p->dstate), p->batch, p->dim, p->seqlen, false, vec, pl)) return SSM_ERR_UNSUPPORTED;
+  if (!make_plan(int(p->dstate), p->batch, p->dim, p->seqlen, false, vec, p->dtype == SSM_BF16, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = nullptr;
   a.nseq = int(p->batch);
   return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
@@ -268,7 +274,7 @@ ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seq
   if (st != SSM_OK) return st;
   if (nseq == 0) return SSM_OK;
   Plan pl;
-  if (!make_plan(int(p->dstate), nseq, p->dim, p->seqlen, true, vec, pl)) return SSM_ERR_UNSUPPORTED;
+  if (!make_plan(int(p->dstate), nseq, p->dim, p->seqlen, true, vec, p->dtype == SSM_BF16, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = cu_seqlens;
   a.nseq = int(nseq);
   return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
@@ -343,7 +349,7 @@ size_t ssm_scan_workspace_size(const ssm_scan_params *p, int64_t nseq) {
   const bool varlen = nseq > 0;
   if (prepare_scan(p, varlen, a, vec) != SSM_OK) return 0;
   Plan pl;
-  if (!make_plan(int(p->dstate), varlen ? nseq : p->batch, p->dim, p->seqlen, varlen, vec, pl)) return 0;
+  if (!make_plan(int(p->dstate), varlen ? nseq : p->batch, p->dim, p->seqlen, varlen, vec, p->dtype == SSM_BF16, pl)) return 0;
   return pl.ws_bytes;
 }
 
