@@ -33,7 +33,8 @@
 // state crosses unit boundaries through a device workspace (release/acquire flag per
 // chain, bounded wait).  With NG > 1 the N states are split across NG warps that share the
 // same channels and steps (more parallelism for narrow problems); their partial outputs
-// are summed through shared memory.
+// are summed through shared memory.  With CPW * SPW < 32 the lanes of one warp form groups
+// that split the states the same way and sum their partial outputs with shuffles.
 //
 // Windows start at the sequence start rounded down to a 16-byte boundary; steps outside
 // [seq_start, seq_end) are made identities (Delta = 0, Delta*u = 0, B = 0) and are not
@@ -82,7 +83,11 @@ struct ChunkCfg {
   static constexpr int kTC = SPW * KI;      // chunk length (time steps)
   static constexpr int kCT = CPW * CW;      // channels per CTA
   static constexpr int kWarps = CW * NG;
-  static constexpr int kNS = N / NG;        // states per warp
+  // lane groups of a warp: when CPW * SPW < 32 the warp's lanes form kLG groups that hold the
+  // same channels and steps and split the states among themselves (their partial y are
+  // summed with shuffles)
+  static constexpr int kLG = 32 / (CPW * SPW);
+  static constexpr int kNS = N / (NG * kLG);  // states per lane group
   static constexpr int kVec = Elem<T>::kVec;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kXPitch = kTC + kVec;  // u/delta/z row pitch (elements): +16 bytes
@@ -104,8 +109,9 @@ struct ChunkCfg {
       size_t(2) * kCT * kNP * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
   static constexpr size_t kSmemBytes = 2 * kXBytes + 2 * kBCBytes + kYBytes + kDBytes + kParamBytes;
   static_assert(KI % 4 == 0 && KI % kVec == 0, "a lane's steps must be whole 16-byte vectors");
-  static_assert(32 % SPW == 0 && CPW * SPW == 32, "lane split");
-  static_assert(N % NG == 0 && KI % NG == 0, "state / step split");
+  static_assert(32 % (CPW * SPW) == 0, "lane split");
+  static_assert(kLG == 1 || NG == 1, "states split either across warps or inside a warp");
+  static_assert(N % (NG * kLG) == 0 && KI % (NG * kLG) == 0, "state / step split");
   static_assert(kXBytes % 16 == 0 && kBCBytes % 16 == 0, "16-byte aligned buffers");
 };
 
@@ -152,9 +158,11 @@ chunk_scan_kernel(const ScanArgs args) {
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int cw = warp % CW, g = warp / CW;        // channel warp, state group
-  const int cg = lane % CPW, seg = lane / CPW;    // interleaved channel groups
+  constexpr int LG = Cfg::kLG;
+  const int lg = lane / (CPW * SPW), lr = lane % (CPW * SPW);  // lane group, lane in group
+  const int cg = lr % CPW, seg = lr / CPW;        // interleaved channel groups
   const int ch = cw * CPW + cg;
-  const int n0 = g * NS;
+  const int n0 = (g * LG + lg) * NS;
 
   if constexpr (VEC) {
     if (threadIdx.x == 0) {
@@ -468,12 +476,30 @@ chunk_scan_kernel(const ScanArgs args) {
       // ---- epilogue: sum of the state groups, skip term, gate, store ----
       // A lane finishes steps [e0, e0 + KE) of its segment: all KI steps when NG == 1,
       // otherwise the g-th slice, after the partial sums went through shared memory.
-      constexpr int KE = KI / NG;
-      const int e0 = g * KE;
+      constexpr int KE = KI / (NG * LG);
+      const int e0 = (g * LG + lg) * KE;
       float yo[KE];
-      if constexpr (NG == 1) {
+      if constexpr (NG == 1 && LG == 1) {
 #pragma unroll
         for (int i = 0; i < KI; ++i) yo[i] = (i & 1) ? y[i / 2].y : y[i / 2].x;
+      } else if constexpr (LG > 1) {
+        // sum over the lane groups (lanes lr + k * CPW * SPW), then keep this group's slice
+#pragma unroll
+        for (int p = 0; p < KP; ++p) {
+#pragma unroll
+          for (int off = CPW * SPW; off < 32; off *= 2) {
+            y[p].x += __shfl_xor_sync(0xffffffffu, y[p].x, off);
+            y[p].y += __shfl_xor_sync(0xffffffffu, y[p].y, off);
+          }
+        }
+        auto yv = [&](int i) { return (i & 1) ? y[i / 2].y : y[i / 2].x; };
+#pragma unroll
+        for (int i = 0; i < KE; ++i) {
+          float v = yv(i);
+#pragma unroll
+          for (int k = 1; k < LG; ++k) v = lg == k ? yv(i + k * KE) : v;  // register indices only
+          yo[i] = v;
+        }
       } else {
         constexpr int YP = Cfg::kYPitch;
         static_assert(32 % KI == 0 && TC % 32 == 0, "a lane's steps lie in one padded block");

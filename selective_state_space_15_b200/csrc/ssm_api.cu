@@ -16,8 +16,10 @@ using ssm::ScanArgs;
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 // Tile shapes: KI steps per lane, SPW segment lanes per channel, CPW channels per warp, CW
-// channel warps and NG state groups per CTA.  Larger states get shorter chunks to bound
-// shared memory; the narrow shapes split the states over several warps for parallelism.
+// channel warps and NG state groups per CTA; when CPW * SPW < 32 the lanes of a warp form
+// 32 / (CPW * SPW) groups that split the states as well.  Larger states get shorter chunks
+// to bound shared memory; the narrow shapes split the states for parallelism (N=16: two
+// lane groups of one channel per warp; N=128: 16 warps).
 struct ShapeInfo {
   int KI, SPW, CPW, CW, NG;
   int ct() const { return CPW * CW; }
@@ -25,7 +27,7 @@ struct ShapeInfo {
 };
 template <int N, bool NARROW> struct Shape;
 template <> struct Shape<16, false> { static constexpr int KI = 16, SPW = 4, CPW = 8, CW = 4, NG = 1; };
-template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW = 2, CW = 4, NG = 2; };
+template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW = 1, CW = 8, NG = 1; };
 template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<128, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 4, NG = 1; };
