@@ -90,18 +90,10 @@ struct ChunkCfg {
   static constexpr int kNS = N / (NG * kLG);  // states per lane group
   static constexpr int kVec = Elem<T>::kVec;
   static constexpr int kThreads = kWarps * 32;
-  // With one channel per warp the 8 lanes of a quarter-warp read 8 segments of the same row,
-  // 2*KI bytes apart; rows are then staged in 128-byte pieces with 16 bytes of padding
-  // after each, so those lanes hit distinct banks.  Step t of a row sits at element
-  // padded(t) = t + (t / kPiece) * kPad.
-  static constexpr bool kSegPad = CPW == 1;
-  static constexpr int kPiece = 128 / int(sizeof(T)), kPad = 16 / int(sizeof(T));
-  static constexpr int kRow = kSegPad ? kTC + kTC / kPiece * kPad : kTC;  // padded row length
-  static constexpr int kXPitch = kRow + kVec;  // u/delta/z row pitch (elements): +16 bytes
-  static constexpr int kBCPitch = kRow;       // B/C row pitch (elements)
+  static constexpr int kXPitch = kTC + kVec;  // u/delta/z row pitch (elements): +16 bytes
   // shared memory layout (bytes), staging double-buffered
   static constexpr size_t kXBytes = size_t(3) * kCT * kXPitch * sizeof(T);  // u, delta, z
-  static constexpr size_t kBCBytes = size_t(2) * N * kBCPitch * sizeof(T);  // B, C
+  static constexpr size_t kBCBytes = size_t(2) * N * kTC * sizeof(T);       // B, C
   // partial y of the state groups, [NG][CT] rows of kYPitch words: 4 words of padding after
   // every 32 steps and 2 after the row put the lanes of a half-warp in distinct banks
   static constexpr int kYPitch = kTC + kTC / 32 * 4 + 2;
@@ -117,7 +109,6 @@ struct ChunkCfg {
       size_t(2) * kCT * kNP * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
   static constexpr size_t kSmemBytes = 2 * kXBytes + 2 * kBCBytes + kYBytes + kDBytes + kParamBytes;
   static_assert(KI % 4 == 0 && KI % kVec == 0, "a lane's steps must be whole 16-byte vectors");
-  static_assert(!kSegPad || (kPiece % KI == 0 && kTC % kPiece == 0), "a lane's steps lie in one piece");
   static_assert(32 % (CPW * SPW) == 0, "lane split");
   static_assert(kLG == 1 || NG == 1, "states split either across warps or inside a warp");
   static_assert(N % (NG * kLG) == 0 && KI % (NG * kLG) == 0, "state / step split");
@@ -130,8 +121,6 @@ __global__ void __launch_bounds__(CW * NG * 32, (CW * NG <= 8 ? 16 / (CW * NG) :
 chunk_scan_kernel(const ScanArgs args) {
   using Cfg = ChunkCfg<T, N, KI, SPW, CPW, CW, NG>;
   constexpr int TC = Cfg::kTC, CT = Cfg::kCT, V = Cfg::kVec, NT = Cfg::kThreads, XP = Cfg::kXPitch;
-  constexpr int BP = Cfg::kBCPitch;
-  auto padded = [](int t) { return Cfg::kSegPad ? t + t / Cfg::kPiece * Cfg::kPad : t; };
   constexpr int NS = Cfg::kNS;
   constexpr int LV = KI / V;  // 16-byte vectors per lane
   constexpr int KP = KI / 2;  // step pairs per lane
@@ -285,16 +274,6 @@ chunk_scan_kernel(const ScanArgs args) {
       const uint32_t row_bytes = uint32_t((wend - wstart) * int64_t(sizeof(T)));
       T *xdst = xs0 + buf * kXElems;
       T *bdst = bc0 + buf * kBCElems;
-      // one bulk copy per row, or one per 128-byte piece of the padded row layout
-      auto copy_row = [&](T *dst, const T *src, uint32_t bytes) {
-        if constexpr (Cfg::kSegPad) {
-          for (uint32_t off = 0; off < bytes; off += 128u)
-            bulk_g2s(dst + off / 128u * (Cfg::kPiece + Cfg::kPad), src + off / sizeof(T),
-                     bytes - off < 128u ? bytes - off : 128u, &bars[buf]);
-        } else {
-          bulk_g2s(dst, src, bytes, &bars[buf]);
-        }
-      };
       fence_proxy_async_smem();
       if (threadIdx.x == 0) mbar_arrive_expect_tx(&bars[buf], row_bytes * uint32_t(nx * nvalid_ch + 2 * N));
       for (int r = threadIdx.x; r < nx * CT + 2 * N; r += NT) {
@@ -302,11 +281,13 @@ chunk_scan_kernel(const ScanArgs args) {
           const int which = r / CT, c2 = r % CT;
           if (c2 >= nvalid_ch) continue;
           const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
-          copy_row(xdst + size_t(r) * XP, base + xbase + (d0 + c2) * args.x_dim_stride + wstart, row_bytes);
+          bulk_g2s(xdst + size_t(r) * XP, base + xbase + (d0 + c2) * args.x_dim_stride + wstart, row_bytes,
+                   &bars[buf]);
         } else {
           const int r2 = r - nx * CT, which = r2 / N, n = r2 % N;
           const T *base = which == 0 ? SSM_GB : SSM_GC;
-          copy_row(bdst + size_t(r2) * BP, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, row_bytes);
+          bulk_g2s(bdst + size_t(r2) * TC, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, row_bytes,
+                   &bars[buf]);
         }
       }
     };
@@ -322,7 +303,7 @@ chunk_scan_kernel(const ScanArgs args) {
         const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
         T val = Elem<T>::from_f32(0.f);
         if (dd < args.dim && t < args.seqlen) val = base[xbase + dd * args.x_dim_stride + t];
-        xdst[size_t(row) * XP + padded(j)] = val;
+        xdst[size_t(row) * XP + j] = val;
       }
       for (int i = threadIdx.x; i < 2 * N * TC; i += NT) {
         const int row = i / TC, j = i % TC;
@@ -331,7 +312,7 @@ chunk_scan_kernel(const ScanArgs args) {
         const T *base = which == 0 ? SSM_GB : SSM_GC;
         T val = Elem<T>::from_f32(0.f);
         if (t < args.seqlen) val = base[bcbase + int64_t(n) * args.bc_state_stride + t];
-        bdst[size_t(row) * BP + padded(j)] = val;
+        bdst[size_t(row) * TC + j] = val;
       }
     };
 
@@ -347,8 +328,8 @@ chunk_scan_kernel(const ScanArgs args) {
 #pragma unroll
       for (int p = 0; p < KP; ++p) y[p] = make_float2(0.f, 0.f);
       if constexpr (!Cfg::kSharedDelta) {
-        const T *ru = X + size_t(ch) * XP + padded(tl0);
-        const T *rd = X + size_t(CT + ch) * XP + padded(tl0);
+        const T *ru = X + size_t(ch) * XP + tl0;
+        const T *rd = X + size_t(CT + ch) * XP + tl0;
         const float bias = bias_s[ch];
 #pragma unroll
         for (int lv = 0; lv < LV; ++lv) {
@@ -376,8 +357,8 @@ chunk_scan_kernel(const ScanArgs args) {
         float *dus = dls + CT * DP;
         for (int i = threadIdx.x; i < CT * TC; i += NT) {
           const int c2 = i / TC, t = i % TC;
-          const float uv = Elem<T>::to_f32(X[size_t(c2) * XP + padded(t)]);
-          float dt = softplus_t<kFast>(Elem<T>::to_f32(X[size_t(CT + c2) * XP + padded(t)]) + bias_s[c2]);
+          const float uv = Elem<T>::to_f32(X[size_t(c2) * XP + t]);
+          float dt = softplus_t<kFast>(Elem<T>::to_f32(X[size_t(CT + c2) * XP + t]) + bias_s[c2]);
           float dtu = dt * uv;
           if constexpr (kMasked) {
             const bool in = t >= rel_lo && t < rel_hi;
@@ -417,8 +398,8 @@ chunk_scan_kernel(const ScanArgs args) {
         constexpr bool FWD = decltype(fwd_tag)::value, OUT = decltype(out_tag)::value;
         const float A2 = FWD ? A2s[ch * NP + n1] : 0.f;
         const float2 A22 = make_float2(A2, A2);
-        const T *rb = Bsm + size_t(n1) * BP + padded(tl0);
-        const T *rc = Csm + size_t(n2) * BP + padded(tl0);
+        const T *rb = Bsm + size_t(n1) * TC + tl0;
+        const T *rc = Csm + size_t(n2) * TC + tl0;
 #pragma unroll
         for (int lv = 0; lv < LV; ++lv) {
           float2 bb[V / 2], cc[V / 2];
@@ -547,8 +528,8 @@ chunk_scan_kernel(const ScanArgs args) {
       }
       if (ch_ok) {
         const float Dd = Dsk[ch];
-        const T *ru = X + size_t(ch) * XP + padded(tl0) + e0;
-        [[maybe_unused]] const T *rz = X + size_t(2 * CT + ch) * XP + padded(tl0) + e0;
+        const T *ru = X + size_t(ch) * XP + tl0 + e0;
+        [[maybe_unused]] const T *rz = X + size_t(2 * CT + ch) * XP + tl0 + e0;
         constexpr int VE = KE < V ? KE : V;  // elements per input vector read
         constexpr int VO = Elem<TO>::kVec;   // output elements per 16-byte store
 #pragma unroll
@@ -607,7 +588,7 @@ chunk_scan_kernel(const ScanArgs args) {
       const int rel_hi = int(min64(t_hi - wstart, TC + 1));
       const T *X = xs0 + buf * kXElems;
       const T *Bsm = bc0 + buf * kBCElems;
-      const T *Csm = Bsm + size_t(N) * BP;
+      const T *Csm = Bsm + size_t(N) * TC;
       if (rel_lo <= 0 && rel_hi >= TC)
         compute_chunk(std::false_type{}, X, Bsm, Csm, wstart, rel_lo, rel_hi);
       else
