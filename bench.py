@@ -127,10 +127,28 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ inputs
 
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's packed batch: every rank scans its own batch (weak scaling)."""
+    return workloads.CONFIGS[WORKLOAD]["seed"] + 1000 * rank
+
+
+def reduce_over_ranks(dist, ms_local: float, tokens_local: float, device):
+    """Job figures from per-rank ones: the slowest rank's time, the sum of all ranks' tokens."""
+    import torch
+    if dist is None:
+        return ms_local, tokens_local
+    t = torch.tensor([ms_local, float(tokens_local)], dtype=torch.float64, device=device)
+    ms = t[0:1].clone()
+    tok = t[1:2].clone()
+    dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    dist.all_reduce(tok, op=dist.ReduceOp.SUM)
+    return float(ms[0]), float(tok[0])
+
+
 def varlen_device_inputs(rank: int, device):
     import torch
     c = workloads.CONFIGS[WORKLOAD]
-    seed = c["seed"] + 1000 * rank
+    seed = rank_seed(rank)
     lens = workloads.varlen_lengths(c["nseq"], c["len_lo"], c["len_hi"], seed)
     inp = workloads.varlen_inputs(lens, c["dim"], c["dstate"], c["dtype"], seed)
     T = inp.meta["total"]
@@ -367,13 +385,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     tokens_local = T * args.steps
-    ms_max, tokens_all = ms_local, tokens_local
-    if dist:
-        t = torch.tensor([ms_local, float(tokens_local)], dtype=torch.float64, device=device)
-        m = t.clone()
-        dist.all_reduce(m[0:1], op=dist.ReduceOp.MAX)
-        dist.all_reduce(m[1:2], op=dist.ReduceOp.SUM)
-        ms_max, tokens_all = float(m[0]), float(m[1])
+    ms_max, tokens_all = reduce_over_ranks(dist, ms_local, tokens_local, device)
     value = tokens_all / (ms_max * 1e-3)
     ms_per_step = ms_max / args.steps
 
@@ -414,11 +426,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = f0.elapsed_time(f1)
     e2e_tokens = T * e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms, float(e2e_tokens)], dtype=torch.float64, device=device)
-        dist.all_reduce(t[0:1], op=dist.ReduceOp.MAX)
-        dist.all_reduce(t[1:2], op=dist.ReduceOp.SUM)
-        e2e_ms, e2e_tokens = float(t[0]), float(t[1])
+    e2e_ms, e2e_tokens = reduce_over_ranks(dist, e2e_ms, e2e_tokens, device)
     e2e_value = e2e_tokens / (e2e_ms * 1e-3)
 
     extra = None
