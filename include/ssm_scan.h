@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 1
+#define SSM_ABI_VERSION 2
 
 typedef enum {
   SSM_OK = 0,
@@ -126,6 +126,22 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_params *p, void *workspace, size_t work
  */
 ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seqlens, int64_t nseq,
                                  void *workspace, size_t workspace_bytes, ssm_stream_t stream);
+
+/*
+ * Packed prefill into a slot-indexed state pool (ufo.work second article §4.2, chunked
+ * prefill; §4.1 state pool): the same scan as ssm_scan_fwd_varlen, but sequence i starts
+ * from pool[slot_ids[i]] and its final state is written back there, so a long prompt can be
+ * fed in pieces over several calls and then decoded with ssm_state_update on the same pool.
+ *   pool     : DEVICE float32 [num_slots][dim][dstate], read and written in place
+ *   slot_ids : DEVICE int32 [nseq]; ids must be distinct (duplicates race).  An id outside
+ *              [0, num_slots) starts that sequence from zero, leaves the pool untouched (y is
+ *              still written) and records SSM_ERR_BAD_SLOT in the device status word.
+ * p->h0 and p->h_last must be NULL (SSM_ERR_INVALID_ARG otherwise).  Workspace as for
+ * ssm_scan_fwd_varlen (ssm_scan_workspace_size with the same nseq).
+ */
+ssm_status_t ssm_scan_fwd_varlen_pool(const ssm_scan_params *p, const int32_t *cu_seqlens, int64_t nseq,
+                                      float *pool, int64_t num_slots, const int32_t *slot_ids,
+                                      void *workspace, size_t workspace_bytes, ssm_stream_t stream);
 
 /*
  * One decode step over a slot-indexed state pool (ufo.work page §4.1 and its second

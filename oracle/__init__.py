@@ -130,6 +130,52 @@ def scan_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, bias=None, z=None, nt
     return {"y": y, "h_last": h_last, "y_mag": y_mag, "h_mag": h_mag}
 
 
+def scan_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=None, bias=None, z=None,
+                     pool_mag=None, nthreads: int = 1):
+    """Packed prefill into a state pool, in place on ``pool`` (float64 [S, dim, N]).
+
+    The serving flow of the ufo.work page's second article, §4.2 (a prompt is prefilled in
+    chunks into the per-request state of the §4.1 pool): sequence i of the packed batch is the
+    fixed-length scan of its columns started from pool[slot_ids[i]], and its final state
+    replaces pool[slot_ids[i]].  An id outside [0, S) starts from zero and writes nothing back.
+    ``pool_mag`` (same shape, optional) carries the magnitude bound of the pool entries and is
+    updated alongside.  Returns y [dim, T] and y_mag.
+    """
+    u, delta, B, C, A = (_f64(x) for x in (u, delta, B, C, A))
+    z, Dskip, bias = (_f64(x) for x in (z, Dskip, bias))
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    dim, T = u.shape
+    N = A.shape[1]
+    S = pool.shape[0]
+    assert pool.shape == (S, dim, N) and pool.dtype == np.float64
+    y = np.zeros((dim, T))
+    y_mag = np.zeros_like(y)
+    for i in range(cu.shape[0] - 1):
+        lo, hi, slot = int(cu[i]), int(cu[i + 1]), int(slot_ids[i])
+        if hi == lo:
+            continue
+        ok = 0 <= slot < S
+        h0 = pool[slot][None] if ok else np.zeros((1, dim, N))
+        col = slice(lo, hi)
+        r = scan(u[None, :, col], delta[None, :, col], B[None, :, col], C[None, :, col], A, Dskip, bias,
+                 None if z is None else z[None, :, col], h0, nthreads=nthreads)
+        y[:, col] = r["y"][0]
+        y_mag[:, col] = r["y_mag"][0]
+        if pool_mag is not None and ok:
+            # scan() starts its magnitude recursion from |h0|; the recursion is linear in its
+            # start, so the bound from pool_mag adds the decayed excess pool_mag - |h0| (>= 0),
+            # run as a scan with no input (u = 0, B = 0)
+            excess = np.maximum(pool_mag[slot] - np.abs(pool[slot]), 0.0)[None]
+            r_ex = scan(np.zeros((1, dim, hi - lo)), delta[None, :, col], np.zeros((1, N, hi - lo)),
+                        C[None, :, col], A, None, bias, None if z is None else z[None, :, col], excess,
+                        nthreads=nthreads)
+            y_mag[:, col] += r_ex["y_mag"][0]
+            pool_mag[slot] = r["h_mag"][0] + r_ex["h_mag"][0]
+        if ok:
+            pool[slot] = r["h_last"][0]
+    return {"y": y, "y_mag": y_mag}
+
+
 def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, bias=None, z=None, pool_mag=None):
     """One decode step, in place on ``pool`` (float64 array [S, dim, N]).
 

@@ -15,11 +15,12 @@ SSM_OK = 0
 _STATUS = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED", 3: "SSM_ERR_CUDA",
            4: "SSM_ERR_BAD_SLOT", 5: "SSM_ERR_TIMEOUT", 6: "SSM_ERR_WORKSPACE"}
 SSM_F32, SSM_BF16 = 0, 1
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 # Every function the header declares; tests check the library exports all of them.
 EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
-            "ssm_get_device_status", "ssm_status_string", "ssm_abi_version", "ssm_scan_fwd_noalloc")
+            "ssm_get_device_status", "ssm_status_string", "ssm_abi_version", "ssm_scan_fwd_noalloc",
+            "ssm_scan_fwd_varlen_pool")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SSM_NOALLOC_SCRATCH_BYTES
 
 
@@ -63,6 +64,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_scan_fwd_noalloc.argtypes = [pp, P]
     lib.ssm_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssm_scan_fwd_varlen.argtypes = [pp, P, I64, P, S, P]
+    lib.ssm_scan_fwd_varlen_pool.argtypes = [pp, P, I64, P, I64, P, P, S, P]
     lib.ssm_state_update.argtypes = [P, I64, P, I64, pp, P]
     lib.ssm_scan_workspace_size.argtypes = [pp, I64]
     lib.ssm_scan_workspace_size.restype = S
@@ -70,7 +72,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_status_string.argtypes = [ctypes.c_int]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_abi_version.argtypes = []
-    for f in ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_get_device_status"):
+    for f in ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_scan_fwd_varlen_pool", "ssm_state_update",
+              "ssm_get_device_status"):
         getattr(lib, f).restype = ctypes.c_int
     if lib.ssm_abi_version() != ABI_VERSION:
         raise RuntimeError(f"libssm_scan ABI {lib.ssm_abi_version()} != binding ABI {ABI_VERSION}")
@@ -217,6 +220,32 @@ def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, 
     _check(lib.ssm_scan_fwd_varlen(ctypes.byref(p), _ptr(cu_seqlens), nseq, _ptr(wbuf), ws, _stream(stream)),
            "ssm_scan_fwd_varlen")
     return y, h_last
+
+
+def scan_fwd_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=None, delta_bias=None, z=None,
+                         y=None, total=None, stream=None, y_dtype=None):
+    """Packed prefill into a state pool: sequence i starts from pool[slot_ids[i]] and its final
+    state is written back there.  pool: float32 [S, D, N]; slot_ids: int32 [nseq].  Returns y."""
+    import torch
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 tensor")
+    if slot_ids.dtype != torch.int32 or not slot_ids.is_contiguous():
+        raise ValueError("slot_ids must be a contiguous int32 tensor")
+    _f32(pool)
+    nseq = cu_seqlens.shape[0] - 1
+    if slot_ids.shape[0] != nseq:
+        raise ValueError("one slot id per sequence")
+    if tuple(pool.shape[1:]) != (u.shape[0], A.shape[1]):
+        raise ValueError("pool must be [S, dim, dstate]")
+    y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
+    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, None, y, None, total)
+    lib = load()
+    ws = lib.ssm_scan_workspace_size(ctypes.byref(p), nseq)
+    wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
+    _check(lib.ssm_scan_fwd_varlen_pool(ctypes.byref(p), _ptr(cu_seqlens), nseq, _ptr(pool), pool.shape[0],
+                                        _ptr(slot_ids), _ptr(wbuf), ws, _stream(stream)),
+           "ssm_scan_fwd_varlen_pool")
+    return y
 
 
 def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, y=None, stream=None,

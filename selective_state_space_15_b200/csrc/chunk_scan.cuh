@@ -53,6 +53,10 @@ struct ScanArgs {
   void *y;
   float *h_last;
   const int32_t *cu_seqlens;  // nullptr: fixed-length batch
+  // state rows: sequence s reads h0 and writes h_last at row state_slots[s] of a [num_slots]
+  // [dim][N] pool (h0 == h_last == the pool) when state_slots is set, else at row s
+  const int32_t *state_slots;
+  int64_t num_slots;
   int64_t dim, seqlen;
   int64_t x_batch_stride, x_dim_stride, bc_batch_stride, bc_state_stride;
   int nseq;    // sequences (batch size or number of packed sequences)
@@ -245,11 +249,22 @@ chunk_scan_kernel(const ScanArgs args) {
     }
     // state entering the unit: h0 (or zero) for a chain's first unit, otherwise the state
     // the previous unit of the chain published
+    // row of this sequence's state in h0 / h_last (a pool slot, or the sequence index); -1:
+    // the slot id is out of range, so the state is neither read nor written
+    int64_t srow = s;
+    if (args.state_slots) {
+      srow = args.state_slots[s];
+      if (srow < 0 || srow >= args.num_slots) {
+        if (threadIdx.x == 0 && tile == 0) report_status(4 /* SSM_ERR_BAD_SLOT */);
+        srow = -1;
+      }
+    }
     if (!PERSIST || kgrp == 0) {
       for (int i = threadIdx.x; i < CT * N; i += NT) {
         const int c2 = i / N, n = i % N;
         const int64_t dd = d0 + c2;
-        carry_s[c2 * NP + n] = (dd < args.dim && args.h0) ? args.h0[(int64_t(s) * args.dim + dd) * N + n] : 0.f;
+        carry_s[c2 * NP + n] =
+            (dd < args.dim && args.h0 && srow >= 0) ? args.h0[(srow * args.dim + dd) * N + n] : 0.f;
       }
     } else {
       if (threadIdx.x == 0) {
@@ -603,11 +618,11 @@ chunk_scan_kernel(const ScanArgs args) {
       __threadfence();
       __syncthreads();
       if (threadIdx.x == 0) atomicExch(args.flags + chain, uint32_t(kgrp + 1));
-    } else if (args.h_last) {
+    } else if (args.h_last && srow >= 0) {
       for (int i = threadIdx.x; i < CT * N; i += NT) {
         const int c2 = i / N, n = i % N;
         const int64_t dd = d0 + c2;
-        if (dd < args.dim) args.h_last[(int64_t(s) * args.dim + dd) * N + n] = carry_s[c2 * NP + n];
+        if (dd < args.dim) args.h_last[(srow * args.dim + dd) * N + n] = carry_s[c2 * NP + n];
       }
     }
     __syncthreads();  // shared state of this unit is dead before the next unit overwrites it

@@ -283,6 +283,30 @@ ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seq
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
+ssm_status_t ssm_scan_fwd_varlen_pool(const ssm_scan_params *p, const int32_t *cu_seqlens, int64_t nseq,
+                                      float *pool, int64_t num_slots, const int32_t *slot_ids,
+                                      void *workspace, size_t workspace_bytes, ssm_stream_t stream) {
+  if (!p || !cu_seqlens || !pool || !slot_ids || nseq < 0 || num_slots <= 0) return SSM_ERR_INVALID_ARG;
+  if (p->h0 || p->h_last) return SSM_ERR_INVALID_ARG;  // the pool holds both
+  if (nseq > (int64_t(1) << 30)) return SSM_ERR_UNSUPPORTED;
+  if (p->seqlen > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;  // int32 offsets
+  ScanArgs a;
+  bool vec = false;
+  ssm_status_t st = prepare_scan(p, true, a, vec);
+  if (st != SSM_OK) return st;
+  if (nseq == 0) return SSM_OK;
+  Plan pl;
+  if (!make_plan(int(p->dstate), nseq, p->dim, p->seqlen, true, vec, p->dtype == SSM_BF16, pl)) return SSM_ERR_UNSUPPORTED;
+  a.cu_seqlens = cu_seqlens;
+  a.nseq = int(nseq);
+  a.h0 = pool;
+  a.h_last = pool;
+  a.state_slots = slot_ids;
+  a.num_slots = num_slots;
+  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
 ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slot_ids, int64_t R,
                               const ssm_scan_params *p, ssm_stream_t stream) {
   if (!p || !pool || !slot_ids || num_slots <= 0 || R < 0) return SSM_ERR_INVALID_ARG;

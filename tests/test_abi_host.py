@@ -74,6 +74,25 @@ def test_null_params_and_varlen_checks(lib):
     assert lib.ssm_scan_fwd_varlen(ctypes.byref(p2), 0x10000, 4, None, 0, None) == 1  # varlen needs batch 1
 
 
+def test_pool_prefill_host_checks(lib):
+    p = _params(seqlen=256)
+    fake = 0x10000
+    f = lib.ssm_scan_fwd_varlen_pool
+    assert f(None, fake, 2, fake, 4, fake, None, 0, None) == 1                     # no params
+    assert f(ctypes.byref(p), None, 2, fake, 4, fake, None, 0, None) == 1          # no cu_seqlens
+    assert f(ctypes.byref(p), fake, 2, None, 4, fake, None, 0, None) == 1          # no pool
+    assert f(ctypes.byref(p), fake, 2, fake, 4, None, None, 0, None) == 1          # no slot ids
+    assert f(ctypes.byref(p), fake, 2, fake, 0, fake, None, 0, None) == 1          # empty pool
+    assert f(ctypes.byref(p), fake, -1, fake, 4, fake, None, 0, None) == 1
+    ph = _params(seqlen=256)
+    ph.h0 = fake
+    assert f(ctypes.byref(ph), fake, 2, fake, 4, fake, None, 0, None) == 1         # the pool holds h0
+    ph = _params(seqlen=256)
+    ph.h_last = fake
+    assert f(ctypes.byref(ph), fake, 2, fake, 4, fake, None, 0, None) == 1         # ... and h_last
+    assert f(ctypes.byref(p), fake, 0, fake, 4, fake, None, 0, None) == 0          # nothing to do
+
+
 def test_state_update_host_checks(lib):
     p = _params(batch=8, seqlen=1, dim=32, dstate=16)
     fake = 0x10000

@@ -274,3 +274,76 @@ def test_workload_generator_is_deterministic_and_bf16_exact():
     # ties round to even: 1 + 2^-8 (exactly halfway between two bf16 values) rounds down to 1
     x = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8], dtype=np.float32)
     np.testing.assert_array_equal(workloads.round_to_bf16(x), np.array([1.0, 1.0 + 2.0 ** -6], dtype=np.float32))
+
+
+def _split_packed(inp, cuts):
+    """Two packed batches holding the first and the rest of each sequence (cut i in sequence i)."""
+    cu = inp.cu_seqlens
+    first, rest = [], []
+    for i in range(len(cu) - 1):
+        lo, hi = int(cu[i]), int(cu[i + 1])
+        first.append(np.arange(lo, lo + cuts[i]))
+        rest.append(np.arange(lo + cuts[i], hi))
+
+    def pack(parts):
+        idx = np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
+        cu2 = np.concatenate([[0], np.cumsum([len(p) for p in parts])]).astype(np.int32)
+        return idx, cu2
+    return pack(first), pack(rest)
+
+
+def test_pool_prefill_from_zero_is_the_varlen_scan():
+    """A pool of zeros: the prefill is the packed scan, and the slots receive its final states."""
+    inp = workloads.varlen_inputs([37, 0, 120, 64], 6, 8, "f32", seed=41)
+    slots = np.array([3, 0, 1, 4], dtype=np.int32)
+    pool = np.zeros((5, 6, 8))
+    got = oracle.scan_varlen_pool(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.cu_seqlens, pool, slots,
+                                  inp.Dskip, inp.bias, inp.z)
+    ref = oracle.scan_varlen(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.cu_seqlens, inp.Dskip, inp.bias, inp.z)
+    assert np.allclose(got["y"], ref["y"], rtol=0, atol=1e-13)
+    for i, s in enumerate(slots):
+        if i == 1:
+            assert np.all(pool[s] == 0.0)                   # empty sequence: the slot is untouched
+        else:
+            assert np.allclose(pool[s], ref["h_last"][i], rtol=0, atol=1e-13)
+    assert np.all(pool[2] == 0.0)                           # slot used by nobody
+
+
+def test_pool_prefill_in_two_pieces_equals_one_call():
+    """Chunked prefill: feeding every prompt in two pieces through the pool gives the same
+    outputs, final states and magnitude bounds as one call (the state is carried exactly)."""
+    rng = np.random.default_rng(42)
+    lens = [37, 5, 120, 64]
+    inp = workloads.varlen_inputs(lens, 6, 8, "f32", seed=42)
+    slots = np.array([2, 0, 4, 1], dtype=np.int32)
+    pool0 = rng.standard_normal((5, 6, 8))
+    mag0 = np.abs(pool0) * 1.5                              # a bound looser than |pool|
+    pool_a, mag_a = pool0.copy(), mag0.copy()
+    one = oracle.scan_varlen_pool(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.cu_seqlens, pool_a, slots,
+                                  inp.Dskip, inp.bias, inp.z, pool_mag=mag_a)
+    (i1, cu1), (i2, cu2) = _split_packed(inp, [10, 0, 77, 64])
+    pool_b, mag_b = pool0.copy(), mag0.copy()
+    y = np.zeros_like(one["y"])
+    y_mag = np.zeros_like(one["y_mag"])
+    for idx, cu in ((i1, cu1), (i2, cu2)):
+        r = oracle.scan_varlen_pool(inp.u[:, idx], inp.delta[:, idx], inp.B[:, idx], inp.C[:, idx], inp.A, cu,
+                                    pool_b, slots, inp.Dskip, inp.bias, inp.z[:, idx], pool_mag=mag_b)
+        y[:, idx] = r["y"]
+        y_mag[:, idx] = r["y_mag"]
+    assert np.allclose(y, one["y"], rtol=1e-12, atol=1e-13)
+    assert np.allclose(pool_b, pool_a, rtol=1e-12, atol=1e-13)
+    assert np.allclose(y_mag, one["y_mag"], rtol=1e-12, atol=1e-13)
+    assert np.allclose(mag_b, mag_a, rtol=1e-12, atol=1e-13)
+    assert np.all(np.abs(one["y"]) <= one["y_mag"] * (1 + 1e-12))
+
+
+def test_pool_prefill_bad_slot_starts_from_zero_and_writes_nothing():
+    inp = workloads.varlen_inputs([20, 30], 4, 8, "f32", seed=43)
+    pool = np.ones((3, 4, 8))
+    before = pool.copy()
+    got = oracle.scan_varlen_pool(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.cu_seqlens, pool,
+                                  np.array([7, 1], dtype=np.int32), inp.Dskip, inp.bias, inp.z)
+    ref = oracle.scan_varlen(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.cu_seqlens, inp.Dskip, inp.bias, inp.z)
+    assert np.allclose(got["y"][:, :20], ref["y"][:, :20], rtol=0, atol=1e-13)   # from zero
+    assert np.array_equal(pool[0], before[0]) and np.array_equal(pool[2], before[2])
+    assert not np.array_equal(pool[1], before[1])
