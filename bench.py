@@ -299,11 +299,70 @@ def decode_run(steps, warmup, hbm_peak):
             "l2": "flushed (256 MB read) before each step", "launch": "CUDA graph replay"}
 
 
+def pool_prefill_run(steps, warmup, sfu_peak):
+    """The varlen workload fed through ssm_scan_fwd_varlen_pool: 16 sequences whose states live
+    in a 64-slot pool (read at the start, written back at the end of each sequence)."""
+    import torch
+    import selective_state_space_15_b200 as ssm
+    stream = torch.cuda.current_stream()
+    device = torch.device("cuda", torch.cuda.current_device())
+    inp, _, dev, T, pitch = varlen_device_inputs(0, device)
+    D, N, nseq = inp.u.shape[0], inp.A.shape[1], inp.meta["nseq"]
+    pool = torch.zeros((64, D, N), dtype=torch.float32, device=device)
+    slots = torch.arange(0, 4 * nseq, 4, dtype=torch.int32, device=device)
+    y = torch.empty((D, pitch), dtype=torch.bfloat16, device=device)
+    ms = time_kernel(lambda: ssm.scan_fwd_varlen_pool(dev["u"], dev["delta"], dev["B"], dev["C"], dev["A"], dev["cu"],
+                                                      pool, slots, dev["Dskip"], dev["bias"], dev["z"], y=y, total=T,
+                                                      stream=stream), steps, warmup, stream)
+    _, ne = scan_counts(T, D, N, 2, 2, nseq)
+    return {"ms": round(ms, 4), "tokens_per_s": T / (ms * 1e-3), "sfu_frac": round(ne / (ms * 1e-3) / sfu_peak, 4)}
+
+
+def decode_loop_run(hbm_peak, loop_steps=100):
+    """A serving-style decode loop: `loop_steps` back-to-back decode steps (inputs cycling over 4
+    token sets) captured in one CUDA graph; the active states (84 MB) stay in L2 between steps."""
+    import torch
+    import selective_state_space_15_b200 as ssm
+    stream = torch.cuda.current_stream()
+    c = workloads.CONFIGS["decode_bf16"]
+    prob = workloads.decode_problem(c["num_slots"], c["dim"], c["dstate"], c["R"], c["dtype"], c["seed"])
+    pool = torch.from_numpy(prob.pool0).cuda()
+    slots = torch.from_numpy(prob.slot_ids).cuda()
+    A, Dsk, bias = (torch.from_numpy(x).cuda() for x in (prob.A, prob.Dskip, prob.bias))
+    bf = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)  # noqa: E731
+    sets = []
+    for k in range(4):
+        x = workloads.decode_step_inputs(prob, k)
+        sets.append([bf(x[n]) for n in ("u", "delta", "z", "B", "C")])
+    ys = [torch.empty_like(sets[0][0]) for _ in range(4)]
+
+    def loop():
+        for i in range(loop_steps):
+            u, dl, z, B, C = sets[i % 4]
+            ssm.state_update(pool, slots, u, dl, B, C, A, Dsk, bias, z, y=ys[i % 4])
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        loop()
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        loop()
+    ms = time_kernel(graph.replay, 5, 3, stream) / loop_steps
+    del graph
+    R, D, N = c["R"], c["dim"], c["dstate"]
+    nb = R * D * N * 4 * 2 + R * D * 2 * 4 + R * N * 2 * 2 + D * (N + 2) * 4
+    return {"ms_per_step": round(ms, 5), "tokens_per_s": R / (ms * 1e-3), "steps_per_graph": loop_steps,
+            "hbm_gbs": round(nb / (ms * 1e-3) / 1e9, 1), "l2": "states resident in L2 between steps"}
+
+
 def secondary(steps, warmup, hbm_peak, sfu_peak):
-    """Kernel-only figures for the long-sequence and decode workloads (single GPU)."""
+    """Kernel-only figures for the long-sequence, pool-prefill and decode workloads (single GPU)."""
     out = {name: long_run(name, max(3, steps // 4), warmup, hbm_peak, sfu_peak)
            for name in ("long_bf16", "long_n128_bf16")}
+    out["varlen_pool_bf16"] = pool_prefill_run(max(3, steps // 4), warmup, sfu_peak)
     out["decode_bf16"] = decode_run(steps, warmup, hbm_peak)
+    out["decode_loop_bf16"] = decode_loop_run(hbm_peak)
     return out
 
 
