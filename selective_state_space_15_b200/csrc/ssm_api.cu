@@ -27,7 +27,7 @@ struct ShapeInfo {
 };
 template <int N, bool NARROW> struct Shape;
 template <> struct Shape<16, false> { static constexpr int KI = 16, SPW = 4, CPW = 8, CW = 4, NG = 1; };
-template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW = 1, CW = 8, NG = 1; };
+template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW = 1, CW = 4, NG = 1; };
 template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<128, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 4, NG = 1; };
