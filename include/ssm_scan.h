@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 2
+#define SSM_ABI_VERSION 3
 
 typedef enum {
   SSM_OK = 0,
@@ -84,6 +84,12 @@ typedef struct CUstream_st *ssm_stream_t;
  *
  * Optional pointers (may be NULL): z (no gate), Dskip (= 0), delta_bias (= 0), h0 (zero
  * state), h_last (final state not written).  Required: u, delta, B, C, A, y.
+ *
+ * Channel groups (scans only; ufo.work page §3.2 splits channels into independent groups):
+ *   with ngroups = G > 1, dim must be a multiple of G and channel d reads B and C of group
+ *   d / (dim / G): B, C become [batch][G][dstate][seqlen] (varlen: [G][dstate][T]) with the
+ *   group stride bc_group_stride (default dstate * bc_state_stride; the default batch
+ *   stride becomes G * dstate * bc_state_stride).  ssm_state_update takes ngroups <= 1 only.
  */
 typedef struct ssm_scan_params {
   ssm_dtype_t dtype;       /* dtype of u, delta, z, B, C (and of y unless y_fp32 is set)       */
@@ -107,6 +113,8 @@ typedef struct ssm_scan_params {
   const float *h0;
   void *y;
   float *h_last;
+  int64_t ngroups;         /* channel groups with their own B, C: 0 or 1 = one group (scans)    */
+  int64_t bc_group_stride; /* 0 -> dstate * bc_state_stride                                    */
 } ssm_scan_params;
 
 /*

@@ -81,9 +81,24 @@ def scan(u, delta, B, C, A, Dskip=None, bias=None, z=None, h0=None, nthreads: in
 
     u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; A: [dim, N]; Dskip, bias: [dim];
     h0: [batch, dim, N] or None (zero state).
+    B, C may also be [batch, G, N, L]: G groups of dim/G consecutive channels, each group
+    with its own B and C (channels are independent, ufo.work page §3.2, so a grouped scan is
+    the scan of each group's channels with that group's B and C).
     Returns dict with y [batch, dim, L], h_last [batch, dim, N] and the magnitudes
     y_mag, h_mag used to scale errors.
     """
+    if np.ndim(B) == 4:
+        G = B.shape[1]
+        dim = np.shape(u)[1]
+        assert dim % G == 0 and np.shape(C) == np.shape(B)
+        dg = dim // G
+        parts = []
+        for g in range(G):
+            sl = slice(g * dg, (g + 1) * dg)
+            sub = lambda x, ax=1: None if x is None else np.asarray(x)[(slice(None),) * ax + (sl,)]  # noqa: E731
+            parts.append(scan(sub(u), sub(delta), np.asarray(B)[:, g], np.asarray(C)[:, g], np.asarray(A)[sl],
+                              sub(Dskip, 0), sub(bias, 0), sub(z), sub(h0), nthreads=nthreads))
+        return {k: np.concatenate([r[k] for r in parts], axis=1) for k in parts[0]}
     u, delta, B, C, A = (_f64(x) for x in (u, delta, B, C, A))
     z, Dskip, bias, h0 = (_f64(x) for x in (z, Dskip, bias, h0))
     batch, dim, L = u.shape
@@ -107,10 +122,26 @@ def scan(u, delta, B, C, A, Dskip=None, bias=None, z=None, h0=None, nthreads: in
 
 
 def scan_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, bias=None, z=None, nthreads: int = 1):
-    """Packed varlen scan. u, delta, z: [dim, T]; B, C: [N, T]; cu_seqlens: [nseq+1].
+    """Packed varlen scan. u, delta, z: [dim, T]; B, C: [N, T] (or [G, N, T]: channel groups as
+    in scan()); cu_seqlens: [nseq+1].
 
     Every sequence starts from h = 0.  Returns y [dim, T], h_last [nseq, dim, N] and magnitudes.
     """
+    if np.ndim(B) == 3:
+        G = B.shape[0]
+        dim = np.shape(u)[0]
+        assert dim % G == 0 and np.shape(C) == np.shape(B)
+        dg = dim // G
+        parts = []
+        for g in range(G):
+            sl = slice(g * dg, (g + 1) * dg)
+            sub = lambda x: None if x is None else np.asarray(x)[sl]  # noqa: E731
+            parts.append(scan_varlen(sub(u), sub(delta), np.asarray(B)[g], np.asarray(C)[g], np.asarray(A)[sl],
+                                     cu_seqlens, sub(Dskip), sub(bias), sub(z), nthreads=nthreads))
+        return {"y": np.concatenate([r["y"] for r in parts], axis=0),
+                "y_mag": np.concatenate([r["y_mag"] for r in parts], axis=0),
+                "h_last": np.concatenate([r["h_last"] for r in parts], axis=1),
+                "h_mag": np.concatenate([r["h_mag"] for r in parts], axis=1)}
     u, delta, B, C, A = (_f64(x) for x in (u, delta, B, C, A))
     z, Dskip, bias = (_f64(x) for x in (z, Dskip, bias))
     cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))

@@ -15,7 +15,7 @@ SSM_OK = 0
 _STATUS = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED", 3: "SSM_ERR_CUDA",
            4: "SSM_ERR_BAD_SLOT", 5: "SSM_ERR_TIMEOUT", 6: "SSM_ERR_WORKSPACE"}
 SSM_F32, SSM_BF16 = 0, 1
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 # Every function the header declares; tests check the library exports all of them.
 EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
@@ -42,6 +42,7 @@ class ScanParams(ctypes.Structure):
         ("B", ctypes.c_void_p), ("C", ctypes.c_void_p),
         ("A", ctypes.c_void_p), ("Dskip", ctypes.c_void_p), ("delta_bias", ctypes.c_void_p),
         ("h0", ctypes.c_void_p), ("y", ctypes.c_void_p), ("h_last", ctypes.c_void_p),
+        ("ngroups", ctypes.c_int64), ("bc_group_stride", ctypes.c_int64),
     ]
 
 
@@ -134,15 +135,18 @@ def _f32(t):
 # ----------------------------------------------------------------------------- scans
 
 def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None):
-    """Fill ScanParams for the fixed-length layout u/delta/z/y [b, D, L], B/C [b, N, L]."""
+    """Fill ScanParams for the fixed-length layout u/delta/z/y [b, D, L], B/C [b, N, L] (or
+    [b, G, N, L]: G channel groups, channel d reading group d // (D / G))."""
     bsz, dim, L = u.shape
     N = A.shape[1]
     _time_contig(u, delta, z, B, C, y)
     for t in (delta, z, y):
         if t is not None and (t.shape != u.shape or t.stride() != u.stride()):
             raise ValueError("delta, z and y must match u's shape and strides")
-    if B.shape != (bsz, N, L) or C.shape != B.shape or C.stride() != B.stride():
-        raise ValueError("B and C must be [batch, dstate, seqlen] with equal strides")
+    G = B.shape[1] if B.dim() == 4 else 1
+    want = (bsz, G, N, L) if B.dim() == 4 else (bsz, N, L)
+    if B.shape != want or C.shape != B.shape or C.stride() != B.stride():
+        raise ValueError("B and C must be [batch, (groups,) dstate, seqlen] with equal strides")
     for t in (A, Dskip, delta_bias, h0, h_last):
         _f32(t)
     p = ScanParams()
@@ -150,7 +154,9 @@ def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None,
     p.y_fp32 = _y_fp32(u, y)
     p.batch, p.dim, p.dstate, p.seqlen = bsz, dim, N, L
     p.x_batch_stride, p.x_dim_stride = u.stride(0), u.stride(1)
-    p.bc_batch_stride, p.bc_state_stride = B.stride(0), B.stride(1)
+    p.bc_batch_stride, p.bc_state_stride = B.stride(0), B.stride(-2)
+    if B.dim() == 4:
+        p.ngroups, p.bc_group_stride = G, B.stride(1)
     p.u, p.delta, p.z, p.B, p.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
     p.A, p.Dskip, p.delta_bias, p.h0 = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(h0)
     p.y, p.h_last = _ptr(y), _ptr(h_last)
@@ -176,7 +182,8 @@ def scan_fwd(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=
 
 def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None,
                   total=None):
-    """ScanParams for the packed layout u/delta/z/y [D, T(+pad)], B/C [N, T(+pad)].
+    """ScanParams for the packed layout u/delta/z/y [D, T(+pad)], B/C [N, T(+pad)] (or
+    [G, N, T(+pad)]: G channel groups).
 
     ``total`` is the number of packed tokens T when the rows are padded beyond it.
     """
@@ -187,8 +194,8 @@ def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=Non
     for t in (delta, z, y):
         if t is not None and (t.shape != u.shape or t.stride() != u.stride()):
             raise ValueError("delta, z and y must match u's shape and strides")
-    if B.shape[0] != N or C.shape != B.shape or C.stride() != B.stride() or B.shape[1] < T:
-        raise ValueError("B and C must be [dstate, >=T] with equal strides")
+    if B.shape[-2] != N or C.shape != B.shape or C.stride() != B.stride() or B.shape[-1] < T or B.dim() > 3:
+        raise ValueError("B and C must be [(groups,) dstate, >=T] with equal strides")
     for t in (A, Dskip, delta_bias, h0, h_last):
         _f32(t)
     p = ScanParams()
@@ -196,7 +203,9 @@ def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=Non
     p.y_fp32 = _y_fp32(u, y)
     p.batch, p.dim, p.dstate, p.seqlen = 1, dim, N, T
     p.x_batch_stride, p.x_dim_stride = 0, u.stride(0)
-    p.bc_batch_stride, p.bc_state_stride = 0, B.stride(0)
+    p.bc_batch_stride, p.bc_state_stride = 0, B.stride(-2)
+    if B.dim() == 3:
+        p.ngroups, p.bc_group_stride = B.shape[0], B.stride(0)
     p.u, p.delta, p.z, p.B, p.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
     p.A, p.Dskip, p.delta_bias, p.h0 = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(h0)
     p.y, p.h_last = _ptr(y), _ptr(h_last)

@@ -60,7 +60,11 @@ struct ScanArgs {
   int64_t dim, seqlen;
   int64_t x_batch_stride, x_dim_stride, bc_batch_stride, bc_state_stride;
   int nseq;    // sequences (batch size or number of packed sequences)
-  int ntiles;  // channel tiles per sequence
+  int ntiles;  // channel tiles per sequence (tiles_per_group per channel group)
+  // channel groups: group g holds channels [g * group_dim, (g + 1) * group_dim) and reads B, C
+  // at offset g * bc_group_stride; a tile never straddles two groups
+  int64_t group_dim, bc_group_stride;
+  int tiles_per_group;
   // persistent scheduling (fixed-length batches only)
   uint32_t *ticket;  // work counter, zero at launch
   uint32_t *flags;   // [nchains] chunk groups completed per chain, zero at launch
@@ -200,7 +204,9 @@ chunk_scan_kernel(const ScanArgs args) {
     }
     const int tile = chain % args.ntiles;
     int s = chain / args.ntiles;
-    const int d0 = tile * CT;
+    const int grp = tile / args.tiles_per_group;
+    const int64_t d0 = int64_t(grp) * args.group_dim + int64_t(tile % args.tiles_per_group) * CT;
+    const int64_t d_end = min64(int64_t(grp + 1) * args.group_dim, args.dim);  // this group's channels
     int64_t t_lo, t_hi, xbase, bcbase;
     if (args.cu_seqlens) {
       if (args.nseq <= kMaxSortedSeqs) {
@@ -231,19 +237,20 @@ chunk_scan_kernel(const ScanArgs args) {
     const int nchunks = t_hi > t_lo ? int((t_hi - w0 + TC - 1) / TC) : 0;
     const int c_begin = PERSIST ? kgrp * args.group : 0;
     const int c_end = PERSIST ? min(c_begin + args.group, nchunks) : nchunks;
-    const int nvalid_ch = int(min64(CT, args.dim - d0));
+    bcbase += int64_t(grp) * args.bc_group_stride;
+    const int nvalid_ch = int(min64(CT, d_end - d0));
     const int64_t d = d0 + ch;
-    const bool ch_ok = d < args.dim;
+    const bool ch_ok = d < d_end;
 
     // per-tile constants
     for (int i = threadIdx.x; i < CT * N; i += NT) {
       const int c2 = i / N, n = i % N;
       const int64_t dd = d0 + c2;
-      A2s[c2 * NP + n] = dd < args.dim ? args.A[dd * N + n] * kLog2e : 0.f;
+      A2s[c2 * NP + n] = dd < d_end ? args.A[dd * N + n] * kLog2e : 0.f;
     }
     for (int i = threadIdx.x; i < CT; i += NT) {
       const int64_t dd = d0 + i;
-      const bool ok = dd < args.dim;
+      const bool ok = dd < d_end;
       Dsk[i] = (ok && args.Dskip) ? args.Dskip[dd] : 0.f;
       bias_s[i] = (ok && args.bias) ? args.bias[dd] : 0.f;
     }
@@ -264,7 +271,7 @@ chunk_scan_kernel(const ScanArgs args) {
         const int c2 = i / N, n = i % N;
         const int64_t dd = d0 + c2;
         carry_s[c2 * NP + n] =
-            (dd < args.dim && args.h0 && srow >= 0) ? args.h0[(srow * args.dim + dd) * N + n] : 0.f;
+            (dd < d_end && args.h0 && srow >= 0) ? args.h0[(srow * args.dim + dd) * N + n] : 0.f;
       }
     } else {
       if (threadIdx.x == 0) {
@@ -317,7 +324,7 @@ chunk_scan_kernel(const ScanArgs args) {
         const int64_t dd = d0 + c2, t = wstart + j;
         const T *base = which == 0 ? SSM_GU : (which == 1 ? SSM_GDL : SSM_GZ);
         T val = Elem<T>::from_f32(0.f);
-        if (dd < args.dim && t < args.seqlen) val = base[xbase + dd * args.x_dim_stride + t];
+        if (dd < d_end && t < args.seqlen) val = base[xbase + dd * args.x_dim_stride + t];
         xdst[size_t(row) * XP + j] = val;
       }
       for (int i = threadIdx.x; i < 2 * N * TC; i += NT) {
@@ -622,7 +629,7 @@ chunk_scan_kernel(const ScanArgs args) {
       for (int i = threadIdx.x; i < CT * N; i += NT) {
         const int c2 = i / N, n = i % N;
         const int64_t dd = d0 + c2;
-        if (dd < args.dim) args.h_last[(srow * args.dim + dd) * N + n] = carry_s[c2 * NP + n];
+        if (dd < d_end) args.h_last[(srow * args.dim + dd) * N + n] = carry_s[c2 * NP + n];
       }
     }
     __syncthreads();  // shared state of this unit is dead before the next unit overwrites it

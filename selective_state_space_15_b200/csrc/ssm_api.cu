@@ -58,13 +58,20 @@ struct Plan {
 // N=128 narrow tile is planned for 16-bit inputs only, whose B/C chunk fits in shared memory)
 constexpr int64_t kNarrowChannels16 = 8192, kNarrowChannels128 = 32768;
 
-bool make_plan(int N, int64_t nseq, int64_t dim, int64_t seqlen, bool varlen, bool vec, bool bf16, Plan &pl) {
+int64_t groups_of(const ssm_scan_params *p) { return p->ngroups > 1 ? p->ngroups : 1; }
+
+bool make_plan(const ssm_scan_params *p, int64_t nseq, bool varlen, bool vec, Plan &pl) {
+  const int N = int(p->dstate);
+  const int64_t dim = p->dim, seqlen = p->seqlen;
+  const bool bf16 = p->dtype == SSM_BF16;
   pl = Plan{};
   pl.persist = !varlen && vec && seqlen > 0;
   pl.narrow = pl.persist && ((N == 16 && nseq * dim < kNarrowChannels16) ||
                              (N == 128 && bf16 && nseq * dim < kNarrowChannels128));
   if (!shape_for(N, pl.narrow, pl.si)) return false;
-  pl.ntiles = (dim + pl.si.ct() - 1) / pl.si.ct();
+  // channel tiles never straddle a group of channels
+  const int64_t G = groups_of(p);
+  pl.ntiles = G * ((dim / G + pl.si.ct() - 1) / pl.si.ct());
   pl.nchains = nseq * pl.ntiles;
   pl.nchunks = pl.persist ? (seqlen + pl.si.tc() - 1) / pl.si.tc() : 0;
   if (pl.persist) {
@@ -175,15 +182,22 @@ ssm_status_t prepare_scan(const ssm_scan_params *p, bool varlen, ScanArgs &a, bo
   a.x_dim_stride = p->x_dim_stride ? p->x_dim_stride : p->seqlen;
   a.x_batch_stride = p->x_batch_stride ? p->x_batch_stride : p->dim * a.x_dim_stride;
   a.bc_state_stride = p->bc_state_stride ? p->bc_state_stride : p->seqlen;
-  a.bc_batch_stride = p->bc_batch_stride ? p->bc_batch_stride : p->dstate * a.bc_state_stride;
+  if (p->ngroups < 0 || p->bc_group_stride < 0) return SSM_ERR_INVALID_ARG;
+  const int64_t G = groups_of(p);
+  if (p->dim % G != 0) return SSM_ERR_INVALID_ARG;
+  a.group_dim = p->dim / G;
+  a.bc_group_stride = p->bc_group_stride ? p->bc_group_stride : p->dstate * a.bc_state_stride;
+  if (G > 1 && a.bc_group_stride < p->dstate * a.bc_state_stride) return SSM_ERR_INVALID_ARG;
+  a.bc_batch_stride = p->bc_batch_stride ? p->bc_batch_stride : G * a.bc_group_stride;
   if (a.x_dim_stride < p->seqlen || a.bc_state_stride < p->seqlen) return SSM_ERR_INVALID_ARG;
   if (!varlen && p->batch > 1 && (a.x_batch_stride < p->dim * a.x_dim_stride ||
-                                  a.bc_batch_stride < p->dstate * a.bc_state_stride))
+                                  a.bc_batch_stride < G * p->dstate * a.bc_state_stride))
     return SSM_ERR_INVALID_ARG;
   const size_t es = elem_size(p->dtype);
   const int64_t V = int64_t(16 / es);
   vec = aligned16(p->u) && aligned16(p->delta) && aligned16(p->B) && aligned16(p->C) && aligned16(p->y) &&
         (!p->z || aligned16(p->z)) && a.x_dim_stride % V == 0 && a.bc_state_stride % V == 0 &&
+        a.bc_group_stride % V == 0 &&
         (varlen || (a.x_batch_stride % V == 0 && a.bc_batch_stride % V == 0));
   return SSM_OK;
 }
@@ -194,6 +208,7 @@ ssm_status_t run_scan(ScanArgs a, const Plan &pl, ssm_dtype_t dt, bool y_fp32, i
     return SSM_ERR_WORKSPACE;
   if (pl.ntiles > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
   a.ntiles = int(pl.ntiles);
+  a.tiles_per_group = int(pl.ntiles / (a.dim / a.group_dim));
   const bool has_z = a.z != nullptr;
   if (dt == SSM_BF16) {
     if (y_fp32) return dispatch_n<__nv_bfloat16, float>(a, pl, N, has_z, vec, ws, st);
@@ -238,7 +253,7 @@ ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_params *p, ssm_stream_t stream)
   if (p->batch == 0) return SSM_OK;
   if (p->batch > (int64_t(1) << 30)) return SSM_ERR_UNSUPPORTED;
   Plan pl;
-  if (!make_plan(int(p->dstate), p->batch, p->dim, p->seqlen, false, vec, p->dtype == SSM_BF16, pl)) return SSM_ERR_UNSUPPORTED;
+  if (!make_plan(p, p->batch, false, vec, pl)) return SSM_ERR_UNSUPPORTED;
   if (pl.ws_bytes > kNoAllocScratchBytes) return SSM_ERR_WORKSPACE;
   void *scratch = nullptr;
   st = noalloc_scratch(&scratch);
@@ -258,7 +273,7 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_params *p, void *workspace, size_t work
   if (p->batch == 0) return SSM_OK;
   if (p->batch > (int64_t(1) << 30)) return SSM_ERR_UNSUPPORTED;
   Plan pl;
-  if (!make_plan(int(p->dstate), p->batch, p->dim, p->seqlen, false, vec, p->dtype == SSM_BF16, pl)) return SSM_ERR_UNSUPPORTED;
+  if (!make_plan(p, p->batch, false, vec, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = nullptr;
   a.nseq = int(p->batch);
   return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
@@ -276,7 +291,7 @@ ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seq
   if (st != SSM_OK) return st;
   if (nseq == 0) return SSM_OK;
   Plan pl;
-  if (!make_plan(int(p->dstate), nseq, p->dim, p->seqlen, true, vec, p->dtype == SSM_BF16, pl)) return SSM_ERR_UNSUPPORTED;
+  if (!make_plan(p, nseq, true, vec, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = cu_seqlens;
   a.nseq = int(nseq);
   return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
@@ -296,7 +311,7 @@ ssm_status_t ssm_scan_fwd_varlen_pool(const ssm_scan_params *p, const int32_t *c
   if (st != SSM_OK) return st;
   if (nseq == 0) return SSM_OK;
   Plan pl;
-  if (!make_plan(int(p->dstate), nseq, p->dim, p->seqlen, true, vec, p->dtype == SSM_BF16, pl)) return SSM_ERR_UNSUPPORTED;
+  if (!make_plan(p, nseq, true, vec, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = cu_seqlens;
   a.nseq = int(nseq);
   a.h0 = pool;
@@ -312,6 +327,7 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
   if (!p || !pool || !slot_ids || num_slots <= 0 || R < 0) return SSM_ERR_INVALID_ARG;
   if (p->dtype != SSM_F32 && p->dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
   if (p->batch != R || p->seqlen != 1 || p->dim <= 0 || p->dstate <= 0) return SSM_ERR_INVALID_ARG;
+  if (p->ngroups > 1) return SSM_ERR_UNSUPPORTED;  // decode takes one B, C per request
   if (!p->u || !p->delta || !p->B || !p->C || !p->A || !p->y) return SSM_ERR_INVALID_ARG;
   const int64_t N = p->dstate;
   if (N % 4 != 0 || N > ssm::kUpdateMaxState) return SSM_ERR_UNSUPPORTED;
@@ -375,7 +391,7 @@ size_t ssm_scan_workspace_size(const ssm_scan_params *p, int64_t nseq) {
   const bool varlen = nseq > 0;
   if (prepare_scan(p, varlen, a, vec) != SSM_OK) return 0;
   Plan pl;
-  if (!make_plan(int(p->dstate), varlen ? nseq : p->batch, p->dim, p->seqlen, varlen, vec, p->dtype == SSM_BF16, pl)) return 0;
+  if (!make_plan(p, varlen ? nseq : p->batch, varlen, vec, pl)) return 0;
   return pl.ws_bytes;
 }
 

@@ -74,6 +74,17 @@ def test_null_params_and_varlen_checks(lib):
     assert lib.ssm_scan_fwd_varlen(ctypes.byref(p2), 0x10000, 4, None, 0, None) == 1  # varlen needs batch 1
 
 
+def test_channel_group_host_checks(lib):
+    assert lib.ssm_scan_fwd(ctypes.byref(_params(ngroups=3)), None, 0, None) == 1       # 64 channels, 3 groups
+    assert lib.ssm_scan_fwd(ctypes.byref(_params(ngroups=-1)), None, 0, None) == 1
+    assert lib.ssm_scan_fwd(ctypes.byref(_params(ngroups=2, bc_group_stride=-8)), None, 0, None) == 1
+    # a group stride shorter than one group's [dstate][seqlen] block
+    assert lib.ssm_scan_fwd(ctypes.byref(_params(ngroups=2, bc_group_stride=100)), None, 0, None) == 1
+    # the decode update takes one B, C per request
+    p = _params(batch=8, seqlen=1, dim=32, dstate=16, ngroups=2)
+    assert lib.ssm_state_update(0x10000, 4, 0x10000, 8, ctypes.byref(p), None) == 2
+
+
 def test_pool_prefill_host_checks(lib):
     p = _params(seqlen=256)
     fake = 0x10000

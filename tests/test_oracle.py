@@ -347,3 +347,47 @@ def test_pool_prefill_bad_slot_starts_from_zero_and_writes_nothing():
     assert np.allclose(got["y"][:, :20], ref["y"][:, :20], rtol=0, atol=1e-13)   # from zero
     assert np.array_equal(pool[0], before[0]) and np.array_equal(pool[2], before[2])
     assert not np.array_equal(pool[1], before[1])
+
+
+def test_grouped_scan_with_equal_groups_is_the_plain_scan():
+    """Channel groups that all carry the same B and C reduce to the ungrouped scan."""
+    inp = workloads.batch_inputs(2, 12, 8, 40, "f32", seed=51)
+    B4 = np.repeat(inp.B[:, None], 3, axis=1)
+    C4 = np.repeat(inp.C[:, None], 3, axis=1)
+    g = oracle.scan(inp.u, inp.delta, B4, C4, inp.A, inp.Dskip, inp.bias, inp.z)
+    r = oracle.scan(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.Dskip, inp.bias, inp.z)
+    for k in ("y", "h_last", "y_mag", "h_mag"):
+        np.testing.assert_array_equal(g[k], r[k])
+
+
+def test_grouped_scan_reads_each_groups_own_b_and_c():
+    """Swapping the B/C of two groups equals swapping which channels sit in which group."""
+    rng = np.random.default_rng(52)
+    bsz, D, N, L, G = 1, 8, 4, 30, 2
+    u, dl, z = (rng.standard_normal((bsz, D, L)) for _ in range(3))
+    B, C = rng.standard_normal((bsz, G, N, L)), rng.standard_normal((bsz, G, N, L))
+    A = -rng.uniform(0.1, 2, size=(D, N))
+    Dk, bias = rng.standard_normal(D), rng.uniform(-3, 0, size=D)
+    out = oracle.scan(u, dl, B, C, A, Dk, bias, z)
+    perm = np.r_[D // 2:D, 0:D // 2]                     # group 1's channels first
+    sw = oracle.scan(u[:, perm], dl[:, perm], B[:, ::-1], C[:, ::-1], A[perm], Dk[perm], bias[perm], z[:, perm])
+    np.testing.assert_array_equal(sw["y"][:, perm.argsort()], out["y"])
+    np.testing.assert_array_equal(sw["h_last"][:, perm.argsort()], out["h_last"])
+    # and group 0 really uses B[:, 0]: a plain scan of its channels with B[:, 0]
+    one = oracle.scan(u[:, :4], dl[:, :4], B[:, 0], C[:, 0], A[:4], Dk[:4], bias[:4], z[:, :4])
+    np.testing.assert_array_equal(out["y"][:, :4], one["y"])
+
+
+def test_grouped_varlen_matches_grouped_fixed_length_per_sequence():
+    inp = workloads.varlen_inputs([23, 40], 6, 4, "f32", seed=53)
+    rng = np.random.default_rng(54)
+    T = inp.meta["total"]
+    B3, C3 = rng.standard_normal((3, 4, T)), rng.standard_normal((3, 4, T))
+    v = oracle.scan_varlen(inp.u, inp.delta, B3, C3, inp.A, inp.cu_seqlens, inp.Dskip, inp.bias, inp.z)
+    cu = inp.cu_seqlens
+    for s in range(2):
+        sl = slice(cu[s], cu[s + 1])
+        f = oracle.scan(inp.u[None, :, sl], inp.delta[None, :, sl], B3[None, :, :, sl], C3[None, :, :, sl], inp.A,
+                        inp.Dskip, inp.bias, inp.z[None, :, sl])
+        np.testing.assert_array_equal(v["y"][:, sl], f["y"][0])
+        np.testing.assert_array_equal(v["h_last"][s], f["h_last"][0])

@@ -232,3 +232,45 @@ def test_persistent_paths_and_workspace():
     ref = oracle.scan(inp.u, inp.delta, inp.B, inp.C, inp.A, z=inp.z)
     check("y", host(y), ref["y"], ref["y_mag"], TOL["bf16"], "bf16")
     assert ssm.device_status() == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape,G", [
+    ((2, 64, 16, 512), 2),      # persistent tiles, one group per 32 channels
+    ((1, 24, 16, 1000), 3),     # narrow tile, 8 channels per group (tiles end at group edges)
+    ((1, 40, 128, 200), 4),     # N=128
+    ((3, 18, 16, 777), 3),      # element-wise staging, 6 channels per group
+])
+def test_channel_groups(shape, G, dtype):
+    """Channel groups: channel d reads B, C of group d // (D / G)."""
+    b, D, N, L = shape
+    inp = workloads.batch_inputs(b, D, N, L, dtype, seed=300 + G + L)
+    rng = np.random.default_rng(301)
+    rnd = lambda: workloads.round_to_bf16(rng.standard_normal((b, G, N, L)).astype(np.float32))  # noqa: E731
+    B4, C4 = (rnd(), rnd()) if dtype == "bf16" else tuple(rng.standard_normal((2, b, G, N, L)).astype(np.float32))
+    u, dl, z = (dev(x, dtype) for x in (inp.u, inp.delta, inp.z))
+    A, Dk, bias = (torch.from_numpy(x).cuda() for x in (inp.A, inp.Dskip, inp.bias))
+    y, hl = ssm.scan_fwd(u, dl, dev(B4, dtype), dev(C4, dtype), A, Dk, bias, z)
+    torch.cuda.synchronize()
+    ref = oracle.scan(inp.u, inp.delta, B4, C4, inp.A, inp.Dskip, inp.bias, inp.z, nthreads=NTHREADS)
+    check("y", host(y), ref["y"], ref["y_mag"], TOL[dtype], dtype)
+    check("h_last", host(hl), ref["h_last"], ref["h_mag"], TOL[dtype])
+
+
+def test_channel_groups_varlen():
+    lengths = [300, 0, 77, 1000]
+    D, N, G = 48, 16, 4
+    inp = workloads.varlen_inputs(lengths, D, N, "bf16", seed=302)
+    T = inp.meta["total"]
+    rng = np.random.default_rng(303)
+    B3, C3 = (workloads.round_to_bf16(rng.standard_normal((G, N, T)).astype(np.float32)) for _ in range(2))
+    pitch = round_up(T, 8)
+    u, dl, z = (dev(x, "bf16", pitch=pitch) for x in (inp.u, inp.delta, inp.z))
+    A, Dk, bias = (torch.from_numpy(x).cuda() for x in (inp.A, inp.Dskip, inp.bias))
+    y, hl = ssm.scan_fwd_varlen(u, dl, dev(B3, "bf16", pitch=pitch), dev(C3, "bf16", pitch=pitch), A,
+                                torch.from_numpy(inp.cu_seqlens).cuda(), Dk, bias, z, total=T)
+    torch.cuda.synchronize()
+    ref = oracle.scan_varlen(inp.u, inp.delta, B3, C3, inp.A, inp.cu_seqlens, inp.Dskip, inp.bias, inp.z,
+                             nthreads=NTHREADS)
+    check("y", host(y, T), ref["y"], ref["y_mag"], TOL["bf16"], "bf16")
+    check("h_last", host(hl), ref["h_last"], ref["h_mag"], TOL["bf16"])
