@@ -109,7 +109,7 @@ ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t str
     if (cudaMemsetAsync(w, 0, pl.carries_off, stream) != cudaSuccess) return SSM_ERR_CUDA;
     const int64_t resident = int64_t(num_sms) * (max_blocks_per_sm > 0 ? max_blocks_per_sm : 1);
     // enough units per CTA for an even spread, as few as possible for low per-unit overhead
-    int64_t group = (pl.nchunks * pl.nchains) / (8 * resident);
+    int64_t group = (pl.nchunks * pl.nchains) / (16 * resident);
     group = group < 1 ? 1 : (group > pl.nchunks ? pl.nchunks : group);
     const int64_t ngroups = (pl.nchunks + group - 1) / group;
     if (pl.nchains * ngroups > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
