@@ -111,7 +111,14 @@ struct ChunkCfg {
   // channels hit distinct banks); with few groups each lane computes its own.
   static constexpr bool kSharedDelta = NG >= 4;
   static constexpr int kDPitch = kTC + 4;
-  static constexpr size_t kDBytes = kSharedDelta ? size_t(2) * kCT * kDPitch * sizeof(float) : 0;
+  // With two lane groups per warp each group evaluates Delta, Delta*u for half of a lane's
+  // steps and the halves meet in a per-warp buffer [2][CPW*SPW][KI+4] (rows padded: distinct
+  // banks for the 8 lanes of a quarter-warp).
+  static constexpr bool kLaneDelta = !kSharedDelta && kLG == 2 && KI / kVec == 2;
+  static constexpr int kXRow = KI + 4;
+  static constexpr size_t kDBytes = kSharedDelta ? size_t(2) * kCT * kDPitch * sizeof(float)
+                                    : kLaneDelta ? size_t(kWarps) * 2 * (CPW * SPW) * kXRow * sizeof(float)
+                                                 : 0;
   static constexpr int kNP = N + 1;         // row pitch of the per-(channel, state) arrays
   static constexpr size_t kParamBytes =
       size_t(2) * kCT * kNP * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
@@ -349,7 +356,57 @@ chunk_scan_kernel(const ScanArgs args) {
       float dsum = 0.f;
 #pragma unroll
       for (int p = 0; p < KP; ++p) y[p] = make_float2(0.f, 0.f);
-      if constexpr (!Cfg::kSharedDelta) {
+      if constexpr (Cfg::kLaneDelta) {
+        // this lane group evaluates vector lg of the lane's KI steps; the other group the rest
+        constexpr int XR = Cfg::kXRow;
+        float *dlw = dls + size_t(warp) * 2 * (CPW * SPW) * XR + size_t(lr) * XR;
+        float *duw = dlw + (CPW * SPW) * XR;
+        const T *ru = X + size_t(ch) * XP + tl0 + lg * V;
+        const T *rd = X + size_t(CT + ch) * XP + tl0 + lg * V;
+        const float bias = bias_s[ch];
+        float2 vu[V / 2], vd[V / 2];
+        unpack16x2<T>(*reinterpret_cast<const uint4 *>(ru), vu);
+        unpack16x2<T>(*reinterpret_cast<const uint4 *>(rd), vd);
+        __syncwarp();  // the previous chunk's reads of the buffer are done
+#pragma unroll
+        for (int e = 0; e < V / 2; e += 2) {
+          float4 l4, u4;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float2 dt = make_float2(softplus_t<kFast>(vd[e + h].x + bias), softplus_t<kFast>(vd[e + h].y + bias));
+            float2 uu;
+            if constexpr (kMasked) {
+              const int i = tl0 + lg * V + 2 * (e + h);
+              dt.x = (i >= rel_lo && i < rel_hi) ? dt.x : 0.f;
+              dt.y = (i + 1 >= rel_lo && i + 1 < rel_hi) ? dt.y : 0.f;
+              uu = make_float2(dt.x != 0.f ? dt.x * vu[e + h].x : 0.f, dt.y != 0.f ? dt.y * vu[e + h].y : 0.f);
+            } else {
+              uu = __fmul2_rn(dt, vu[e + h]);
+            }
+            if (h == 0) {
+              l4.x = dt.x; l4.y = dt.y; u4.x = uu.x; u4.y = uu.y;
+            } else {
+              l4.z = dt.x; l4.w = dt.y; u4.z = uu.x; u4.w = uu.y;
+            }
+          }
+          *reinterpret_cast<float4 *>(dlw + lg * V + 2 * e) = l4;
+          *reinterpret_cast<float4 *>(duw + lg * V + 2 * e) = u4;
+        }
+        __syncwarp();  // both halves written
+        float2 ds = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < KI / 4; ++q) {
+          const float4 l4 = reinterpret_cast<const float4 *>(dlw)[q];
+          const float4 u4 = reinterpret_cast<const float4 *>(duw)[q];
+          dl[2 * q] = make_float2(l4.x, l4.y);
+          dl[2 * q + 1] = make_float2(l4.z, l4.w);
+          du[2 * q] = make_float2(u4.x, u4.y);
+          du[2 * q + 1] = make_float2(u4.z, u4.w);
+          ds = __fadd2_rn(ds, dl[2 * q]);
+          ds = __fadd2_rn(ds, dl[2 * q + 1]);
+        }
+        dsum = ds.x + ds.y;
+      } else if constexpr (!Cfg::kSharedDelta) {
         const T *ru = X + size_t(ch) * XP + tl0;
         const T *rd = X + size_t(CT + ch) * XP + tl0;
         const float bias = bias_s[ch];
