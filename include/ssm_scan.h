@@ -37,8 +37,9 @@
  *   - Supported state sizes: dstate in {16, 32, 64, 128} for the scans, any multiple of 4
  *     up to 128 for the decode update.  Other values return SSM_ERR_UNSUPPORTED.
  *   - Fast path: when every tensor base is 16-byte aligned and every row stride is a
- *     multiple of 16 bytes, inputs are staged with 16-byte asynchronous copies.  Other
- *     layouts are accepted and take a slower element-wise staging path.
+ *     multiple of 16 bytes, inputs are staged with TMA bulk copies, and rows are read up to
+ *     the sequence length rounded up to 16 bytes (the row stride covers it).  Other layouts
+ *     are accepted and take a slower element-wise staging path.
  */
 #ifndef SSM_SCAN_H_
 #define SSM_SCAN_H_

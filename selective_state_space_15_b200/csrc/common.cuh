@@ -13,7 +13,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
-// MUFU approximations (PTX ISA: ex2/lg2/rcp .approx).
+// MUFU approximations (PTX ISA: ex2/lg2 .approx).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -22,11 +22,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float rcp_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -130,15 +125,6 @@ template <bool kFast> __device__ __forceinline__ float silu_t(float z) {
   return kFast ? silu_fast(z) : silu_precise(z);
 }
 
-// 16-byte global->shared asynchronous copy; `src_bytes` < 16 zero-fills the remainder
-// (src_bytes == 0 reads nothing).
-__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gmem_src, int src_bytes) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(gmem_src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 // ---- TMA bulk copies completing on an mbarrier (PTX ISA: cp.async.bulk, mbarrier) ----
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
