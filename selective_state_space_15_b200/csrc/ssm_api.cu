@@ -19,29 +19,34 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 // channel warps and NG state groups per CTA; when CPW * SPW < 32 the lanes of a warp form
 // 32 / (CPW * SPW) groups that split the states as well.  Larger states get shorter chunks
 // to bound shared memory; the narrow shapes split the states for parallelism (N=16: two
-// lane groups of one channel per warp; N=128: 16 warps).
+// lane groups of one channel per warp; N=128: 16 warps).  32-bit inputs can take a shape of
+// their own (F32): the narrow N=16 one halves the chunk so that four CTAs fit per SM.
 struct ShapeInfo {
   int KI, SPW, CPW, CW, NG;
   int ct() const { return CPW * CW; }
   int tc() const { return SPW * KI; }
 };
-template <int N, bool NARROW> struct Shape;
+template <int N, bool NARROW, bool F32 = false> struct Shape;
+template <int N, bool NARROW> struct Shape<N, NARROW, true> : Shape<N, NARROW, false> {};
 template <> struct Shape<16, false> { static constexpr int KI = 16, SPW = 4, CPW = 8, CW = 4, NG = 1; };
 template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW = 1, CW = 4, NG = 1; };
+template <> struct Shape<16, true, true> { static constexpr int KI = 8, SPW = 16, CPW = 1, CW = 4, NG = 1; };
 template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<128, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 4, NG = 1; };
 template <> struct Shape<128, true> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 1, NG = 16; };
-template <int N, bool NARROW> ShapeInfo shape_of() {
-  using S = Shape<N, NARROW>;
+template <int N, bool NARROW, bool F32> ShapeInfo shape_of() {
+  using S = Shape<N, NARROW, F32>;
   return ShapeInfo{S::KI, S::SPW, S::CPW, S::CW, S::NG};
 }
-bool shape_for(int N, bool narrow, ShapeInfo &si) {
+bool shape_for(int N, bool narrow, bool f32, ShapeInfo &si) {
   switch (N) {
-    case 16: si = narrow ? shape_of<16, true>() : shape_of<16, false>(); return true;
-    case 32: si = shape_of<32, false>(); return true;
-    case 64: si = shape_of<64, false>(); return true;
-    case 128: si = narrow ? shape_of<128, true>() : shape_of<128, false>(); return true;
+    case 16:
+      si = narrow ? (f32 ? shape_of<16, true, true>() : shape_of<16, true, false>()) : shape_of<16, false, false>();
+      return true;
+    case 32: si = shape_of<32, false, false>(); return true;
+    case 64: si = shape_of<64, false, false>(); return true;
+    case 128: si = narrow ? shape_of<128, true, false>() : shape_of<128, false, false>(); return true;
     default: return false;
   }
 }
@@ -68,7 +73,7 @@ bool make_plan(const ssm_scan_params *p, int64_t nseq, bool varlen, bool vec, Pl
   pl.persist = !varlen && vec && seqlen > 0;
   pl.narrow = pl.persist && ((N == 16 && nseq * dim < kNarrowChannels16) ||
                              (N == 128 && bf16 && nseq * dim < kNarrowChannels128));
-  if (!shape_for(N, pl.narrow, pl.si)) return false;
+  if (!shape_for(N, pl.narrow, p->dtype == SSM_F32, pl.si)) return false;
   // channel tiles never straddle a group of channels
   const int64_t G = groups_of(p);
   pl.ntiles = G * ((dim / G + pl.si.ct() - 1) / pl.si.ct());
@@ -84,7 +89,7 @@ bool make_plan(const ssm_scan_params *p, int64_t nseq, bool varlen, bool vec, Pl
 
 template <typename T, typename TO, int N, bool NARROW, bool HAS_Z, bool VEC, bool PERSIST>
 ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t stream) {
-  using S = Shape<N, NARROW>;
+  using S = Shape<N, NARROW, sizeof(T) == 4>;
   using Cfg = ssm::ChunkCfg<T, N, S::KI, S::SPW, S::CPW, S::CW, S::NG>;
   auto kern = ssm::chunk_scan_kernel<T, TO, N, S::KI, S::SPW, S::CPW, S::CW, S::NG, HAS_Z, VEC, PERSIST>;
   static int configured_device = -1;  // the attribute is set once per device function per device
@@ -108,9 +113,17 @@ ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t str
     unsigned char *w = static_cast<unsigned char *>(ws);
     if (cudaMemsetAsync(w, 0, pl.carries_off, stream) != cudaSuccess) return SSM_ERR_CUDA;
     const int64_t resident = int64_t(num_sms) * (max_blocks_per_sm > 0 ? max_blocks_per_sm : 1);
-    // enough units per CTA for an even spread, as few as possible for low per-unit overhead
-    int64_t group = (pl.nchunks * pl.nchains) / (16 * resident);
-    group = group < 1 ? 1 : (group > pl.nchunks ? pl.nchunks : group);
+    // The units of one chain run one after another, so splitting a chain only evens out the
+    // load when there are more chains than CTA slots.  Then: enough units per slot for an even
+    // spread (about 16), and at least kMinGroup chunks per unit to keep the per-unit overhead
+    // (ticket, hand-off, first load) small; otherwise a chain is a single unit.
+    constexpr int64_t kMinGroup = 6;
+    int64_t group = pl.nchunks;
+    if (pl.nchains > resident) {
+      group = (pl.nchunks * pl.nchains) / (16 * resident);
+      group = group < kMinGroup ? kMinGroup : group;
+      group = group > pl.nchunks ? pl.nchunks : group;
+    }
     const int64_t ngroups = (pl.nchunks + group - 1) / group;
     if (pl.nchains * ngroups > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
     a.ticket = reinterpret_cast<uint32_t *>(w);
@@ -172,7 +185,7 @@ ssm_status_t prepare_scan(const ssm_scan_params *p, bool varlen, ScanArgs &a, bo
   if (varlen && p->batch != 1) return SSM_ERR_INVALID_ARG;
   if (!p->u || !p->delta || !p->B || !p->C || !p->A || !p->y) return SSM_ERR_INVALID_ARG;
   ShapeInfo probe;
-  if (p->dstate > 128 || !shape_for(int(p->dstate), false, probe)) return SSM_ERR_UNSUPPORTED;
+  if (p->dstate > 128 || !shape_for(int(p->dstate), false, false, probe)) return SSM_ERR_UNSUPPORTED;
   if (p->dim > (int64_t(1) << 31) || p->seqlen > (int64_t(1) << 40)) return SSM_ERR_UNSUPPORTED;
   a = ScanArgs{};
   a.u = p->u; a.delta = p->delta; a.z = p->z; a.B = p->B; a.C = p->C;

@@ -206,13 +206,16 @@ def test_persistent_paths_and_workspace():
     units through the workspace); narrow problems split the states over two warps."""
     import ctypes
     lib = ssm.load()
-    for (b, D, L, seed) in [(1, 8, 4096, 21), (3, 40, 2304, 22), (2, 2048 + 8, 512, 23)]:
-        inp = workloads.batch_inputs(b, D, 16, L, "bf16", seed=seed)
-        y, hl = run_batch(inp, "bf16", y_dtype=torch.float32)
+    # more chains than CTA slots split into several units handed on through the workspace
+    # (3 x 1000 and 3 x 1100 channels); fewer chains run as one unit each
+    for (b, D, L, seed, dt) in [(1, 8, 4096, 21, "bf16"), (3, 40, 2304, 22, "bf16"), (2, 2048 + 8, 512, 23, "bf16"),
+                                (3, 1000, 2304, 27, "bf16"), (1, 8, 4100, 25, "f32"), (3, 1100, 1540, 26, "f32")]:
+        inp = workloads.batch_inputs(b, D, 16, L, dt, seed=seed)
+        y, hl = run_batch(inp, dt, y_dtype=torch.float32)
         ch = np.arange(0, D, max(1, D // 24))
         ref = oracle_batch(inp, channels=ch)
-        check("y", y[:, ch], ref["y"], ref["y_mag"], TOL["bf16"], "f32")
-        check("h_last", hl[:, ch], ref["h_last"], ref["h_mag"], TOL["bf16"])
+        check("y", y[:, ch], ref["y"], ref["y_mag"], TOL[dt], "f32")
+        check("h_last", hl[:, ch], ref["h_last"], ref["h_mag"], TOL[dt])
     # the workspace size is reported and enforced
     inp = workloads.batch_inputs(1, 8, 16, 256, "bf16", seed=24)
     u, dl, z, B, C = (dev(x, "bf16") for x in (inp.u, inp.delta, inp.z, inp.B, inp.C))
