@@ -99,9 +99,12 @@ struct ChunkCfg {
   static constexpr int kVec = Elem<T>::kVec;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kXPitch = kTC + kVec;  // u/delta/z row pitch (elements): +16 bytes
+  // B/C row pitch (elements).  With lane groups, the two groups of a quarter-warp read
+  // neighbouring states at the same steps: 16 bytes of padding put them in distinct banks.
+  static constexpr int kBCPitch = kTC + (kLG > 1 ? 16 / int(sizeof(T)) : 0);
   // shared memory layout (bytes), staging double-buffered
   static constexpr size_t kXBytes = size_t(3) * kCT * kXPitch * sizeof(T);  // u, delta, z
-  static constexpr size_t kBCBytes = size_t(2) * N * kTC * sizeof(T);       // B, C
+  static constexpr size_t kBCBytes = size_t(2) * N * kBCPitch * sizeof(T);  // B, C
   // partial y of the state groups, [NG][CT] rows of kYPitch words: 4 words of padding after
   // every 32 steps and 2 after the row put the lanes of a half-warp in distinct banks
   static constexpr int kYPitch = kTC + kTC / 32 * 4 + 2;
@@ -112,12 +115,13 @@ struct ChunkCfg {
   static constexpr bool kSharedDelta = NG >= 4;
   static constexpr int kDPitch = kTC + 4;
   // With two lane groups per warp each group evaluates Delta, Delta*u for half of a lane's
-  // steps and the halves meet in a per-warp buffer [2][CPW*SPW][KI+4] (rows padded: distinct
-  // banks for the 8 lanes of a quarter-warp).
+  // steps and the halves meet in a per-warp buffer of float4: [2][KI/4][kXQ], one column per
+  // lane pair.  The row pitch kXQ (16 + 16/kVec float4) puts a half's writes from the two
+  // groups of a quarter-warp in distinct banks.
   static constexpr bool kLaneDelta = !kSharedDelta && kLG == 2 && KI / kVec == 2;
-  static constexpr int kXRow = KI + 4;
+  static constexpr int kXQ = CPW * SPW + 16 / kVec;
   static constexpr size_t kDBytes = kSharedDelta ? size_t(2) * kCT * kDPitch * sizeof(float)
-                                    : kLaneDelta ? size_t(kWarps) * 2 * (CPW * SPW) * kXRow * sizeof(float)
+                                    : kLaneDelta ? size_t(kWarps) * 2 * (KI / 4) * kXQ * 16
                                                  : 0;
   static constexpr int kNP = N + 1;         // row pitch of the per-(channel, state) arrays
   static constexpr size_t kParamBytes =
@@ -174,10 +178,13 @@ chunk_scan_kernel(const ScanArgs args) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int cw = warp % CW, g = warp / CW;        // channel warp, state group
   constexpr int LG = Cfg::kLG;
-  const int lg = lane / (CPW * SPW), lr = lane % (CPW * SPW);  // lane group, lane in group
+  // lane = (seg * CPW + cg) * LG + lg: the lane groups are interleaved, so a quarter-warp
+  // holds 8 / LG segments of every group
+  const int lg = lane % LG, lr = lane / LG;       // lane group, lane in group
   const int cg = lr % CPW, seg = lr / CPW;        // interleaved channel groups
   const int ch = cw * CPW + cg;
-  const int n0 = (g * LG + lg) * NS;
+  // this lane's states: nb, nb + LG, ..., nb + (NS - 1) * LG (the groups' states interleave)
+  const int nb = g * LG * NS + lg;
 
   if constexpr (VEC) {
     if (threadIdx.x == 0) {
@@ -315,7 +322,7 @@ chunk_scan_kernel(const ScanArgs args) {
         } else {
           const int r2 = r - nx * CT, which = r2 / N, n = r2 % N;
           const T *base = which == 0 ? SSM_GB : SSM_GC;
-          bulk_g2s(bdst + size_t(r2) * TC, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, row_bytes,
+          bulk_g2s(bdst + size_t(r2) * Cfg::kBCPitch, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, row_bytes,
                    &bars[buf]);
         }
       }
@@ -341,7 +348,7 @@ chunk_scan_kernel(const ScanArgs args) {
         const T *base = which == 0 ? SSM_GB : SSM_GC;
         T val = Elem<T>::from_f32(0.f);
         if (t < args.seqlen) val = base[bcbase + int64_t(n) * args.bc_state_stride + t];
-        bdst[size_t(row) * TC + j] = val;
+        bdst[size_t(row) * Cfg::kBCPitch + j] = val;
       }
     };
 
@@ -358,9 +365,9 @@ chunk_scan_kernel(const ScanArgs args) {
       for (int p = 0; p < KP; ++p) y[p] = make_float2(0.f, 0.f);
       if constexpr (Cfg::kLaneDelta) {
         // this lane group evaluates vector lg of the lane's KI steps; the other group the rest
-        constexpr int XR = Cfg::kXRow;
-        float *dlw = dls + size_t(warp) * 2 * (CPW * SPW) * XR + size_t(lr) * XR;
-        float *duw = dlw + (CPW * SPW) * XR;
+        // float4 q of the lane pair's Delta (rows 0 .. KI/4-1) and Delta*u (rows KI/4 ..)
+        constexpr int XQ = Cfg::kXQ, Q = KI / 4;
+        float4 *xw = reinterpret_cast<float4 *>(dls) + size_t(warp) * 2 * Q * XQ + lr;
         const T *ru = X + size_t(ch) * XP + tl0 + lg * V;
         const T *rd = X + size_t(CT + ch) * XP + tl0 + lg * V;
         const float bias = bias_s[ch];
@@ -389,15 +396,16 @@ chunk_scan_kernel(const ScanArgs args) {
               l4.z = dt.x; l4.w = dt.y; u4.z = uu.x; u4.w = uu.y;
             }
           }
-          *reinterpret_cast<float4 *>(dlw + lg * V + 2 * e) = l4;
-          *reinterpret_cast<float4 *>(duw + lg * V + 2 * e) = u4;
+          const int q = lg * (V / 4) + e / 2;
+          xw[q * XQ] = l4;
+          xw[(Q + q) * XQ] = u4;
         }
         __syncwarp();  // both halves written
         float2 ds = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q = 0; q < KI / 4; ++q) {
-          const float4 l4 = reinterpret_cast<const float4 *>(dlw)[q];
-          const float4 u4 = reinterpret_cast<const float4 *>(duw)[q];
+        for (int q = 0; q < Q; ++q) {
+          const float4 l4 = xw[q * XQ];
+          const float4 u4 = xw[(Q + q) * XQ];
           dl[2 * q] = make_float2(l4.x, l4.y);
           dl[2 * q + 1] = make_float2(l4.z, l4.w);
           du[2 * q] = make_float2(u4.x, u4.y);
@@ -477,8 +485,8 @@ chunk_scan_kernel(const ScanArgs args) {
         constexpr bool FWD = decltype(fwd_tag)::value, OUT = decltype(out_tag)::value;
         const float A2 = FWD ? A2s[ch * NP + n1] : 0.f;
         const float2 A22 = make_float2(A2, A2);
-        const T *rb = Bsm + size_t(n1) * TC + tl0;
-        const T *rc = Csm + size_t(n2) * TC + tl0;
+        const T *rb = Bsm + size_t(n1) * Cfg::kBCPitch + tl0;
+        const T *rc = Csm + size_t(n2) * Cfg::kBCPitch + tl0;
 #pragma unroll
         for (int lv = 0; lv < LV; ++lv) {
           float2 bb[V / 2], cc[V / 2];
@@ -520,15 +528,15 @@ chunk_scan_kernel(const ScanArgs args) {
         float P = ex2_approx(dsum * A2);  // product of the lane's a_i
 #pragma unroll
         for (int off = 1; off < SPW; off *= 2) {
-          const float Pu = __shfl_up_sync(0xffffffffu, P, off * CPW);
-          const float Gu = __shfl_up_sync(0xffffffffu, G, off * CPW);
+          const float Pu = __shfl_up_sync(0xffffffffu, P, off * CPW * LG);
+          const float Gu = __shfl_up_sync(0xffffffffu, G, off * CPW * LG);
           if (seg >= off) {
             G = fmaf(P, Gu, G);
             P *= Pu;
           }
         }
-        float Pe = __shfl_up_sync(0xffffffffu, P, CPW);
-        float Ge = __shfl_up_sync(0xffffffffu, G, CPW);
+        float Pe = __shfl_up_sync(0xffffffffu, P, CPW * LG);
+        float Ge = __shfl_up_sync(0xffffffffu, G, CPW * LG);
         if (seg == 0) {
           Pe = 1.f;
           Ge = 0.f;
@@ -541,15 +549,15 @@ chunk_scan_kernel(const ScanArgs args) {
         using yes = std::true_type;
         using no = std::false_type;
         float G = 0.f, h = 0.f;
-        steps(yes{}, no{}, n0, n0, G, h);
-        h = scan_state(n0, G);
+        steps(yes{}, no{}, nb, nb, G, h);
+        h = scan_state(nb, G);
 #pragma unroll 1
-        for (int n = n0 + 1; n < n0 + NS; ++n) {
+        for (int n = nb + LG; n < nb + NS * LG; n += LG) {
           G = 0.f;
-          steps(yes{}, yes{}, n, n - 1, G, h);
+          steps(yes{}, yes{}, n, n - LG, G, h);
           h = scan_state(n, G);
         }
-        steps(no{}, yes{}, n0 + NS - 1, n0 + NS - 1, G, h);
+        steps(no{}, yes{}, nb + (NS - 1) * LG, nb + (NS - 1) * LG, G, h);
       }
 
       // ---- epilogue: sum of the state groups, skip term, gate, store ----
@@ -562,11 +570,11 @@ chunk_scan_kernel(const ScanArgs args) {
 #pragma unroll
         for (int i = 0; i < KI; ++i) yo[i] = (i & 1) ? y[i / 2].y : y[i / 2].x;
       } else if constexpr (LG > 1) {
-        // sum over the lane groups (lanes lr + k * CPW * SPW), then keep this group's slice
+        // sum over the lane groups (lanes lr * LG + k), then keep this group's slice
 #pragma unroll
         for (int p = 0; p < KP; ++p) {
 #pragma unroll
-          for (int off = CPW * SPW; off < 32; off *= 2) {
+          for (int off = 1; off < LG; off *= 2) {
             y[p].x += __shfl_xor_sync(0xffffffffu, y[p].x, off);
             y[p].y += __shfl_xor_sync(0xffffffffu, y[p].y, off);
           }
@@ -667,7 +675,7 @@ chunk_scan_kernel(const ScanArgs args) {
       const int rel_hi = int(min64(t_hi - wstart, TC + 1));
       const T *X = xs0 + buf * kXElems;
       const T *Bsm = bc0 + buf * kBCElems;
-      const T *Csm = Bsm + size_t(N) * TC;
+      const T *Csm = Bsm + size_t(N) * Cfg::kBCPitch;
       if (rel_lo <= 0 && rel_hi >= TC)
         compute_chunk(std::false_type{}, X, Bsm, Csm, wstart, rel_lo, rel_hi);
       else
