@@ -126,12 +126,20 @@ struct ChunkCfg {
   static constexpr int kNP = N + 1;         // row pitch of the per-(channel, state) arrays
   static constexpr size_t kParamBytes =
       size_t(2) * kCT * kNP * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
-  static constexpr size_t kSmemBytes = 2 * kXBytes + 2 * kBCBytes + kYBytes + kDBytes + kParamBytes;
+  // 16-bit B/C of the wide N=16 tile are widened to float32 once per chunk (double-buffered
+  // [2][2][N][TC]), so the state loop loads them without converting; their 16-bit copies
+  // then need a single staging buffer (a chunk's copy lands after the previous one was
+  // widened).
+  static constexpr bool kBF = sizeof(T) == 2 && N == 16 && kLG == 1 && NG == 1;
+  static constexpr size_t kBCAll = (kBF ? 1 : 2) * kBCBytes;  // 16-bit B/C staging
+  static constexpr size_t kBFBytes = kBF ? size_t(2) * 2 * N * kTC * sizeof(float) : 0;
+  static constexpr size_t kSmemBytes = 2 * kXBytes + kBCAll + kYBytes + kDBytes + kBFBytes + kParamBytes;
   static_assert(KI % 4 == 0 && KI % kVec == 0, "a lane's steps must be whole 16-byte vectors");
   static_assert(32 % (CPW * SPW) == 0, "lane split");
   static_assert(kLG == 1 || NG == 1, "states split either across warps or inside a warp");
   static_assert(N % (NG * kLG) == 0 && KI % (NG * kLG) == 0, "state / step split");
   static_assert(kXBytes % 16 == 0 && kBCBytes % 16 == 0, "16-byte aligned buffers");
+  static_assert(!kBF || kBCPitch == kTC, "widened B/C rows are unpadded");
 };
 
 template <typename T, typename TO, int N, int KI, int SPW, int CPW, int CW, int NG, bool HAS_Z, bool VEC,
@@ -150,13 +158,16 @@ chunk_scan_kernel(const ScanArgs args) {
   extern __shared__ __align__(16) unsigned char smem[];
   T *const xs0 = reinterpret_cast<T *>(smem);                     // [2][3][CT][XP]
   T *const bc0 = reinterpret_cast<T *>(smem + 2 * Cfg::kXBytes);  // [2][2][N][TC]
-  float *ypart = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes);  // [NG][CT][YP]
+  float *ypart = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + Cfg::kBCAll);  // [NG][CT][YP]
   // [CT][N] arrays use a row pitch of N + 1 words, so the channels of a warp hit distinct banks
   constexpr int NP = Cfg::kNP;
-  float *dls = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes);  // [2][CT][DP]
+  float *dls = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + Cfg::kBCAll + Cfg::kYBytes);  // [2][CT][DP]
   constexpr int DP = Cfg::kDPitch;
-  float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + 2 * Cfg::kBCBytes + Cfg::kYBytes +
-                                         Cfg::kDBytes);  // [CT][NP]
+  float *const bcf = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + Cfg::kBCAll + Cfg::kYBytes +
+                                               Cfg::kDBytes);  // [2][2][N][TC] (kBF only)
+  constexpr size_t kBFElems = size_t(2) * N * TC;
+  float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + Cfg::kBCAll + Cfg::kYBytes +
+                                         Cfg::kDBytes + Cfg::kBFBytes);  // [CT][NP]
   float *carry_s = A2s + CT * NP;                                 // [CT][NP]
   float *Dsk = carry_s + CT * NP;                                 // [CT]
   float *bias_s = Dsk + CT;                                       // [CT]
@@ -309,7 +320,7 @@ chunk_scan_kernel(const ScanArgs args) {
       const int64_t wend = min64(wstart + TC, seqlen_r);
       const uint32_t row_bytes = uint32_t((wend - wstart) * int64_t(sizeof(T)));
       T *xdst = xs0 + buf * kXElems;
-      T *bdst = bc0 + buf * kBCElems;
+      T *bdst = bc0 + (Cfg::kBF ? 0 : buf * kBCElems);
       fence_proxy_async_smem();
       if (threadIdx.x == 0) mbar_arrive_expect_tx(&bars[buf], row_bytes * uint32_t(nx * nvalid_ch + 2 * N));
       for (int r = threadIdx.x; r < nx * CT + 2 * N; r += NT) {
@@ -348,14 +359,17 @@ chunk_scan_kernel(const ScanArgs args) {
         const T *base = which == 0 ? SSM_GB : SSM_GC;
         T val = Elem<T>::from_f32(0.f);
         if (t < args.seqlen) val = base[bcbase + int64_t(n) * args.bc_state_stride + t];
-        bdst[size_t(row) * Cfg::kBCPitch + j] = val;
+        if constexpr (Cfg::kBF)
+          bcf[buf * kBFElems + size_t(row) * TC + j] = Elem<T>::to_f32(val);
+        else
+          bdst[size_t(row) * Cfg::kBCPitch + j] = val;
       }
     };
 
     // One chunk of the lane's work; the masked instance handles chunks that straddle a
     // sequence end.
-    auto compute_chunk = [&](auto masked_tag, const T *X, const T *Bsm, const T *Csm, int64_t wstart, int rel_lo,
-                             int rel_hi) {
+    auto compute_chunk = [&](auto masked_tag, const T *X, const T *Bsm, const T *Csm, const float *Bf, int64_t wstart,
+                             int rel_lo, int rel_hi) {
       constexpr bool kMasked = decltype(masked_tag)::value;
       const int tl0 = seg * KI;  // chunk-local first step of this lane
       // ---- prologue: Delta and Delta*u for the lane's KI steps (as pairs of steps) ----
@@ -485,13 +499,29 @@ chunk_scan_kernel(const ScanArgs args) {
         constexpr bool FWD = decltype(fwd_tag)::value, OUT = decltype(out_tag)::value;
         const float A2 = FWD ? A2s[ch * NP + n1] : 0.f;
         const float2 A22 = make_float2(A2, A2);
-        const T *rb = Bsm + size_t(n1) * Cfg::kBCPitch + tl0;
-        const T *rc = Csm + size_t(n2) * Cfg::kBCPitch + tl0;
+        [[maybe_unused]] const T *rb = Bsm + size_t(n1) * Cfg::kBCPitch + tl0;
+        [[maybe_unused]] const T *rc = Csm + size_t(n2) * Cfg::kBCPitch + tl0;
+        [[maybe_unused]] const float4 *rbf = reinterpret_cast<const float4 *>(Bf + size_t(n1) * TC + tl0);
+        [[maybe_unused]] const float4 *rcf = reinterpret_cast<const float4 *>(Bf + size_t(N + n2) * TC + tl0);
+        // V/2 step pairs of float32 B (or C) from shared memory
+        auto ldf = [](const float4 *q, float2 (&o)[V / 2]) {
+#pragma unroll
+          for (int k = 0; k < V / 4; ++k) {
+            const float4 v = q[k];
+            o[2 * k] = make_float2(v.x, v.y);
+            o[2 * k + 1] = make_float2(v.z, v.w);
+          }
+        };
 #pragma unroll
         for (int lv = 0; lv < LV; ++lv) {
           float2 bb[V / 2], cc[V / 2];
-          if constexpr (FWD) unpack16x2<T>(*reinterpret_cast<const uint4 *>(rb + lv * V), bb);
-          if constexpr (OUT) unpack16x2<T>(*reinterpret_cast<const uint4 *>(rc + lv * V), cc);
+          if constexpr (Cfg::kBF) {
+            if constexpr (FWD) ldf(rbf + lv * (V / 4), bb);
+            if constexpr (OUT) ldf(rcf + lv * (V / 4), cc);
+          } else {
+            if constexpr (FWD) unpack16x2<T>(*reinterpret_cast<const uint4 *>(rb + lv * V), bb);
+            if constexpr (OUT) unpack16x2<T>(*reinterpret_cast<const uint4 *>(rc + lv * V), cc);
+          }
 #pragma unroll
           for (int e = 0; e < V / 2; ++e) {
             const int p = lv * (V / 2) + e;
@@ -663,6 +693,18 @@ chunk_scan_kernel(const ScanArgs args) {
       const int64_t wstart = w0 + int64_t(c) * TC;
       if constexpr (VEC) {
         mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
+        if constexpr (Cfg::kBF) {
+          // widen the chunk's 16-bit B/C (the single staging copy) into its float32 buffer
+          float *dst = bcf + buf * kBFElems;
+          for (int i = threadIdx.x; i < 2 * N * TC / V; i += NT) {
+            float f[V];
+            unpack16<T>(*reinterpret_cast<const uint4 *>(bc0 + size_t(i) * V), f);
+#pragma unroll
+            for (int k = 0; k < V / 4; ++k)
+              reinterpret_cast<float4 *>(dst + size_t(i) * V)[k] =
+                  make_float4(f[4 * k], f[4 * k + 1], f[4 * k + 2], f[4 * k + 3]);
+          }
+        }
       } else {
         stage_scalar(buf, c);
       }
@@ -676,10 +718,11 @@ chunk_scan_kernel(const ScanArgs args) {
       const T *X = xs0 + buf * kXElems;
       const T *Bsm = bc0 + buf * kBCElems;
       const T *Csm = Bsm + size_t(N) * Cfg::kBCPitch;
+      const float *Bf = bcf + buf * kBFElems;
       if (rel_lo <= 0 && rel_hi >= TC)
-        compute_chunk(std::false_type{}, X, Bsm, Csm, wstart, rel_lo, rel_hi);
+        compute_chunk(std::false_type{}, X, Bsm, Csm, Bf, wstart, rel_lo, rel_hi);
       else
-        compute_chunk(std::true_type{}, X, Bsm, Csm, wstart, rel_lo, rel_hi);
+        compute_chunk(std::true_type{}, X, Bsm, Csm, Bf, wstart, rel_lo, rel_hi);
     }
 
     // ------------------------------------------------------------- hand the state on
