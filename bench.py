@@ -17,6 +17,7 @@ import ctypes
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -48,11 +49,16 @@ def peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the CUDA sources with comments and blank lines removed (a comment edit keeps
+    the committed ncu counters valid; any code change invalidates them)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_15_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+        h.update(name.encode() + "\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()[:16]
 
 

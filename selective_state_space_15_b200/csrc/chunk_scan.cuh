@@ -14,15 +14,17 @@
 // No h_t ever leaves registers; only y and the final state are written.  Each exponential
 // exp(Delta A) is evaluated once.
 //
-// Lanes are interleaved: lane = seg * CPW + cg.  The CPW channel groups of an 8-lane
-// shared-memory phase therefore read the same B/C words (broadcast), and the distinct
-// segments of a phase hit distinct banks.
+// Lanes are interleaved: lane = (seg * CPW + cg) * LG + lg.  The CPW channel groups of an
+// 8-lane shared-memory phase therefore read the same B/C words (broadcast), and the distinct
+// segments of a phase hit distinct banks; with LG = 2 lane groups (which take alternate
+// states) a phase holds 4 segments of both groups, whose rows sit 16 bytes apart in banks.
 //
 // Staging.  The u, delta, z rows of the tile and the B, C rows of the chunk window are copied
 // into shared memory (double-buffered) while the previous chunk is computed: one TMA bulk
 // copy per row (cp.async.bulk completing on an mbarrier) when every row is 16-byte aligned,
-// element-wise loads otherwise.  B and C stay in the input dtype in shared memory (a bf16
-// value is widened in a register when used), which halves their shared-memory traffic.
+// element-wise loads otherwise.  In the wide N=16 tile 16-bit B and C are widened to float32
+// once per chunk by the whole CTA (shared by its 32 channels); the other tiles keep them in
+// the input dtype in shared memory and widen a value in a register when it is used.
 // u/delta/z rows are padded by 16 bytes so that the channel groups of a phase read
 // different banks.  Chunks that lie entirely inside the sequence skip all masking.
 //
