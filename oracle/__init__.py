@@ -14,7 +14,9 @@ Definitions followed (cited by page title and section; see ``ssm_oracle.c`` for 
     y_t = C_t h_t;
   * discosf.com "企业官网建设流程全解析" §1.1 (skip term D x) and §1.3 (Δ = softplus(·));
   * ufo.work §4.2 -- packed sequences restart from h = 0 at each cu_seqlens boundary;
-  * ufo.work §4.1 -- single-token update of a persistent per-request state.
+  * ufo.work §4.1 -- single-token update of a persistent per-request state;
+  * discosf.com §1.2 -- the zero-order-hold input matrix Bbar = (ΔA)^-1 (exp(ΔA) - I) ΔB,
+    chosen with ``zoh=True`` (default: Bbar = ΔB).
 """
 from __future__ import annotations
 
@@ -52,11 +54,11 @@ def _load():
             lib = ctypes.CDLL(build())
             P = ctypes.c_void_p
             I = ctypes.c_int64
-            lib.oracle_scan.argtypes = [I, I, I, I] + [P] * 13 + [ctypes.c_int]
+            lib.oracle_scan.argtypes = [I, I, I, I] + [P] * 13 + [ctypes.c_int, ctypes.c_int]
             lib.oracle_scan.restype = ctypes.c_int
-            lib.oracle_scan_varlen.argtypes = [I, I, I] + [P] * 8 + [P, I] + [P] * 4 + [ctypes.c_int]
+            lib.oracle_scan_varlen.argtypes = [I, I, I] + [P] * 8 + [P, I] + [P] * 4 + [ctypes.c_int, ctypes.c_int]
             lib.oracle_scan_varlen.restype = ctypes.c_int
-            lib.oracle_state_update.argtypes = [I, I, I, P, P, P, I] + [P] * 9
+            lib.oracle_state_update.argtypes = [I, I, I, P, P, P, I] + [P] * 10 + [ctypes.c_int]
             lib.oracle_state_update.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -76,7 +78,7 @@ def default_threads() -> int:
     return max(1, os.cpu_count() or 1)
 
 
-def scan(u, delta, B, C, A, Dskip=None, bias=None, z=None, h0=None, nthreads: int = 1):
+def scan(u, delta, B, C, A, Dskip=None, bias=None, z=None, h0=None, nthreads: int = 1, zoh: bool = False):
     """Fixed-length batch scan.
 
     u, delta, z: [batch, dim, L]; B, C: [batch, N, L]; A: [dim, N]; Dskip, bias: [dim];
@@ -84,6 +86,7 @@ def scan(u, delta, B, C, A, Dskip=None, bias=None, z=None, h0=None, nthreads: in
     B, C may also be [batch, G, N, L]: G groups of dim/G consecutive channels, each group
     with its own B and C (channels are independent, ufo.work page §3.2, so a grouped scan is
     the scan of each group's channels with that group's B and C).
+    ``zoh``: zero-order-hold input matrix instead of Bbar = Δ B.
     Returns dict with y [batch, dim, L], h_last [batch, dim, N] and the magnitudes
     y_mag, h_mag used to scale errors.
     """
@@ -97,7 +100,7 @@ def scan(u, delta, B, C, A, Dskip=None, bias=None, z=None, h0=None, nthreads: in
             sl = slice(g * dg, (g + 1) * dg)
             sub = lambda x, ax=1: None if x is None else np.asarray(x)[(slice(None),) * ax + (sl,)]  # noqa: E731
             parts.append(scan(sub(u), sub(delta), np.asarray(B)[:, g], np.asarray(C)[:, g], np.asarray(A)[sl],
-                              sub(Dskip, 0), sub(bias, 0), sub(z), sub(h0), nthreads=nthreads))
+                              sub(Dskip, 0), sub(bias, 0), sub(z), sub(h0), nthreads=nthreads, zoh=zoh))
         return {k: np.concatenate([r[k] for r in parts], axis=1) for k in parts[0]}
     u, delta, B, C, A = (_f64(x) for x in (u, delta, B, C, A))
     z, Dskip, bias, h0 = (_f64(x) for x in (z, Dskip, bias, h0))
@@ -115,13 +118,14 @@ def scan(u, delta, B, C, A, Dskip=None, bias=None, z=None, h0=None, nthreads: in
     h_mag = np.empty_like(h_last)
     rc = _load().oracle_scan(batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C),
                              _ptr(A), _ptr(Dskip), _ptr(bias), _ptr(h0), _ptr(y), _ptr(h_last),
-                             _ptr(y_mag), _ptr(h_mag), int(nthreads))
+                             _ptr(y_mag), _ptr(h_mag), int(bool(zoh)), int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_scan rejected its arguments (code {rc})")
     return {"y": y, "h_last": h_last, "y_mag": y_mag, "h_mag": h_mag}
 
 
-def scan_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, bias=None, z=None, nthreads: int = 1):
+def scan_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, bias=None, z=None, nthreads: int = 1,
+                zoh: bool = False):
     """Packed varlen scan. u, delta, z: [dim, T]; B, C: [N, T] (or [G, N, T]: channel groups as
     in scan()); cu_seqlens: [nseq+1].
 
@@ -137,7 +141,7 @@ def scan_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, bias=None, z=None, nt
             sl = slice(g * dg, (g + 1) * dg)
             sub = lambda x: None if x is None else np.asarray(x)[sl]  # noqa: E731
             parts.append(scan_varlen(sub(u), sub(delta), np.asarray(B)[g], np.asarray(C)[g], np.asarray(A)[sl],
-                                     cu_seqlens, sub(Dskip), sub(bias), sub(z), nthreads=nthreads))
+                                     cu_seqlens, sub(Dskip), sub(bias), sub(z), nthreads=nthreads, zoh=zoh))
         return {"y": np.concatenate([r["y"] for r in parts], axis=0),
                 "y_mag": np.concatenate([r["y_mag"] for r in parts], axis=0),
                 "h_last": np.concatenate([r["h_last"] for r in parts], axis=1),
@@ -155,14 +159,14 @@ def scan_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, bias=None, z=None, nt
     h_mag = np.empty_like(h_last)
     rc = _load().oracle_scan_varlen(dim, N, T, _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C),
                                     _ptr(A), _ptr(Dskip), _ptr(bias), _ptr(cu), nseq, _ptr(y),
-                                    _ptr(h_last), _ptr(y_mag), _ptr(h_mag), int(nthreads))
+                                    _ptr(h_last), _ptr(y_mag), _ptr(h_mag), int(bool(zoh)), int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_scan_varlen rejected its arguments (code {rc})")
     return {"y": y, "h_last": h_last, "y_mag": y_mag, "h_mag": h_mag}
 
 
 def scan_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=None, bias=None, z=None,
-                     pool_mag=None, nthreads: int = 1):
+                     pool_mag=None, nthreads: int = 1, zoh: bool = False):
     """Packed prefill into a state pool, in place on ``pool`` (float64 [S, dim, N]).
 
     The serving flow of the ufo.work page's second article, §4.2 (a prompt is prefilled in
@@ -189,7 +193,7 @@ def scan_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=None, 
         h0 = pool[slot][None] if ok else np.zeros((1, dim, N))
         col = slice(lo, hi)
         r = scan(u[None, :, col], delta[None, :, col], B[None, :, col], C[None, :, col], A, Dskip, bias,
-                 None if z is None else z[None, :, col], h0, nthreads=nthreads)
+                 None if z is None else z[None, :, col], h0, nthreads=nthreads, zoh=zoh)
         y[:, col] = r["y"][0]
         y_mag[:, col] = r["y_mag"][0]
         if pool_mag is not None and ok:
@@ -199,7 +203,7 @@ def scan_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=None, 
             excess = np.maximum(pool_mag[slot] - np.abs(pool[slot]), 0.0)[None]
             r_ex = scan(np.zeros((1, dim, hi - lo)), delta[None, :, col], np.zeros((1, N, hi - lo)),
                         C[None, :, col], A, None, bias, None if z is None else z[None, :, col], excess,
-                        nthreads=nthreads)
+                        nthreads=nthreads, zoh=zoh)
             y_mag[:, col] += r_ex["y_mag"][0]
             pool_mag[slot] = r["h_mag"][0] + r_ex["h_mag"][0]
         if ok:
@@ -207,7 +211,8 @@ def scan_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=None, 
     return {"y": y, "y_mag": y_mag}
 
 
-def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, bias=None, z=None, pool_mag=None):
+def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, bias=None, z=None, pool_mag=None,
+                 zoh: bool = False):
     """One decode step, in place on ``pool`` (float64 array [S, dim, N]).
 
     slot_ids: [R]; u, delta, z: [R, dim]; B, C: [R, N].  ``pool_mag`` (same shape as pool, or
@@ -226,7 +231,7 @@ def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, bias=None, z=Non
     y_mag = np.empty_like(y)
     rc = _load().oracle_state_update(S, dim, N, _ptr(pool), _ptr(pool_mag), _ptr(ids), R, _ptr(u),
                                      _ptr(delta), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(Dskip),
-                                     _ptr(bias), _ptr(y), _ptr(y_mag))
+                                     _ptr(bias), _ptr(y), _ptr(y_mag), int(bool(zoh)))
     if rc != 0:
         raise ValueError(f"oracle_state_update rejected its arguments (code {rc})")
     return {"y": y, "y_mag": y_mag}

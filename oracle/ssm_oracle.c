@@ -17,6 +17,9 @@
  *     zero at every sequence start (cu_seqlens boundaries).
  *   - ufo.work page §4.1 / its second article §4.1: a one-token state update over a persistent
  *     state pool indexed per request.
+ *   - discosf.com §1.2 (and ufo.work §1.1, "or by a zero-order hold"): the zero-order-hold
+ *     input matrix Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B, selected per call
+ *     (zoh != 0) instead of Bbar = Delta B.
  * Readings where the pages are silent: the bias sits inside the softplus; the optional SiLU(z)
  * gate multiplies the whole output C h + D u and never feeds back into h; y uses h_t (not h_{t-1}).
  *
@@ -25,7 +28,7 @@
  * chunking and no reassociation.  Threads (optional) only split independent channels.
  *
  * Alongside each result the oracle runs an absolute-value recursion
- *   habs_t = Abar_t habs_{t-1} + |Delta_t B_t u_t|       (habs_{-1} = |h0|)
+ *   habs_t = Abar_t habs_{t-1} + |Bbar_t u_t|            (habs_{-1} = |h0|)
  *   ymag_t = |g(z_t)| (sum_n |C_t[n]| habs_t[n] + |D u_t|)
  * which bounds |h| and |y| from above; tests divide errors by these magnitudes.
  *
@@ -49,10 +52,21 @@ static double softplus(double x) { return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(
 /* SiLU(z) = z * sigmoid(z) = z / (1 + e^-z). */
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
+/* Input coefficient of one step for one (channel, state): Bbar_t[n] = coef * B_t[n].
+ * Euler (ufo.work §1.1): coef = Delta.  Zero-order hold (discosf.com §1.2): A is diagonal, so
+ * (Delta A)^-1 (exp(Delta A) - 1) Delta is the scalar expm1(x) / x * Delta with x = Delta A;
+ * at x = 0 (A = 0 or Delta = 0) the quotient is 1. */
+static double input_coef(int zoh, double dt, double a) {
+  if (!zoh) return dt;
+  const double x = dt * a;
+  return x == 0.0 ? dt : expm1(x) / x * dt;
+}
+
 /* One channel of one sequence.  u, delta, z, y point at the channel's row (stride 1 in time);
  * B and C point at the sequence's block, one row per state index, row stride bc_stride. */
 typedef struct {
   int64_t dstate, len, bc_stride;
+  int zoh;                                 /* nonzero: zero-order-hold Bbar */
   const double *u, *delta, *z, *B, *C, *A; /* A: this channel's dstate values */
   double dskip, bias;
   const double *h0;                        /* dstate values or NULL */
@@ -73,7 +87,7 @@ static void scan_channel(const chan_job *j) {
     double acc = 0.0, acc_abs = 0.0;
     for (int64_t n = 0; n < N; ++n) {
       const double abar = exp(dt * j->A[n]);                   /* Abar = exp(Delta A) */
-      const double bx = dt * j->B[n * j->bc_stride + t] * ut;  /* Bbar x = Delta B u  */
+      const double bx = input_coef(j->zoh, dt, j->A[n]) * j->B[n * j->bc_stride + t] * ut; /* Bbar x */
       h[n] = abar * h[n] + bx;                                 /* h_t = Abar h_{t-1} + Bbar x_t */
       ha[n] = abar * ha[n] + fabs(bx);
       const double c = j->C[n * j->bc_stride + t];
@@ -131,7 +145,7 @@ int oracle_scan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
                 const double *u, const double *delta, const double *z,
                 const double *B, const double *C, const double *A,
                 const double *Dskip, const double *bias, const double *h0,
-                double *y, double *h_last, double *y_mag, double *h_mag, int nthreads) {
+                double *y, double *h_last, double *y_mag, double *h_mag, int zoh, int nthreads) {
   if (batch < 0 || dim < 0 || dstate <= 0 || seqlen < 0) return 1;
   const int64_t njobs = batch * dim;
   chan_job *jobs = (chan_job *)calloc((size_t)(njobs > 0 ? njobs : 1), sizeof(chan_job));
@@ -139,7 +153,7 @@ int oracle_scan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
     for (int64_t d = 0; d < dim; ++d) {
       chan_job *j = &jobs[b * dim + d];
       const int64_t xo = (b * dim + d) * seqlen, so = (b * dim + d) * dstate;
-      j->dstate = dstate; j->len = seqlen; j->bc_stride = seqlen;
+      j->dstate = dstate; j->len = seqlen; j->bc_stride = seqlen; j->zoh = zoh;
       j->u = u + xo; j->delta = delta + xo; j->z = z ? z + xo : NULL;
       j->B = B + b * dstate * seqlen; j->C = C + b * dstate * seqlen;
       j->A = A + d * dstate;
@@ -159,7 +173,7 @@ int oracle_scan_varlen(int64_t dim, int64_t dstate, int64_t total,
                        const double *B, const double *C, const double *A,
                        const double *Dskip, const double *bias,
                        const int64_t *cu_seqlens, int64_t nseq,
-                       double *y, double *h_last, double *y_mag, double *h_mag, int nthreads) {
+                       double *y, double *h_last, double *y_mag, double *h_mag, int zoh, int nthreads) {
   if (dim < 0 || dstate <= 0 || total < 0 || nseq < 0) return 1;
   if (cu_seqlens[0] != 0 || cu_seqlens[nseq] != total) return 2;
   for (int64_t s = 0; s < nseq; ++s)
@@ -170,7 +184,7 @@ int oracle_scan_varlen(int64_t dim, int64_t dstate, int64_t total,
     for (int64_t d = 0; d < dim; ++d) {
       chan_job *j = &jobs[s * dim + d];
       const int64_t t0 = cu_seqlens[s], xo = d * total + t0, so = (s * dim + d) * dstate;
-      j->dstate = dstate; j->len = cu_seqlens[s + 1] - t0; j->bc_stride = total;
+      j->dstate = dstate; j->len = cu_seqlens[s + 1] - t0; j->bc_stride = total; j->zoh = zoh;
       j->u = u + xo; j->delta = delta + xo; j->z = z ? z + xo : NULL;
       j->B = B + t0; j->C = C + t0;
       j->A = A + d * dstate;
@@ -192,7 +206,7 @@ int oracle_state_update(int64_t num_slots, int64_t dim, int64_t dstate,
                         const double *u, const double *delta, const double *z,
                         const double *B, const double *C, const double *A,
                         const double *Dskip, const double *bias,
-                        double *y, double *y_mag) {
+                        double *y, double *y_mag, int zoh) {
   if (num_slots < 0 || dim < 0 || dstate <= 0 || R < 0) return 1;
   for (int64_t r = 0; r < R; ++r)
     if (slot_ids[r] < 0 || slot_ids[r] >= num_slots) return 4;
@@ -206,7 +220,7 @@ int oracle_state_update(int64_t num_slots, int64_t dim, int64_t dstate,
       double acc = 0.0, acc_abs = 0.0;
       for (int64_t n = 0; n < dstate; ++n) {
         const double abar = exp(dt * A[d * dstate + n]);
-        const double bx = dt * B[r * dstate + n] * ut;
+        const double bx = input_coef(zoh, dt, A[d * dstate + n]) * B[r * dstate + n] * ut;
         h[n] = abar * h[n] + bx;
         const double hm = ha ? (ha[n] = abar * ha[n] + fabs(bx)) : fabs(h[n]);
         const double c = C[r * dstate + n];

@@ -391,3 +391,78 @@ def test_grouped_varlen_matches_grouped_fixed_length_per_sequence():
                         inp.Dskip, inp.bias, inp.z[None, :, sl])
         np.testing.assert_array_equal(v["y"][:, sl], f["y"][0])
         np.testing.assert_array_equal(v["h_last"][s], f["h_last"][0])
+
+
+# ---- zero-order hold (discosf.com §1.2: Bbar = (Δ A)^-1 (exp(Δ A) - I) Δ B) ----
+
+def _zoh_exact_reference(p):
+    """The continuous system h' = A h + B u with u and B held over each step of length Δ, solved
+    exactly per (channel, state) by the matrix exponential of the augmented system
+    [[A, B u], [0, 0]] Δ (scipy's Padé expm; independent of the oracle's closed form)."""
+    from scipy.linalg import expm
+    b, D, L = p["u"].shape
+    N = p["A"].shape[1]
+    h = p["h0"].copy() if p["h0"] is not None else np.zeros((b, D, N))
+    y = np.zeros((b, D, L))
+    for bb in range(b):
+        for d in range(D):
+            for t in range(L):
+                dt = np.logaddexp(0.0, p["delta"][bb, d, t] + p["bias"][d])
+                acc = 0.0
+                for n in range(N):
+                    M = np.array([[p["A"][d, n], p["B"][bb, n, t] * p["u"][bb, d, t]], [0.0, 0.0]]) * dt
+                    h[bb, d, n] = (expm(M) @ np.array([h[bb, d, n], 1.0]))[0]
+                    acc += p["C"][bb, n, t] * h[bb, d, n]
+                yt = acc + p["Dskip"][d] * p["u"][bb, d, t]
+                if p["z"] is not None:
+                    zz = p["z"][bb, d, t]
+                    yt *= zz / (1.0 + np.exp(-zz))
+                y[bb, d, t] = yt
+    return y, h
+
+
+@pytest.mark.parametrize("seed,A_range", [(90, (0.2, 3.0)), (91, (1e-4, 0.05)), (92, (2.0, 40.0))])
+def test_zoh_step_is_the_exact_ode_solution(seed, A_range):
+    rng = np.random.default_rng(seed)
+    p = _rand_problem(rng, 2, 3, 4, 7, A_range=A_range)
+    out = oracle.scan(p["u"], p["delta"], p["B"], p["C"], p["A"], p["Dskip"], p["bias"], p["z"], p["h0"], zoh=True)
+    y_ref, h_ref = _zoh_exact_reference(p)
+    np.testing.assert_allclose(out["y"], y_ref, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(out["h_last"], h_ref, rtol=1e-11, atol=1e-12)
+    # and it is not the Euler input matrix
+    eul = oracle.scan(p["u"], p["delta"], p["B"], p["C"], p["A"], p["Dskip"], p["bias"], p["z"], p["h0"])
+    assert np.abs(eul["h_last"] - h_ref).max() > 1e-6
+
+
+def test_zoh_with_A_zero_is_euler():
+    rng = np.random.default_rng(93)
+    p = _rand_problem(rng, 1, 3, 4, 9)
+    p["A"][:] = 0.0
+    a = oracle.scan(p["u"], p["delta"], p["B"], p["C"], p["A"], p["Dskip"], p["bias"], p["z"], p["h0"], zoh=True)
+    e = oracle.scan(p["u"], p["delta"], p["B"], p["C"], p["A"], p["Dskip"], p["bias"], p["z"], p["h0"])
+    assert np.array_equal(a["y"], e["y"]) and np.array_equal(a["h_last"], e["h_last"])
+
+
+def test_zoh_varlen_and_decode_agree_with_the_fixed_length_scan():
+    rng = np.random.default_rng(94)
+    D, N = 3, 4
+    lengths = [5, 0, 3, 8]
+    T = sum(lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    p = _rand_problem(rng, 1, D, N, T, h0=False)
+    v = oracle.scan_varlen(p["u"][0], p["delta"][0], p["B"][0], p["C"][0], p["A"], cu, p["Dskip"], p["bias"],
+                           p["z"][0], zoh=True)
+    pool = np.zeros((len(lengths), D, N))
+    for i, (lo, hi) in enumerate(zip(cu[:-1], cu[1:])):
+        sl = slice(lo, hi)
+        r = oracle.scan(p["u"][:, :, sl], p["delta"][:, :, sl], p["B"][:, :, sl], p["C"][:, :, sl], p["A"],
+                        p["Dskip"], p["bias"], p["z"][:, :, sl], zoh=True)
+        np.testing.assert_allclose(v["y"][:, sl], r["y"][0], rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(v["h_last"][i], r["h_last"][0], rtol=1e-13, atol=1e-14)
+        # the same sequence token by token through the decode step
+        for t in range(lo, hi):
+            dec = oracle.state_update(pool, [i], p["u"][0, :, t][None], p["delta"][0, :, t][None],
+                                      p["B"][0, :, t][None], p["C"][0, :, t][None], p["A"], p["Dskip"], p["bias"],
+                                      p["z"][0, :, t][None], zoh=True)
+            np.testing.assert_allclose(dec["y"][0], v["y"][:, t], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(pool[i], v["h_last"][i], rtol=1e-12, atol=1e-13)
