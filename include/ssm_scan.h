@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 3
+#define SSM_ABI_VERSION 4
 
 typedef enum {
   SSM_OK = 0,
@@ -64,6 +64,16 @@ typedef enum {
 } ssm_status_t;
 
 typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
+
+/*
+ * Discretisation of the input matrix (A is diagonal: one value per (channel, state)).
+ *   SSM_DISC_EULER: Bbar = Delta B ("会议长序列建模…" page, ufo.work, §1.1); the default.
+ *   SSM_DISC_ZOH:   zero-order hold, Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B
+ *                   ("企业官网建设流程全解析" page, discosf.com, §1.2), i.e. (exp(Delta A) - 1) / A * B
+ *                   per (channel, state), and Delta B where A = 0.
+ * Abar = exp(Delta A) in both.
+ */
+typedef enum { SSM_DISC_EULER = 0, SSM_DISC_ZOH = 1 } ssm_discretization_t;
 
 /* Opaque CUDA stream handle; pass a cudaStream_t (they are the same pointer type). */
 typedef struct CUstream_st *ssm_stream_t;
@@ -116,6 +126,7 @@ typedef struct ssm_scan_params {
   float *h_last;
   int64_t ngroups;         /* channel groups with their own B, C: 0 or 1 = one group (scans)    */
   int64_t bc_group_stride; /* 0 -> dstate * bc_state_stride                                    */
+  int32_t discretization;  /* ssm_discretization_t; other values -> SSM_ERR_INVALID_ARG (all calls) */
 } ssm_scan_params;
 
 /*

@@ -15,7 +15,8 @@ SSM_OK = 0
 _STATUS = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED", 3: "SSM_ERR_CUDA",
            4: "SSM_ERR_BAD_SLOT", 5: "SSM_ERR_TIMEOUT", 6: "SSM_ERR_WORKSPACE"}
 SSM_F32, SSM_BF16 = 0, 1
-ABI_VERSION = 3
+ABI_VERSION = 4
+DISC_EULER, DISC_ZOH = 0, 1  # ssm_discretization_t
 
 # Every function the header declares; tests check the library exports all of them.
 EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
@@ -42,7 +43,7 @@ class ScanParams(ctypes.Structure):
         ("B", ctypes.c_void_p), ("C", ctypes.c_void_p),
         ("A", ctypes.c_void_p), ("Dskip", ctypes.c_void_p), ("delta_bias", ctypes.c_void_p),
         ("h0", ctypes.c_void_p), ("y", ctypes.c_void_p), ("h_last", ctypes.c_void_p),
-        ("ngroups", ctypes.c_int64), ("bc_group_stride", ctypes.c_int64),
+        ("ngroups", ctypes.c_int64), ("bc_group_stride", ctypes.c_int64), ("discretization", ctypes.c_int32),
     ]
 
 
@@ -134,7 +135,7 @@ def _f32(t):
 
 # ----------------------------------------------------------------------------- scans
 
-def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None):
+def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None, zoh=False):
     """Fill ScanParams for the fixed-length layout u/delta/z/y [b, D, L], B/C [b, N, L] (or
     [b, G, N, L]: G channel groups, channel d reading group d // (D / G))."""
     bsz, dim, L = u.shape
@@ -160,19 +161,21 @@ def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None,
     p.u, p.delta, p.z, p.B, p.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
     p.A, p.Dskip, p.delta_bias, p.h0 = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(h0)
     p.y, p.h_last = _ptr(y), _ptr(h_last)
+    p.discretization = DISC_ZOH if zoh else DISC_EULER
     return p
 
 
 def scan_fwd(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None,
-             return_last_state=True, stream=None, y_dtype=None):
+             return_last_state=True, stream=None, y_dtype=None, zoh=False):
     """Selective scan over a fixed-length batch.  Returns (y, h_last).
 
-    y is allocated in ``y_dtype`` (default: the input dtype; float32 is also accepted)."""
+    y is allocated in ``y_dtype`` (default: the input dtype; float32 is also accepted).
+    ``zoh``: zero-order-hold input matrix instead of Bbar = Delta B."""
     import torch
     y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
     if h_last is None and return_last_state:
         h_last = torch.empty((u.shape[0], u.shape[1], A.shape[1]), device=u.device, dtype=torch.float32)
-    p = scan_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last)
+    p = scan_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last, zoh)
     lib = load()
     ws = lib.ssm_scan_workspace_size(ctypes.byref(p), 0)
     wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
@@ -181,7 +184,7 @@ def scan_fwd(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=
 
 
 def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None,
-                  total=None):
+                  total=None, zoh=False):
     """ScanParams for the packed layout u/delta/z/y [D, T(+pad)], B/C [N, T(+pad)] (or
     [G, N, T(+pad)]: G channel groups).
 
@@ -209,11 +212,12 @@ def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=Non
     p.u, p.delta, p.z, p.B, p.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
     p.A, p.Dskip, p.delta_bias, p.h0 = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(h0)
     p.y, p.h_last = _ptr(y), _ptr(h_last)
+    p.discretization = DISC_ZOH if zoh else DISC_EULER
     return p
 
 
 def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, z=None, h0=None, y=None,
-                    h_last=None, total=None, return_last_state=True, stream=None, y_dtype=None):
+                    h_last=None, total=None, return_last_state=True, stream=None, y_dtype=None, zoh=False):
     """Packed variable-length scan.  cu_seqlens: int32 device tensor [nseq+1].  Returns (y, h_last)."""
     import torch
     if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
@@ -222,7 +226,7 @@ def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, 
     y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
     if h_last is None and return_last_state:
         h_last = torch.empty((nseq, u.shape[0], A.shape[1]), device=u.device, dtype=torch.float32)
-    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last, total)
+    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last, total, zoh)
     lib = load()
     ws = lib.ssm_scan_workspace_size(ctypes.byref(p), nseq)
     wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
@@ -232,7 +236,7 @@ def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, 
 
 
 def scan_fwd_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=None, delta_bias=None, z=None,
-                         y=None, total=None, stream=None, y_dtype=None):
+                         y=None, total=None, stream=None, y_dtype=None, zoh=False):
     """Packed prefill into a state pool: sequence i starts from pool[slot_ids[i]] and its final
     state is written back there.  pool: float32 [S, D, N]; slot_ids: int32 [nseq].  Returns y."""
     import torch
@@ -247,7 +251,7 @@ def scan_fwd_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=No
     if tuple(pool.shape[1:]) != (u.shape[0], A.shape[1]):
         raise ValueError("pool must be [S, dim, dstate]")
     y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
-    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, None, y, None, total)
+    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, None, y, None, total, zoh)
     lib = load()
     ws = lib.ssm_scan_workspace_size(ctypes.byref(p), nseq)
     wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
@@ -258,7 +262,7 @@ def scan_fwd_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=No
 
 
 def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, y=None, stream=None,
-                 y_dtype=None):
+                 y_dtype=None, zoh=False):
     """One decode step in place on ``pool`` [S, D, N] float32.  u/delta/z [R, D]; B/C [R, N]."""
     import torch
     if slot_ids.dtype != torch.int32 or not slot_ids.is_contiguous():
@@ -283,6 +287,7 @@ def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, delta_bias=None,
         raise ValueError("B and C must share the row stride")
     p.u, p.delta, p.z, p.B, p.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
     p.A, p.Dskip, p.delta_bias, p.y = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(y)
+    p.discretization = DISC_ZOH if zoh else DISC_EULER
     _check(load().ssm_state_update(_ptr(pool), S, _ptr(slot_ids), R, ctypes.byref(p), _stream(stream)),
            "ssm_state_update")
     return y

@@ -136,6 +136,8 @@ struct ChunkCfg {
   static constexpr size_t kBCAll = (kBF ? 1 : 2) * kBCBytes;  // 16-bit B/C staging
   static constexpr size_t kBFBytes = kBF ? size_t(2) * 2 * N * kTC * sizeof(float) : 0;
   static constexpr size_t kSmemBytes = 2 * kXBytes + kBCAll + kYBytes + kDBytes + kBFBytes + kParamBytes;
+  // 1/A per (channel, state) after the parameters, for the zero-order hold only
+  static constexpr size_t kInvABytes = size_t(kCT) * kNP * sizeof(float);
   static_assert(KI % 4 == 0 && KI % kVec == 0, "a lane's steps must be whole 16-byte vectors");
   static_assert(32 % (CPW * SPW) == 0, "lane split");
   static_assert(kLG == 1 || NG == 1, "states split either across warps or inside a warp");
@@ -145,7 +147,7 @@ struct ChunkCfg {
 };
 
 template <typename T, typename TO, int N, int KI, int SPW, int CPW, int CW, int NG, bool HAS_Z, bool VEC,
-          bool PERSIST>
+          bool PERSIST, bool ZOH>
 __global__ void __launch_bounds__(CW * NG * 32, (CW * NG <= 8 ? 16 / (CW * NG) : 1))
 chunk_scan_kernel(const ScanArgs args) {
   using Cfg = ChunkCfg<T, N, KI, SPW, CPW, CW, NG>;
@@ -174,6 +176,7 @@ chunk_scan_kernel(const ScanArgs args) {
   float *Dsk = carry_s + CT * NP;                                 // [CT]
   float *bias_s = Dsk + CT;                                       // [CT]
   int *order = reinterpret_cast<int *>(bias_s + CT);              // [kMaxSortedSeqs]
+  float *invAs = reinterpret_cast<float *>(order + kMaxSortedSeqs);  // [CT][NP] 1/A (ZOH only)
   __shared__ __align__(8) uint64_t bars[2];                      // chunk-arrival barriers
   __shared__ int unit_sh;
 
@@ -273,7 +276,9 @@ chunk_scan_kernel(const ScanArgs args) {
     for (int i = threadIdx.x; i < CT * N; i += NT) {
       const int c2 = i / N, n = i % N;
       const int64_t dd = d0 + c2;
-      A2s[c2 * NP + n] = dd < d_end ? args.A[dd * N + n] * kLog2e : 0.f;
+      const float av = dd < d_end ? args.A[dd * N + n] : 0.f;
+      A2s[c2 * NP + n] = av * kLog2e;
+      if constexpr (ZOH) invAs[c2 * NP + n] = inv_or_zero(av);
     }
     for (int i = threadIdx.x; i < CT; i += NT) {
       const int64_t dd = d0 + i;
@@ -335,8 +340,8 @@ chunk_scan_kernel(const ScanArgs args) {
         } else {
           const int r2 = r - nx * CT, which = r2 / N, n = r2 % N;
           const T *base = which == 0 ? SSM_GB : SSM_GC;
-          bulk_g2s(bdst + size_t(r2) * Cfg::kBCPitch, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, row_bytes,
-                   &bars[buf]);
+          bulk_g2s(bdst + size_t(r2) * Cfg::kBCPitch, base + bcbase + int64_t(n) * args.bc_state_stride + wstart,
+                   row_bytes, &bars[buf]);
         }
       }
     };
@@ -402,9 +407,10 @@ chunk_scan_kernel(const ScanArgs args) {
               const int i = tl0 + lg * V + 2 * (e + h);
               dt.x = (i >= rel_lo && i < rel_hi) ? dt.x : 0.f;
               dt.y = (i + 1 >= rel_lo && i + 1 < rel_hi) ? dt.y : 0.f;
-              uu = make_float2(dt.x != 0.f ? dt.x * vu[e + h].x : 0.f, dt.y != 0.f ? dt.y * vu[e + h].y : 0.f);
+              uu = make_float2(dt.x != 0.f ? (ZOH ? vu[e + h].x : dt.x * vu[e + h].x) : 0.f,
+                               dt.y != 0.f ? (ZOH ? vu[e + h].y : dt.y * vu[e + h].y) : 0.f);
             } else {
-              uu = __fmul2_rn(dt, vu[e + h]);
+              uu = ZOH ? vu[e + h] : __fmul2_rn(dt, vu[e + h]);
             }
             if (h == 0) {
               l4.x = dt.x; l4.y = dt.y; u4.x = uu.x; u4.y = uu.y;
@@ -448,9 +454,10 @@ chunk_scan_kernel(const ScanArgs args) {
               dt.x = (i >= rel_lo && i < rel_hi) ? dt.x : 0.f;
               dt.y = (i + 1 >= rel_lo && i + 1 < rel_hi) ? dt.y : 0.f;
               // select, so a non-finite u outside the sequence stays out
-              du[p] = make_float2(dt.x != 0.f ? dt.x * vu[e].x : 0.f, dt.y != 0.f ? dt.y * vu[e].y : 0.f);
+              du[p] = make_float2(dt.x != 0.f ? (ZOH ? vu[e].x : dt.x * vu[e].x) : 0.f,
+                                  dt.y != 0.f ? (ZOH ? vu[e].y : dt.y * vu[e].y) : 0.f);
             } else {
-              du[p] = __fmul2_rn(dt, vu[e]);
+              du[p] = ZOH ? vu[e] : __fmul2_rn(dt, vu[e]);
             }
             dl[p] = dt;
             dsum += dt.x + dt.y;
@@ -462,7 +469,7 @@ chunk_scan_kernel(const ScanArgs args) {
           const int c2 = i / TC, t = i % TC;
           const float uv = Elem<T>::to_f32(X[size_t(c2) * XP + t]);
           float dt = softplus_t<kFast>(Elem<T>::to_f32(X[size_t(CT + c2) * XP + t]) + bias_s[c2]);
-          float dtu = dt * uv;
+          float dtu = ZOH ? uv : dt * uv;
           if constexpr (kMasked) {
             const bool in = t >= rel_lo && t < rel_hi;
             dt = in ? dt : 0.f;
@@ -501,6 +508,8 @@ chunk_scan_kernel(const ScanArgs args) {
         constexpr bool FWD = decltype(fwd_tag)::value, OUT = decltype(out_tag)::value;
         const float A2 = FWD ? A2s[ch * NP + n1] : 0.f;
         const float2 A22 = make_float2(A2, A2);
+        [[maybe_unused]] float2 IA2;
+        if constexpr (FWD && ZOH) IA2 = make_float2(invAs[ch * NP + n1], invAs[ch * NP + n1]);
         [[maybe_unused]] const T *rb = Bsm + size_t(n1) * Cfg::kBCPitch + tl0;
         [[maybe_unused]] const T *rc = Csm + size_t(n2) * Cfg::kBCPitch + tl0;
         [[maybe_unused]] const float4 *rbf = reinterpret_cast<const float4 *>(Bf + size_t(n1) * TC + tl0);
@@ -539,12 +548,17 @@ chunk_scan_kernel(const ScanArgs args) {
               const float2 x = __fmul2_rn(dl[p], A22);
               a[2 * p] = ex2_approx(x.x);
               a[2 * p + 1] = ex2_approx(x.y);
+              // Euler: du = Delta*u is the input coefficient times u; zero-order hold: du = u,
+              // scaled by the coefficient (a - 1)/A
+              float2 q = du[p];
+              if constexpr (ZOH)
+                q = __fmul2_rn(q, zoh_coef2(dl[p], __fmul2_rn(x, make_float2(kLn2, kLn2)),
+                                            make_float2(a[2 * p], a[2 * p + 1]), IA2));
               if constexpr (kMasked) {
                 // stale B outside the window never reaches h (du is 0 there, B may be non-finite)
-                b[p] = make_float2(du[p].x != 0.f ? du[p].x * bb[e].x : 0.f,
-                                   du[p].y != 0.f ? du[p].y * bb[e].y : 0.f);
+                b[p] = make_float2(du[p].x != 0.f ? q.x * bb[e].x : 0.f, du[p].y != 0.f ? q.y * bb[e].y : 0.f);
               } else {
-                b[p] = __fmul2_rn(du[p], bb[e]);
+                b[p] = __fmul2_rn(q, bb[e]);
               }
               G = fmaf(a[2 * p], G, b[p].x);
               G = fmaf(a[2 * p + 1], G, b[p].y);

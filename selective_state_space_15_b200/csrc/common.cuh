@@ -125,6 +125,27 @@ template <bool kFast> __device__ __forceinline__ float silu_t(float z) {
   return kFast ? silu_fast(z) : silu_precise(z);
 }
 
+// Zero-order-hold input coefficient ("企业官网建设流程全解析" page, discosf.com, §1.2:
+// Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B).  For a diagonal A the coefficient of B is
+// c = (e^x - 1) / x * Delta with x = Delta A, which equals (a - 1) / A with a = e^x as the
+// recurrence already computes it.  Where |x| < 1/4, a - 1 would cancel, so the series
+// e^x - 1 = x (1 + x/2 + x^2/6 + x^3/24 + x^4/120 + ...) gives c = Delta (1 + x/2 + ...)
+// (truncation below |x|^5/720 < 1.4e-6 relative); elsewhere |a - 1| >= 0.22 and the error of
+// the MUFU exponential stays near 1e-6 relative.  invA = 1/A, or 0 where A = 0 (then x = 0
+// and the series is taken).  Both branches are evaluated and selected; the unselected one
+// may be inf/nan, which a select does not propagate.  Two coefficients at a time, in packed
+// f32x2 arithmetic.
+__device__ __forceinline__ float inv_or_zero(float a) { return a != 0.f ? 1.f / a : 0.f; }
+__device__ __forceinline__ float2 zoh_coef2(float2 dt, float2 x, float2 a, float2 invA) {
+  float2 s = __ffma2_rn(x, make_float2(1.f / 120.f, 1.f / 120.f), make_float2(1.f / 24.f, 1.f / 24.f));
+  s = __ffma2_rn(x, s, make_float2(1.f / 6.f, 1.f / 6.f));
+  s = __ffma2_rn(x, s, make_float2(0.5f, 0.5f));
+  s = __ffma2_rn(x, s, make_float2(1.f, 1.f));
+  const float2 near = __fmul2_rn(dt, s);
+  const float2 far = __fmul2_rn(__fadd2_rn(a, make_float2(-1.f, -1.f)), invA);
+  return make_float2(fabsf(x.x) < 0.25f ? near.x : far.x, fabsf(x.y) < 0.25f ? near.y : far.y);
+}
+
 
 // ---- TMA bulk copies completing on an mbarrier (PTX ISA: cp.async.bulk, mbarrier) ----
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

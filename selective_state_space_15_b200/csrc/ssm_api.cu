@@ -87,21 +87,21 @@ bool make_plan(const ssm_scan_params *p, int64_t nseq, bool varlen, bool vec, Pl
   return true;
 }
 
-template <typename T, typename TO, int N, bool NARROW, bool HAS_Z, bool VEC, bool PERSIST>
+template <typename T, typename TO, int N, bool NARROW, bool HAS_Z, bool VEC, bool PERSIST, bool ZOH>
 ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t stream) {
   using S = Shape<N, NARROW, sizeof(T) == 4>;
   using Cfg = ssm::ChunkCfg<T, N, S::KI, S::SPW, S::CPW, S::CW, S::NG>;
-  auto kern = ssm::chunk_scan_kernel<T, TO, N, S::KI, S::SPW, S::CPW, S::CW, S::NG, HAS_Z, VEC, PERSIST>;
+  auto kern = ssm::chunk_scan_kernel<T, TO, N, S::KI, S::SPW, S::CPW, S::CW, S::NG, HAS_Z, VEC, PERSIST, ZOH>;
+  constexpr size_t kSmem = Cfg::kSmemBytes + (ZOH ? Cfg::kInvABytes : 0);
   static int configured_device = -1;  // the attribute is set once per device function per device
   static int max_blocks_per_sm = 0;
   static int num_sms = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
   if (configured_device != dev) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
       return SSM_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&max_blocks_per_sm, kern, Cfg::kThreads, Cfg::kSmemBytes) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&max_blocks_per_sm, kern, Cfg::kThreads, kSmem) !=
         cudaSuccess)
       return SSM_ERR_CUDA;
     if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SSM_ERR_CUDA;
@@ -135,44 +135,51 @@ ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t str
     blocks = a.total_units < resident ? a.total_units : resident;
   }
   if (blocks > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
-  kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(a);
+  kern<<<unsigned(blocks), Cfg::kThreads, kSmem, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
-template <typename T, typename TO, int N, bool NARROW>
+template <typename T, typename TO, int N, bool NARROW, bool ZOH>
 ssm_status_t dispatch_zvp(const ScanArgs &a, const Plan &pl, bool has_z, bool vec, void *ws, cudaStream_t st) {
   if (pl.persist) {
-    if (has_z) return launch_chunk<T, TO, N, NARROW, true, true, true>(a, pl, ws, st);
-    return launch_chunk<T, TO, N, NARROW, false, true, true>(a, pl, ws, st);
+    if (has_z) return launch_chunk<T, TO, N, NARROW, true, true, true, ZOH>(a, pl, ws, st);
+    return launch_chunk<T, TO, N, NARROW, false, true, true, ZOH>(a, pl, ws, st);
   }
   if constexpr (NARROW) {
     return SSM_ERR_UNSUPPORTED;  // the narrow shape is only planned for persistent launches
   } else {
     if (has_z)
-      return vec ? launch_chunk<T, TO, N, false, true, true, false>(a, pl, ws, st)
-                 : launch_chunk<T, TO, N, false, true, false, false>(a, pl, ws, st);
-    return vec ? launch_chunk<T, TO, N, false, false, true, false>(a, pl, ws, st)
-               : launch_chunk<T, TO, N, false, false, false, false>(a, pl, ws, st);
+      return vec ? launch_chunk<T, TO, N, false, true, true, false, ZOH>(a, pl, ws, st)
+                 : launch_chunk<T, TO, N, false, true, false, false, ZOH>(a, pl, ws, st);
+    return vec ? launch_chunk<T, TO, N, false, false, true, false, ZOH>(a, pl, ws, st)
+               : launch_chunk<T, TO, N, false, false, false, false, ZOH>(a, pl, ws, st);
+  }
+}
+
+template <typename T, typename TO, bool ZOH>
+ssm_status_t dispatch_n(const ScanArgs &a, const Plan &pl, int N, bool has_z, bool vec, void *ws,
+                        cudaStream_t st) {
+  switch (N) {
+    case 16: return pl.narrow ? dispatch_zvp<T, TO, 16, true, ZOH>(a, pl, has_z, vec, ws, st)
+                              : dispatch_zvp<T, TO, 16, false, ZOH>(a, pl, has_z, vec, ws, st);
+    case 32: return dispatch_zvp<T, TO, 32, false, ZOH>(a, pl, has_z, vec, ws, st);
+    case 64: return dispatch_zvp<T, TO, 64, false, ZOH>(a, pl, has_z, vec, ws, st);
+    case 128:
+      if constexpr (std::is_same<T, float>::value) {
+        return dispatch_zvp<T, TO, 128, false, ZOH>(a, pl, has_z, vec, ws, st);  // no narrow plan for float32
+      } else {
+        return pl.narrow ? dispatch_zvp<T, TO, 128, true, ZOH>(a, pl, has_z, vec, ws, st)
+                         : dispatch_zvp<T, TO, 128, false, ZOH>(a, pl, has_z, vec, ws, st);
+      }
+    default: return SSM_ERR_UNSUPPORTED;
   }
 }
 
 template <typename T, typename TO>
-ssm_status_t dispatch_n(const ScanArgs &a, const Plan &pl, int N, bool has_z, bool vec, void *ws,
-                        cudaStream_t st) {
-  switch (N) {
-    case 16: return pl.narrow ? dispatch_zvp<T, TO, 16, true>(a, pl, has_z, vec, ws, st)
-                              : dispatch_zvp<T, TO, 16, false>(a, pl, has_z, vec, ws, st);
-    case 32: return dispatch_zvp<T, TO, 32, false>(a, pl, has_z, vec, ws, st);
-    case 64: return dispatch_zvp<T, TO, 64, false>(a, pl, has_z, vec, ws, st);
-    case 128:
-      if constexpr (std::is_same<T, float>::value) {
-        return dispatch_zvp<T, TO, 128, false>(a, pl, has_z, vec, ws, st);  // no narrow plan for float32
-      } else {
-        return pl.narrow ? dispatch_zvp<T, TO, 128, true>(a, pl, has_z, vec, ws, st)
-                         : dispatch_zvp<T, TO, 128, false>(a, pl, has_z, vec, ws, st);
-      }
-    default: return SSM_ERR_UNSUPPORTED;
-  }
+ssm_status_t dispatch_disc(const ScanArgs &a, const Plan &pl, int N, bool has_z, bool vec, bool zoh, void *ws,
+                           cudaStream_t st) {
+  return zoh ? dispatch_n<T, TO, true>(a, pl, N, has_z, vec, ws, st)
+             : dispatch_n<T, TO, false>(a, pl, N, has_z, vec, ws, st);
 }
 
 size_t elem_size(ssm_dtype_t t) { return t == SSM_BF16 ? 2 : 4; }
@@ -181,6 +188,7 @@ size_t elem_size(ssm_dtype_t t) { return t == SSM_BF16 ? 2 : 4; }
 ssm_status_t prepare_scan(const ssm_scan_params *p, bool varlen, ScanArgs &a, bool &vec) {
   if (!p) return SSM_ERR_INVALID_ARG;
   if (p->dtype != SSM_F32 && p->dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+  if (p->discretization != SSM_DISC_EULER && p->discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
   if (p->dim <= 0 || p->dstate <= 0 || p->seqlen < 0 || p->batch < 0) return SSM_ERR_INVALID_ARG;
   if (varlen && p->batch != 1) return SSM_ERR_INVALID_ARG;
   if (!p->u || !p->delta || !p->B || !p->C || !p->A || !p->y) return SSM_ERR_INVALID_ARG;
@@ -215,8 +223,8 @@ ssm_status_t prepare_scan(const ssm_scan_params *p, bool varlen, ScanArgs &a, bo
   return SSM_OK;
 }
 
-ssm_status_t run_scan(ScanArgs a, const Plan &pl, ssm_dtype_t dt, bool y_fp32, int N, bool vec, void *ws,
-                      size_t ws_bytes, cudaStream_t st) {
+ssm_status_t run_scan(ScanArgs a, const Plan &pl, ssm_dtype_t dt, bool y_fp32, int N, bool vec, bool zoh,
+                      void *ws, size_t ws_bytes, cudaStream_t st) {
   if (pl.ws_bytes > 0 && (ws == nullptr || ws_bytes < pl.ws_bytes || (reinterpret_cast<uintptr_t>(ws) & 15)))
     return SSM_ERR_WORKSPACE;
   if (pl.ntiles > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
@@ -224,10 +232,10 @@ ssm_status_t run_scan(ScanArgs a, const Plan &pl, ssm_dtype_t dt, bool y_fp32, i
   a.tiles_per_group = int(pl.ntiles / (a.dim / a.group_dim));
   const bool has_z = a.z != nullptr;
   if (dt == SSM_BF16) {
-    if (y_fp32) return dispatch_n<__nv_bfloat16, float>(a, pl, N, has_z, vec, ws, st);
-    return dispatch_n<__nv_bfloat16, __nv_bfloat16>(a, pl, N, has_z, vec, ws, st);
+    if (y_fp32) return dispatch_disc<__nv_bfloat16, float>(a, pl, N, has_z, vec, zoh, ws, st);
+    return dispatch_disc<__nv_bfloat16, __nv_bfloat16>(a, pl, N, has_z, vec, zoh, ws, st);
   }
-  return dispatch_n<float, float>(a, pl, N, has_z, vec, ws, st);
+  return dispatch_disc<float, float>(a, pl, N, has_z, vec, zoh, ws, st);
 }
 
 // Scratch for ssm_scan_fwd_noalloc: a static device array that every GPU loading the
@@ -254,6 +262,32 @@ ssm_status_t noalloc_scratch(void **out) {
   return SSM_OK;
 }
 
+// Decode launches: the N = 16 kernel (one warp per 32 channels, coalesced quads), else G
+// states per thread.
+template <typename T, typename TO, bool ZOH>
+void launch_update_disc(const ssm::UpdateArgs &a, int G, bool has_z, dim3 blocks, cudaStream_t st) {
+  using namespace ssm;
+  if (a.dstate == 16) {
+    const dim3 b16(unsigned((a.dim + kUpdateThreads - 1) / kUpdateThreads), blocks.y);
+    if (has_z) state_update16_kernel<T, TO, true, ZOH><<<b16, kUpdateThreads, 0, st>>>(a);
+    else state_update16_kernel<T, TO, false, ZOH><<<b16, kUpdateThreads, 0, st>>>(a);
+    return;
+  }
+  auto go = [&](auto g_tag) {
+    constexpr int GG = decltype(g_tag)::value;
+    if (has_z) state_update_kernel<T, TO, true, GG, ZOH><<<blocks, kUpdateThreads, 0, st>>>(a);
+    else state_update_kernel<T, TO, false, GG, ZOH><<<blocks, kUpdateThreads, 0, st>>>(a);
+  };
+  if (G == 16) go(std::integral_constant<int, 16>{});
+  else if (G == 8) go(std::integral_constant<int, 8>{});
+  else go(std::integral_constant<int, 4>{});
+}
+template <typename T, typename TO>
+void launch_update(const ssm::UpdateArgs &a, int G, bool has_z, bool zoh, dim3 blocks, cudaStream_t st) {
+  if (zoh) launch_update_disc<T, TO, true>(a, G, has_z, blocks, st);
+  else launch_update_disc<T, TO, false>(a, G, has_z, blocks, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -273,7 +307,8 @@ ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_params *p, ssm_stream_t stream)
   if (st != SSM_OK) return st;
   a.cu_seqlens = nullptr;
   a.nseq = int(p->batch);
-  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, scratch, kNoAllocScratchBytes,
+  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, p->discretization == SSM_DISC_ZOH,
+                  scratch, kNoAllocScratchBytes,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -289,7 +324,8 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_params *p, void *workspace, size_t work
   if (!make_plan(p, p->batch, false, vec, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = nullptr;
   a.nseq = int(p->batch);
-  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
+  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, p->discretization == SSM_DISC_ZOH,
+                  workspace, workspace_bytes,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -307,7 +343,8 @@ ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_params *p, const int32_t *cu_seq
   if (!make_plan(p, nseq, true, vec, pl)) return SSM_ERR_UNSUPPORTED;
   a.cu_seqlens = cu_seqlens;
   a.nseq = int(nseq);
-  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
+  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, p->discretization == SSM_DISC_ZOH,
+                  workspace, workspace_bytes,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -331,7 +368,8 @@ ssm_status_t ssm_scan_fwd_varlen_pool(const ssm_scan_params *p, const int32_t *c
   a.h_last = pool;
   a.state_slots = slot_ids;
   a.num_slots = num_slots;
-  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, workspace, workspace_bytes,
+  return run_scan(a, pl, p->dtype, p->y_fp32 != 0, int(p->dstate), vec, p->discretization == SSM_DISC_ZOH,
+                  workspace, workspace_bytes,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -340,6 +378,7 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
   if (!p || !pool || !slot_ids || num_slots <= 0 || R < 0) return SSM_ERR_INVALID_ARG;
   if (p->dtype != SSM_F32 && p->dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
   if (p->batch != R || p->seqlen != 1 || p->dim <= 0 || p->dstate <= 0) return SSM_ERR_INVALID_ARG;
+  if (p->discretization != SSM_DISC_EULER && p->discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
   if (p->ngroups > 1) return SSM_ERR_UNSUPPORTED;  // decode takes one B, C per request
   if (!p->u || !p->delta || !p->B || !p->C || !p->A || !p->y) return SSM_ERR_INVALID_ARG;
   const int64_t N = p->dstate;
@@ -363,38 +402,11 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
   if (gx > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
   const dim3 blocks(unsigned(gx), unsigned(R < 65535 ? R : 65535));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool has_z = p->z != nullptr;
+  const bool has_z = p->z != nullptr, zoh = p->discretization == SSM_DISC_ZOH;
   using bf16 = __nv_bfloat16;
-#define SSM_UPDATE_LAUNCH(T, TO)                                                                          \
-  do {                                                                                                     \
-    if (G == 16) {                                                                                         \
-      if (has_z) ssm::state_update_kernel<T, TO, true, 16><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);      \
-      else ssm::state_update_kernel<T, TO, false, 16><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);           \
-    } else if (G == 8) {                                                                                   \
-      if (has_z) ssm::state_update_kernel<T, TO, true, 8><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);       \
-      else ssm::state_update_kernel<T, TO, false, 8><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);            \
-    } else {                                                                                               \
-      if (has_z) ssm::state_update_kernel<T, TO, true, 4><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);       \
-      else ssm::state_update_kernel<T, TO, false, 4><<<blocks, ssm::kUpdateThreads, 0, st>>>(a);            \
-    }                                                                                                      \
-  } while (0)
-  if (N == 16) {  // one warp per 32 channels, coalesced quads
-    const dim3 b16(unsigned((p->dim + ssm::kUpdateThreads - 1) / ssm::kUpdateThreads), blocks.y);
-#define SSM_UPDATE16(T, TO)                                                                         \
-  (has_z ? ssm::state_update16_kernel<T, TO, true><<<b16, ssm::kUpdateThreads, 0, st>>>(a)          \
-         : ssm::state_update16_kernel<T, TO, false><<<b16, ssm::kUpdateThreads, 0, st>>>(a))
-    if (p->dtype == SSM_BF16 && !p->y_fp32) SSM_UPDATE16(bf16, bf16);
-    else if (p->dtype == SSM_BF16) SSM_UPDATE16(bf16, float);
-    else SSM_UPDATE16(float, float);
-#undef SSM_UPDATE16
-  } else if (p->dtype == SSM_BF16 && !p->y_fp32) {
-    SSM_UPDATE_LAUNCH(bf16, bf16);
-  } else if (p->dtype == SSM_BF16) {
-    SSM_UPDATE_LAUNCH(bf16, float);
-  } else {
-    SSM_UPDATE_LAUNCH(float, float);
-  }
-#undef SSM_UPDATE_LAUNCH
+  if (p->dtype == SSM_BF16 && !p->y_fp32) launch_update<bf16, bf16>(a, G, has_z, zoh, blocks, st);
+  else if (p->dtype == SSM_BF16) launch_update<bf16, float>(a, G, has_z, zoh, blocks, st);
+  else launch_update<float, float>(a, G, has_z, zoh, blocks, st);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

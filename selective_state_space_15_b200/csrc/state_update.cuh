@@ -10,7 +10,8 @@
 // block (every channel of the request reads the same values).  Consecutive threads take
 // consecutive channels, so a warp streams one contiguous run of the pool row.  When a
 // channel is split over several threads (dstate > 16) their partial C.h go through shared
-// memory.
+// memory.  With ZOH the input coefficient is the zero-order hold's (a - 1)/A instead of
+// Delta (zoh_coef2 in common.cuh).
 #pragma once
 
 #include "common.cuh"
@@ -34,7 +35,7 @@ constexpr int kUpdateMaxState = 128;
 
 // Grid: x over the channels of one request (kUpdateThreads / tpc per block), y strides over
 // the requests.  G states per thread (4, 8 or 16; G divides dstate).
-template <typename T, typename TO, bool HAS_Z, int G>
+template <typename T, typename TO, bool HAS_Z, int G, bool ZOH>
 __global__ void __launch_bounds__(kUpdateThreads) state_update_kernel(const UpdateArgs args) {
   constexpr bool kFast = Elem<T>::kFast;
   static_assert(G % 4 == 0 && G <= 16, "state group");
@@ -83,8 +84,16 @@ __global__ void __launch_bounds__(kUpdateThreads) state_update_kernel(const Upda
         const float2 x23 = __fmul2_rn(dtl, make_float2(av[k].z, av[k].w));
         const float2 a01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
         const float2 a23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-        const float2 h01 = __ffma2_rn(a01, make_float2(h[k].x, h[k].y), __fmul2_rn(dtu, make_float2(b4.x, b4.y)));
-        const float2 h23 = __ffma2_rn(a23, make_float2(h[k].z, h[k].w), __fmul2_rn(dtu, make_float2(b4.z, b4.w)));
+        float2 q01 = dtu, q23 = dtu;  // input coefficient times u
+        if constexpr (ZOH) {
+          const float2 DT = make_float2(dt, dt), U = make_float2(uval, uval), L = make_float2(kLn2, kLn2);
+          const float2 i01 = make_float2(inv_or_zero(av[k].x), inv_or_zero(av[k].y));
+          const float2 i23 = make_float2(inv_or_zero(av[k].z), inv_or_zero(av[k].w));
+          q01 = __fmul2_rn(U, zoh_coef2(DT, __fmul2_rn(x01, L), a01, i01));
+          q23 = __fmul2_rn(U, zoh_coef2(DT, __fmul2_rn(x23, L), a23, i23));
+        }
+        const float2 h01 = __ffma2_rn(a01, make_float2(h[k].x, h[k].y), __fmul2_rn(q01, make_float2(b4.x, b4.y)));
+        const float2 h23 = __ffma2_rn(a23, make_float2(h[k].z, h[k].w), __fmul2_rn(q23, make_float2(b4.z, b4.w)));
         acc2 = __ffma2_rn(make_float2(c4.x, c4.y), h01, acc2);
         acc2 = __ffma2_rn(make_float2(c4.z, c4.w), h23, acc2);
         h[k] = make_float4(h01.x, h01.y, h23.x, h23.y);
@@ -113,7 +122,7 @@ __global__ void __launch_bounds__(kUpdateThreads) state_update_kernel(const Upda
 // per-channel terms (softplus, Delta*u, gate) for one channel, 8m + j, and hands Delta to the
 // other three lanes of the channel with shuffles; C.h is reduced over the 4 lanes of a
 // channel, and lane l writes y for its own channel.
-template <typename T, typename TO, bool HAS_Z>
+template <typename T, typename TO, bool HAS_Z, bool ZOH>
 __global__ void __launch_bounds__(kUpdateThreads, 4) state_update16_kernel(const UpdateArgs args) {
   constexpr bool kFast = Elem<T>::kFast;
   constexpr int N = 16;
@@ -147,7 +156,7 @@ __global__ void __launch_bounds__(kUpdateThreads, 4) state_update16_kernel(const
                                   Elem<T>::to_f32(Br[3]));
     const float4 c4 = make_float4(Elem<T>::to_f32(Cr[0]), Elem<T>::to_f32(Cr[1]), Elem<T>::to_f32(Cr[2]),
                                   Elem<T>::to_f32(Cr[3]));
-    // this lane's own channel: Delta, Delta*u, u, gate
+    // this lane's own channel: Delta, Delta*u (zero-order hold: u), u, gate
     float dtl = 0.f, dtu = 0.f, uval = 0.f, zval = 0.f;
     if (own_ok) {
       const int64_t xo = r * args.x_stride + c_own;
@@ -155,7 +164,7 @@ __global__ void __launch_bounds__(kUpdateThreads, 4) state_update16_kernel(const
       const float dt = softplus_t<kFast>(Elem<T>::to_f32(static_cast<const T *>(args.delta)[xo]) +
                                          (args.bias ? args.bias[c_own] : 0.f));
       dtl = dt * kLog2e;
-      dtu = dt * uval;
+      dtu = ZOH ? uval : dt * uval;
       if constexpr (HAS_Z) zval = Elem<T>::to_f32(static_cast<const T *>(args.z)[xo]);
     }
     float own_sum = 0.f;
@@ -169,8 +178,16 @@ __global__ void __launch_bounds__(kUpdateThreads, 4) state_update16_kernel(const
       const float2 x23 = __fmul2_rn(L2, make_float2(av[k].z, av[k].w));
       const float2 a01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
       const float2 a23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-      const float2 h01 = __ffma2_rn(a01, make_float2(h[k].x, h[k].y), __fmul2_rn(DU, make_float2(b4.x, b4.y)));
-      const float2 h23 = __ffma2_rn(a23, make_float2(h[k].z, h[k].w), __fmul2_rn(DU, make_float2(b4.z, b4.w)));
+      float2 q01 = DU, q23 = DU;  // input coefficient times u
+      if constexpr (ZOH) {
+        const float2 L = make_float2(kLn2, kLn2), DT = __fmul2_rn(L2, L);
+        const float2 i01 = make_float2(inv_or_zero(av[k].x), inv_or_zero(av[k].y));
+        const float2 i23 = make_float2(inv_or_zero(av[k].z), inv_or_zero(av[k].w));
+        q01 = __fmul2_rn(DU, zoh_coef2(DT, __fmul2_rn(x01, L), a01, i01));
+        q23 = __fmul2_rn(DU, zoh_coef2(DT, __fmul2_rn(x23, L), a23, i23));
+      }
+      const float2 h01 = __ffma2_rn(a01, make_float2(h[k].x, h[k].y), __fmul2_rn(q01, make_float2(b4.x, b4.y)));
+      const float2 h23 = __ffma2_rn(a23, make_float2(h[k].z, h[k].w), __fmul2_rn(q23, make_float2(b4.z, b4.w)));
       h[k] = make_float4(h01.x, h01.y, h23.x, h23.y);
       float2 p2 = __fmul2_rn(make_float2(c4.x, c4.y), h01);
       p2 = __ffma2_rn(make_float2(c4.z, c4.w), h23, p2);

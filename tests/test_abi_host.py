@@ -35,6 +35,20 @@ def test_library_exports_every_declared_function(lib):
         assert hasattr(lib, name), name
 
 
+def test_binding_struct_mirrors_the_header():
+    """ScanParams lists the fields of ssm_scan_params in the header's order."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct ssm_scan_params \{(.*?)\} ssm_scan_params;", src, flags=re.S).group(1)
+    names = []
+    for decl in filter(None, (d.strip() for d in body.split(";"))):
+        # "type name" or "type *a, *b, *c": the declarators are the words after the type
+        first, *rest = decl.split(",")
+        names.append(re.findall(r"(\w+)$", first)[0])
+        names += [re.sub(r"[*\s]", "", r) for r in rest]
+    assert names == [f[0] for f in ssm.ScanParams._fields_]
+    assert (ssm.DISC_EULER, ssm.DISC_ZOH) == (0, 1)
+
+
 def test_abi_version_and_status_strings(lib):
     assert lib.ssm_abi_version() == ssm.ABI_VERSION
     for code, name in ssm._STATUS.items():
@@ -59,6 +73,7 @@ def _params(**kw):
     ("dstate", 24, 2), ("dstate", 256, 2),
     ("x_dim_stride", 100, 1),           # row stride shorter than the sequence
     ("bc_state_stride", 100, 1),
+    ("discretization", 2, 1), ("discretization", -1, 1),   # neither Euler nor zero-order hold
 ])
 def test_scan_rejects_bad_arguments_on_host(lib, field, value, code):
     p = _params(**{field: value})
@@ -118,6 +133,8 @@ def test_state_update_host_checks(lib):
     p3 = _params(batch=8, seqlen=2, dim=32, dstate=16)
     assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p3), None) == 1     # one token only
     assert lib.ssm_state_update(fake + 4, 4, fake, 8, ctypes.byref(p), None) == 1  # pool not 16-byte aligned
+    p4 = _params(batch=8, seqlen=1, dim=32, dstate=16, discretization=3)
+    assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p4), None) == 1     # unknown discretisation
 
 
 def test_workspace_size_query_is_host_only(lib):
