@@ -347,6 +347,24 @@ def pool_prefill_run(steps, warmup, sfu_peak):
     return {"ms": round(ms, 4), "tokens_per_s": T / (ms * 1e-3), "sfu_frac": round(ne / (ms * 1e-3) / sfu_peak, 4)}
 
 
+def varlen_zoh_run(steps, warmup, sfu_peak):
+    """The varlen workload with the zero-order-hold input matrix (ssm_scan_fwd_varlen, zoh)."""
+    import torch
+    import selective_state_space_15_b200 as ssm
+    stream = torch.cuda.current_stream()
+    device = torch.device("cuda", torch.cuda.current_device())
+    inp, _, dev, T, pitch = varlen_device_inputs(0, device)
+    D, N, nseq = inp.u.shape[0], inp.A.shape[1], inp.meta["nseq"]
+    y = torch.empty((D, pitch), dtype=torch.bfloat16, device=device)
+    hl = torch.empty((nseq, D, N), dtype=torch.float32, device=device)
+    ms = time_kernel(lambda: ssm.scan_fwd_varlen(dev["u"], dev["delta"], dev["B"], dev["C"], dev["A"], dev["cu"],
+                                                 dev["Dskip"], dev["bias"], dev["z"], y=y, h_last=hl, total=T,
+                                                 stream=stream, zoh=True), steps, warmup, stream)
+    _, ne = scan_counts(T, D, N, 2, 2, nseq)
+    return {"ms": round(ms, 4), "tokens_per_s": T / (ms * 1e-3), "sfu_frac": round(ne / (ms * 1e-3) / sfu_peak, 4),
+            "discretization": "zero-order hold"}
+
+
 def decode_loop_run(hbm_peak, loop_steps=100):
     """A serving-style decode loop: `loop_steps` back-to-back decode steps (inputs cycling over 4
     token sets) captured in one CUDA graph; the active states (84 MB) stay in L2 between steps."""
@@ -391,6 +409,7 @@ def secondary(steps, warmup, hbm_peak, sfu_peak):
     out.update({name: long_run(name, max(3, steps // 4), warmup, hbm_peak, sfu_peak)
                 for name in ("long_bf16", "long_n128_bf16")})
     out["varlen_pool_bf16"] = pool_prefill_run(max(3, steps // 4), warmup, sfu_peak)
+    out["varlen_zoh_bf16"] = varlen_zoh_run(max(3, steps // 4), warmup, sfu_peak)
     out["decode_bf16"] = decode_run(steps, warmup, hbm_peak)
     out["decode_loop_bf16"] = decode_loop_run(hbm_peak)
     return out
