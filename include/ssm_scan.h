@@ -34,8 +34,8 @@
  *     (then y is float32).  A, Dskip, delta_bias and all states (h0, h_last, the decode pool)
  *     are float32.  Arithmetic is float32; a bf16 y is rounded to nearest-even once, at the
  *     store.
- *   - Supported state sizes: dstate in {16, 32, 64, 128} for the scans, any multiple of 4
- *     up to 128 for the decode update.  Other values return SSM_ERR_UNSUPPORTED.
+ *   - Supported state sizes: dstate in {16, 32, 64, 128, 256} for the scans, any multiple of
+ *     4 up to 256 for the decode update.  Other values return SSM_ERR_UNSUPPORTED.
  *   - Fast path: when every tensor base is 16-byte aligned and every row stride is a
  *     multiple of 16 bytes, inputs are staged with TMA bulk copies, and rows are read up to
  *     the sequence length rounded up to 16 bytes (the row stride covers it).  Other layouts

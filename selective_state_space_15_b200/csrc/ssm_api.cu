@@ -35,6 +35,9 @@ template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW
 template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<128, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 4, NG = 1; };
 template <> struct Shape<128, true> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 1, NG = 16; };
+// N=256: 8 warps share an 8-channel tile and take 32 states each (per-(channel, state) arrays
+// and the B/C chunk of a wider tile would not fit in shared memory)
+template <> struct Shape<256, false> { static constexpr int KI = 8, SPW = 4, CPW = 8, CW = 1, NG = 8; };
 template <int N, bool NARROW, bool F32> ShapeInfo shape_of() {
   using S = Shape<N, NARROW, F32>;
   return ShapeInfo{S::KI, S::SPW, S::CPW, S::CW, S::NG};
@@ -47,6 +50,7 @@ bool shape_for(int N, bool narrow, bool f32, ShapeInfo &si) {
     case 32: si = shape_of<32, false, false>(); return true;
     case 64: si = shape_of<64, false, false>(); return true;
     case 128: si = narrow ? shape_of<128, true, false>() : shape_of<128, false, false>(); return true;
+    case 256: si = shape_of<256, false, false>(); return true;
     default: return false;
   }
 }
@@ -171,6 +175,7 @@ ssm_status_t dispatch_n(const ScanArgs &a, const Plan &pl, int N, bool has_z, bo
         return pl.narrow ? dispatch_zvp<T, TO, 128, true, ZOH>(a, pl, has_z, vec, ws, st)
                          : dispatch_zvp<T, TO, 128, false, ZOH>(a, pl, has_z, vec, ws, st);
       }
+    case 256: return dispatch_zvp<T, TO, 256, false, ZOH>(a, pl, has_z, vec, ws, st);
     default: return SSM_ERR_UNSUPPORTED;
   }
 }
@@ -193,7 +198,7 @@ ssm_status_t prepare_scan(const ssm_scan_params *p, bool varlen, ScanArgs &a, bo
   if (varlen && p->batch != 1) return SSM_ERR_INVALID_ARG;
   if (!p->u || !p->delta || !p->B || !p->C || !p->A || !p->y) return SSM_ERR_INVALID_ARG;
   ShapeInfo probe;
-  if (p->dstate > 128 || !shape_for(int(p->dstate), false, false, probe)) return SSM_ERR_UNSUPPORTED;
+  if (p->dstate > 256 || !shape_for(int(p->dstate), false, false, probe)) return SSM_ERR_UNSUPPORTED;
   if (p->dim > (int64_t(1) << 31) || p->seqlen > (int64_t(1) << 40)) return SSM_ERR_UNSUPPORTED;
   a = ScanArgs{};
   a.u = p->u; a.delta = p->delta; a.z = p->z; a.B = p->B; a.C = p->C;

@@ -31,7 +31,7 @@ struct UpdateArgs {
 };
 
 constexpr int kUpdateThreads = 256;
-constexpr int kUpdateMaxState = 128;
+constexpr int kUpdateMaxState = 256;
 
 // Grid: x over the channels of one request (kUpdateThreads / tpc per block), y strides over
 // the requests.  G states per thread (4, 8 or 16; G divides dstate).

@@ -70,7 +70,7 @@ def _params(**kw):
 @pytest.mark.parametrize("field,value,code", [
     ("u", None, 1), ("delta", None, 1), ("B", None, 1), ("C", None, 1), ("A", None, 1), ("y", None, 1),
     ("dim", 0, 1), ("dstate", 0, 1), ("seqlen", -1, 1), ("batch", -1, 1), ("dtype", 7, 1),
-    ("dstate", 24, 2), ("dstate", 256, 2),
+    ("dstate", 24, 2), ("dstate", 512, 2), ("dstate", 200, 2),
     ("x_dim_stride", 100, 1),           # row stride shorter than the sequence
     ("bc_state_stride", 100, 1),
     ("discretization", 2, 1), ("discretization", -1, 1),   # neither Euler nor zero-order hold
@@ -128,8 +128,8 @@ def test_state_update_host_checks(lib):
     assert lib.ssm_state_update(fake, 4, fake, 7, ctypes.byref(p), None) == 1      # batch != R
     p2 = _params(batch=8, seqlen=1, dim=32, dstate=10)
     assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p2), None) == 2     # not a multiple of 4
-    p2 = _params(batch=8, seqlen=1, dim=32, dstate=132)
-    assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p2), None) == 2     # above 128
+    p2 = _params(batch=8, seqlen=1, dim=32, dstate=260)
+    assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p2), None) == 2     # above 256
     p3 = _params(batch=8, seqlen=2, dim=32, dstate=16)
     assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p3), None) == 1     # one token only
     assert lib.ssm_state_update(fake + 4, 4, fake, 8, ctypes.byref(p), None) == 1  # pool not 16-byte aligned

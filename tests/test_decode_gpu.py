@@ -27,7 +27,7 @@ def _step(prob, pool_t, slots_t, step, A, D, bias):
 
 
 @pytest.mark.parametrize("dtype,N", [("bf16", 16), ("f32", 16), ("bf16", 64), ("f32", 128), ("f32", 4), ("bf16", 8),
-                                     ("f32", 12), ("bf16", 24), ("bf16", 48)])
+                                     ("f32", 12), ("bf16", 24), ("bf16", 48), ("bf16", 256), ("f32", 200)])
 def test_decode_small_matches_oracle_and_leaves_other_slots(dtype, N):
     prob = workloads.decode_problem(num_slots=37, dim=48, dstate=N, R=11, dtype=dtype, seed=5)
     pool_t = torch.from_numpy(prob.pool0).cuda()

@@ -53,6 +53,8 @@ def oracle_batch(inp, channels=None, h0=None, gate=True):
     (1, 24, 32, 515),
     (1, 12, 64, 300),
     (1, 10, 128, 200),
+    (2, 20, 256, 160),    # N=256: 8 warps split the states of an 8-channel tile
+    (1, 9, 256, 77),      # N=256, element-wise staging, tail tile
 ])
 def test_batch_small_full(shape, dtype):
     b, D, N, L = shape
@@ -125,6 +127,19 @@ def test_varlen_small_full(lengths, pitch_mult, dtype):
     inp = workloads.varlen_inputs(lengths, D, N, dtype, seed=len(lengths) + sum(lengths))
     T = inp.meta["total"]
     y, hl = _varlen_run(inp, dtype, round_up(T, pitch_mult))
+    ref = oracle.scan_varlen(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.cu_seqlens, inp.Dskip, inp.bias, inp.z,
+                             nthreads=NTHREADS)
+    check("y", y, ref["y"], ref["y_mag"], TOL[dtype], dtype)
+    check("h_last", hl, ref["h_last"], ref["h_mag"], TOL[dtype])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_varlen_dstate_256(dtype):
+    lengths = [100, 0, 37, 300, 1]
+    D, N = 20, 256
+    inp = workloads.varlen_inputs(lengths, D, N, dtype, seed=256)
+    T = inp.meta["total"]
+    y, hl = _varlen_run(inp, dtype, round_up(T, 8))
     ref = oracle.scan_varlen(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.cu_seqlens, inp.Dskip, inp.bias, inp.z,
                              nthreads=NTHREADS)
     check("y", y, ref["y"], ref["y_mag"], TOL[dtype], dtype)

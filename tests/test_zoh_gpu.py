@@ -45,6 +45,7 @@ def _widen_range(inp):
     (1, 24, 32, 512),
     (1, 12, 64, 304),
     (1, 10, 128, 200),     # N=128 (narrow 16-warp tile for bf16)
+    (1, 9, 256, 160),      # N=256
 ])
 def test_zoh_batch_matches_oracle(shape, dtype):
     b, D, N, L = shape
