@@ -48,17 +48,30 @@ def peaks():
         return 6650.0, 1965.0, "fallback"
 
 
+# The timed scan kernel is defined by these sources and by the tile-shape line of its
+# workload (the wide N=16 tile) in ssm_api.cu.
+KERNEL_SOURCES = ("chunk_scan.cuh", "common.cuh")
+KERNEL_SHAPE_LINE = "template <> struct Shape<16, false>"
+
+
+def _code_only(text: str) -> str:
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources with comments and blank lines removed (a comment edit keeps
-    the committed ncu counters valid; any code change invalidates them)."""
+    """Hash of the timed scan kernel's code: its sources without comments and blank lines,
+    plus its tile-shape line.  Comment edits and changes to other kernels or to host code
+    keep the committed ncu counters valid; a change to the kernel's code or tile does not."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_15_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
-            text = f.read()
-        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
-        h.update(name.encode() + "\n".join(ln for ln in lines if ln).encode())
+            h.update(name.encode() + _code_only(f.read()).encode())
+    with open(os.path.join(csrc, "ssm_api.cu"), encoding="utf-8") as f:
+        shape = [ln.strip() for ln in f if ln.startswith(KERNEL_SHAPE_LINE)]
+    h.update("\n".join(shape).encode())
     return h.hexdigest()[:16]
 
 

@@ -41,6 +41,10 @@
 // Windows start at the sequence start rounded down to a 16-byte boundary; steps outside
 // [seq_start, seq_end) are made identities (Delta = 0, Delta*u = 0, B = 0) and are not
 // stored, which also resets the state at packed-sequence boundaries ("ufo.work" §4.2).
+//
+// Discretisation.  Euler (B-bar = Delta B) by default; with ZOH the zero-order hold of the
+// "企业官网建设流程全解析" page (discosf.com), §1.2: the lane keeps u instead of Delta*u and
+// scales it per (step, state) by (exp(Delta A) - 1) / A (zoh_coef2 in common.cuh).
 #pragma once
 
 #include <type_traits>

@@ -145,3 +145,28 @@ def test_workspace_size_query_is_host_only(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(FileNotFoundError):
         ssm.load(str(tmp_path / "nope.so"))
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    """bench.kernel_source_hash: comment edits keep the committed ncu counters, code edits void them."""
+    import shutil
+    import sys
+    root = os.path.dirname(os.path.dirname(__file__))
+    sys.path.insert(0, root)
+    import bench
+    csrc = os.path.join(root, "selective_state_space_15_b200", "csrc")
+    fake = tmp_path / "selective_state_space_15_b200" / "csrc"
+    fake.mkdir(parents=True)
+    for name in os.listdir(csrc):
+        shutil.copy(os.path.join(csrc, name), fake / name)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.kernel_source_hash()
+    src = fake / "chunk_scan.cuh"
+    text = src.read_text()
+    src.write_text("// a new comment line\n" + text.replace("namespace ssm {", "namespace ssm {  /* note */", 1))
+    assert bench.kernel_source_hash() == base
+    src.write_text(text.replace("constexpr int kMaxSortedSeqs = 64;", "constexpr int kMaxSortedSeqs = 32;"))
+    assert bench.kernel_source_hash() != base
+    src.write_text(text)
+    (fake / "state_update.cuh").write_text("// decode kernel changed\nint x;\n")
+    assert bench.kernel_source_hash() == base
