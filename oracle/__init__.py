@@ -16,7 +16,9 @@ Definitions followed (cited by page title and section; see ``ssm_oracle.c`` for 
   * ufo.work §4.2 -- packed sequences restart from h = 0 at each cu_seqlens boundary;
   * ufo.work §4.1 -- single-token update of a persistent per-request state;
   * discosf.com §1.2 -- the zero-order-hold input matrix Bbar = (ΔA)^-1 (exp(ΔA) - I) ΔB,
-    chosen with ``zoh=True`` (default: Bbar = ΔB).
+    chosen with ``zoh=True`` (default: Bbar = ΔB);
+  * ufo.work §2.2 -- the training backward pass; ``scan_bwd`` returns the gradients that the
+    forward definition fixes (reverse-mode derivative of ``scan``).
 """
 from __future__ import annotations
 
@@ -60,6 +62,8 @@ def _load():
             lib.oracle_scan_varlen.restype = ctypes.c_int
             lib.oracle_state_update.argtypes = [I, I, I, P, P, P, I] + [P] * 10 + [ctypes.c_int]
             lib.oracle_state_update.restype = ctypes.c_int
+            lib.oracle_scan_bwd.argtypes = [I, I, I, I] + [P] * 20 + [ctypes.c_int, ctypes.c_int]
+            lib.oracle_scan_bwd.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -235,6 +239,37 @@ def state_update(pool, slot_ids, u, delta, B, C, A, Dskip=None, bias=None, z=Non
     if rc != 0:
         raise ValueError(f"oracle_state_update rejected its arguments (code {rc})")
     return {"y": y, "y_mag": y_mag}
+
+
+def scan_bwd(u, delta, B, C, A, dy, Dskip=None, bias=None, z=None, h0=None, dh_last=None, nthreads: int = 1,
+             zoh: bool = False):
+    """Gradients of the fixed-length batch scan (the reverse-mode derivative of ``scan``).
+
+    Given dy = dL/dy [batch, dim, L] and optionally dh_last = dL/dh_last [batch, dim, N],
+    returns du, ddelta, dz (None without z) [batch, dim, L]; dB, dC [batch, N, L];
+    dA [dim, N]; dDskip, dbias [dim]; dh0 [batch, dim, N] (the gradient for the initial state,
+    whether or not one is given).  The ufo.work page, §2.2, describes how training keeps or
+    recomputes the states for this pass; the values are fixed by the forward definition.
+    """
+    u, delta, B, C, A, dy = (_f64(x) for x in (u, delta, B, C, A, dy))
+    z, Dskip, bias, h0, dh_last = (_f64(x) for x in (z, Dskip, bias, h0, dh_last))
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    assert delta.shape == u.shape and dy.shape == u.shape and B.shape == (batch, N, L) and C.shape == B.shape
+    assert A.shape == (dim, N)
+    for x, shape in ((z, u.shape), (h0, (batch, dim, N)), (dh_last, (batch, dim, N))):
+        assert x is None or x.shape == shape
+    out = {"du": np.empty_like(u), "ddelta": np.empty_like(u), "dz": np.empty_like(u) if z is not None else None,
+           "dB": np.empty_like(B), "dC": np.empty_like(C), "dA": np.empty_like(A),
+           "dDskip": np.empty(dim), "dbias": np.empty(dim), "dh0": np.empty((batch, dim, N))}
+    rc = _load().oracle_scan_bwd(batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C), _ptr(A),
+                                 _ptr(Dskip), _ptr(bias), _ptr(h0), _ptr(dy), _ptr(dh_last),
+                                 _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dB"]),
+                                 _ptr(out["dC"]), _ptr(out["dA"]), _ptr(out["dDskip"]), _ptr(out["dbias"]),
+                                 _ptr(out["dh0"]), int(bool(zoh)), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_scan_bwd rejected its arguments (code {rc})")
+    return out
 
 
 def scaled_error(x, ref, mag) -> float:

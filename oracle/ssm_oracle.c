@@ -240,3 +240,215 @@ int oracle_state_update(int64_t num_slots, int64_t dim, int64_t dstate,
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------------------------------
+ * Backward (the adjoint of oracle_scan).  The ufo.work page, §2.2, discusses how a training
+ * backward pass keeps or recomputes the states h_t; what it computes is fixed by the forward
+ * definition: the gradients of a scalar loss L, given dL/dy (dy) and optionally dL/dh_last
+ * (dh_last), with respect to every input.  This is the plain reverse-mode derivative of the
+ * loop above: the forward states of a channel are recomputed and stored, then the loop runs
+ * backwards over t.
+ *
+ *   y_t   = yraw_t g(z_t),  yraw_t = sum_n C_t[n] h_t[n] + D u_t,  g = SiLU (1 without z)
+ *   h_t   = a_t h_{t-1} + c_t B_t u_t,  a_t = exp(Delta_t A),  c_t = input_coef(Delta_t, A)
+ *   Delta = softplus(delta + bias)
+ *
+ * Outputs: du, ddelta, dz : [batch][dim][seqlen];  dB, dC : [batch][dstate][seqlen];
+ * dA : [dim][dstate];  dDskip, dbias : [dim];  dh0 : [batch][dim][dstate] (optional).
+ */
+
+static double sigmoid(double x) {
+  if (x >= 0.0) return 1.0 / (1.0 + exp(-x));
+  const double e = exp(x);
+  return e / (1.0 + e);
+}
+
+/* d/dz SiLU(z) = sigma(z) (1 + z (1 - sigma(z))). */
+static double silu_grad(double z) {
+  const double s = sigmoid(z);
+  return s * (1.0 + z * (1.0 - s));
+}
+
+/* Partial derivatives of the input coefficient c(Delta, A).  Euler: c = Delta.  Zero-order
+ * hold: c = expm1(x)/x * Delta with x = Delta A, so dc/dDelta = exp(x) and
+ * dc/dA = Delta^2 phi'(x) with phi(x) = expm1(x)/x, phi'(x) = (x e^x - expm1(x)) / x^2; near
+ * x = 0 the series phi'(x) = sum_{k>=1} k x^(k-1) / (k+1)! avoids the cancellation. */
+static void input_coef_grad(int zoh, double dt, double a, double *dc_ddt, double *dc_da) {
+  if (!zoh) {
+    *dc_ddt = 1.0;
+    *dc_da = 0.0;
+    return;
+  }
+  const double x = dt * a;
+  *dc_ddt = exp(x);
+  double dphi;
+  if (fabs(x) < 1e-2) {
+    double term = 1.0, fact = 2.0;           /* x^(k-1), (k+1)! */
+    dphi = 0.0;
+    for (int k = 1; k <= 8; ++k) {
+      dphi += k * term / fact;
+      term *= x;
+      fact *= (double)(k + 2);
+    }
+  } else {
+    dphi = (x * exp(x) - expm1(x)) / (x * x);
+  }
+  *dc_da = dt * dt * dphi;
+}
+
+typedef struct {
+  chan_job f;                 /* forward description of the channel (y fields unused)   */
+  int64_t b, d;               /* batch row and channel                                 */
+  const double *dy;           /* len values                                            */
+  const double *dh_last;      /* dstate values or NULL                                 */
+  double *du, *ddelta, *dz;   /* len values (dz only with a gate)                      */
+  double *dh0;                /* dstate values or NULL                                 */
+} bwd_job;
+
+typedef struct {
+  const bwd_job *jobs;
+  int64_t njobs, first, step;
+  int64_t dim, dstate, seqlen;
+  /* this worker's accumulators */
+  double *dB, *dC;            /* [batch][dstate][seqlen] */
+  double *dA;                 /* [dim][dstate]           */
+  double *dDskip, *dbias;     /* [dim]                   */
+} bwd_worker;
+
+static void scan_channel_bwd(const bwd_job *j, bwd_worker *w) {
+  const chan_job *f = &j->f;
+  const int64_t N = f->dstate, L = f->len;
+  double *H = (double *)malloc(sizeof(double) * (size_t)(N * (L > 0 ? L : 1)));
+  double *hprev0 = (double *)malloc(sizeof(double) * (size_t)N);
+  double *dh = (double *)malloc(sizeof(double) * (size_t)N);
+  /* forward: states h_t for every step */
+  for (int64_t n = 0; n < N; ++n) hprev0[n] = f->h0 ? f->h0[n] : 0.0;
+  for (int64_t t = 0; t < L; ++t) {
+    const double dt = softplus(f->delta[t] + f->bias);
+    for (int64_t n = 0; n < N; ++n) {
+      const double hp = t > 0 ? H[(t - 1) * N + n] : hprev0[n];
+      const double c = input_coef(f->zoh, dt, f->A[n]);
+      H[t * N + n] = exp(dt * f->A[n]) * hp + c * f->B[n * f->bc_stride + t] * f->u[t];
+    }
+  }
+  /* backward over t */
+  for (int64_t n = 0; n < N; ++n) dh[n] = j->dh_last ? j->dh_last[n] : 0.0;
+  double *dB = w->dB + j->b * N * w->seqlen, *dC = w->dC + j->b * N * w->seqlen;
+  double *dA = w->dA + j->d * N;
+  for (int64_t t = L - 1; t >= 0; --t) {
+    const double ut = f->u[t];
+    const double s = f->delta[t] + f->bias;
+    const double dt = softplus(s);
+    double yraw = f->dskip * ut;
+    for (int64_t n = 0; n < N; ++n) yraw += f->C[n * f->bc_stride + t] * H[t * N + n];
+    double dyraw = j->dy[t];
+    if (f->z) {
+      j->dz[t] = j->dy[t] * yraw * silu_grad(f->z[t]);
+      dyraw *= silu(f->z[t]);
+    }
+    w->dDskip[j->d] += dyraw * ut;
+    double du = dyraw * f->dskip;
+    double ddt = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+      const double Bt = f->B[n * f->bc_stride + t], Ct = f->C[n * f->bc_stride + t];
+      const double hp = t > 0 ? H[(t - 1) * N + n] : hprev0[n];
+      const double a = exp(dt * f->A[n]);
+      const double c = input_coef(f->zoh, dt, f->A[n]);
+      double dc_ddt, dc_da;
+      input_coef_grad(f->zoh, dt, f->A[n], &dc_ddt, &dc_da);
+      dh[n] += dyraw * Ct;                     /* y_t reads h_t */
+      dC[n * w->seqlen + t] += dyraw * H[t * N + n];
+      const double dcoef = dh[n] * Bt * ut;    /* h_t = a h_{t-1} + c B u */
+      dB[n * w->seqlen + t] += dh[n] * c * ut;
+      du += dh[n] * c * Bt;
+      const double da = dh[n] * hp;
+      ddt += da * a * f->A[n] + dcoef * dc_ddt;
+      dA[n] += da * a * dt + dcoef * dc_da;
+      dh[n] *= a;                              /* on to h_{t-1} */
+    }
+    j->du[t] = du;
+    const double dd = ddt * sigmoid(s);        /* softplus' = sigmoid */
+    j->ddelta[t] = dd;
+    w->dbias[j->d] += dd;
+  }
+  if (j->dh0)
+    for (int64_t n = 0; n < N; ++n) j->dh0[n] = dh[n];
+  free(H);
+  free(hprev0);
+  free(dh);
+}
+
+static void *bwd_worker_run(void *p) {
+  bwd_worker *w = (bwd_worker *)p;
+  for (int64_t i = w->first; i < w->njobs; i += w->step) scan_channel_bwd(&w->jobs[i], w);
+  return NULL;
+}
+
+/* Gradients of the fixed-length batch scan.  Optional: z (then dz is written), Dskip, bias,
+ * h0, dh_last, dh0.  The per-channel outputs are written; the shared ones (dB, dC, dA,
+ * dDskip, dbias) are summed over every (batch, channel, t) that uses them. */
+int oracle_scan_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                    const double *u, const double *delta, const double *z,
+                    const double *B, const double *C, const double *A,
+                    const double *Dskip, const double *bias, const double *h0,
+                    const double *dy, const double *dh_last,
+                    double *du, double *ddelta, double *dz, double *dB, double *dC, double *dA,
+                    double *dDskip, double *dbias, double *dh0, int zoh, int nthreads) {
+  if (batch < 0 || dim < 0 || dstate <= 0 || seqlen < 0) return 1;
+  const int64_t njobs = batch * dim;
+  bwd_job *jobs = (bwd_job *)calloc((size_t)(njobs > 0 ? njobs : 1), sizeof(bwd_job));
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t d = 0; d < dim; ++d) {
+      bwd_job *j = &jobs[b * dim + d];
+      const int64_t xo = (b * dim + d) * seqlen, so = (b * dim + d) * dstate;
+      chan_job *f = &j->f;
+      f->dstate = dstate; f->len = seqlen; f->bc_stride = seqlen; f->zoh = zoh;
+      f->u = u + xo; f->delta = delta + xo; f->z = z ? z + xo : NULL;
+      f->B = B + b * dstate * seqlen; f->C = C + b * dstate * seqlen;
+      f->A = A + d * dstate;
+      f->dskip = Dskip ? Dskip[d] : 0.0; f->bias = bias ? bias[d] : 0.0;
+      f->h0 = h0 ? h0 + so : NULL;
+      j->b = b; j->d = d;
+      j->dy = dy + xo; j->dh_last = dh_last ? dh_last + so : NULL;
+      j->du = du + xo; j->ddelta = ddelta + xo; j->dz = z ? dz + xo : NULL;
+      j->dh0 = dh0 ? dh0 + so : NULL;
+    }
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > njobs) nthreads = njobs > 0 ? (int)njobs : 1;
+  const size_t nbc = (size_t)(batch * dstate * seqlen), na = (size_t)(dim * dstate);
+  bwd_worker *ws = (bwd_worker *)calloc((size_t)nthreads, sizeof(bwd_worker));
+  for (int i = 0; i < nthreads; ++i) {
+    bwd_worker *w = &ws[i];
+    w->jobs = jobs; w->njobs = njobs; w->first = i; w->step = nthreads;
+    w->dim = dim; w->dstate = dstate; w->seqlen = seqlen;
+    w->dB = (double *)calloc(nbc ? nbc : 1, sizeof(double));
+    w->dC = (double *)calloc(nbc ? nbc : 1, sizeof(double));
+    w->dA = (double *)calloc(na ? na : 1, sizeof(double));
+    w->dDskip = (double *)calloc((size_t)(dim ? dim : 1), sizeof(double));
+    w->dbias = (double *)calloc((size_t)(dim ? dim : 1), sizeof(double));
+  }
+  if (nthreads == 1) {
+    bwd_worker_run(&ws[0]);
+  } else {
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, bwd_worker_run, &ws[i]);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+  }
+  /* the workers' partial sums, in worker order */
+  memset(dB, 0, sizeof(double) * nbc);
+  memset(dC, 0, sizeof(double) * nbc);
+  memset(dA, 0, sizeof(double) * na);
+  memset(dDskip, 0, sizeof(double) * (size_t)dim);
+  memset(dbias, 0, sizeof(double) * (size_t)dim);
+  for (int i = 0; i < nthreads; ++i) {
+    bwd_worker *w = &ws[i];
+    for (size_t k = 0; k < nbc; ++k) { dB[k] += w->dB[k]; dC[k] += w->dC[k]; }
+    for (size_t k = 0; k < na; ++k) dA[k] += w->dA[k];
+    for (int64_t k = 0; k < dim; ++k) { dDskip[k] += w->dDskip[k]; dbias[k] += w->dbias[k]; }
+    free(w->dB); free(w->dC); free(w->dA); free(w->dDskip); free(w->dbias);
+  }
+  free(ws);
+  free(jobs);
+  return 0;
+}

@@ -466,3 +466,74 @@ def test_zoh_varlen_and_decode_agree_with_the_fixed_length_scan():
                                       p["z"][0, :, t][None], zoh=True)
             np.testing.assert_allclose(dec["y"][0], v["y"][:, t], rtol=1e-12, atol=1e-13)
         np.testing.assert_allclose(pool[i], v["h_last"][i], rtol=1e-12, atol=1e-13)
+
+
+# ---- backward: the reverse-mode derivative of the scan (ufo.work §2.2 discusses how training
+# ---- keeps or recomputes the states; the values follow from the forward definition) ----
+
+_GRAD_OF = {"u": "du", "delta": "ddelta", "z": "dz", "B": "dB", "C": "dC", "A": "dA", "Dskip": "dDskip",
+            "bias": "dbias", "h0": "dh0"}
+
+
+@pytest.mark.parametrize("zoh", [False, True])
+@pytest.mark.parametrize("gate,h0,A_range,seed", [(True, True, (0.2, 3.0), 400), (False, False, (1e-4, 0.05), 401),
+                                                  (True, False, (2.0, 40.0), 402)])
+def test_backward_matches_central_differences(zoh, gate, h0, A_range, seed):
+    """<grad, V> equals the central difference of L = <dy, y> + <dh_last, h_last> along V, for a
+    random direction V of every input (fp64, step 1e-6)."""
+    rng = np.random.default_rng(seed + 10 * zoh)
+    p = _rand_problem(rng, 2, 3, 4, 9, gate=gate, h0=h0, A_range=A_range)
+    p["A"][0, 1] = 0.0                              # the A = 0 limit of the zero-order hold
+    if p["h0"] is None:
+        p["h0"] = np.zeros((2, 3, 4))
+    dy = rng.standard_normal(p["u"].shape)
+    dhl = rng.standard_normal((2, 3, 4))
+    g = oracle.scan_bwd(p["u"], p["delta"], p["B"], p["C"], p["A"], dy, p["Dskip"], p["bias"], p["z"], p["h0"],
+                        dhl, zoh=zoh)
+
+    def loss(q):
+        r = oracle.scan(q["u"], q["delta"], q["B"], q["C"], q["A"], q["Dskip"], q["bias"], q["z"], q["h0"], zoh=zoh)
+        return float((r["y"] * dy).sum() + (r["h_last"] * dhl).sum())
+
+    eps = 1e-6
+    for name, gname in _GRAD_OF.items():
+        if p[name] is None:
+            assert g[gname] is None
+            continue
+        V = rng.standard_normal(p[name].shape)
+        plus, minus = dict(p), dict(p)
+        plus[name] = p[name] + eps * V
+        minus[name] = p[name] - eps * V
+        fd = (loss(plus) - loss(minus)) / (2 * eps)
+        an = float((g[gname] * V).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_backward_of_the_cumulative_sum_case():
+    """A = 0, Euler, no gate, no skip: h_t = sum_{s<=t} Delta_s B_s u_s and y_t = C_t . h_t, so
+    dC_t = sum_d dy_t h_t and dB_s = sum_d Delta_s u_s sum_{t>=s} dy_t C_t (reverse cumsum)."""
+    rng = np.random.default_rng(403)
+    b, D, N, L = 2, 3, 4, 11
+    p = _rand_problem(rng, b, D, N, L, gate=False, h0=False)
+    p["A"][:] = 0.0
+    dy = rng.standard_normal((b, D, L))
+    g = oracle.scan_bwd(p["u"], p["delta"], p["B"], p["C"], p["A"], dy, None, p["bias"])
+    dt = np.logaddexp(0.0, p["delta"] + p["bias"][None, :, None])            # [b, D, L]
+    h = np.cumsum(dt[:, :, None, :] * p["B"][:, None] * p["u"][:, :, None, :], axis=-1)   # [b, D, N, L]
+    dC = np.einsum("bdt,bdnt->bnt", dy, h)
+    rc = np.flip(np.cumsum(np.flip(dy[:, :, None, :] * p["C"][:, None], -1), -1), -1)       # sum_{t>=s}
+    dB = np.einsum("bds,bdns->bns", dt * p["u"], rc)
+    np.testing.assert_allclose(g["dC"], dC, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dB"], dB, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dDskip"], np.einsum("bdt,bdt->d", dy, p["u"]), rtol=1e-12, atol=1e-12)
+
+
+def test_backward_is_independent_of_the_thread_count():
+    rng = np.random.default_rng(404)
+    p = _rand_problem(rng, 3, 5, 4, 13)
+    dy = rng.standard_normal(p["u"].shape)
+    args = (p["u"], p["delta"], p["B"], p["C"], p["A"], dy, p["Dskip"], p["bias"], p["z"], p["h0"])
+    g1 = oracle.scan_bwd(*args, nthreads=1)
+    g4 = oracle.scan_bwd(*args, nthreads=4)
+    for k in g1:
+        np.testing.assert_allclose(g4[k], g1[k], rtol=1e-13, atol=1e-13, err_msg=k)
