@@ -270,7 +270,8 @@ def long_run(name, steps, warmup, hbm_peak, sfu_peak, seqlen=None):
     g.manual_seed(c["seed"])
     mk = lambda *s: torch.randn(*s, generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)  # noqa: E731
     u, dl, z, B, C = mk(1, D, L), mk(1, D, L), mk(1, D, L), mk(1, N, L), mk(1, N, L)
-    A, Dsk, bias = (torch.from_numpy(x).cuda() for x in workloads.channel_params(np.random.default_rng(c["seed"]), D, N))
+    params = workloads.channel_params(np.random.default_rng(c["seed"]), D, N)
+    A, Dsk, bias = (torch.from_numpy(x).cuda() for x in params)
     y = torch.empty_like(u)
     hl = torch.empty(1, D, N, device="cuda")
     ms = time_kernel(lambda: ssm.scan_fwd(u, dl, B, C, A, Dsk, bias, z, y=y, h_last=hl), steps, warmup, stream)
@@ -596,11 +597,14 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_desc(T), "tokens_per_step_rank0": T, "global_batch_tokens": tokens_all / args.steps,
-                   "l2": "inputs 0.58 GB per step > 126 MB L2; no flush", "parallelism": f"dp{world} (independent batches)"},
+        "config": {"workload": workload_desc(T), "tokens_per_step_rank0": T,
+                   "global_batch_tokens": tokens_all / args.steps,
+                   "l2": "inputs 0.58 GB per step > 126 MB L2; no flush",
+                   "parallelism": f"dp{world} (independent batches)"},
         "roofline": {"bound": "alu", "unit": "Gexp/s", "achieved": nexps / launch_s / 1e9, "peak": sfu_peak / 1e9,
                      "frac": nexps / launch_s / sfu_peak, "traffic": traffic,
-                     "peak_note": f"MUFU: {N_SM} SMs x {SFU_PER_CLK_PER_SM} ex2/clk x {sm_max:.0f} MHz; exps/token = D(N+2)"},
+                     "peak_note": f"MUFU: {N_SM} SMs x {SFU_PER_CLK_PER_SM} ex2/clk x {sm_max:.0f} MHz; "
+                                  "exps/token = D(N+2)"},
         "roofline_hbm": {"bound": "hbm", "unit": "GB/s", "achieved": nbytes / launch_s / 1e9, "peak": hbm_peak,
                          "frac": nbytes / launch_s / 1e9 / hbm_peak, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": nbytes},
@@ -644,7 +648,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-secondary", action="store_true", help="skip the long-sequence/decode figures")
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "long_bf16", "long_n128_bf16", "decode_bf16", "tiny_f32", "batch_f32"],
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=[WORKLOAD, "long_bf16", "long_n128_bf16", "decode_bf16", "tiny_f32", "batch_f32"],
                     help="with --kernel-only: time another workload's kernel alone (for ncu captures)")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="with --kernel-only and a long workload: a shorter sequence (profiler captures)")

@@ -234,7 +234,8 @@ def test_extreme_steps():
     # Δ ≈ 30: abar = e^-30 wipes the previous state, h_t ≈ Δ B_t u_t, no overflow
     big = oracle.scan(u, np.full((1, D, L), 30.0), B, C, A, h0=h0)
     assert np.all(np.isfinite(big["y"]))
-    np.testing.assert_allclose(big["h_last"][0], 30.0 * B[0, :, -1][None, :] * u[0, :, -1][:, None], rtol=1e-11, atol=1e-10)
+    np.testing.assert_allclose(big["h_last"][0], 30.0 * B[0, :, -1][None, :] * u[0, :, -1][:, None],
+                               rtol=1e-11, atol=1e-10)
     # Δ ≈ e^-50: abar ≈ 1 and the input term vanishes, so the state stays h0
     tiny = oracle.scan(u, np.full((1, D, L), -50.0), B, C, A, h0=h0)
     np.testing.assert_allclose(tiny["h_last"], h0, rtol=1e-15, atol=1e-20)
