@@ -538,3 +538,27 @@ def test_backward_is_independent_of_the_thread_count():
     g4 = oracle.scan_bwd(*args, nthreads=4)
     for k in g1:
         np.testing.assert_allclose(g4[k], g1[k], rtol=1e-13, atol=1e-13, err_msg=k)
+
+
+# ---- the chunked SSD form (ufo.work second article §1.1, §2.2), scalar A per head ----
+
+@pytest.mark.parametrize("chunk", [1, 5, 16, 64])
+def test_ssd_chunked_form_equals_the_sequential_scan(chunk):
+    from oracle import ssd
+    rng = np.random.default_rng(500 + chunk)
+    H, P, N, L = 3, 4, 8, 37
+    x = rng.standard_normal((H, P, L))
+    dt = np.exp(rng.uniform(np.log(1e-3), np.log(0.5), size=(H, L)))
+    A = -rng.uniform(0.5, 8.0, size=H)
+    B = rng.standard_normal((N, L))
+    C = rng.standard_normal((N, L))
+    h0 = rng.standard_normal((H, P, N))
+    y, hl = ssd.ssd_chunked(x, dt, A, B, C, chunk, h0)
+    # the same problem as a scan over H*P channels: every channel of head h has A[d, :] = A_h
+    # and delta with softplus(delta) = dt (no bias, skip or gate)
+    D = H * P
+    delta = np.repeat(np.log(np.expm1(dt)), P, axis=0)[None]            # [1, D, L]
+    ref = oracle.scan(x.reshape(1, D, L), delta, B[None], C[None], np.repeat(A, P)[:, None] * np.ones((D, N)),
+                      h0=h0.reshape(1, D, N))
+    np.testing.assert_allclose(y.reshape(D, L), ref["y"][0], rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(hl.reshape(D, N), ref["h_last"][0], rtol=1e-10, atol=1e-11)
