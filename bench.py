@@ -196,15 +196,16 @@ def scan_counts(T, D, N, in_bytes, out_bytes, nseq):
 # ------------------------------------------------------------------------------ CPU oracle
 
 class CpuOracle:
-    """The fp64 oracle on all host cores over a bounded channel sample of the packed batch.
+    """The fp64 oracle on the host cores (all of them, or ``threads``) over a bounded channel
+    sample of the packed batch.
 
     Channels are independent, so the sample's time scales to the full batch by D / channels."""
 
-    def __init__(self, inp, budget_s: float):
+    def __init__(self, inp, budget_s: float, threads: int | None = None):
         import oracle
         oracle.build()
         self.oracle, self.inp = oracle, inp
-        self.threads = oracle.default_threads()
+        self.threads = threads or oracle.default_threads()
         self.D = inp.u.shape[0]
         self.T = inp.meta["total"]
         n0 = min(self.D, max(self.threads, 8))
@@ -226,8 +227,12 @@ class CpuOracle:
                           f"channels, scaled by {self.D}/{self.nch}; {t:.2f} s wall"}
 
 
-def cpu_oracle_rate(inp, budget_s: float = 12.0):
-    return CpuOracle(inp, budget_s).measure()
+def cpu_oracle_rate(inp, budget_s: float = 12.0, single_budget_s: float = 6.0):
+    """The oracle on all host cores, with the single-thread rate beside it."""
+    out = CpuOracle(inp, budget_s).measure()
+    one = CpuOracle(inp, single_budget_s, threads=1).measure()
+    out["single_thread"] = {"value": one["value"], "unit": "tokens/s", "cores": 1, "sample": one["sample"]}
+    return out
 
 
 # ------------------------------------------------------------------------------ timing
