@@ -134,6 +134,23 @@ def test_varlen_small_full(lengths, pitch_mult, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_varlen_many_sequences(dtype):
+    """More packed sequences than the kernel ranks by length (64): CTAs take them in order."""
+    rng = np.random.default_rng(77)
+    lengths = [int(x) for x in rng.integers(0, 60, size=150)]
+    lengths[3] = 0
+    lengths[100] = 200
+    D, N = 24, 16
+    inp = workloads.varlen_inputs(lengths, D, N, dtype, seed=78)
+    T = inp.meta["total"]
+    y, hl = _varlen_run(inp, dtype, round_up(T, 8))
+    ref = oracle.scan_varlen(inp.u, inp.delta, inp.B, inp.C, inp.A, inp.cu_seqlens, inp.Dskip, inp.bias, inp.z,
+                             nthreads=NTHREADS)
+    check("y", y, ref["y"], ref["y_mag"], TOL[dtype], dtype)
+    check("h_last", hl, ref["h_last"], ref["h_mag"], TOL[dtype])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_varlen_dstate_256(dtype):
     lengths = [100, 0, 37, 300, 1]
     D, N = 20, 256
