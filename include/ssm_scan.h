@@ -211,6 +211,17 @@ const char *ssm_status_string(ssm_status_t s);
 /* SSM_ABI_VERSION of the built library. */
 int ssm_abi_version(void);
 
+/*
+ * TEST HOOK -- not for production use.  The next fixed-length scan that runs on the
+ * persistent grid (rows 16-byte aligned, more than one chunk) splits every chain into
+ * one-chunk units and starts its unit counter past the first chunk group: no unit of that
+ * group runs, so the units after it wait for a hand-off that never comes.  Their wait is
+ * bounded; on giving up the kernel records SSM_ERR_TIMEOUT in the status word and finishes
+ * with unusable outputs, and the context stays usable.  The hook applies to one launch and
+ * then clears itself.  It lets a test show that the hand-off wait cannot hang the GPU.
+ */
+void ssm_test_drop_first_handoff(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,7 +21,7 @@ DISC_EULER, DISC_ZOH = 0, 1  # ssm_discretization_t
 # Every function the header declares; tests check the library exports all of them.
 EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
             "ssm_get_device_status", "ssm_status_string", "ssm_abi_version", "ssm_scan_fwd_noalloc",
-            "ssm_scan_fwd_varlen_pool")
+            "ssm_scan_fwd_varlen_pool", "ssm_test_drop_first_handoff")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SSM_NOALLOC_SCRATCH_BYTES
 
 
@@ -74,6 +74,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_status_string.argtypes = [ctypes.c_int]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_abi_version.argtypes = []
+    lib.ssm_test_drop_first_handoff.argtypes = []
+    lib.ssm_test_drop_first_handoff.restype = None
     for f in ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_scan_fwd_varlen_pool", "ssm_state_update",
               "ssm_get_device_status"):
         getattr(lib, f).restype = ctypes.c_int

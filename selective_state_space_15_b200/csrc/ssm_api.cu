@@ -3,6 +3,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "ssm_scan.h"
@@ -69,6 +70,9 @@ constexpr int64_t kNarrowChannels16 = 8192, kNarrowChannels128 = 32768;
 
 int64_t groups_of(const ssm_scan_params *p) { return p->ngroups > 1 ? p->ngroups : 1; }
 
+// Test hook (ssm_test_drop_first_handoff): consumed by the next persistent launch.
+std::atomic<bool> g_test_drop_first_handoff{false};
+
 bool make_plan(const ssm_scan_params *p, int64_t nseq, bool varlen, bool vec, Plan &pl) {
   const int N = int(p->dstate);
   const int64_t dim = p->dim, seqlen = p->seqlen;
@@ -128,6 +132,8 @@ ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t str
       group = group < kMinGroup ? kMinGroup : group;
       group = group > pl.nchunks ? pl.nchunks : group;
     }
+    const bool drop_first = g_test_drop_first_handoff.exchange(false);
+    if (drop_first) group = 1;
     const int64_t ngroups = (pl.nchunks + group - 1) / group;
     if (pl.nchains * ngroups > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
     a.ticket = reinterpret_cast<uint32_t *>(w);
@@ -137,6 +143,11 @@ ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t str
     a.group = int(group);
     a.total_units = int(pl.nchains * ngroups);
     blocks = a.total_units < resident ? a.total_units : resident;
+    if (drop_first) {  // the unit counter starts past the first chunk group
+      const uint32_t start = uint32_t(pl.nchains);
+      if (cudaMemcpyAsync(w, &start, sizeof(start), cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    }
   }
   if (blocks > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
   kern<<<unsigned(blocks), Cfg::kThreads, kSmem, stream>>>(a);
@@ -449,5 +460,7 @@ const char *ssm_status_string(ssm_status_t s) {
 }
 
 int ssm_abi_version(void) { return SSM_ABI_VERSION; }
+
+void ssm_test_drop_first_handoff(void) { g_test_drop_first_handoff.store(true); }
 
 }  // extern "C"

@@ -269,6 +269,22 @@ def test_persistent_paths_and_workspace():
     assert ssm.device_status() == 0
 
 
+def test_handoff_wait_is_bounded_and_reported():
+    """The wait for the state handed on between the units of a chain is bounded: with the test
+    hook no unit of the first chunk group runs, the later units give up waiting, the kernel
+    records SSM_ERR_TIMEOUT, and the next call on the same context is correct."""
+    inp = workloads.batch_inputs(1, 8, 16, 1024, "bf16", seed=31)   # 2 chains of 4 chunks
+    ssm.load().ssm_test_drop_first_handoff()
+    run_batch(inp, "bf16")                      # outputs unusable
+    assert ssm.device_status() == 5             # SSM_ERR_TIMEOUT, read and cleared
+    assert ssm.device_status() == 0
+    y, hl = run_batch(inp, "bf16")
+    ref = oracle_batch(inp)
+    check("y", y, ref["y"], ref["y_mag"], TOL["bf16"], "bf16")
+    check("h_last", hl, ref["h_last"], ref["h_mag"], TOL["bf16"])
+    assert ssm.device_status() == 0
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("shape,G", [
     ((2, 64, 16, 512), 2),      # persistent tiles, one group per 32 channels
