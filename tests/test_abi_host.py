@@ -170,3 +170,20 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     src.write_text(text)
     (fake / "state_update.cuh").write_text("// decode kernel changed\nint x;\n")
     assert bench.kernel_source_hash() == base
+
+
+def test_product_path_never_touches_the_oracle():
+    """The library, its binding and its header name no oracle module, file or symbol, and the
+    oracle names nothing of the library: the two share no code."""
+    root = os.path.dirname(os.path.dirname(__file__))
+    pkg = os.path.join(root, "selective_state_space_15_b200")
+    product = [os.path.join(pkg, f) for f in os.listdir(pkg) if f.endswith(".py")]
+    product += [os.path.join(pkg, "csrc", f) for f in os.listdir(os.path.join(pkg, "csrc"))]
+    product += [HEADER]
+    for path in product:
+        text = open(path, encoding="utf-8").read()
+        assert not re.search(r"\boracle\b", text), path
+    for name in ("ssm_oracle.c", "__init__.py", "brute.py", "ssd.py"):
+        text = open(os.path.join(root, "oracle", name), encoding="utf-8").read()
+        assert "selective_state_space_15_b200" not in text and "ssm_scan.h" not in text, name
+        assert not re.search(r"\bcsrc\b|chunk_scan|state_update\.cuh", text), name
