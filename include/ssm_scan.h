@@ -56,7 +56,7 @@ extern "C" {
 typedef enum {
   SSM_OK = 0,
   SSM_ERR_INVALID_ARG = 1, /* null pointer where one is required, bad size/stride/alignment  */
-  SSM_ERR_UNSUPPORTED = 2, /* a valid request this build has no kernel for (e.g. dstate = 24) */
+  SSM_ERR_UNSUPPORTED = 2, /* a valid request the library has no kernel for (e.g. dstate = 24) */
   SSM_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch error, no device, ...)      */
   SSM_ERR_BAD_SLOT = 4,    /* device-detected: a decode slot id outside [0, num_slots)       */
   SSM_ERR_TIMEOUT = 5,     /* device-detected: a bounded wait on another CTA gave up          */
