@@ -7,14 +7,18 @@
  *     h_t[n]  = exp(Delta_t * A[d,n]) * h_{t-1}[n] + Delta_t * B[b,n,t] * u[b,d,t]
  *     y[b,d,t] = (sum_n C[b,n,t] * h_t[n] + Dskip[d] * u[b,d,t]) * silu(z[b,d,t])
  *
+ * (with `discretization = SSM_DISC_ZOH` the input term Delta_t * B is replaced by the
+ * zero-order hold's (exp(Delta_t A[d,n]) - 1) / A[d,n] * B; see ssm_discretization_t)
+ *
  * Sources (web pages on the subject, cited by title and section):
  *   - "会议长序列建模状态空间模型加速：深度剖析Mamba硬件感知算子融合与选择性扫描并行化策略"
  *     (ufo.work) §1.1: the recurrence with Abar = exp(Delta A), Bbar = Delta B, y = C h and
  *     input-dependent Delta, B, C; §3.1: chunk transfer operators composed across chunks;
  *     §4.1: a persistent state pool and a one-token update kernel; §4.2: packed sequences with
  *     cu_seqlens and a state reset at each boundary.
- *   - "企业官网建设流程全解析" (discosf.com) §1.1: the skip term y = C h + D x; §1.3:
- *     Delta = softplus of a per-token linear map (here: delta + per-channel bias).
+ *   - "企业官网建设流程全解析" (discosf.com) §1.1: the skip term y = C h + D x; §1.2: the
+ *     zero-order-hold discretisation; §1.3: Delta = softplus of a per-token linear map (here:
+ *     delta + per-channel bias).
  *   The pages do not fix the bias placement or the output gate; this library puts the bias
  *   inside the softplus and multiplies the whole output by silu(z) = z * sigmoid(z) when z is
  *   given.  The gated value never feeds back into the state.
