@@ -26,3 +26,40 @@ def test_zoh_coefficient_formula_in_float32():
     rel = np.abs(coef - exact) / np.abs(exact)
     assert rel.max() < 2e-6, rel.max()
     assert np.abs(x).max() > 100 and np.abs(x).min() < 1e-6   # both branches and their far ends
+
+
+def test_fast_softplus_formula_in_float32():
+    """The 16-bit-input softplus: w = e^x, log1p(w) by the alternating series
+    w (1 - w (1/2 - w/3 + w^2/4 - w^3/5 + w^4/6 - w^5/7)) for w < 1/8, else ln2 log2(1 + w),
+    and x itself above 15.  Restated in float32 (the MUFU ex2/lg2 stood in for by float32
+    exp2/log2 perturbed by 2 ulp), it stays within 5e-6 relative of fp64 softplus over the
+    deltas and biases of the workloads and beyond (the largest errors, ~2e-6 near x = -29,
+    come from rounding x log2(e) to float32 before the exponential), far inside the 3e-3
+    bf16 budget."""
+    f = np.float32
+    xs = np.linspace(-30.0, 30.0, 200001).astype(f)
+    ulp2 = f(1 + 2 * 2.0 ** -23)
+    w = (np.exp2(xs * f(np.log2(np.e))) * ulp2).astype(f)
+    with np.errstate(over="ignore", invalid="ignore"):        # the unselected series at large w
+        p = (w * f(-1 / 7) + f(1 / 6)).astype(f)
+        for c in (-1 / 5, 1 / 4, -1 / 3, 1 / 2):
+            p = (w * p + f(c)).astype(f)
+        series = (w * (-w * p + f(1))).astype(f)
+    via_log = (f(np.log(2.0)) * (np.log2(f(1) + w) * ulp2)).astype(f)
+    r = np.where(w < f(0.125), series, via_log)
+    got = np.where(xs > f(15), xs, r)
+    ref = np.logaddexp(0.0, xs.astype(np.float64))
+    assert (np.abs(got - ref) / ref).max() < 5e-6
+
+
+def test_fast_silu_formula_in_float32():
+    """The 16-bit-input gate silu(z) = z/2 (1 + tanh(z/2)): with a tanh carrying a relative
+    error of 2^-11 (the documented bound of the approximate MUFU tanh; about 1e-5 measured),
+    the gate stays within 1e-3 of z sigmoid(z) relative to |z|, inside the 3e-3 bf16 budget."""
+    f = np.float32
+    z = np.linspace(-40.0, 40.0, 100001).astype(f)
+    hz = (f(0.5) * z).astype(f)
+    t = (np.tanh(hz) * f(1 + 2.0 ** -11)).astype(f)
+    got = (hz * t + hz).astype(f)
+    ref = z.astype(np.float64) / (1.0 + np.exp(-z.astype(np.float64)))
+    assert (np.abs(got - ref) / np.maximum(np.abs(z), 1e-30)).max() < 1e-3
