@@ -562,3 +562,19 @@ def test_ssd_chunked_form_equals_the_sequential_scan(chunk):
                       h0=h0.reshape(1, D, N))
     np.testing.assert_allclose(y.reshape(D, L), ref["y"][0], rtol=1e-10, atol=1e-11)
     np.testing.assert_allclose(hl.reshape(D, N), ref["h_last"][0], rtol=1e-10, atol=1e-11)
+
+
+@pytest.mark.parametrize("chunk,zoh", [(1, False), (4, False), (64, False), (3, True)])
+def test_chunk_checkpointed_backward_equals_the_unchunked_one(chunk, zoh):
+    """ufo.work §2.2 / its second article §3.1: keeping only chunk-boundary states and
+    recomputing the inside of each chunk during the backward gives the same gradients."""
+    from oracle import bwd_chunked
+    rng = np.random.default_rng(600 + chunk)
+    p = _rand_problem(rng, 2, 3, 4, 11)
+    dy = rng.standard_normal(p["u"].shape)
+    dhl = rng.standard_normal((2, 3, 4))
+    args = (p["u"], p["delta"], p["B"], p["C"], p["A"], dy, p["Dskip"], p["bias"], p["z"], p["h0"], dhl)
+    ref = oracle.scan_bwd(*args, zoh=zoh)
+    got = bwd_chunked.scan_bwd_chunked(*args, chunk=chunk, zoh=zoh)
+    for k in ref:
+        np.testing.assert_allclose(got[k], ref[k], rtol=1e-11, atol=1e-12, err_msg=k)
