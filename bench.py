@@ -48,10 +48,10 @@ def peaks():
         return 6650.0, 1965.0, "fallback"
 
 
-# The timed scan kernel is defined by these sources and by the tile-shape line of its
-# workload (the wide N=16 tile) in ssm_api.cu.
-KERNEL_SOURCES = ("chunk_scan.cuh", "common.cuh")
-KERNEL_SHAPE_LINE = "template <> struct Shape<16, false>"
+# The timed scan kernel (the lane-sequential one, which the varlen workload takes) is defined
+# by these sources and by the lines of ssm_api.cu that fix its tile (lanes per channel, chunk).
+KERNEL_SOURCES = ("seq_scan.cuh", "common.cuh")
+KERNEL_SHAPE_MARKERS = ("constexpr int seq_lpc(", "constexpr int TC = ", "constexpr int kSeqMaxCtasPerSm")
 
 
 def _code_only(text: str) -> str:
@@ -70,7 +70,7 @@ def kernel_source_hash() -> str:
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode() + _code_only(f.read()).encode())
     with open(os.path.join(csrc, "ssm_api.cu"), encoding="utf-8") as f:
-        shape = [ln.strip() for ln in f if ln.startswith(KERNEL_SHAPE_LINE)]
+        shape = [ln.strip() for ln in f if any(m in ln for m in KERNEL_SHAPE_MARKERS)]
     h.update("\n".join(shape).encode())
     return h.hexdigest()[:16]
 

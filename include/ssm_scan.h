@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 4
+#define SSM_ABI_VERSION 5
 
 typedef enum {
   SSM_OK = 0,
@@ -78,6 +78,23 @@ typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
  * Abar = exp(Delta A) in both.
  */
 typedef enum { SSM_DISC_EULER = 0, SSM_DISC_ZOH = 1 } ssm_discretization_t;
+
+/*
+ * Kernel choice for the prefill scans (ssm_scan_fwd, ssm_scan_fwd_varlen,
+ * ssm_scan_fwd_varlen_pool, ssm_scan_fwd_noalloc).  Both compute the same recurrence; they
+ * differ in where the parallelism comes from.
+ *   SSM_ALGO_AUTO:       the library picks (the default).
+ *   SSM_ALGO_CHUNKED:    chunks of every sequence are split into time segments across the
+ *                        lanes of a warp and composed with the chunk transfer operators
+ *                        (ufo.work page, §3.1); suits few, long sequences.  Every case.
+ *   SSM_ALGO_SEQUENTIAL: every lane walks time step by step for one channel and a group of
+ *                        its states (no composition); suits many channels x sequences.
+ *                        dstate 16 or 32, Euler discretisation, 16-byte aligned rows only;
+ *                        other cases return SSM_ERR_UNSUPPORTED.
+ * AUTO takes SEQUENTIAL when it applies and there are at least 16384 (sequence, channel)
+ * pairs, CHUNKED otherwise.  Other values -> SSM_ERR_INVALID_ARG.
+ */
+typedef enum { SSM_ALGO_AUTO = 0, SSM_ALGO_CHUNKED = 1, SSM_ALGO_SEQUENTIAL = 2 } ssm_algorithm_t;
 
 /* Opaque CUDA stream handle; pass a cudaStream_t (they are the same pointer type). */
 typedef struct CUstream_st *ssm_stream_t;
@@ -131,6 +148,7 @@ typedef struct ssm_scan_params {
   int64_t ngroups;         /* channel groups with their own B, C: 0 or 1 = one group (scans)    */
   int64_t bc_group_stride; /* 0 -> dstate * bc_state_stride                                    */
   int32_t discretization;  /* ssm_discretization_t; other values -> SSM_ERR_INVALID_ARG (all calls) */
+  int32_t algorithm;       /* ssm_algorithm_t (prefill scans; ignored by ssm_state_update)        */
 } ssm_scan_params;
 
 /*

@@ -15,8 +15,10 @@ SSM_OK = 0
 _STATUS = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED", 3: "SSM_ERR_CUDA",
            4: "SSM_ERR_BAD_SLOT", 5: "SSM_ERR_TIMEOUT", 6: "SSM_ERR_WORKSPACE"}
 SSM_F32, SSM_BF16 = 0, 1
-ABI_VERSION = 4
+ABI_VERSION = 5
 DISC_EULER, DISC_ZOH = 0, 1  # ssm_discretization_t
+ALGO_AUTO, ALGO_CHUNKED, ALGO_SEQUENTIAL = 0, 1, 2  # ssm_algorithm_t
+_ALGO = {"auto": ALGO_AUTO, "chunked": ALGO_CHUNKED, "sequential": ALGO_SEQUENTIAL}
 
 # Every function the header declares; tests check the library exports all of them.
 EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
@@ -44,6 +46,7 @@ class ScanParams(ctypes.Structure):
         ("A", ctypes.c_void_p), ("Dskip", ctypes.c_void_p), ("delta_bias", ctypes.c_void_p),
         ("h0", ctypes.c_void_p), ("y", ctypes.c_void_p), ("h_last", ctypes.c_void_p),
         ("ngroups", ctypes.c_int64), ("bc_group_stride", ctypes.c_int64), ("discretization", ctypes.c_int32),
+        ("algorithm", ctypes.c_int32),
     ]
 
 
@@ -128,6 +131,15 @@ def _time_contig(*ts):
             raise ValueError("the time (last) axis must have stride 1")
 
 
+def _algo(algorithm) -> int:
+    """ssm_algorithm_t code for 'auto' / 'chunked' / 'sequential' (or the code itself)."""
+    if isinstance(algorithm, str):
+        if algorithm not in _ALGO:
+            raise ValueError(f"algorithm must be one of {sorted(_ALGO)}")
+        return _ALGO[algorithm]
+    return int(algorithm)
+
+
 def _f32(t):
     import torch
     if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
@@ -137,7 +149,8 @@ def _f32(t):
 
 # ----------------------------------------------------------------------------- scans
 
-def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None, zoh=False):
+def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None, zoh=False,
+                algorithm="auto"):
     """Fill ScanParams for the fixed-length layout u/delta/z/y [b, D, L], B/C [b, N, L] (or
     [b, G, N, L]: G channel groups, channel d reading group d // (D / G))."""
     bsz, dim, L = u.shape
@@ -164,20 +177,22 @@ def scan_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None,
     p.A, p.Dskip, p.delta_bias, p.h0 = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(h0)
     p.y, p.h_last = _ptr(y), _ptr(h_last)
     p.discretization = DISC_ZOH if zoh else DISC_EULER
+    p.algorithm = _algo(algorithm)
     return p
 
 
 def scan_fwd(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None,
-             return_last_state=True, stream=None, y_dtype=None, zoh=False):
+             return_last_state=True, stream=None, y_dtype=None, zoh=False, algorithm="auto"):
     """Selective scan over a fixed-length batch.  Returns (y, h_last).
 
     y is allocated in ``y_dtype`` (default: the input dtype; float32 is also accepted).
-    ``zoh``: zero-order-hold input matrix instead of Bbar = Delta B."""
+    ``zoh``: zero-order-hold input matrix instead of Bbar = Delta B.  ``algorithm``: 'auto',
+    'chunked' or 'sequential' (ssm_algorithm_t)."""
     import torch
     y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
     if h_last is None and return_last_state:
         h_last = torch.empty((u.shape[0], u.shape[1], A.shape[1]), device=u.device, dtype=torch.float32)
-    p = scan_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last, zoh)
+    p = scan_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last, zoh, algorithm)
     lib = load()
     ws = lib.ssm_scan_workspace_size(ctypes.byref(p), 0)
     wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
@@ -186,7 +201,7 @@ def scan_fwd(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=
 
 
 def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=None, y=None, h_last=None,
-                  total=None, zoh=False):
+                  total=None, zoh=False, algorithm="auto"):
     """ScanParams for the packed layout u/delta/z/y [D, T(+pad)], B/C [N, T(+pad)] (or
     [G, N, T(+pad)]: G channel groups).
 
@@ -215,11 +230,13 @@ def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=Non
     p.A, p.Dskip, p.delta_bias, p.h0 = _ptr(A), _ptr(Dskip), _ptr(delta_bias), _ptr(h0)
     p.y, p.h_last = _ptr(y), _ptr(h_last)
     p.discretization = DISC_ZOH if zoh else DISC_EULER
+    p.algorithm = _algo(algorithm)
     return p
 
 
 def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, z=None, h0=None, y=None,
-                    h_last=None, total=None, return_last_state=True, stream=None, y_dtype=None, zoh=False):
+                    h_last=None, total=None, return_last_state=True, stream=None, y_dtype=None, zoh=False,
+                    algorithm="auto"):
     """Packed variable-length scan.  cu_seqlens: int32 device tensor [nseq+1].  Returns (y, h_last)."""
     import torch
     if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
@@ -228,7 +245,7 @@ def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, 
     y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
     if h_last is None and return_last_state:
         h_last = torch.empty((nseq, u.shape[0], A.shape[1]), device=u.device, dtype=torch.float32)
-    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last, total, zoh)
+    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, y, h_last, total, zoh, algorithm)
     lib = load()
     ws = lib.ssm_scan_workspace_size(ctypes.byref(p), nseq)
     wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
@@ -238,7 +255,7 @@ def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, 
 
 
 def scan_fwd_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=None, delta_bias=None, z=None,
-                         y=None, total=None, stream=None, y_dtype=None, zoh=False):
+                         y=None, total=None, stream=None, y_dtype=None, zoh=False, algorithm="auto"):
     """Packed prefill into a state pool: sequence i starts from pool[slot_ids[i]] and its final
     state is written back there.  pool: float32 [S, D, N]; slot_ids: int32 [nseq].  Returns y."""
     import torch
@@ -253,7 +270,7 @@ def scan_fwd_varlen_pool(u, delta, B, C, A, cu_seqlens, pool, slot_ids, Dskip=No
     if tuple(pool.shape[1:]) != (u.shape[0], A.shape[1]):
         raise ValueError("pool must be [S, dim, dstate]")
     y = torch.empty_like(u, dtype=y_dtype or u.dtype) if y is None else y
-    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, None, y, None, total, zoh)
+    p = varlen_params(u, delta, B, C, A, Dskip, delta_bias, z, None, y, None, total, zoh, algorithm)
     lib = load()
     ws = lib.ssm_scan_workspace_size(ctypes.byref(p), nseq)
     wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None

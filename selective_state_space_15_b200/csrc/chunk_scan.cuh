@@ -53,44 +53,6 @@
 
 namespace ssm {
 
-struct ScanArgs {
-  const void *u, *delta, *z, *B, *C;
-  const float *A, *Dskip, *bias, *h0;
-  void *y;
-  float *h_last;
-  const int32_t *cu_seqlens;  // nullptr: fixed-length batch
-  // state rows: sequence s reads h0 and writes h_last at row state_slots[s] of a [num_slots]
-  // [dim][N] pool (h0 == h_last == the pool) when state_slots is set, else at row s
-  const int32_t *state_slots;
-  int64_t num_slots;
-  int64_t dim, seqlen;
-  int64_t x_batch_stride, x_dim_stride, bc_batch_stride, bc_state_stride;
-  int nseq;    // sequences (batch size or number of packed sequences)
-  int ntiles;  // channel tiles per sequence (tiles_per_group per channel group)
-  // channel groups: group g holds channels [g * group_dim, (g + 1) * group_dim) and reads B, C
-  // at offset g * bc_group_stride; a tile never straddles two groups
-  int64_t group_dim, bc_group_stride;
-  int tiles_per_group;
-  // persistent scheduling (fixed-length batches only)
-  uint32_t *ticket;  // work counter, zero at launch
-  uint32_t *flags;   // [nchains] chunk groups completed per chain, zero at launch
-  float *carries;    // [nchains][CT][N] state at the end of the last completed group
-  int nchains;       // nseq * ntiles
-  int group;         // chunks per work unit
-  int total_units;   // nchains * ceil(nchunks / group)
-};
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Packed sequences are visited longest first (CTAs with low indices start first), which
-// keeps the tail short when lengths differ; the ordering is computed in each CTA, so it is
-// only done for modest sequence counts.
-constexpr int kMaxSortedSeqs = 64;
-
 // CW warps hold distinct channel groups; NG warps share them and split the N states.
 template <typename T, int N, int KI, int SPW, int CPW, int CW, int NG>
 struct ChunkCfg {
@@ -711,8 +673,9 @@ chunk_scan_kernel(const ScanArgs args) {
     for (int c = c_begin; c < c_end; ++c, ++gc) {
       const int buf = int(gc & 1u);
       const int64_t wstart = w0 + int64_t(c) * TC;
+      bool landed = true;
       if constexpr (VEC) {
-        mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
+        landed = mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
         if constexpr (Cfg::kBF) {
           // widen the chunk's 16-bit B/C (the single staging copy) into its float32 buffer
           float *dst = bcf + buf * kBFElems;
@@ -728,7 +691,15 @@ chunk_scan_kernel(const ScanArgs args) {
       } else {
         stage_scalar(buf, c);
       }
-      __syncthreads();  // chunk c visible to all; everyone is done with chunk c-1's buffers
+      // chunk c visible to all; everyone is done with chunk c-1's buffers
+      if (__syncthreads_or(!landed)) {
+        // a copy did not land within the bounded wait (SSM_ERR_TIMEOUT is recorded): give up
+        // on this CTA's work, once more waiting (bounded) for the copy in flight so that it
+        // does not write shared memory after the CTA has exited; units that wait for this
+        // chain's hand-off then time out as well instead of waiting for ever
+        mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
+        return;
+      }
       if constexpr (VEC) {
         if (c + 1 < c_end) issue_chunk(buf ^ 1, c + 1);  // streams in while chunk c is computed
       }

@@ -31,24 +31,22 @@ __device__ __forceinline__ float lg2_approx(float x) {
 __device__ __forceinline__ float softplus_precise(float x) {
   return x > 20.f ? x : log1pf(expf(x));
 }
-// Fast form (bf16 inputs): w = e^x through ex2; log1p(w) from the alternating series
-// w - w^2/2 + ... + w^7/7 when w < 1/8 (truncation error below w^8/8, i.e. relative
-// error < 3e-7), else ln2 * log2(1 + w) through lg2, whose absolute error (~1e-7) is small
-// against a result of at least log(1.125) = 0.118 there.
-// Both branches are evaluated and selected (no divergence); the unselected one may be
-// inf/nan for large x, which a select does not propagate.
+// Fast form (one MUFU operation): softplus(x) = max(x, 0) + log1p(w) with w = e^-|x| in
+// (0, 1], and log1p(w) = w q(w) where q(w) = log1p(w) / w is smooth on [0, 1] (q(0) = 1,
+// q(1) = ln 2).  q is a degree-7 polynomial fitted to it in relative error (weighted least
+// squares on Chebyshev nodes, refined towards equal ripple); evaluated in float32 by Horner's
+// rule it stays within 4e-7 of log1p(w) relative, for every w in [0, 1].  No branch, no
+// select: for x -> -inf, w flushes to 0 and the result to 0; for x -> +inf it is x.
 __device__ __forceinline__ float softplus_fast(float x) {
-  const float w = ex2_approx(x * kLog2e);
-  float p = fmaf(w, -1.f / 7.f, 1.f / 6.f);
-  p = fmaf(w, p, -1.f / 5.f);
-  p = fmaf(w, p, 1.f / 4.f);
-  p = fmaf(w, p, -1.f / 3.f);
-  p = fmaf(w, p, 1.f / 2.f);
-  // log1p(w) = w - w^2 (1/2 - w/3 + w^2/4 - ...) = w * (1 - w * p)
-  const float series = w * fmaf(-w, p, 1.f);
-  const float viaLog = kLn2 * lg2_approx(1.f + w);
-  const float r = w < 0.125f ? series : viaLog;
-  return x > 15.f ? x : r;
+  const float w = ex2_approx(-fabsf(x) * kLog2e);
+  float q = fmaf(w, -0.00853909645229578f, 0.044089239090681076f);
+  q = fmaf(w, q, -0.10768117010593414f);
+  q = fmaf(w, q, 0.17745204269886017f);
+  q = fmaf(w, q, -0.24495449662208557f);
+  q = fmaf(w, q, 0.33275479078292847f);
+  q = fmaf(w, q, -0.4999740421772003f);
+  q = fmaf(w, q, 0.9999998211860657f);
+  return fmaf(w, q, fmaxf(x, 0.f));
 }
 
 // silu(z) = z * sigmoid(z) = z / (1 + e^-z).
@@ -199,5 +197,44 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   report_status(5 /* SSM_ERR_TIMEOUT */);
   return false;
 }
+
+// ---- arguments of the prefill scan kernels (filled by the host API) ----
+struct ScanArgs {
+  const void *u, *delta, *z, *B, *C;
+  const float *A, *Dskip, *bias, *h0;
+  void *y;
+  float *h_last;
+  const int32_t *cu_seqlens;  // nullptr: fixed-length batch
+  // state rows: sequence s reads h0 and writes h_last at row state_slots[s] of a [num_slots]
+  // [dim][N] pool (h0 == h_last == the pool) when state_slots is set, else at row s
+  const int32_t *state_slots;
+  int64_t num_slots;
+  int64_t dim, seqlen;
+  int64_t x_batch_stride, x_dim_stride, bc_batch_stride, bc_state_stride;
+  int nseq;    // sequences (batch size or number of packed sequences)
+  int ntiles;  // channel tiles per sequence (tiles_per_group per channel group)
+  // channel groups: group g holds channels [g * group_dim, (g + 1) * group_dim) and reads B, C
+  // at offset g * bc_group_stride; a tile never straddles two groups
+  int64_t group_dim, bc_group_stride;
+  int tiles_per_group;
+  // persistent scheduling (fixed-length batches only)
+  uint32_t *ticket;  // work counter, zero at launch
+  uint32_t *flags;   // [nchains] chunk groups completed per chain, zero at launch
+  float *carries;    // [nchains][CT][N] state at the end of the last completed group
+  int nchains;       // nseq * ntiles
+  int group;         // chunks per work unit
+  int total_units;   // nchains * ceil(nchunks / group) (chunked kernel); units (lane-sequential kernel)
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Packed sequences are visited longest first (CTAs with low indices start first), which
+// keeps the tail short when lengths differ; the ordering is computed in each CTA, so it is
+// only done for modest sequence counts.
+constexpr int kMaxSortedSeqs = 64;
 
 }  // namespace ssm

@@ -4,10 +4,13 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "ssm_scan.h"
 #include "chunk_scan.cuh"
+#include "seq_scan.cuh"
 #include "state_update.cuh"
 
 namespace {
@@ -15,6 +18,36 @@ namespace {
 using ssm::ScanArgs;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Per (kernel, device) launch facts: the dynamic shared-memory attribute is set and the
+// occupancy queried once per device, under a lock, so host threads that drive different
+// GPUs (or the same one) can launch concurrently.
+struct LaunchInfo {
+  ssm_status_t status = SSM_OK;
+  int blocks_per_sm = 0;
+  int num_sms = 0;
+};
+std::mutex g_launch_mutex;
+std::map<std::pair<const void *, int>, LaunchInfo> g_launch_info;
+
+ssm_status_t launch_info(const void *kern, int threads, size_t smem, LaunchInfo &out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_launch_mutex);
+  auto it = g_launch_info.find({kern, dev});
+  if (it == g_launch_info.end()) {
+    LaunchInfo li;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&li.blocks_per_sm, kern, threads, smem) != cudaSuccess ||
+        cudaDeviceGetAttribute(&li.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      li.status = SSM_ERR_CUDA;
+    }
+    if (li.blocks_per_sm < 1) li.blocks_per_sm = 1;
+    it = g_launch_info.emplace(std::make_pair(kern, dev), li).first;
+  }
+  out = it->second;
+  return out.status;
+}
 
 // Tile shapes: KI steps per lane, SPW segment lanes per channel, CPW channels per warp, CW
 // channel warps and NG state groups per CTA; when CPW * SPW < 32 the lanes of a warp form
@@ -60,6 +93,7 @@ bool shape_for(int N, bool narrow, bool f32, ShapeInfo &si) {
 // one CTA per (sequence, tile) otherwise.
 struct Plan {
   bool persist = false, narrow = false;
+  bool seq = false;  // lane-sequential kernel (seq_scan.cuh) instead of the chunked one
   ShapeInfo si{};
   int64_t ntiles = 0, nchains = 0, nchunks = 0;
   size_t flags_off = 0, carries_off = 0, ws_bytes = 0;
@@ -73,11 +107,41 @@ int64_t groups_of(const ssm_scan_params *p) { return p->ngroups > 1 ? p->ngroups
 // Test hook (ssm_test_drop_first_handoff): consumed by the next persistent launch.
 std::atomic<bool> g_test_drop_first_handoff{false};
 
+// Lane-sequential kernel: lanes per channel (LPC: 4 lanes of 4 states for dstate 16, of 8
+// for dstate 32; a CTA of four warps then holds 32 channels), the resident CTAs per SM it is
+// launched with (0: as many as fit), and the number of (sequence, channel) pairs from which
+// AUTO prefers it.  Units are (sequence, 32-channel tile) pairs, about twice as many as CTA
+// slots on the packed workloads, so that the longest-first ticket can even out the tail.
+#ifndef SSM_SEQ_LPC16
+#define SSM_SEQ_LPC16 4
+#endif
+#ifndef SSM_SEQ_MAX_CTAS
+#define SSM_SEQ_MAX_CTAS 0
+#endif
+constexpr int seq_lpc(int N) { return N == 16 ? SSM_SEQ_LPC16 : 4; }
+constexpr int kSeqMaxCtasPerSm = SSM_SEQ_MAX_CTAS;
+constexpr int64_t kSeqMinPairs = 16384;
+bool seq_supported(const ssm_scan_params *p, bool vec) {
+  return vec && (p->dstate == 16 || p->dstate == 32) && p->discretization == SSM_DISC_EULER;
+}
+
+// Returns false when the requested algorithm has no kernel for this problem.
 bool make_plan(const ssm_scan_params *p, int64_t nseq, bool varlen, bool vec, Plan &pl) {
   const int N = int(p->dstate);
   const int64_t dim = p->dim, seqlen = p->seqlen;
   const bool bf16 = p->dtype == SSM_BF16;
   pl = Plan{};
+  if (p->algorithm == SSM_ALGO_SEQUENTIAL ||
+      (p->algorithm == SSM_ALGO_AUTO && seq_supported(p, vec) && nseq * dim >= kSeqMinPairs)) {
+    if (!seq_supported(p, vec)) return false;
+    pl.seq = true;
+    const int64_t G = groups_of(p);
+    const int64_t ct = int64_t(4) * (32 / seq_lpc(N));
+    pl.ntiles = G * ((dim / G + ct - 1) / ct);
+    pl.nchains = nseq * pl.ntiles;
+    pl.ws_bytes = 16;  // the unit ticket
+    return true;
+  }
   pl.persist = !varlen && vec && seqlen > 0;
   pl.narrow = pl.persist && ((N == 16 && nseq * dim < kNarrowChannels16) ||
                              (N == 128 && bf16 && nseq * dim < kNarrowChannels128));
@@ -101,20 +165,9 @@ ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t str
   using Cfg = ssm::ChunkCfg<T, N, S::KI, S::SPW, S::CPW, S::CW, S::NG>;
   auto kern = ssm::chunk_scan_kernel<T, TO, N, S::KI, S::SPW, S::CPW, S::CW, S::NG, HAS_Z, VEC, PERSIST, ZOH>;
   constexpr size_t kSmem = Cfg::kSmemBytes + (ZOH ? Cfg::kInvABytes : 0);
-  static int configured_device = -1;  // the attribute is set once per device function per device
-  static int max_blocks_per_sm = 0;
-  static int num_sms = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
-  if (configured_device != dev) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
-      return SSM_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&max_blocks_per_sm, kern, Cfg::kThreads, kSmem) !=
-        cudaSuccess)
-      return SSM_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SSM_ERR_CUDA;
-    configured_device = dev;
-  }
+  LaunchInfo li;
+  if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, kSmem, li) != SSM_OK) return SSM_ERR_CUDA;
+  const int max_blocks_per_sm = li.blocks_per_sm, num_sms = li.num_sms;
   if (pl.nchains == 0) return SSM_OK;
   int64_t blocks = pl.nchains;
   if constexpr (PERSIST) {
@@ -152,6 +205,38 @@ ssm_status_t launch_chunk(ScanArgs a, const Plan &pl, void *ws, cudaStream_t str
   if (blocks > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
   kern<<<unsigned(blocks), Cfg::kThreads, kSmem, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// Lane-sequential kernel: a persistent grid over (sequence, channel tile) units taken from a
+// ticket in the workspace (zeroed here, on the stream).
+template <typename T, typename TO, int N, bool HAS_Z>
+ssm_status_t launch_seq(ScanArgs a, const Plan &pl, void *ws, cudaStream_t stream) {
+  constexpr int LPC = seq_lpc(N);
+  constexpr int TC = sizeof(T) == 2 ? 32 : 16;  // 64-byte rows either way
+  using Cfg = ssm::SeqCfg<T, N, LPC, TC>;
+  auto kern = ssm::seq_scan_kernel<T, TO, N, LPC, TC, HAS_Z>;
+  LaunchInfo li;
+  if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
+    return SSM_ERR_CUDA;
+  if (pl.nchains == 0) return SSM_OK;
+  if (pl.nchains > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+  if (cudaMemsetAsync(ws, 0, 16, stream) != cudaSuccess) return SSM_ERR_CUDA;
+  a.ticket = static_cast<uint32_t *>(ws);
+  a.total_units = int(pl.nchains);
+  const int per_sm = kSeqMaxCtasPerSm > 0 && kSeqMaxCtasPerSm < li.blocks_per_sm ? kSeqMaxCtasPerSm : li.blocks_per_sm;
+  const int64_t resident = int64_t(li.num_sms) * per_sm;
+  const int64_t blocks = pl.nchains < resident ? pl.nchains : resident;
+  kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+template <typename T, typename TO>
+ssm_status_t dispatch_seq(const ScanArgs &a, const Plan &pl, int N, bool has_z, void *ws, cudaStream_t st) {
+  switch (N) {
+    case 16: return has_z ? launch_seq<T, TO, 16, true>(a, pl, ws, st) : launch_seq<T, TO, 16, false>(a, pl, ws, st);
+    case 32: return has_z ? launch_seq<T, TO, 32, true>(a, pl, ws, st) : launch_seq<T, TO, 32, false>(a, pl, ws, st);
+    default: return SSM_ERR_UNSUPPORTED;
+  }
 }
 
 template <typename T, typename TO, int N, bool NARROW, bool ZOH>
@@ -205,6 +290,8 @@ ssm_status_t prepare_scan(const ssm_scan_params *p, bool varlen, ScanArgs &a, bo
   if (!p) return SSM_ERR_INVALID_ARG;
   if (p->dtype != SSM_F32 && p->dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
   if (p->discretization != SSM_DISC_EULER && p->discretization != SSM_DISC_ZOH) return SSM_ERR_INVALID_ARG;
+  if (p->algorithm != SSM_ALGO_AUTO && p->algorithm != SSM_ALGO_CHUNKED && p->algorithm != SSM_ALGO_SEQUENTIAL)
+    return SSM_ERR_INVALID_ARG;
   if (p->dim <= 0 || p->dstate <= 0 || p->seqlen < 0 || p->batch < 0) return SSM_ERR_INVALID_ARG;
   if (varlen && p->batch != 1) return SSM_ERR_INVALID_ARG;
   if (!p->u || !p->delta || !p->B || !p->C || !p->A || !p->y) return SSM_ERR_INVALID_ARG;
@@ -247,6 +334,12 @@ ssm_status_t run_scan(ScanArgs a, const Plan &pl, ssm_dtype_t dt, bool y_fp32, i
   a.ntiles = int(pl.ntiles);
   a.tiles_per_group = int(pl.ntiles / (a.dim / a.group_dim));
   const bool has_z = a.z != nullptr;
+  if (pl.seq) {
+    if (dt == SSM_BF16)
+      return y_fp32 ? dispatch_seq<__nv_bfloat16, float>(a, pl, N, has_z, ws, st)
+                    : dispatch_seq<__nv_bfloat16, __nv_bfloat16>(a, pl, N, has_z, ws, st);
+    return dispatch_seq<float, float>(a, pl, N, has_z, ws, st);
+  }
   if (dt == SSM_BF16) {
     if (y_fp32) return dispatch_disc<__nv_bfloat16, float>(a, pl, N, has_z, vec, zoh, ws, st);
     return dispatch_disc<__nv_bfloat16, __nv_bfloat16>(a, pl, N, has_z, vec, zoh, ws, st);

@@ -74,6 +74,7 @@ def _params(**kw):
     ("x_dim_stride", 100, 1),           # row stride shorter than the sequence
     ("bc_state_stride", 100, 1),
     ("discretization", 2, 1), ("discretization", -1, 1),   # neither Euler nor zero-order hold
+    ("algorithm", 3, 1), ("algorithm", -1, 1),             # no such kernel choice
 ])
 def test_scan_rejects_bad_arguments_on_host(lib, field, value, code):
     p = _params(**{field: value})
@@ -137,6 +138,38 @@ def test_state_update_host_checks(lib):
     assert lib.ssm_state_update(fake, 4, fake, 8, ctypes.byref(p4), None) == 1     # unknown discretisation
 
 
+def test_algorithm_choice_on_host(lib):
+    """The sequential kernel takes dstate 16 and 32 with the Euler input matrix and 16-byte
+    aligned rows; other requests for it are refused before anything runs.  AUTO takes it from
+    16384 (sequence, channel) pairs on; its workspace is the 16-byte unit ticket."""
+    seq, chunked = ssm.ALGO_SEQUENTIAL, ssm.ALGO_CHUNKED
+    f = lib.ssm_scan_fwd
+    assert f(ctypes.byref(_params(dstate=64, algorithm=seq)), None, 0, None) == 2
+    assert f(ctypes.byref(_params(discretization=ssm.DISC_ZOH, algorithm=seq)), None, 0, None) == 2
+    assert f(ctypes.byref(_params(x_dim_stride=129, seqlen=128, algorithm=seq)), None, 0, None) == 2  # odd rows
+    assert f(ctypes.byref(_params(algorithm=seq)), None, 0, None) == 6          # needs its ticket
+    size = lib.ssm_scan_workspace_size
+    assert size(ctypes.byref(_params(algorithm=seq)), 0) == 16
+    assert size(ctypes.byref(_params(dstate=32, algorithm=seq)), 0) == 16
+    # AUTO: 16 x 1024 pairs -> sequential; 1 x 1024 -> chunked (persistent: ticket, flags, carries)
+    assert size(ctypes.byref(_params(batch=16, dim=1024)), 0) == 16
+    assert size(ctypes.byref(_params(batch=1, dim=1024)), 0) > 16
+    assert size(ctypes.byref(_params(batch=16, dim=1024, algorithm=chunked)), 0) > 16
+    # packed sequences: 16 sequences x 2048 channels take the sequential kernel, 4 x 2048 the
+    # chunked one (one CTA per sequence and tile: no workspace)
+    assert size(ctypes.byref(_params(dim=2048, seqlen=4096)), 16) == 16
+    assert size(ctypes.byref(_params(dim=2048, seqlen=4096)), 4) == 0
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch(lib):
+    """ssm_scan_fwd_noalloc refuses, on the host and before anything runs, a problem whose
+    scratch need exceeds SSM_NOALLOC_SCRATCH_BYTES (here the chunked kernel's hand-off carries
+    of 2048 chains, 4.2 MB)."""
+    p = _params(batch=64, dim=1024, seqlen=4096, algorithm=ssm.ALGO_CHUNKED)
+    assert lib.ssm_scan_workspace_size(ctypes.byref(p), 0) > ssm.NOALLOC_SCRATCH_BYTES
+    assert lib.ssm_scan_fwd_noalloc(ctypes.byref(p), None) == 6                  # SSM_ERR_WORKSPACE
+
+
 def test_workspace_size_query_is_host_only(lib):
     p = _params()
     assert lib.ssm_scan_workspace_size(ctypes.byref(p), 0) >= 0
@@ -161,14 +194,21 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
         shutil.copy(os.path.join(csrc, name), fake / name)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     base = bench.kernel_source_hash()
-    src = fake / "chunk_scan.cuh"
+    src = fake / "seq_scan.cuh"
     text = src.read_text()
     src.write_text("// a new comment line\n" + text.replace("namespace ssm {", "namespace ssm {  /* note */", 1))
     assert bench.kernel_source_hash() == base
-    src.write_text(text.replace("constexpr int kMaxSortedSeqs = 64;", "constexpr int kMaxSortedSeqs = 32;"))
+    src.write_text(text.replace("static constexpr int kWarps = 4;", "static constexpr int kWarps = 8;"))
     assert bench.kernel_source_hash() != base
     src.write_text(text)
+    api = fake / "ssm_api.cu"
+    api_text = api.read_text()
+    api.write_text(api_text.replace("constexpr int seq_lpc(int N) {", "constexpr int seq_lpc(int N) { /**/ ", 1)
+                   .replace("? 2 : 4;", "? 4 : 4;", 1))
+    assert bench.kernel_source_hash() != base                      # the tile of the timed kernel
+    api.write_text(api_text)
     (fake / "state_update.cuh").write_text("// decode kernel changed\nint x;\n")
+    (fake / "chunk_scan.cuh").write_text("// chunked kernel changed\nint y;\n")
     assert bench.kernel_source_hash() == base
 
 
