@@ -51,7 +51,7 @@ def peaks():
 # The timed scan kernel (the lane-sequential one, which the varlen workload takes) is defined
 # by these sources and by the lines of ssm_api.cu that fix its tile (lanes per channel, chunk).
 KERNEL_SOURCES = ("seq_scan.cuh", "common.cuh")
-KERNEL_SHAPE_MARKERS = ("constexpr int seq_lpc(", "constexpr int TC = ", "constexpr int kSeqMaxCtasPerSm")
+KERNEL_SHAPE_MARKERS = ("#define SSM_SEQ_", "constexpr int seq_lpc(", "constexpr int TC = ", "constexpr int kSeq")
 
 
 def _code_only(text: str) -> str:

@@ -197,6 +197,52 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
                               const ssm_scan_params *p, ssm_stream_t stream);
 
 /*
+ * Gradients of the fixed-length batch scan: the reverse-mode derivative of ssm_scan_fwd's
+ * outputs y and h_last with respect to u, delta, z, B, C, A, Dskip, delta_bias and h0, for
+ * training.  It follows the schedule of the "会议长序列建模…" page (ufo.work), §2.2 (strategy B:
+ * keep checkpoints, recompute the rest) and its second article, §3.1 (chunk-level checkpoints):
+ * a forward pass keeps only the state every few steps (in the workspace), then the sequence
+ * is walked backwards, each short stretch recomputed from its checkpoint and the adjoint
+ * recurrence dh_{t-1} = exp(Delta_t A) (dh_t + C_t dyraw_t) carried from the end.
+ *
+ * `p` describes the forward problem exactly as for ssm_scan_fwd (the same inputs).  Supported:
+ * dstate 16, ngroups <= 1, the Euler input matrix (p->discretization = SSM_DISC_EULER), and
+ * every tensor base and row stride 16-byte aligned (the forward's fast path; dy, du, ddelta and
+ * dz included).  Other cases return SSM_ERR_UNSUPPORTED before anything runs.
+ *
+ * Every gradient is overwritten (not accumulated into).  "The dtype of y" below is the input
+ * dtype, or float32 when p->y_fp32 is set.
+ *   dy          : [batch][dim][seqlen] in the dtype of y, strides as u (required)
+ *   dh_last     : [batch][dim][dstate] float32, gradient of h_last, or NULL (zero)
+ *   du, ddelta  : [batch][dim][seqlen] in the dtype of y, strides as u (required)
+ *   dz          : the same; required when p->z is given, ignored otherwise
+ *   dB, dC      : [batch][dstate][seqlen] float32, contiguous (required)
+ *   dA          : [dim][dstate] float32 (required)
+ *   dDskip, ddelta_bias : [dim] float32, or NULL (not computed)
+ *   dh0         : [batch][dim][dstate] float32, or NULL (not computed)
+ * The workspace (ssm_scan_bwd_workspace_size bytes, 16-byte aligned) holds the checkpoints
+ * and per-tile partial sums of dB and dC; its contents on entry do not matter.
+ */
+typedef struct ssm_scan_grads {
+  const void *dy;
+  const float *dh_last;
+  void *du;
+  void *ddelta;
+  void *dz;
+  float *dB;
+  float *dC;
+  float *dA;
+  float *dDskip;
+  float *ddelta_bias;
+  float *dh0;
+} ssm_scan_grads;
+ssm_status_t ssm_scan_bwd(const ssm_scan_params *p, const ssm_scan_grads *g, void *workspace,
+                          size_t workspace_bytes, ssm_stream_t stream);
+
+/* Bytes of device workspace ssm_scan_bwd needs for this problem (0 if it is not supported). */
+size_t ssm_scan_bwd_workspace_size(const ssm_scan_params *p);
+
+/*
  * Allocation-free variant of ssm_scan_fwd.  (The pages have no counterpart; this is a
  * library convenience.)
  *

@@ -23,7 +23,8 @@ _ALGO = {"auto": ALGO_AUTO, "chunked": ALGO_CHUNKED, "sequential": ALGO_SEQUENTI
 # Every function the header declares; tests check the library exports all of them.
 EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
             "ssm_get_device_status", "ssm_status_string", "ssm_abi_version", "ssm_scan_fwd_noalloc",
-            "ssm_scan_fwd_varlen_pool", "ssm_test_drop_first_handoff")
+            "ssm_scan_fwd_varlen_pool", "ssm_test_drop_first_handoff", "ssm_scan_bwd",
+            "ssm_scan_bwd_workspace_size")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SSM_NOALLOC_SCRATCH_BYTES
 
 
@@ -50,6 +51,12 @@ class ScanParams(ctypes.Structure):
     ]
 
 
+class ScanGrads(ctypes.Structure):
+    """Mirror of ssm_scan_grads."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dy", "dh_last", "du", "ddelta", "dz", "dB", "dC", "dA", "dDskip",
+                                                 "ddelta_bias", "dh0")]
+
+
 _lib = None
 
 
@@ -73,6 +80,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_state_update.argtypes = [P, I64, P, I64, pp, P]
     lib.ssm_scan_workspace_size.argtypes = [pp, I64]
     lib.ssm_scan_workspace_size.restype = S
+    lib.ssm_scan_bwd.argtypes = [pp, ctypes.POINTER(ScanGrads), P, S, P]
+    lib.ssm_scan_bwd_workspace_size.argtypes = [pp]
+    lib.ssm_scan_bwd_workspace_size.restype = S
     lib.ssm_get_device_status.argtypes = [P]
     lib.ssm_status_string.argtypes = [ctypes.c_int]
     lib.ssm_status_string.restype = ctypes.c_char_p
@@ -80,7 +90,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_test_drop_first_handoff.argtypes = []
     lib.ssm_test_drop_first_handoff.restype = None
     for f in ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_scan_fwd_varlen_pool", "ssm_state_update",
-              "ssm_get_device_status"):
+              "ssm_get_device_status", "ssm_scan_bwd"):
         getattr(lib, f).restype = ctypes.c_int
     if lib.ssm_abi_version() != ABI_VERSION:
         raise RuntimeError(f"libssm_scan ABI {lib.ssm_abi_version()} != binding ABI {ABI_VERSION}")
@@ -232,6 +242,45 @@ def varlen_params(u, delta, B, C, A, Dskip=None, delta_bias=None, z=None, h0=Non
     p.discretization = DISC_ZOH if zoh else DISC_EULER
     p.algorithm = _algo(algorithm)
     return p
+
+
+def scan_bwd(u, delta, B, C, A, dy, Dskip=None, delta_bias=None, z=None, h0=None, dh_last=None, stream=None,
+             zoh=False, grad_dtype=None, want_dh0=True):
+    """Gradients of scan_fwd (fixed-length batch) given dy (and optionally dh_last).
+
+    Returns a dict with du, ddelta, dz (None without z) [b, D, L] in ``grad_dtype`` (default: the
+    input dtype; float32 is also accepted), dB, dC [b, N, L], dA [D, N], dDskip, dbias [D] and
+    dh0 [b, D, N] (float32)."""
+    import torch
+    gdt = grad_dtype or u.dtype
+    if dy.dtype != gdt:
+        raise TypeError("dy must have the gradient dtype")
+    bsz, dim, L = u.shape
+    N = A.shape[1]
+    out = {"du": torch.empty_like(u, dtype=gdt), "ddelta": torch.empty_like(u, dtype=gdt),
+           "dz": torch.empty_like(u, dtype=gdt) if z is not None else None,
+           "dB": torch.empty((bsz, N, L), device=u.device, dtype=torch.float32),
+           "dC": torch.empty((bsz, N, L), device=u.device, dtype=torch.float32),
+           "dA": torch.empty((dim, N), device=u.device, dtype=torch.float32),
+           "dDskip": torch.empty(dim, device=u.device, dtype=torch.float32) if Dskip is not None else None,
+           "dbias": torch.empty(dim, device=u.device, dtype=torch.float32) if delta_bias is not None else None,
+           "dh0": torch.empty((bsz, dim, N), device=u.device, dtype=torch.float32) if want_dh0 else None}
+    for t in (dy, out["du"], out["ddelta"], out["dz"]):
+        if t is not None and t.stride() != u.stride():
+            raise ValueError("dy and the per-step gradients must have u's strides")
+    p = scan_params(u, delta, B, C, A, Dskip, delta_bias, z, h0, None, None, zoh)
+    p.y_fp32 = 1 if (gdt == torch.float32 and u.dtype != torch.float32) else 0
+    _f32(dh_last)
+    g = ScanGrads()
+    g.dy, g.dh_last = _ptr(dy), _ptr(dh_last)
+    g.du, g.ddelta, g.dz = _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"])
+    g.dB, g.dC, g.dA = _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dA"])
+    g.dDskip, g.ddelta_bias, g.dh0 = _ptr(out["dDskip"]), _ptr(out["dbias"]), _ptr(out["dh0"])
+    lib = load()
+    ws = lib.ssm_scan_bwd_workspace_size(ctypes.byref(p))
+    wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
+    _check(lib.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g), _ptr(wbuf), ws, _stream(stream)), "ssm_scan_bwd")
+    return out
 
 
 def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, z=None, h0=None, y=None,

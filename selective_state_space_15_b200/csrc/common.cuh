@@ -224,6 +224,10 @@ struct ScanArgs {
   int nchains;       // nseq * ntiles
   int group;         // chunks per work unit
   int total_units;   // nchains * ceil(nchunks / group) (chunked kernel); units (lane-sequential kernel)
+  // checkpoint mode of the lane-sequential kernel (the backward's first pass): the state
+  // entering every 8-step block is stored to ckpt[b][block][dim][N]; y is not computed
+  float *ckpt;
+  int64_t ckpt_blocks;  // blocks per sequence: ceil(seqlen / 8)
 };
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {

@@ -1,0 +1,528 @@
+// Backward pass of the selective scan (gradients for training), lane-sequential.
+//
+// Schedule ("ufo.work" page, §2.2, strategy B: keep checkpoints, recompute the rest; its
+// second article, §3.1: chunk-level checkpoints).  A first launch (the lane-sequential
+// forward kernel in checkpoint mode) stores the state entering every 8-step block.  This
+// kernel then walks each (sequence, channel tile) from the end: for every 8-step block it
+// recomputes a_t = exp(Delta_t A) and h_t from the block's checkpoint, keeping them in
+// registers, and runs the adjoint recurrence backwards through the block:
+//
+//   dyraw_t  = dy_t silu(z_t)                 dz_t = dy_t yraw_t silu'(z_t)
+//   dh      += dyraw_t C_t                    (y_t reads h_t)
+//   dC_t    += dyraw_t h_t                    dB_t += dh Delta_t u_t       (summed over channels)
+//   du_t     = dyraw_t D + Delta_t sum_n dh B_t
+//   dDelta_t = sum_n (dh h_{t-1} a_t A + dh B_t u_t)      ddelta_t = dDelta_t sigmoid(delta_t + bias)
+//   dA      += dh h_{t-1} a_t Delta_t         dh *= a_t                   (on to h_{t-1})
+//
+// with yraw_t = sum_n C_t h_t + D u_t (the ungated output).  dh starts from dh_last and ends
+// as dh0.  Each exponential of the forward is evaluated twice in total (checkpoint pass and
+// recompute), none a third time.
+//
+// Lanes: LPC = 4 lanes share a channel and split its states (NS = N / 4 each); a warp holds
+// 8 channels, a CTA four warps (32 channels).  Per block a lane evaluates the per-step terms
+// (softplus, its derivative, the gate) for 2 of the 8 steps and hands them to the channel's
+// other lanes by shuffles; sums over the states (yraw, du, dDelta) are reduced across those 4
+// lanes.  The sums over channels (dB, dC) go through shared memory: every lane writes its
+// per-state terms, each warp adds its 8 channels, the four warps meet in a per-chunk
+// accumulator, and the CTA writes one partial row per (tile, sequence, state) to the
+// workspace; a last kernel adds the tiles' partials.  dA, dDskip and dbias are summed in
+// registers and added to their outputs with atomics once per unit.
+//
+// Staging is the forward's: TMA bulk copies of the u, delta, z, dy rows and the B, C rows of a
+// chunk (here in reverse chunk order), double-buffered, with B and C widened to float32 in a
+// [step][state] layout once per chunk.
+#pragma once
+
+#include "common.cuh"
+#include "seq_scan.cuh"
+
+namespace ssm {
+
+struct BwdArgs {
+  const void *dy;          // [batch][dim][seqlen], dtype TG, strides as u
+  const float *dh_last;    // [batch][dim][N] or nullptr
+  void *du, *ddelta, *dz;  // [batch][dim][seqlen], dtype TG
+  float *dA, *dDskip, *dbias, *dh0;
+  const float *ckpt;       // [batch][ckpt_blocks][dim][N]: state entering each 8-step block
+  float *partials;         // [ntiles][batch][2][N][seqlen]: per-tile sums of dB (0) and dC (1)
+  int64_t ckpt_blocks;
+};
+
+// sigmoid(x) from w = e^-|x| (which the softplus already has): 1/(1+w) for x > 0, w/(1+w) else.
+__device__ __forceinline__ float sigmoid_from_w(float x, float w) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + w));
+  return (x > 0.f ? 1.f : w) * r;
+}
+
+template <typename T, typename TG, int N, int TC>
+struct BwdCfg {
+  static constexpr int kLPC = 4;
+  static constexpr int kNS = N / kLPC;
+  static constexpr int kCPW = 32 / kLPC;  // 8 channels per warp
+  static constexpr int kWarps = 4;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kCT = kWarps * kCPW;
+  static constexpr int kSub = 8 / kLPC;   // steps of an 8-step block a lane prepares: 2
+  static constexpr int kXP = TC + 8;      // staged row pitch (elements), as in the forward
+  static constexpr size_t kXElems = size_t(3) * kCT * kXP;     // u, delta, z
+  static constexpr size_t kYElems = size_t(kCT) * kXP;         // dy (dtype TG)
+  static constexpr size_t kBCElems = size_t(2) * N * TC;
+  static constexpr int kCOff = TC * N + 16;
+  static constexpr size_t kBFElems = size_t(2) * TC * N + 16;
+  // per warp: the per-state dB, dC terms of one 8-step block, [8][2][LPC][CPW] groups of NS
+  static constexpr size_t kPartElems = size_t(8) * 2 * kLPC * kCPW * kNS;
+  static constexpr size_t kAccElems = size_t(2) * N * TC;     // [2: dB, dC][N][TC], per buffer
+  static constexpr size_t kOffY = 2 * kXElems * sizeof(T);
+  static constexpr size_t kOffBC = kOffY + 2 * kYElems * sizeof(TG);
+  static constexpr size_t kOffBF = (kOffBC + 2 * kBCElems * sizeof(T) + 15) / 16 * 16;
+  static constexpr size_t kOffPart = kOffBF + 2 * kBFElems * sizeof(float);
+  static constexpr size_t kOffAcc = kOffPart + kWarps * kPartElems * sizeof(float);
+  static constexpr size_t kSmemBytes = kOffAcc + 2 * kAccElems * sizeof(float);
+  static_assert(kNS % 4 == 0, "whole float4 groups of states per lane");
+  static_assert(TC % 8 == 0 && (kXP * sizeof(T)) % 16 == 0 && (kXP * sizeof(TG)) % 16 == 0, "16-byte rows");
+  static_assert(kOffY % 16 == 0 && kOffBF % 16 == 0 && kOffPart % 16 == 0, "aligned buffers");
+};
+
+template <typename T, typename TG, int N, int TC, bool HAS_Z>
+__global__ void __launch_bounds__(128, 3) seq_bwd_kernel(const ScanArgs args, const BwdArgs bw) {
+  using Cfg = BwdCfg<T, TG, N, TC>;
+  constexpr int LPC = Cfg::kLPC, NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT, NT = Cfg::kThreads;
+  constexpr int XP = Cfg::kXP, SUB = Cfg::kSub;
+  constexpr int V = Elem<T>::kVec;
+  constexpr bool kFast = Elem<T>::kFast;
+  constexpr int nx = HAS_Z ? 3 : 2;
+
+  extern __shared__ __align__(16) unsigned char smem[];
+  T *const xs0 = reinterpret_cast<T *>(smem);                                   // [2][3][CT][XP]
+  TG *const ys0 = reinterpret_cast<TG *>(smem + Cfg::kOffY);                    // [2][CT][XP]
+  T *const bcs0 = reinterpret_cast<T *>(smem + Cfg::kOffBC);                    // [2][2][N][TC]
+  float *const bf0 = reinterpret_cast<float *>(smem + Cfg::kOffBF);             // [2][kBFElems]
+  float *const part0 = reinterpret_cast<float *>(smem + Cfg::kOffPart);         // [W][kPartElems]
+  float *const acc0 = reinterpret_cast<float *>(smem + Cfg::kOffAcc);           // [2][2][N][TC]
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int unit_sh;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int g = lane % LPC, c = lane / LPC;
+  const int ch = warp * CPW + c;
+  const int lbase = lane - g;
+  const int64_t L = args.seqlen;
+  const int64_t seqlen_r = (L + V - 1) / V * V;
+  float *const part = part0 + size_t(warp) * Cfg::kPartElems;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_init_fence();
+  }
+  for (int i = threadIdx.x; i < int(2 * Cfg::kAccElems); i += NT) acc0[i] = 0.f;
+  __syncthreads();
+  uint32_t gc = 0;
+
+  for (;;) {
+    if (threadIdx.x == 0) unit_sh = int(atomicAdd(args.ticket, 1u));
+    __syncthreads();
+    const int unit = unit_sh;
+    if (unit >= args.total_units) break;
+    const int tile = unit % args.ntiles;
+    const int s = unit / args.ntiles;
+    const int64_t d0 = int64_t(tile) * CT;
+    const int nvalid = int(min64(CT, args.dim - d0));
+    const int64_t d = d0 + ch;
+    const bool ch_ok = d < args.dim;
+    const int64_t xbase = int64_t(s) * args.x_batch_stride;
+    const int64_t bcbase = int64_t(s) * args.bc_batch_stride;
+    const int nchunks = L > 0 ? int((L + TC - 1) / TC) : 0;
+
+    float2 A2[NS / 2], An[NS / 2], dh[NS / 2], dAacc[NS / 2];
+    float bias = 0.f, Dd = 0.f, dDacc = 0.f, dbacc = 0.f;
+#pragma unroll
+    for (int p = 0; p < NS / 2; ++p) {
+      A2[p] = An[p] = dh[p] = dAacc[p] = make_float2(0.f, 0.f);
+    }
+    if (ch_ok) {
+      const float *Ar = args.A + d * N + g * NS;
+#pragma unroll
+      for (int p = 0; p < NS / 2; ++p) {
+        An[p] = make_float2(Ar[2 * p], Ar[2 * p + 1]);
+        A2[p] = make_float2(An[p].x * kLog2e, An[p].y * kLog2e);
+      }
+      if (bw.dh_last) {
+        const float *hr = bw.dh_last + (int64_t(s) * args.dim + d) * N + g * NS;
+#pragma unroll
+        for (int p = 0; p < NS / 2; ++p) dh[p] = make_float2(hr[2 * p], hr[2 * p + 1]);
+      }
+      bias = args.bias ? args.bias[d] : 0.f;
+      Dd = args.Dskip ? args.Dskip[d] : 0.f;
+    }
+
+    auto issue_chunk = [&](int buf, int cc) {
+      const int64_t wstart = int64_t(cc) * TC;
+      const int64_t wend = min64(wstart + TC, seqlen_r);
+      const uint32_t rows_t = uint32_t((wend - wstart) * int64_t(sizeof(T)));
+      const uint32_t rows_g = uint32_t((wend - wstart) * int64_t(sizeof(TG)));
+      T *xd = xs0 + buf * Cfg::kXElems;
+      TG *yd = ys0 + buf * Cfg::kYElems;
+      T *bd = bcs0 + buf * Cfg::kBCElems;
+      fence_proxy_async_smem();
+      if (threadIdx.x == 0)
+        mbar_arrive_expect_tx(&bars[buf], rows_t * uint32_t(nx * nvalid + 2 * N) + rows_g * uint32_t(nvalid));
+      for (int r = threadIdx.x; r < (nx + 1) * CT + 2 * N; r += NT) {
+        if (r < nx * CT) {
+          const int which = r / CT, c2 = r % CT;
+          if (c2 >= nvalid) continue;
+          const T *base = static_cast<const T *>(which == 0 ? args.u : (which == 1 ? args.delta : args.z));
+          bulk_g2s(xd + size_t(r) * XP, base + xbase + (d0 + c2) * args.x_dim_stride + wstart, rows_t, &bars[buf]);
+        } else if (r < (nx + 1) * CT) {
+          const int c2 = r - nx * CT;
+          if (c2 >= nvalid) continue;
+          bulk_g2s(yd + size_t(c2) * XP,
+                   static_cast<const TG *>(bw.dy) + xbase + (d0 + c2) * args.x_dim_stride + wstart, rows_g, &bars[buf]);
+        } else {
+          const int r2 = r - (nx + 1) * CT, which = r2 / N, n = r2 % N;
+          const T *base = static_cast<const T *>(which == 0 ? args.B : args.C);
+          bulk_g2s(bd + size_t(r2) * TC, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, rows_t,
+                   &bars[buf]);
+        }
+      }
+    };
+
+    // the chunk accumulator `acc` (dB, dC summed over the CTA's channels) -> the tile's partial
+    // rows, then cleared for its next use
+    auto flush_acc = [&](int abuf, int cc) {
+      float *acc = acc0 + abuf * Cfg::kAccElems;
+      const int64_t wstart = int64_t(cc) * TC;
+      for (int i = threadIdx.x; i < 2 * N * TC; i += NT) {
+        const int row = i / TC, t = i % TC;  // row = which * N + n
+        if (wstart + t < L)
+          bw.partials[((int64_t(tile) * args.nseq + s) * 2 * N + row) * L + wstart + t] = acc[i];
+        acc[i] = 0.f;
+      }
+    };
+
+    // one 8-step block, from the end of the block to its start
+    auto block = [&](auto masked_tag, const T *X, const TG *Y, const float *Bf, float *acc, int64_t wstart, int sb) {
+      constexpr bool kMasked = decltype(masked_tag)::value;
+      const int k0 = sb * 8;                      // chunk-local first step of the block
+      const int64_t gblk = (wstart + k0) / 8;     // block index in the sequence
+      const int rel_hi = int(min64(L - (wstart + k0), 8));  // steps of the block inside the sequence
+      // ---- this lane's SUB steps: softplus, its derivative, the gate
+      const int c0 = k0 + g * SUB;
+      float uv[SUB], dv[SUB], zv[SUB], gv[SUB], dm[SUB], um[SUB], sg[SUB], zs[SUB], zd[SUB];
+      load_sub<T, SUB>(X + size_t(ch) * XP + c0, uv);
+      load_sub<T, SUB>(X + size_t(CT + ch) * XP + c0, dv);
+      if constexpr (HAS_Z) load_sub<T, SUB>(X + size_t(2 * CT + ch) * XP + c0, zv);
+      load_sub<TG, SUB>(Y + size_t(ch) * XP + c0, gv);
+#pragma unroll
+      for (int j = 0; j < SUB; ++j) {
+        const float x = dv[j] + bias;
+        float dt, sgm;
+        if constexpr (kFast) {
+          const float w = ex2_approx(-fabsf(x) * kLog2e);
+          float q = fmaf(w, -0.00853909645229578f, 0.044089239090681076f);
+          q = fmaf(w, q, -0.10768117010593414f);
+          q = fmaf(w, q, 0.17745204269886017f);
+          q = fmaf(w, q, -0.24495449662208557f);
+          q = fmaf(w, q, 0.33275479078292847f);
+          q = fmaf(w, q, -0.4999740421772003f);
+          q = fmaf(w, q, 0.9999998211860657f);
+          dt = fmaf(w, q, fmaxf(x, 0.f));
+          sgm = sigmoid_from_w(x, w);
+        } else {
+          dt = softplus_precise(x);
+          sgm = 1.f / (1.f + expf(-x));
+        }
+        float du = dt * uv[j], gy = gv[j];
+        if constexpr (kMasked) {
+          const bool in = g * SUB + j < rel_hi;
+          dt = in ? dt : 0.f;
+          du = in ? du : 0.f;  // selects: non-finite inputs past the end stay out
+          gy = in ? gy : 0.f;
+        }
+        dm[j] = dt;
+        um[j] = du;
+        sg[j] = sgm;
+        gv[j] = gy;
+        if constexpr (HAS_Z) {
+          // silu(z) = z s, silu'(z) = s (1 + z (1 - s)), s = sigmoid(z)
+          const float s_ = kFast ? fmaf(0.5f, tanh_approx(0.5f * zv[j]), 0.5f) : 1.f / (1.f + expf(-zv[j]));
+          zs[j] = zv[j] * s_;
+          zd[j] = s_ * fmaf(zv[j], 1.f - s_, 1.f);
+        }
+      }
+      float dl[8], dU[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        dl[k] = __shfl_sync(0xffffffffu, dm[k % SUB], lbase + k / SUB);
+        dU[k] = __shfl_sync(0xffffffffu, um[k % SUB], lbase + k / SUB);
+      }
+      // ---- recompute a_t and h_t over the block from its checkpoint
+      float2 hin[NS / 2];
+#pragma unroll
+      for (int p = 0; p < NS / 2; ++p) hin[p] = make_float2(0.f, 0.f);
+      if (ch_ok) {
+        const float *ck = bw.ckpt + ((int64_t(s) * bw.ckpt_blocks + gblk) * args.dim + d) * N + g * NS;
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q) {
+          const float4 v = reinterpret_cast<const float4 *>(ck)[q];
+          hin[2 * q] = make_float2(v.x, v.y);
+          hin[2 * q + 1] = make_float2(v.z, v.w);
+        }
+      }
+      float2 a[8][NS / 2], h[8][NS / 2];
+      float yp[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int t = k0 + k;
+        const float2 dd = make_float2(dl[k], dl[k]), uu = make_float2(dU[k], dU[k]);
+        float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q) {
+          float4 b4 = reinterpret_cast<const float4 *>(Bf + t * N + g * NS)[q];
+          float4 c4 = reinterpret_cast<const float4 *>(Bf + Cfg::kCOff + t * N + g * NS)[q];
+          if constexpr (kMasked) {
+            if (k >= rel_hi) b4 = c4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int p = 2 * q + e;
+            const float2 bp = e ? make_float2(b4.z, b4.w) : make_float2(b4.x, b4.y);
+            const float2 cp = e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+            const float2 x = __fmul2_rn(dd, A2[p]);
+            a[k][p] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            h[k][p] = __ffma2_rn(a[k][p], k ? h[k - 1][p] : hin[p], __fmul2_rn(uu, bp));
+            acc2 = __ffma2_rn(cp, h[k][p], acc2);
+          }
+        }
+        yp[k] = acc2.x + acc2.y;
+      }
+      // ---- sum C h over the channel's lanes for this lane's steps (recursive halving)
+#pragma unroll
+      for (int lev = 0; (1 << lev) < LPC; ++lev) {
+        const int off = LPC >> (lev + 1), half = 8 >> (lev + 1);
+        const bool upper = (g & off) != 0;
+#pragma unroll
+        for (int j = 0; j < half; ++j) {
+          const float send = upper ? yp[j] : yp[half + j];
+          const float keep = upper ? yp[half + j] : yp[j];
+          yp[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      // ---- the gate's gradient and the ungated output's, for this lane's steps
+      float dym[SUB], dzv[SUB];
+#pragma unroll
+      for (int j = 0; j < SUB; ++j) {
+        const float yraw = fmaf(Dd, uv[j], yp[j]);
+        if constexpr (HAS_Z) {
+          dzv[j] = gv[j] * yraw * zd[j];
+          dym[j] = gv[j] * zs[j];
+        } else {
+          dzv[j] = 0.f;
+          dym[j] = gv[j];
+        }
+        if constexpr (kMasked) {
+          const bool in = g * SUB + j < rel_hi;  // past the end: zero, whatever z and u hold there
+          dzv[j] = in ? dzv[j] : 0.f;
+          dym[j] = in ? dym[j] : 0.f;
+          uv[j] = in ? uv[j] : 0.f;
+        }
+      }
+      float dr[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) dr[k] = __shfl_sync(0xffffffffu, dym[k % SUB], lbase + k / SUB);
+      // ---- the adjoint recurrence, last step first
+      float s1[8], s2[8];
+#pragma unroll
+      for (int k = 7; k >= 0; --k) {
+        const int t = k0 + k;
+        const float2 dd = make_float2(dl[k], dl[k]), uu = make_float2(dU[k], dU[k]);
+        const float2 dyr = make_float2(dr[k], dr[k]);
+        float2 S1 = make_float2(0.f, 0.f), S2 = make_float2(0.f, 0.f);
+        float *pb = part + ((size_t(k) * 2 + 0) * LPC * CPW + size_t(g) * CPW + c) * NS;  // dB terms
+        float *pc = part + ((size_t(k) * 2 + 1) * LPC * CPW + size_t(g) * CPW + c) * NS;  // dC terms
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q) {
+          float4 b4 = reinterpret_cast<const float4 *>(Bf + t * N + g * NS)[q];
+          float4 c4 = reinterpret_cast<const float4 *>(Bf + Cfg::kCOff + t * N + g * NS)[q];
+          if constexpr (kMasked) {
+            if (k >= rel_hi) b4 = c4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          float2 tb[2], tc[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int p = 2 * q + e;
+            const float2 bp = e ? make_float2(b4.z, b4.w) : make_float2(b4.x, b4.y);
+            const float2 cp = e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+            dh[p] = __ffma2_rn(dyr, cp, dh[p]);                 // y_t reads h_t
+            tc[e] = __fmul2_rn(dyr, h[k][p]);                    // dC_t term of this channel
+            tb[e] = __fmul2_rn(dh[p], uu);                       // dB_t term: dh Delta u
+            S1 = __ffma2_rn(dh[p], bp, S1);                      // sum_n dh B
+            const float2 daa = __fmul2_rn(__fmul2_rn(dh[p], k ? h[k - 1][p] : hin[p]), a[k][p]);
+            S2 = __ffma2_rn(daa, An[p], S2);                     // sum_n dh h_{t-1} a A
+            dAacc[p] = __ffma2_rn(daa, dd, dAacc[p]);            // dA += dh h_{t-1} a Delta
+            dh[p] = __fmul2_rn(dh[p], a[k][p]);                  // on to h_{t-1}
+          }
+          reinterpret_cast<float4 *>(pb)[q] = make_float4(tb[0].x, tb[0].y, tb[1].x, tb[1].y);
+          reinterpret_cast<float4 *>(pc)[q] = make_float4(tc[0].x, tc[0].y, tc[1].x, tc[1].y);
+        }
+        s1[k] = S1.x + S1.y;
+        s2[k] = S2.x + S2.y;
+      }
+      // ---- sums over the channel's lanes of sum_n dh B and sum_n dh h a A, for this lane's steps
+#pragma unroll
+      for (int lev = 0; (1 << lev) < LPC; ++lev) {
+        const int off = LPC >> (lev + 1), half = 8 >> (lev + 1);
+        const bool upper = (g & off) != 0;
+#pragma unroll
+        for (int j = 0; j < half; ++j) {
+          const float send1 = upper ? s1[j] : s1[half + j], keep1 = upper ? s1[half + j] : s1[j];
+          const float send2 = upper ? s2[j] : s2[half + j], keep2 = upper ? s2[half + j] : s2[j];
+          s1[j] = keep1 + __shfl_xor_sync(0xffffffffu, send1, off);
+          s2[j] = keep2 + __shfl_xor_sync(0xffffffffu, send2, off);
+        }
+      }
+      if (ch_ok) {
+        float odu[SUB], odd[SUB];
+#pragma unroll
+        for (int j = 0; j < SUB; ++j) {
+          odu[j] = fmaf(dym[j], Dd, dm[j] * s1[j]);              // du = dyraw D + Delta sum dh B
+          odd[j] = fmaf(uv[j], s1[j], s2[j]) * sg[j];            // (sum dh h a A + u sum dh B) sigmoid
+          if constexpr (kMasked) {
+            const bool in = g * SUB + j < rel_hi;
+            odd[j] = in ? odd[j] : 0.f;
+            odu[j] = in ? odu[j] : 0.f;
+          }
+          dDacc = fmaf(dym[j], uv[j], dDacc);
+          dbacc += odd[j];
+        }
+        const int64_t off = xbase + d * args.x_dim_stride + wstart + c0;
+        TG *gdu = static_cast<TG *>(bw.du) + off;
+        TG *gdd = static_cast<TG *>(bw.ddelta) + off;
+        [[maybe_unused]] TG *gdz = HAS_Z ? static_cast<TG *>(bw.dz) + off : nullptr;
+        if (!kMasked || g * SUB + SUB <= rel_hi) {
+          store_sub<TG, SUB>(gdu, odu);
+          store_sub<TG, SUB>(gdd, odd);
+          if constexpr (HAS_Z) store_sub<TG, SUB>(gdz, dzv);
+        } else {
+#pragma unroll
+          for (int j = 0; j < SUB; ++j)
+            if (g * SUB + j < rel_hi) {
+              gdu[j] = Elem<TG>::from_f32(odu[j]);
+              gdd[j] = Elem<TG>::from_f32(odd[j]);
+              if constexpr (HAS_Z) gdz[j] = Elem<TG>::from_f32(dzv[j]);
+            }
+        }
+      }
+      // ---- dB, dC: add the warp's 8 channels, then into the CTA's chunk accumulator
+      __syncwarp();
+      for (int o = lane; o < 8 * 2 * LPC * (NS / 4); o += 32) {
+        // output group o = ((k * 2 + which) * LPC + gg) * (NS / 4) + q: 4 states of one step
+        const int q = o % (NS / 4), gg = (o / (NS / 4)) % LPC, which = (o / (NS / 4 * LPC)) % 2;
+        const int k = o / (NS / 4 * LPC * 2);
+        const float *src = part + ((size_t(k) * 2 + which) * LPC * CPW + size_t(gg) * CPW) * NS + q * 4;
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int cc = 0; cc < CPW; ++cc) {
+          const float4 v = *reinterpret_cast<const float4 *>(src + cc * NS);
+          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+        }
+        float *dst = acc + (size_t(which) * N + gg * NS + q * 4) * TC + k0 + k;
+        atomicAdd(dst, sum.x);
+        atomicAdd(dst + TC, sum.y);
+        atomicAdd(dst + 2 * TC, sum.z);
+        atomicAdd(dst + 3 * TC, sum.w);
+      }
+      __syncwarp();  // the warp's terms are consumed before the next block rewrites them
+    };
+
+    // ------------------------------------------------------------- chunks, last first
+    if (nchunks > 0) issue_chunk(int(gc & 1u), nchunks - 1);
+    int prev_acc = -1;  // accumulator of the chunk done before this one (to be flushed)
+    for (int cc = nchunks - 1; cc >= 0; --cc, ++gc) {
+      const int buf = int(gc & 1u);
+      const int64_t wstart = int64_t(cc) * TC;
+      const bool landed = mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
+      {
+        const T *bs = bcs0 + buf * Cfg::kBCElems;
+        float *bfw = bf0 + buf * Cfg::kBFElems;
+        for (int i = threadIdx.x; i < 2 * N * (TC / 8); i += NT) {
+          const int row = i % (2 * N), blk = i / (2 * N);
+          float f[8];
+          load_sub<T, 8>(bs + size_t(row) * TC + blk * 8, f);
+          float *dst = bfw + (row >= N ? Cfg::kCOff : 0) + blk * 8 * N + row % N;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) dst[j * N] = f[j];
+        }
+      }
+      // chunk cc widened; every warp is done with chunk cc+1 (its buffers and accumulator)
+      if (__syncthreads_or(!landed)) {
+        mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);  // no copy left writing shared memory
+        return;
+      }
+      if (prev_acc >= 0) flush_acc(prev_acc, cc + 1);
+      if (cc > 0) issue_chunk(buf ^ 1, cc - 1);
+      const T *X = xs0 + buf * Cfg::kXElems;
+      const TG *Y = ys0 + buf * Cfg::kYElems;
+      const float *Bf = bf0 + buf * Cfg::kBFElems;
+      float *acc = acc0 + buf * Cfg::kAccElems;
+#pragma unroll 1
+      for (int sb = TC / 8 - 1; sb >= 0; --sb) {
+        if (wstart + sb * 8 >= L) continue;  // a block wholly past the end (uniform)
+        if (wstart + sb * 8 + 8 <= L)
+          block(std::false_type{}, X, Y, Bf, acc, wstart, sb);
+        else
+          block(std::true_type{}, X, Y, Bf, acc, wstart, sb);
+      }
+      prev_acc = buf;
+    }
+    __syncthreads();
+    if (prev_acc >= 0) flush_acc(prev_acc, 0);
+
+    // ------------------------------------------------------------- per-unit results
+    if (ch_ok) {
+      if (bw.dh0) {
+        float *hr = bw.dh0 + (int64_t(s) * args.dim + d) * N + g * NS;
+#pragma unroll
+        for (int p = 0; p < NS / 2; ++p) {
+          hr[2 * p] = dh[p].x;
+          hr[2 * p + 1] = dh[p].y;
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < NS / 2; ++p) {
+        atomicAdd(bw.dA + d * N + g * NS + 2 * p, dAacc[p].x);
+        atomicAdd(bw.dA + d * N + g * NS + 2 * p + 1, dAacc[p].y);
+      }
+    }
+    // dDskip and dbias: this lane's steps, summed over the channel's lanes
+#pragma unroll
+    for (int off = 1; off < LPC; off *= 2) {
+      dDacc += __shfl_xor_sync(0xffffffffu, dDacc, off);
+      dbacc += __shfl_xor_sync(0xffffffffu, dbacc, off);
+    }
+    if (ch_ok && g == 0) {
+      if (bw.dDskip) atomicAdd(bw.dDskip + d, dDacc);
+      if (bw.dbias) atomicAdd(bw.dbias + d, dbacc);
+    }
+    __syncthreads();  // shared state of this unit is dead before the next unit overwrites it
+  }
+}
+
+// dB, dC = the sum of the tiles' partial rows.  One thread per (sequence, which, state, step).
+__global__ void __launch_bounds__(256) bwd_reduce_tiles_kernel(const float *partials, float *dB, float *dC,
+                                                              int64_t ntiles, int64_t per_tile, int64_t per_which,
+                                                              int64_t L) {
+  // per_tile = batch * 2 * N * L (one tile's partials); element e of it = ((s * 2 + which) * N + n) * L + t
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < per_tile;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    float sum = 0.f;
+    for (int64_t tl = 0; tl < ntiles; ++tl) sum += partials[tl * per_tile + e];
+    const int64_t row = e / L, t = e % L;          // row = (s * 2 + which) * N + n
+    const int64_t n = row % per_which, sw = row / per_which;
+    const int64_t s = sw / 2, which = sw % 2;
+    (which ? dC : dB)[(s * per_which + n) * L + t] = sum;
+  }
+}
+
+}  // namespace ssm

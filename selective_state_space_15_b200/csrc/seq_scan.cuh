@@ -38,11 +38,11 @@
 
 namespace ssm {
 
-template <typename T, int N, int LPC, int TC>
+template <typename T, int N, int LPC, int TC, int W>
 struct SeqCfg {
   static constexpr int kNS = N / LPC;       // states per lane
   static constexpr int kCPW = 32 / LPC;     // channels per warp
-  static constexpr int kWarps = 4;
+  static constexpr int kWarps = W;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kCT = kWarps * kCPW;  // channels per CTA
   static constexpr int kSub = 8 / LPC;      // steps of an 8-step block that a lane prepares
@@ -110,14 +110,16 @@ template <typename TO, int SUB> __device__ __forceinline__ void store_sub(TO *p,
   }
 }
 
-template <typename T, typename TO, int N, int LPC, int TC, bool HAS_Z>
-__global__ void __launch_bounds__(128, 4) seq_scan_kernel(const ScanArgs args) {
-  using Cfg = SeqCfg<T, N, LPC, TC>;
+// CKPT: checkpoint mode (fixed-length batches): the state entering every 8-step block is
+// stored to args.ckpt and nothing else is written (no y, no final state).
+template <typename T, typename TO, int N, int LPC, int TC, int W, bool HAS_Z, bool CKPT = false>
+__global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs args) {
+  using Cfg = SeqCfg<T, N, LPC, TC, W>;
   constexpr int NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT, NT = Cfg::kThreads, XP = Cfg::kXP;
   constexpr int SUB = Cfg::kSub;
   constexpr int V = Elem<T>::kVec;
   constexpr bool kFast = Elem<T>::kFast;
-  constexpr int nx = HAS_Z ? 3 : 2;
+  constexpr int nx = CKPT ? 2 : (HAS_Z ? 3 : 2);
 
   extern __shared__ __align__(16) unsigned char smem[];
   T *const xs0 = reinterpret_cast<T *>(smem);           // [2][3][CT][XP]
@@ -278,6 +280,15 @@ __global__ void __launch_bounds__(128, 4) seq_scan_kernel(const ScanArgs args) {
             dU[k] = __shfl_sync(0xffffffffu, um[k % SUB], lbase + k / SUB);
           }
         }
+        if constexpr (CKPT) {
+          // the state entering this block (steps before the sequence start are identities)
+          const int64_t gblk = (wstart - w0) / 8 + blk;  // blocks past the sequence end are not stored
+          if (ch_ok && gblk < args.ckpt_blocks) {
+            float *ck = args.ckpt + ((int64_t(s) * args.ckpt_blocks + gblk) * args.dim + d) * N + g * NS;
+#pragma unroll
+            for (int p = 0; p < NS / 2; ++p) reinterpret_cast<float2 *>(ck)[p] = h[p];
+          }
+        }
         // ---- the recurrence over the block's 8 steps for this lane's NS states
         float yp[8];
 #pragma unroll
@@ -289,7 +300,7 @@ __global__ void __launch_bounds__(128, 4) seq_scan_kernel(const ScanArgs args) {
 #pragma unroll
           for (int q = 0; q < NS / 4; ++q) {
             bq[q] = reinterpret_cast<const float4 *>(Bb + t * N)[q];
-            cq[q] = reinterpret_cast<const float4 *>(Cb + t * N)[q];
+            cq[q] = CKPT ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<const float4 *>(Cb + t * N)[q];
           }
           float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
@@ -306,10 +317,11 @@ __global__ void __launch_bounds__(128, 4) seq_scan_kernel(const ScanArgs args) {
               bb.y = dU[k] != 0.f ? bb.y : 0.f;
             }
             h[p] = __ffma2_rn(a, h[p], bb);
-            acc = __ffma2_rn(cp, h[p], acc);
+            if constexpr (!CKPT) acc = __ffma2_rn(cp, h[p], acc);
           }
           yp[k] = acc.x + acc.y;
         }
+        if constexpr (CKPT) continue;
         // ---- sum y over the channel's LPC lanes by recursive halving: at each level a lane
         // keeps the half of its step range picked by one bit of g and sends the other half to
         // the partner lane; lane g ends with steps [g SUB, (g + 1) SUB)
@@ -386,7 +398,7 @@ __global__ void __launch_bounds__(128, 4) seq_scan_kernel(const ScanArgs args) {
     }
 
     // ------------------------------------------------------------- final state
-    if (args.h_last && srow >= 0 && ch_ok) {
+    if (!CKPT && args.h_last && srow >= 0 && ch_ok) {
       float *hr = args.h_last + (srow * args.dim + d) * N + g * NS;
 #pragma unroll
       for (int p = 0; p < NS / 2; ++p) {

@@ -3,6 +3,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <atomic>
 #include <map>
 #include <mutex>
@@ -11,6 +12,7 @@
 #include "ssm_scan.h"
 #include "chunk_scan.cuh"
 #include "seq_scan.cuh"
+#include "seq_bwd.cuh"
 #include "state_update.cuh"
 
 namespace {
@@ -118,7 +120,11 @@ std::atomic<bool> g_test_drop_first_handoff{false};
 #ifndef SSM_SEQ_MAX_CTAS
 #define SSM_SEQ_MAX_CTAS 0
 #endif
+#ifndef SSM_SEQ_WARPS
+#define SSM_SEQ_WARPS 4
+#endif
 constexpr int seq_lpc(int N) { return N == 16 ? SSM_SEQ_LPC16 : 4; }
+constexpr int kSeqWarps = SSM_SEQ_WARPS;
 constexpr int kSeqMaxCtasPerSm = SSM_SEQ_MAX_CTAS;
 constexpr int64_t kSeqMinPairs = 16384;
 bool seq_supported(const ssm_scan_params *p, bool vec) {
@@ -136,7 +142,7 @@ bool make_plan(const ssm_scan_params *p, int64_t nseq, bool varlen, bool vec, Pl
     if (!seq_supported(p, vec)) return false;
     pl.seq = true;
     const int64_t G = groups_of(p);
-    const int64_t ct = int64_t(4) * (32 / seq_lpc(N));
+    const int64_t ct = int64_t(kSeqWarps) * (32 / seq_lpc(N));
     pl.ntiles = G * ((dim / G + ct - 1) / ct);
     pl.nchains = nseq * pl.ntiles;
     pl.ws_bytes = 16;  // the unit ticket
@@ -213,8 +219,8 @@ template <typename T, typename TO, int N, bool HAS_Z>
 ssm_status_t launch_seq(ScanArgs a, const Plan &pl, void *ws, cudaStream_t stream) {
   constexpr int LPC = seq_lpc(N);
   constexpr int TC = sizeof(T) == 2 ? 32 : 16;  // 64-byte rows either way
-  using Cfg = ssm::SeqCfg<T, N, LPC, TC>;
-  auto kern = ssm::seq_scan_kernel<T, TO, N, LPC, TC, HAS_Z>;
+  using Cfg = ssm::SeqCfg<T, N, LPC, TC, kSeqWarps>;
+  auto kern = ssm::seq_scan_kernel<T, TO, N, LPC, TC, kSeqWarps, HAS_Z>;
   LaunchInfo li;
   if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
     return SSM_ERR_CUDA;
@@ -397,6 +403,86 @@ void launch_update(const ssm::UpdateArgs &a, int G, bool has_z, bool zoh, dim3 b
   else launch_update_disc<T, TO, false>(a, G, has_z, blocks, st);
 }
 
+// ---- backward (ssm_scan_bwd) ----
+// Workspace: two unit tickets (16 bytes each), the checkpoints [batch][ceil(L/8)][dim][N] and
+// the per-tile partial sums of dB and dC [tiles][batch][2][N][L], all float32.
+constexpr int kBwdTC16 = 32;  // chunk of the backward kernel for 16-bit inputs (64-byte rows)
+struct BwdPlan {
+  int64_t nblk = 0, ntiles = 0, nunits = 0;
+  size_t off_ckpt = 0, off_part = 0, bytes = 0;
+};
+bool make_bwd_plan(const ssm_scan_params *p, bool vec, BwdPlan &bp) {
+  if (!vec || p->dstate != 16 || groups_of(p) != 1 || p->discretization != SSM_DISC_EULER) return false;
+  constexpr int64_t CT = 32;  // BwdCfg::kCT
+  bp.nblk = (p->seqlen + 7) / 8;
+  bp.ntiles = (p->dim + CT - 1) / CT;
+  bp.nunits = p->batch * bp.ntiles;
+  bp.off_ckpt = 32;
+  const size_t ckpt = size_t(p->batch) * bp.nblk * p->dim * p->dstate * sizeof(float);
+  bp.off_part = (bp.off_ckpt + ckpt + 255) / 256 * 256;
+  bp.bytes = bp.off_part + size_t(bp.ntiles) * p->batch * 2 * p->dstate * p->seqlen * sizeof(float);
+  return true;
+}
+
+template <typename T, typename TG, bool HAS_Z>
+ssm_status_t launch_bwd(ScanArgs a, const ssm::BwdArgs &bwa, const BwdPlan &bp, const ssm_scan_params *p,
+                        float *dB, float *dC, unsigned char *ws, cudaStream_t st) {
+  constexpr int N = 16;
+  // 1. checkpoints: the lane-sequential forward in checkpoint mode
+  {
+    constexpr int LPC = seq_lpc(N);
+    constexpr int TC = sizeof(T) == 2 ? 32 : 16;
+    using Cfg = ssm::SeqCfg<T, N, LPC, TC, kSeqWarps>;
+    auto kern = ssm::seq_scan_kernel<T, T, N, LPC, TC, kSeqWarps, false, true>;
+    LaunchInfo li;
+    if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
+      return SSM_ERR_CUDA;
+    const int64_t ct = Cfg::kCT;
+    ScanArgs f = a;
+    f.ntiles = int((p->dim + ct - 1) / ct);
+    f.tiles_per_group = f.ntiles;
+    f.group_dim = p->dim;
+    f.nseq = int(p->batch);
+    f.total_units = int(p->batch * f.ntiles);
+    f.ticket = reinterpret_cast<uint32_t *>(ws);
+    f.ckpt = reinterpret_cast<float *>(ws + bp.off_ckpt);
+    f.ckpt_blocks = bp.nblk;
+    f.y = nullptr;
+    f.h_last = nullptr;
+    const int64_t blocks = std::min<int64_t>(f.total_units, int64_t(li.num_sms) * li.blocks_per_sm);
+    kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, st>>>(f);
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+  }
+  // 2. the backward walk
+  {
+    constexpr int TC = sizeof(T) == 2 ? kBwdTC16 : 16;
+    using Cfg = ssm::BwdCfg<T, TG, N, TC>;
+    auto kern = ssm::seq_bwd_kernel<T, TG, N, TC, HAS_Z>;
+    LaunchInfo li;
+    if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
+      return SSM_ERR_CUDA;
+    ScanArgs b = a;
+    b.ntiles = int(bp.ntiles);
+    b.nseq = int(p->batch);
+    b.total_units = int(bp.nunits);
+    b.ticket = reinterpret_cast<uint32_t *>(ws + 16);
+    const int64_t blocks = std::min<int64_t>(bp.nunits, int64_t(li.num_sms) * li.blocks_per_sm);
+    kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, st>>>(b, bwa);
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+  }
+  // 3. dB, dC from the tiles' partial sums
+  {
+    const int64_t per_tile = p->batch * 2 * N * p->seqlen;
+    const int64_t blocks = std::min<int64_t>((per_tile + 255) / 256, 148 * 16);
+    if (blocks > 0) {
+      ssm::bwd_reduce_tiles_kernel<<<unsigned(blocks), 256, 0, st>>>(bwa.partials, dB, dC, bp.ntiles, per_tile, N,
+                                                                     p->seqlen);
+      if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+    }
+  }
+  return SSM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -517,6 +603,67 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
   else if (p->dtype == SSM_BF16) launch_update<bf16, float>(a, G, has_z, zoh, blocks, st);
   else launch_update<float, float>(a, G, has_z, zoh, blocks, st);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+ssm_status_t ssm_scan_bwd(const ssm_scan_params *p, const ssm_scan_grads *g, void *workspace,
+                          size_t workspace_bytes, ssm_stream_t stream) {
+  ScanArgs a;
+  bool vec = false;
+  ssm_status_t st = prepare_scan(p, false, a, vec);
+  if (st != SSM_OK) return st;
+  if (!g || !g->dy || !g->du || !g->ddelta || !g->dB || !g->dC || !g->dA) return SSM_ERR_INVALID_ARG;
+  if (p->z && !g->dz) return SSM_ERR_INVALID_ARG;
+  const bool aligned = aligned16(g->dy) && aligned16(g->du) && aligned16(g->ddelta) && (!p->z || aligned16(g->dz));
+  BwdPlan bp;
+  if (!aligned || !make_bwd_plan(p, vec, bp)) return SSM_ERR_UNSUPPORTED;
+  if (p->batch > (int64_t(1) << 30) || bp.nunits > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < bp.bytes || !aligned16(workspace)) return SSM_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  const size_t nd = size_t(p->dim);
+  if (cudaMemsetAsync(ws, 0, 32, cs) != cudaSuccess ||
+      cudaMemsetAsync(g->dA, 0, nd * p->dstate * sizeof(float), cs) != cudaSuccess ||
+      (g->dDskip && cudaMemsetAsync(g->dDskip, 0, nd * sizeof(float), cs) != cudaSuccess) ||
+      (g->ddelta_bias && cudaMemsetAsync(g->ddelta_bias, 0, nd * sizeof(float), cs) != cudaSuccess))
+    return SSM_ERR_CUDA;
+  if (p->batch == 0) return SSM_OK;
+  if (p->seqlen == 0) {  // nothing to walk: dh0 = dh_last, dB, dC empty
+    if (g->dh0) {
+      const size_t nb = size_t(p->batch) * nd * p->dstate * sizeof(float);
+      if ((g->dh_last ? cudaMemcpyAsync(g->dh0, g->dh_last, nb, cudaMemcpyDeviceToDevice, cs)
+                      : cudaMemsetAsync(g->dh0, 0, nb, cs)) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    }
+    return SSM_OK;
+  }
+  ssm::BwdArgs bwa{};
+  bwa.dy = g->dy; bwa.dh_last = g->dh_last;
+  bwa.du = g->du; bwa.ddelta = g->ddelta; bwa.dz = g->dz;
+  bwa.dA = g->dA; bwa.dDskip = p->Dskip ? g->dDskip : nullptr; bwa.dbias = p->delta_bias ? g->ddelta_bias : nullptr;
+  bwa.dh0 = g->dh0;
+  bwa.ckpt = reinterpret_cast<const float *>(ws + bp.off_ckpt);
+  bwa.partials = reinterpret_cast<float *>(ws + bp.off_part);
+  bwa.ckpt_blocks = bp.nblk;
+  a.cu_seqlens = nullptr;
+  using bf16 = __nv_bfloat16;
+  const bool has_z = p->z != nullptr;
+  if (p->dtype == SSM_BF16 && !p->y_fp32)
+    return has_z ? launch_bwd<bf16, bf16, true>(a, bwa, bp, p, g->dB, g->dC, ws, cs)
+                 : launch_bwd<bf16, bf16, false>(a, bwa, bp, p, g->dB, g->dC, ws, cs);
+  if (p->dtype == SSM_BF16)
+    return has_z ? launch_bwd<bf16, float, true>(a, bwa, bp, p, g->dB, g->dC, ws, cs)
+                 : launch_bwd<bf16, float, false>(a, bwa, bp, p, g->dB, g->dC, ws, cs);
+  return has_z ? launch_bwd<float, float, true>(a, bwa, bp, p, g->dB, g->dC, ws, cs)
+               : launch_bwd<float, float, false>(a, bwa, bp, p, g->dB, g->dC, ws, cs);
+}
+
+size_t ssm_scan_bwd_workspace_size(const ssm_scan_params *p) {
+  ScanArgs a;
+  bool vec = false;
+  if (prepare_scan(p, false, a, vec) != SSM_OK) return 0;
+  BwdPlan bp;
+  if (!make_bwd_plan(p, vec, bp)) return 0;
+  return bp.bytes;
 }
 
 size_t ssm_scan_workspace_size(const ssm_scan_params *p, int64_t nseq) {

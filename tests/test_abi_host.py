@@ -161,6 +161,37 @@ def test_algorithm_choice_on_host(lib):
     assert size(ctypes.byref(_params(dim=2048, seqlen=4096)), 4) == 0
 
 
+def test_backward_host_checks(lib):
+    """ssm_scan_bwd refuses bad or unsupported requests on the host, before anything runs."""
+    fake = 0x10000
+    g = ssm.ScanGrads()
+    for name in ("dy", "du", "ddelta", "dz", "dB", "dC", "dA"):
+        setattr(g, name, fake)
+    f = lib.ssm_scan_bwd
+    p = _params()
+    assert f(ctypes.byref(p), None, None, 0, None) == 1                              # no gradients
+    g_missing = ssm.ScanGrads()
+    g_missing.dy = fake
+    assert f(ctypes.byref(p), ctypes.byref(g_missing), None, 0, None) == 1         # outputs missing
+    pz = _params()
+    pz.z = fake
+    g_noz = ssm.ScanGrads()
+    for name in ("dy", "du", "ddelta", "dB", "dC", "dA"):
+        setattr(g_noz, name, fake)
+    assert f(ctypes.byref(pz), ctypes.byref(g_noz), None, 0, None) == 1            # z given, no dz
+    assert f(ctypes.byref(_params(dstate=32)), ctypes.byref(g), None, 0, None) == 2
+    assert f(ctypes.byref(_params(discretization=ssm.DISC_ZOH)), ctypes.byref(g), None, 0, None) == 2
+    assert f(ctypes.byref(_params(dim=64, ngroups=2)), ctypes.byref(g), None, 0, None) == 2
+    assert f(ctypes.byref(_params(x_dim_stride=130, seqlen=128)), ctypes.byref(g), None, 0, None) == 2
+    assert f(ctypes.byref(p), ctypes.byref(g), None, 0, None) == 6                  # SSM_ERR_WORKSPACE
+    # workspace: checkpoints every 8 steps and per-32-channel-tile partial rows of dB and dC
+    need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(p))
+    ckpt = 1 * (128 // 8) * 64 * 16 * 4
+    part = 2 * 1 * 2 * 16 * 128 * 4
+    assert ckpt + part <= need <= ckpt + part + 512
+    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(_params(dstate=32))) == 0
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
     """ssm_scan_fwd_noalloc refuses, on the host and before anything runs, a problem whose
     scratch need exceeds SSM_NOALLOC_SCRATCH_BYTES (here the chunked kernel's hand-off carries
@@ -198,13 +229,12 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     text = src.read_text()
     src.write_text("// a new comment line\n" + text.replace("namespace ssm {", "namespace ssm {  /* note */", 1))
     assert bench.kernel_source_hash() == base
-    src.write_text(text.replace("static constexpr int kWarps = 4;", "static constexpr int kWarps = 8;"))
+    src.write_text(text.replace("static constexpr int kXP = TC + 8;", "static constexpr int kXP = TC + 16;"))
     assert bench.kernel_source_hash() != base
     src.write_text(text)
     api = fake / "ssm_api.cu"
     api_text = api.read_text()
-    api.write_text(api_text.replace("constexpr int seq_lpc(int N) {", "constexpr int seq_lpc(int N) { /**/ ", 1)
-                   .replace("? 2 : 4;", "? 4 : 4;", 1))
+    api.write_text(api_text.replace("#define SSM_SEQ_LPC16 4", "#define SSM_SEQ_LPC16 2", 1))
     assert bench.kernel_source_hash() != base                      # the tile of the timed kernel
     api.write_text(api_text)
     (fake / "state_update.cuh").write_text("// decode kernel changed\nint x;\n")

@@ -32,12 +32,17 @@ def _lib():
 
 
 def _batch(inp, dtype, h0=None, gate=True, y_dtype=None, algorithm=SEQ):
-    u, dl = dev(inp.u, dtype), dev(inp.delta, dtype)
-    z = dev(inp.z, dtype) if gate else None
-    B, C = dev(inp.B, dtype), dev(inp.C, dtype)
+    """Rows padded to a 16-byte pitch (NaN in the padding) when L is not a multiple of 8: the
+    sequential kernel takes 16-byte aligned rows only."""
+    L = inp.u.shape[-1]
+    pitch = round_up(L, 8)
+    u, dl = dev(inp.u, dtype, pitch=pitch)[..., :L], dev(inp.delta, dtype, pitch=pitch)[..., :L]
+    z = dev(inp.z, dtype, pitch=pitch)[..., :L] if gate else None
+    B, C = dev(inp.B, dtype, pitch=pitch)[..., :L], dev(inp.C, dtype, pitch=pitch)[..., :L]
     A, D, bias = (torch.from_numpy(x).cuda() for x in (inp.A, inp.Dskip, inp.bias))
     h0t = torch.from_numpy(h0).cuda() if h0 is not None else None
-    y, hl = ssm.scan_fwd(u, dl, B, C, A, D, bias, z, h0t, y_dtype=y_dtype, algorithm=algorithm)
+    y = torch.empty(u.shape[:-1] + (pitch,), device="cuda", dtype=y_dtype or u.dtype)[..., :L]
+    y, hl = ssm.scan_fwd(u, dl, B, C, A, D, bias, z, h0t, y=y, algorithm=algorithm)
     torch.cuda.synchronize()
     return host(y), host(hl)
 
