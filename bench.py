@@ -48,10 +48,10 @@ def peaks():
         return 6650.0, 1965.0, "fallback"
 
 
-# The timed scan kernel (the lane-sequential one, which the varlen workload takes) is defined
-# by these sources and by the lines of ssm_api.cu that fix its tile (lanes per channel, chunk).
-KERNEL_SOURCES = ("seq_scan.cuh", "common.cuh")
-KERNEL_SHAPE_MARKERS = ("#define SSM_SEQ_", "constexpr int seq_lpc(", "constexpr int TC = ", "constexpr int kSeq")
+# The timed scan kernel (the chunked one, which the varlen workload takes) is defined by these
+# sources and by the tile-shape line of its workload (the wide N=16 tile) in ssm_api.cu.
+KERNEL_SOURCES = ("chunk_scan.cuh", "common.cuh")
+KERNEL_SHAPE_MARKERS = ("template <> struct Shape<16, false>",)
 
 
 def _code_only(text: str) -> str:
@@ -608,8 +608,14 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"dp{world} (independent batches)"},
         "roofline": {"bound": "alu", "unit": "Gexp/s", "achieved": nexps / launch_s / 1e9, "peak": sfu_peak / 1e9,
                      "frac": nexps / launch_s / sfu_peak, "traffic": traffic,
-                     "peak_note": f"MUFU: {N_SM} SMs x {SFU_PER_CLK_PER_SM} ex2/clk x {sm_max:.0f} MHz; "
-                                  "exps/token = D(N+2)"},
+                     "peak_note": f"MUFU: {N_SM} SMs x {SFU_PER_CLK_PER_SM} results/clk (15.96 measured, "
+                                  f"profiles/mufu_rate_b200.md) x {sm_max:.0f} MHz; counted: D(N+2) exponentials "
+                                  "per token (N exp(Delta A), one in softplus, one in the gate) -- the algorithm's "
+                                  "lower bound",
+                     "mufu_ops_per_token_kernel": D * (N + 3),
+                     "mufu_note": "the timed (chunked) kernel issues D(N+3) MUFU operations per token: the N "
+                                  "exponentials, one ex2 per 16-step lane segment and state for the segment "
+                                  "product (D N / 16), one in softplus, one tanh in the gate"},
         "roofline_hbm": {"bound": "hbm", "unit": "GB/s", "achieved": nbytes / launch_s / 1e9, "peak": hbm_peak,
                          "frac": nbytes / launch_s / 1e9 / hbm_peak, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": nbytes},

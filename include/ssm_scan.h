@@ -91,8 +91,8 @@ typedef enum { SSM_DISC_EULER = 0, SSM_DISC_ZOH = 1 } ssm_discretization_t;
  *                        its states (no composition); suits many channels x sequences.
  *                        dstate 16 or 32, Euler discretisation, 16-byte aligned rows only;
  *                        other cases return SSM_ERR_UNSUPPORTED.
- * AUTO takes SEQUENTIAL when it applies and there are at least 16384 (sequence, channel)
- * pairs, CHUNKED otherwise.  Other values -> SSM_ERR_INVALID_ARG.
+ * AUTO takes CHUNKED (the faster of the two on every workload measured).  Other values ->
+ * SSM_ERR_INVALID_ARG.
  */
 typedef enum { SSM_ALGO_AUTO = 0, SSM_ALGO_CHUNKED = 1, SSM_ALGO_SEQUENTIAL = 2 } ssm_algorithm_t;
 
@@ -205,7 +205,8 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
  * is walked backwards, each short stretch recomputed from its checkpoint and the adjoint
  * recurrence dh_{t-1} = exp(Delta_t A) (dh_t + C_t dyraw_t) carried from the end.
  *
- * `p` describes the forward problem exactly as for ssm_scan_fwd (the same inputs).  Supported:
+ * `p` describes the forward problem as for ssm_scan_fwd (the same inputs; p->y and p->h_last
+ * are not used and may be NULL).  Supported:
  * dstate 16, ngroups <= 1, the Euler input matrix (p->discretization = SSM_DISC_EULER), and
  * every tensor base and row stride 16-byte aligned (the forward's fast path; dy, du, ddelta and
  * dz included).  Other cases return SSM_ERR_UNSUPPORTED before anything runs.
@@ -241,6 +242,45 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params *p, const ssm_scan_grads *g, voi
 
 /* Bytes of device workspace ssm_scan_bwd needs for this problem (0 if it is not supported). */
 size_t ssm_scan_bwd_workspace_size(const ssm_scan_params *p);
+
+/*
+ * SSD (Mamba-2) chunked form of the scan on the tensor cores: the second article of the
+ * "会议长序列建模…" page (ufo.work), "Mamba-2/SSD架构下的矩阵化加速范式…", §1.1 (the scan as masked
+ * attention, Y = (mask o (C B^T)) V with V = Delta x) and §2.2 (the mask carries the decay
+ * exp(A sum Delta) from a prefix sum), with the state carried between chunks.  A is one scalar
+ * per head and Delta one value per (head, step), shared by the head's headdim channels; B and C
+ * are shared by all heads.  For head h, channel p and state n:
+ *     h_t[p][n] = exp(dt[h][t] A[h]) h_{t-1}[p][n] + dt[h][t] B[n][t] x[h][p][t]
+ *     y[h][p][t] = sum_n C[n][t] h_t[p][n]
+ * -- the selective scan with A[d][n] = A[h] for the channels d of head h and Delta given
+ * directly (no softplus, no skip term, no gate).  Computed in chunks of 128 steps as four
+ * dense products per chunk on tcgen05 (float16 operands, float32 accumulation).
+ *   x      : DEVICE bf16 [batch][nheads][headdim][seqlen]
+ *   dt     : DEVICE float32 [batch][nheads][seqlen], the step Delta (> 0)
+ *   A      : DEVICE float32 [nheads] (< 0 for a decaying state)
+ *   B, C   : DEVICE bf16 [batch][dstate][seqlen]
+ *   h0     : DEVICE float32 [batch][nheads][headdim][dstate] or NULL (zero)
+ *   y      : DEVICE bf16 [batch][nheads][headdim][seqlen] (written)
+ *   h_last : DEVICE float32 [batch][nheads][headdim][dstate] or NULL (not written)
+ * Supported: headdim 64, dstate 128, seqlen a multiple of 8, 16-byte aligned x, B, C;
+ * SSM_ERR_UNSUPPORTED otherwise.  Contiguous tensors.  No workspace.
+ */
+typedef struct ssm_ssd_params {
+  int64_t batch;
+  int64_t nheads;
+  int64_t headdim;
+  int64_t dstate;
+  int64_t seqlen;
+  const void *x;
+  const float *dt;
+  const float *A;
+  const void *B;
+  const void *C;
+  const float *h0;
+  void *y;
+  float *h_last;
+} ssm_ssd_params;
+ssm_status_t ssm_ssd_fwd(const ssm_ssd_params *p, ssm_stream_t stream);
 
 /*
  * Allocation-free variant of ssm_scan_fwd.  (The pages have no counterpart; this is a

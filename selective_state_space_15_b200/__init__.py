@@ -24,7 +24,7 @@ _ALGO = {"auto": ALGO_AUTO, "chunked": ALGO_CHUNKED, "sequential": ALGO_SEQUENTI
 EXPORTED = ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_state_update", "ssm_scan_workspace_size",
             "ssm_get_device_status", "ssm_status_string", "ssm_abi_version", "ssm_scan_fwd_noalloc",
             "ssm_scan_fwd_varlen_pool", "ssm_test_drop_first_handoff", "ssm_scan_bwd",
-            "ssm_scan_bwd_workspace_size")
+            "ssm_scan_bwd_workspace_size", "ssm_ssd_fwd")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SSM_NOALLOC_SCRATCH_BYTES
 
 
@@ -49,6 +49,13 @@ class ScanParams(ctypes.Structure):
         ("ngroups", ctypes.c_int64), ("bc_group_stride", ctypes.c_int64), ("discretization", ctypes.c_int32),
         ("algorithm", ctypes.c_int32),
     ]
+
+
+class SsdParams(ctypes.Structure):
+    """Mirror of ssm_ssd_params."""
+    _fields_ = [("batch", ctypes.c_int64), ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("seqlen", ctypes.c_int64)] + \
+               [(n, ctypes.c_void_p) for n in ("x", "dt", "A", "B", "C", "h0", "y", "h_last")]
 
 
 class ScanGrads(ctypes.Structure):
@@ -82,6 +89,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_scan_workspace_size.restype = S
     lib.ssm_scan_bwd.argtypes = [pp, ctypes.POINTER(ScanGrads), P, S, P]
     lib.ssm_scan_bwd_workspace_size.argtypes = [pp]
+    lib.ssm_ssd_fwd.argtypes = [ctypes.POINTER(SsdParams), P]
     lib.ssm_scan_bwd_workspace_size.restype = S
     lib.ssm_get_device_status.argtypes = [P]
     lib.ssm_status_string.argtypes = [ctypes.c_int]
@@ -90,7 +98,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_test_drop_first_handoff.argtypes = []
     lib.ssm_test_drop_first_handoff.restype = None
     for f in ("ssm_scan_fwd", "ssm_scan_fwd_varlen", "ssm_scan_fwd_varlen_pool", "ssm_state_update",
-              "ssm_get_device_status", "ssm_scan_bwd"):
+              "ssm_get_device_status", "ssm_scan_bwd", "ssm_ssd_fwd"):
         getattr(lib, f).restype = ctypes.c_int
     if lib.ssm_abi_version() != ABI_VERSION:
         raise RuntimeError(f"libssm_scan ABI {lib.ssm_abi_version()} != binding ABI {ABI_VERSION}")
@@ -281,6 +289,30 @@ def scan_bwd(u, delta, B, C, A, dy, Dskip=None, delta_bias=None, z=None, h0=None
     wbuf = torch.empty(ws, device=u.device, dtype=torch.uint8) if ws else None
     _check(lib.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g), _ptr(wbuf), ws, _stream(stream)), "ssm_scan_bwd")
     return out
+
+
+def ssd_fwd(x, dt, A, B, C, h0=None, y=None, h_last=None, return_last_state=True, stream=None):
+    """SSD chunked form (tensor cores): x [b, H, P, L] bf16, dt [b, H, L] float32 (the step, > 0),
+    A [H] float32, B, C [b, N, L] bf16, h0 [b, H, P, N] float32 or None.  Returns (y, h_last)."""
+    import torch
+    bsz, H, P, L = x.shape
+    N = B.shape[1]
+    for t in (x, B, C):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("x, B and C must be contiguous bfloat16")
+    for t in (dt, A, h0, h_last):
+        _f32(t)
+    if tuple(dt.shape) != (bsz, H, L) or tuple(B.shape) != (bsz, N, L) or C.shape != B.shape:
+        raise ValueError("dt must be [b, H, L] and B, C [b, N, L]")
+    y = torch.empty_like(x) if y is None else y
+    if h_last is None and return_last_state:
+        h_last = torch.empty((bsz, H, P, N), device=x.device, dtype=torch.float32)
+    p = SsdParams()
+    p.batch, p.nheads, p.headdim, p.dstate, p.seqlen = bsz, H, P, N, L
+    p.x, p.dt, p.A, p.B, p.C = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C)
+    p.h0, p.y, p.h_last = _ptr(h0), _ptr(y), _ptr(h_last)
+    _check(load().ssm_ssd_fwd(ctypes.byref(p), _stream(stream)), "ssm_ssd_fwd")
+    return y, h_last
 
 
 def scan_fwd_varlen(u, delta, B, C, A, cu_seqlens, Dskip=None, delta_bias=None, z=None, h0=None, y=None,

@@ -234,12 +234,12 @@ __global__ void __launch_bounds__(128, 3) seq_bwd_kernel(const ScanArgs args, co
           sgm = 1.f / (1.f + expf(-x));
         }
         float du = dt * uv[j], gy = gv[j];
-        if constexpr (kMasked) {
-          const bool in = g * SUB + j < rel_hi;
-          dt = in ? dt : 0.f;
-          du = in ? du : 0.f;  // selects: non-finite inputs past the end stay out
-          gy = in ? gy : 0.f;
-        }
+        // a channel past the end of a ragged tile, or a step past the end of the sequence, takes
+        // no part (its staged rows are stale; selects keep non-finite values out of the sums)
+        const bool in = ch_ok && (!kMasked || g * SUB + j < rel_hi);
+        dt = in ? dt : 0.f;
+        du = in ? du : 0.f;
+        gy = in ? gy : 0.f;
         dm[j] = dt;
         um[j] = du;
         sg[j] = sgm;
@@ -321,8 +321,8 @@ __global__ void __launch_bounds__(128, 3) seq_bwd_kernel(const ScanArgs args, co
           dzv[j] = 0.f;
           dym[j] = gv[j];
         }
-        if constexpr (kMasked) {
-          const bool in = g * SUB + j < rel_hi;  // past the end: zero, whatever z and u hold there
+        {
+          const bool in = ch_ok && (!kMasked || g * SUB + j < rel_hi);  // zero, whatever z and u hold
           dzv[j] = in ? dzv[j] : 0.f;
           dym[j] = in ? dym[j] : 0.f;
           uv[j] = in ? uv[j] : 0.f;

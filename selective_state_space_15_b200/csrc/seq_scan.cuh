@@ -9,21 +9,24 @@
 // channels (and sequences) alone, so the host picks this kernel only when there are enough
 // of them to fill the GPU; a single long sequence goes to the chunked kernel instead.
 //
-// Per step and lane: x = Delta * A log2(e) and a = ex2(x) for NS states, b = (Delta u) B,
-// h = a h + b and y += C h, all in packed f32x2 arithmetic over pairs of states.  The LPC
-// lanes of a channel split its per-step work: in every block of 8 steps, lane g evaluates
-// softplus(delta + bias) and Delta u for steps [g SUB, (g + 1) SUB) (SUB = 8 / LPC) and the
-// values reach the other lanes by shuffles; after the block, the LPC partial sums of y are
-// reduced by recursive halving so that lane g ends with the full y of the same SUB steps,
-// which it gates (silu(z), skip term D u) and stores.
+// Per step and lane: x = Delta A log2(e) and a = ex2(x) for NS states, b = (Delta u) B,
+// h = a h + b and y += C h.  The arithmetic is packed f32x2 over pairs of consecutive steps of
+// one state (x, b and the y update; the recurrence itself is a scalar chain per state), so no
+// operand has to be duplicated into a register pair.  Delta = softplus(delta + bias) and
+// Delta u are evaluated once per (step, channel) by the whole CTA when a chunk lands, into
+// shared memory, where the LPC lanes of a channel read them; after every block of 8 steps the
+// LPC partial sums of y are reduced by recursive halving so that lane g ends with the full y
+// of steps [g SUB, (g + 1) SUB) (SUB = 8 / LPC), which it gates (silu(z), skip term D u) and
+// stores.
 //
 // Staging.  A CTA (four warps, CT channels of one sequence) copies the u, delta, z rows of
 // its channels and the B, C rows of a TC-step chunk into shared memory with TMA bulk copies
 // (cp.async.bulk completing on an mbarrier, no multicast), double-buffered: chunk c + 1
-// streams in while chunk c is computed.  B and C are then widened to float32 once per chunk
-// into a [step][state] layout, so that a lane reads the NS values of its states at one step
-// with 16-byte loads that every channel of the CTA shares (broadcast).  Row pitches are
-// padded so that the lanes of a load phase read distinct banks.
+// streams in while chunk c is computed.  When a chunk has landed the CTA widens B and C to
+// float32 (rows padded by 16 bytes so that the rows of a load phase hit distinct banks) and
+// evaluates Delta and Delta u into double-buffered float32 rows; a lane then reads four steps
+// of a state's B or C, or of its channel's Delta, with one 16-byte load that the other
+// channels' lanes share (broadcast).
 //
 // Scheduling.  Work units are (sequence, channel tile) pairs taken from an atomic ticket by
 // a persistent grid.  Packed sequences are visited longest first (ranked in every CTA from
@@ -45,19 +48,22 @@ struct SeqCfg {
   static constexpr int kWarps = W;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kCT = kWarps * kCPW;  // channels per CTA
-  static constexpr int kSub = 8 / LPC;      // steps of an 8-step block that a lane prepares
+  static constexpr int kSub = 8 / LPC;      // steps of an 8-step block that a lane finishes
   // u/delta/z row pitch (elements): one 8-step block of padding, so that the channels of a
-  // load phase (whose lanes read 8 consecutive steps of a row between them) hit distinct banks
+  // load phase hit distinct banks
   static constexpr int kXP = TC + 8;
   static constexpr size_t kXElems = size_t(3) * kCT * kXP;  // one staging buffer: u, delta, z
   static constexpr size_t kBCElems = size_t(2) * N * TC;    // one staging buffer: B, C
-  // widened float32 B then C, each [TC][N]; C starts 16 words after B's end so that the
-  // widening threads of B and C write distinct banks
-  static constexpr int kCOff = TC * N + 16;
-  static constexpr size_t kBFElems = size_t(2) * TC * N + 16;
+  // widened float32 rows (B then C, 2N rows of pitch kBP) and Delta, Delta u rows ([2][CT][kBP]):
+  // 16 bytes of padding per row, and each group of NS state rows (the rows one lane reads)
+  // shifted by 16 bytes more, so that the LPC lanes of a channel read distinct banks
+  static constexpr int kBP = TC + 4;
+  static constexpr size_t kBFElems = size_t(2) * N * kBP + 2 * LPC * 4;
+  __host__ __device__ static constexpr int bf_row(int r) { return r * kBP + (r / kNS) * 4; }
+  static constexpr size_t kDLElems = size_t(2) * kCT * kBP;
   static constexpr size_t kSmemBytes = 2 * kXElems * sizeof(T) + 2 * kBCElems * sizeof(T) +
-                                       2 * kBFElems * sizeof(float) + kMaxSortedSeqs * sizeof(int);
-  static_assert(N % LPC == 0 && kNS % 4 == 0, "whole 16-byte groups of states per lane");
+                                       2 * (kBFElems + kDLElems) * sizeof(float) + kMaxSortedSeqs * sizeof(int);
+  static_assert(N % LPC == 0 && kNS % 2 == 0, "whole pairs of states per lane");
   static_assert(8 % LPC == 0 && TC % 8 == 0, "8-step blocks");
   static_assert((kXP * sizeof(T)) % 16 == 0 && (TC * sizeof(T)) % 16 == 0, "16-byte rows");
   static_assert(((size_t(2) * kXElems + 2 * kBCElems) * sizeof(T)) % 16 == 0, "aligned float buffers");
@@ -113,7 +119,7 @@ template <typename TO, int SUB> __device__ __forceinline__ void store_sub(TO *p,
 // CKPT: checkpoint mode (fixed-length batches): the state entering every 8-step block is
 // stored to args.ckpt and nothing else is written (no y, no final state).
 template <typename T, typename TO, int N, int LPC, int TC, int W, bool HAS_Z, bool CKPT = false>
-__global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs args) {
+__global__ void __launch_bounds__(W * 32, (LPC == 1 ? 8 : 16) / W) seq_scan_kernel(const ScanArgs args) {
   using Cfg = SeqCfg<T, N, LPC, TC, W>;
   constexpr int NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT, NT = Cfg::kThreads, XP = Cfg::kXP;
   constexpr int SUB = Cfg::kSub;
@@ -124,15 +130,16 @@ __global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs
   extern __shared__ __align__(16) unsigned char smem[];
   T *const xs0 = reinterpret_cast<T *>(smem);           // [2][3][CT][XP]
   T *const bcs0 = xs0 + 2 * Cfg::kXElems;               // [2][2][N][TC]
-  float *const bf0 = reinterpret_cast<float *>(bcs0 + 2 * Cfg::kBCElems);  // [2][kBFElems]
-  int *const order = reinterpret_cast<int *>(bf0 + 2 * Cfg::kBFElems);     // [kMaxSortedSeqs]
+  float *const bf0 = reinterpret_cast<float *>(bcs0 + 2 * Cfg::kBCElems);  // [2][2N][BP]
+  float *const dl0 = bf0 + 2 * Cfg::kBFElems;                               // [2][2][CT][BP]
+  int *const order = reinterpret_cast<int *>(dl0 + 2 * Cfg::kDLElems);      // [kMaxSortedSeqs]
+  constexpr int BP = Cfg::kBP;
   __shared__ __align__(8) uint64_t bars[2];
   __shared__ int unit_sh;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int g = lane % LPC;                  // state group: states [g NS, (g + 1) NS)
   const int ch = warp * CPW + lane / LPC;    // channel within the tile
-  const int lbase = lane - g;                // first lane of this channel
   const int64_t seqlen_r = (args.seqlen + V - 1) / V * V;
 
   if (threadIdx.x == 0) {
@@ -195,24 +202,28 @@ __global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs
     }
 
     // per-lane constants and the state entering the sequence
-    float2 A2[NS / 2], h[NS / 2];
-    float bias = 0.f, Dd = 0.f;
+    // per-lane constants (A log2(e) of each state, duplicated for step-pair arithmetic) and the
+    // state entering the sequence
+    float2 A2[NS];
+    float h[NS];
+    float Dd = 0.f;
+    [[maybe_unused]] float bias = 0.f;
 #pragma unroll
-    for (int p = 0; p < NS / 2; ++p) {
-      A2[p] = make_float2(0.f, 0.f);
-      h[p] = make_float2(0.f, 0.f);
+    for (int n = 0; n < NS; ++n) {
+      A2[n] = make_float2(0.f, 0.f);
+      h[n] = 0.f;
     }
     if (ch_ok) {
       const float *Ar = args.A + d * N + g * NS;
 #pragma unroll
-      for (int p = 0; p < NS / 2; ++p) A2[p] = make_float2(Ar[2 * p] * kLog2e, Ar[2 * p + 1] * kLog2e);
+      for (int n = 0; n < NS; ++n) A2[n] = make_float2(Ar[n] * kLog2e, Ar[n] * kLog2e);
       if (args.h0 && srow >= 0) {
         const float *hr = args.h0 + (srow * args.dim + d) * N + g * NS;
 #pragma unroll
-        for (int p = 0; p < NS / 2; ++p) h[p] = make_float2(hr[2 * p], hr[2 * p + 1]);
+        for (int n = 0; n < NS; ++n) h[n] = hr[n];
       }
-      bias = args.bias ? args.bias[d] : 0.f;
       Dd = args.Dskip ? args.Dskip[d] : 0.f;
+      bias = args.bias ? args.bias[d] : 0.f;
     }
 
     // TMA: chunk c's u/delta/z rows of the tile and B/C rows into buffer `buf`
@@ -241,43 +252,43 @@ __global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs
     };
 
     // One chunk of this lane's steps; the masked instance handles chunks that straddle a
-    // sequence boundary or the end of the rows.
-    auto compute_chunk = [&](auto masked_tag, const T *X, const float *Bf, int64_t wstart, int rel_lo,
-                             int rel_hi) {
+    // sequence boundary or the end of the rows (Delta and Delta u are already zero there).
+    auto compute_chunk = [&](auto masked_tag, const T *X, const float *Bf, const float *Dl, int64_t wstart,
+                             int rel_lo, int rel_hi) {
       constexpr bool kMasked = decltype(masked_tag)::value;
-      const T *ru = X + size_t(ch) * XP;
-      const T *rd = X + size_t(CT + ch) * XP;
+      [[maybe_unused]] const T *ru = X + size_t(ch) * XP;
       [[maybe_unused]] const T *rz = X + size_t(2 * CT + ch) * XP;
-      const float *Bb = Bf + g * NS;
-      const float *Cb = Bf + Cfg::kCOff + g * NS;
+      const float *Bb = Bf + Cfg::bf_row(g * NS);       // rows of this lane's states
+      const float *Cb = Bf + Cfg::bf_row(N + g * NS);
+      const float *rdl = Dl + size_t(ch) * BP;           // Delta of this channel
+      const float *rdu = Dl + size_t(CT + ch) * BP;      // Delta u
 #pragma unroll 1
       for (int blk = 0; blk < TC / 8; ++blk) {
-        // ---- Delta and Delta*u: this lane's SUB steps, then all 8 from the channel's lanes
-        const int c0 = blk * 8 + g * SUB;
-        float uv[SUB], dv[SUB], dm[SUB], um[SUB];
-        load_sub<T, SUB>(ru + c0, uv);
-        load_sub<T, SUB>(rd + c0, dv);
-#pragma unroll
-        for (int j = 0; j < SUB; ++j) {
-          float dt = softplus_t<kFast>(dv[j] + bias);
-          float du = dt * uv[j];
-          if constexpr (kMasked) {
-            const bool in = c0 + j >= rel_lo && c0 + j < rel_hi;
-            dt = in ? dt : 0.f;
-            du = in ? du : 0.f;  // select: a non-finite u outside the sequence stays out
-          }
-          dm[j] = dt;
-          um[j] = du;
-        }
         float dl[8], dU[8];
+        if constexpr (LPC == 1) {
+          // the lane owns its channel: Delta and Delta u of the block's 8 steps, here
+          float uv[8], dv[8];
+          load_sub<T, 8>(ru + blk * 8, uv);
+          load_sub<T, 8>(X + size_t(CT + ch) * XP + blk * 8, dv);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if constexpr (LPC == 1) {
-            dl[k] = dm[k];
-            dU[k] = um[k];
-          } else {
-            dl[k] = __shfl_sync(0xffffffffu, dm[k % SUB], lbase + k / SUB);
-            dU[k] = __shfl_sync(0xffffffffu, um[k % SUB], lbase + k / SUB);
+          for (int j = 0; j < 8; ++j) {
+            const float dt = softplus_t<kFast>(dv[j] + bias);
+            if constexpr (kMasked) {
+              const bool in = blk * 8 + j >= rel_lo && blk * 8 + j < rel_hi;
+              dl[j] = in ? dt : 0.f;
+              dU[j] = in ? dt * uv[j] : 0.f;  // select: a non-finite u outside the sequence stays out
+            } else {
+              dl[j] = dt;
+              dU[j] = dt * uv[j];
+            }
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const float4 l4 = reinterpret_cast<const float4 *>(rdl + blk * 8)[q];
+            const float4 u4 = reinterpret_cast<const float4 *>(rdu + blk * 8)[q];
+            dl[4 * q] = l4.x; dl[4 * q + 1] = l4.y; dl[4 * q + 2] = l4.z; dl[4 * q + 3] = l4.w;
+            dU[4 * q] = u4.x; dU[4 * q + 1] = u4.y; dU[4 * q + 2] = u4.z; dU[4 * q + 3] = u4.w;
           }
         }
         if constexpr (CKPT) {
@@ -286,42 +297,48 @@ __global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs
           if (ch_ok && gblk < args.ckpt_blocks) {
             float *ck = args.ckpt + ((int64_t(s) * args.ckpt_blocks + gblk) * args.dim + d) * N + g * NS;
 #pragma unroll
-            for (int p = 0; p < NS / 2; ++p) reinterpret_cast<float2 *>(ck)[p] = h[p];
+            for (int n = 0; n < NS; n += 2) *reinterpret_cast<float2 *>(ck + n) = make_float2(h[n], h[n + 1]);
           }
         }
-        // ---- the recurrence over the block's 8 steps for this lane's NS states
-        float yp[8];
+        // ---- the recurrence over the block's 8 steps for this lane's NS states, in step pairs
+        float2 yp2[4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int t = blk * 8 + k;
-          const float2 dd = make_float2(dl[k], dl[k]);
-          const float2 uu = make_float2(dU[k], dU[k]);
-          float4 bq[NS / 4], cq[NS / 4];
+        for (int k2 = 0; k2 < 4; ++k2) yp2[k2] = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int q = 0; q < NS / 4; ++q) {
-            bq[q] = reinterpret_cast<const float4 *>(Bb + t * N)[q];
-            cq[q] = CKPT ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<const float4 *>(Cb + t * N)[q];
-          }
-          float2 acc = make_float2(0.f, 0.f);
+        for (int q = 0; q < 2; ++q) {
 #pragma unroll
-          for (int p = 0; p < NS / 2; ++p) {
-            const float4 b4 = bq[p / 2], c4 = cq[p / 2];
-            const float2 bp = (p & 1) ? make_float2(b4.z, b4.w) : make_float2(b4.x, b4.y);
-            const float2 cp = (p & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
-            const float2 x = __fmul2_rn(dd, A2[p]);
-            const float2 a = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            float2 bb = __fmul2_rn(uu, bp);
-            if constexpr (kMasked) {
-              // stale B outside the sequence never reaches h (Delta*u is 0 there, B may be non-finite)
-              bb.x = dU[k] != 0.f ? bb.x : 0.f;
-              bb.y = dU[k] != 0.f ? bb.y : 0.f;
+          for (int n = 0; n < NS; ++n) {
+            const float4 b4 = reinterpret_cast<const float4 *>(Bb + size_t(n) * BP + blk * 8)[q];
+            [[maybe_unused]] float4 c4;
+            if constexpr (!CKPT) c4 = reinterpret_cast<const float4 *>(Cb + size_t(n) * BP + blk * 8)[q];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int k2 = 2 * q + e;
+              const float2 dd = make_float2(dl[2 * k2], dl[2 * k2 + 1]);
+              const float2 uu = make_float2(dU[2 * k2], dU[2 * k2 + 1]);
+              const float2 x = __fmul2_rn(dd, A2[n]);
+              const float2 a = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              float2 bb = __fmul2_rn(uu, e ? make_float2(b4.z, b4.w) : make_float2(b4.x, b4.y));
+              if constexpr (kMasked) {
+                // stale B outside the sequence never reaches h (Delta u is 0 there, B may be non-finite)
+                bb.x = uu.x != 0.f ? bb.x : 0.f;
+                bb.y = uu.y != 0.f ? bb.y : 0.f;
+              }
+              const float h0v = fmaf(a.x, h[n], bb.x);
+              h[n] = fmaf(a.y, h0v, bb.y);
+              if constexpr (!CKPT)
+                yp2[k2] = __ffma2_rn(e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y), make_float2(h0v, h[n]),
+                                     yp2[k2]);
             }
-            h[p] = __ffma2_rn(a, h[p], bb);
-            if constexpr (!CKPT) acc = __ffma2_rn(cp, h[p], acc);
           }
-          yp[k] = acc.x + acc.y;
         }
         if constexpr (CKPT) continue;
+        float yp[8];
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          yp[2 * k2] = yp2[k2].x;
+          yp[2 * k2 + 1] = yp2[k2].y;
+        }
         // ---- sum y over the channel's LPC lanes by recursive halving: at each level a lane
         // keeps the half of its step range picked by one bit of g and sends the other half to
         // the partner lane; lane g ends with steps [g SUB, (g + 1) SUB)
@@ -339,7 +356,9 @@ __global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs
         }
         // ---- skip term, gate, store this lane's SUB steps
         if (ch_ok) {
-          float zv[SUB], o[SUB];
+          const int c0 = blk * 8 + g * SUB;
+          float uv[SUB], zv[SUB], o[SUB];
+          load_sub<T, SUB>(ru + c0, uv);
           if constexpr (HAS_Z) load_sub<T, SUB>(rz + c0, zv);
 #pragma unroll
           for (int j = 0; j < SUB; ++j) {
@@ -365,17 +384,46 @@ __global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs
       const int buf = int(gc & 1u);
       const int64_t wstart = w0 + int64_t(c) * TC;
       const bool landed = mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
+      const int rel_lo = int(max64(t_lo - wstart, -1));
+      const int rel_hi = int(min64(t_hi - wstart, TC + 1));
       {
-        // widen the chunk's B and C to float32, [step][state]
+        // widen the chunk's B and C to float32 rows
         const T *bs = bcs0 + buf * Cfg::kBCElems;
         float *bf = bf0 + buf * Cfg::kBFElems;
         for (int i = threadIdx.x; i < 2 * N * (TC / 8); i += NT) {
           const int row = i % (2 * N), blk = i / (2 * N);
           float f[8];
           load_sub<T, 8>(bs + size_t(row) * TC + blk * 8, f);
-          float *dst = bf + (row >= N ? Cfg::kCOff : 0) + blk * 8 * N + row % N;
+          float4 *dst = reinterpret_cast<float4 *>(bf + Cfg::bf_row(row) + blk * 8);
+          dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+          dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+        // Delta = softplus(delta + bias) and Delta u, once per (step, channel), for the LPC
+        // lanes of a channel to share; steps outside the sequence are identities (Delta =
+        // Delta u = 0).  With LPC = 1 the lane evaluates its own.
+        const T *Xs = xs0 + buf * Cfg::kXElems;
+        float *dlw = dl0 + buf * Cfg::kDLElems;
+        for (int i = threadIdx.x; i < (LPC > 1 ? CT * (TC / 8) : 0); i += NT) {
+          const int c2 = i % CT, blk = i / CT;
+          const int64_t dd = d0 + c2;
+          const float bias = (dd < d_end && args.bias) ? args.bias[dd] : 0.f;
+          float uv[8], dv[8], o1[8], o2[8];
+          load_sub<T, 8>(Xs + size_t(c2) * XP + blk * 8, uv);
+          load_sub<T, 8>(Xs + size_t(CT + c2) * XP + blk * 8, dv);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) dst[j * N] = f[j];
+          for (int j = 0; j < 8; ++j) {
+            const int t = blk * 8 + j;
+            const bool in = t >= rel_lo && t < rel_hi;
+            const float dt = softplus_t<kFast>(dv[j] + bias);
+            o1[j] = in ? dt : 0.f;
+            o2[j] = in ? dt * uv[j] : 0.f;  // select: a non-finite u outside the sequence stays out
+          }
+          float4 *w1 = reinterpret_cast<float4 *>(dlw + size_t(c2) * BP + blk * 8);
+          float4 *w2 = reinterpret_cast<float4 *>(dlw + size_t(CT + c2) * BP + blk * 8);
+          w1[0] = make_float4(o1[0], o1[1], o1[2], o1[3]);
+          w1[1] = make_float4(o1[4], o1[5], o1[6], o1[7]);
+          w2[0] = make_float4(o2[0], o2[1], o2[2], o2[3]);
+          w2[1] = make_float4(o2[4], o2[5], o2[6], o2[7]);
         }
       }
       // chunk c widened; every warp is done with chunk c-1's buffers
@@ -387,24 +435,20 @@ __global__ void __launch_bounds__(W * 32, 16 / W) seq_scan_kernel(const ScanArgs
         return;
       }
       if (c + 1 < nchunks) issue_chunk(buf ^ 1, c + 1);  // streams in while chunk c is computed
-      const int rel_lo = int(max64(t_lo - wstart, -1));
-      const int rel_hi = int(min64(t_hi - wstart, TC + 1));
       const T *X = xs0 + buf * Cfg::kXElems;
       const float *Bf = bf0 + buf * Cfg::kBFElems;
+      const float *Dl = dl0 + buf * Cfg::kDLElems;
       if (rel_lo <= 0 && rel_hi >= TC)
-        compute_chunk(std::false_type{}, X, Bf, wstart, rel_lo, rel_hi);
+        compute_chunk(std::false_type{}, X, Bf, Dl, wstart, rel_lo, rel_hi);
       else
-        compute_chunk(std::true_type{}, X, Bf, wstart, rel_lo, rel_hi);
+        compute_chunk(std::true_type{}, X, Bf, Dl, wstart, rel_lo, rel_hi);
     }
 
     // ------------------------------------------------------------- final state
     if (!CKPT && args.h_last && srow >= 0 && ch_ok) {
       float *hr = args.h_last + (srow * args.dim + d) * N + g * NS;
 #pragma unroll
-      for (int p = 0; p < NS / 2; ++p) {
-        hr[2 * p] = h[p].x;
-        hr[2 * p + 1] = h[p].y;
-      }
+      for (int n = 0; n < NS; ++n) hr[n] = h[n];
     }
     __syncthreads();  // shared state of this unit is dead before the next unit overwrites it
   }

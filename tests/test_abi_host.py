@@ -140,8 +140,8 @@ def test_state_update_host_checks(lib):
 
 def test_algorithm_choice_on_host(lib):
     """The sequential kernel takes dstate 16 and 32 with the Euler input matrix and 16-byte
-    aligned rows; other requests for it are refused before anything runs.  AUTO takes it from
-    16384 (sequence, channel) pairs on; its workspace is the 16-byte unit ticket."""
+    aligned rows; other requests for it are refused before anything runs.  Its workspace is the
+    16-byte unit ticket; AUTO takes the chunked kernel."""
     seq, chunked = ssm.ALGO_SEQUENTIAL, ssm.ALGO_CHUNKED
     f = lib.ssm_scan_fwd
     assert f(ctypes.byref(_params(dstate=64, algorithm=seq)), None, 0, None) == 2
@@ -151,14 +151,12 @@ def test_algorithm_choice_on_host(lib):
     size = lib.ssm_scan_workspace_size
     assert size(ctypes.byref(_params(algorithm=seq)), 0) == 16
     assert size(ctypes.byref(_params(dstate=32, algorithm=seq)), 0) == 16
-    # AUTO: 16 x 1024 pairs -> sequential; 1 x 1024 -> chunked (persistent: ticket, flags, carries)
-    assert size(ctypes.byref(_params(batch=16, dim=1024)), 0) == 16
-    assert size(ctypes.byref(_params(batch=1, dim=1024)), 0) > 16
+    # AUTO takes the chunked kernel: persistent fixed-length units (ticket, flags, carries) and,
+    # for packed sequences, one CTA per sequence and tile (no workspace)
+    assert size(ctypes.byref(_params(batch=16, dim=1024)), 0) > 16
     assert size(ctypes.byref(_params(batch=16, dim=1024, algorithm=chunked)), 0) > 16
-    # packed sequences: 16 sequences x 2048 channels take the sequential kernel, 4 x 2048 the
-    # chunked one (one CTA per sequence and tile: no workspace)
-    assert size(ctypes.byref(_params(dim=2048, seqlen=4096)), 16) == 16
-    assert size(ctypes.byref(_params(dim=2048, seqlen=4096)), 4) == 0
+    assert size(ctypes.byref(_params(dim=2048, seqlen=4096)), 16) == 0
+    assert size(ctypes.byref(_params(dim=2048, seqlen=4096, algorithm=seq)), 16) == 16
 
 
 def test_backward_host_checks(lib):
@@ -225,20 +223,21 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
         shutil.copy(os.path.join(csrc, name), fake / name)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     base = bench.kernel_source_hash()
-    src = fake / "seq_scan.cuh"
+    src = fake / "chunk_scan.cuh"
     text = src.read_text()
     src.write_text("// a new comment line\n" + text.replace("namespace ssm {", "namespace ssm {  /* note */", 1))
     assert bench.kernel_source_hash() == base
-    src.write_text(text.replace("static constexpr int kXP = TC + 8;", "static constexpr int kXP = TC + 16;"))
+    src.write_text(text.replace("static constexpr int kNP = N + 1;", "static constexpr int kNP = N + 2;"))
     assert bench.kernel_source_hash() != base
     src.write_text(text)
     api = fake / "ssm_api.cu"
     api_text = api.read_text()
-    api.write_text(api_text.replace("#define SSM_SEQ_LPC16 4", "#define SSM_SEQ_LPC16 2", 1))
+    api.write_text(api_text.replace("template <> struct Shape<16, false> { static constexpr int KI = 16,",
+                                    "template <> struct Shape<16, false> { static constexpr int KI = 8,", 1))
     assert bench.kernel_source_hash() != base                      # the tile of the timed kernel
     api.write_text(api_text)
     (fake / "state_update.cuh").write_text("// decode kernel changed\nint x;\n")
-    (fake / "chunk_scan.cuh").write_text("// chunked kernel changed\nint y;\n")
+    (fake / "seq_scan.cuh").write_text("// sequential kernel changed\nint y;\n")
     assert bench.kernel_source_hash() == base
 
 

@@ -103,7 +103,7 @@ def test_bwd_small_full(shape, dtype):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_bwd_no_gate_no_initial_state(dtype):
-    b, D, N, L = 2, 48, 16, 300
+    b, D, N, L = 2, 48, 16, 304
     inp = workloads.batch_inputs(b, D, N, L, dtype, seed=810, gate=False)
     dy = draw_dy((b, D, L), dtype, 811)
     got = run_bwd(inp, dtype, dy, gate=False)

@@ -158,3 +158,31 @@ def config_inputs(name: str):
         lens = varlen_lengths(c["nseq"], c["len_lo"], c["len_hi"], c["seed"])
         return varlen_inputs(lens, c["dim"], c["dstate"], c["dtype"], c["seed"])
     return decode_problem(c["num_slots"], c["dim"], c["dstate"], c["R"], c["dtype"], c["seed"])
+
+
+@dataclass
+class SsdInputs:
+    """Host arrays for one SSD (scalar-A-per-head) problem: x [b, H, P, L] and B, C [b, N, L]
+    bf16-exact float32; dt [b, H, L] > 0, A [H] < 0 and h0 [b, H, P, N] float32."""
+    x: np.ndarray
+    dt: np.ndarray
+    A: np.ndarray
+    B: np.ndarray
+    C: np.ndarray
+    h0: np.ndarray | None
+    meta: dict = field(default_factory=dict)
+
+
+def ssd_inputs(batch, nheads, headdim, dstate, seqlen, seed=5, h0=False) -> SsdInputs:
+    """x, B, C ~ N(0, 1) rounded to bf16; dt log-uniform in [1e-3, 1e-1] per (sequence, head,
+    step); A[h] = -exp(U[log 0.5, log 16]) per head (slow and fast decays); h0 ~ N(0, 1) when
+    asked for."""
+    rng = np.random.default_rng([seed, 55])
+    x = _normal(rng, (batch, nheads, headdim, seqlen), "bf16")
+    B = _normal(rng, (batch, dstate, seqlen), "bf16")
+    C = _normal(rng, (batch, dstate, seqlen), "bf16")
+    dt = np.exp(rng.uniform(np.log(1e-3), np.log(1e-1), size=(batch, nheads, seqlen))).astype(np.float32)
+    A = (-np.exp(rng.uniform(np.log(0.5), np.log(16.0), size=nheads))).astype(np.float32)
+    hz = rng.standard_normal((batch, nheads, headdim, dstate), dtype=np.float32) if h0 else None
+    return SsdInputs(x, dt, A, B, C, hz, meta=dict(batch=batch, nheads=nheads, headdim=headdim, dstate=dstate,
+                                                   seqlen=seqlen, seed=seed))
