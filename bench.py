@@ -422,6 +422,55 @@ def decode_loop_run(hbm_peak, loop_steps=100):
             "hbm_gbs": round(nb / (ms * 1e-3) / 1e9, 1), "l2": "states resident in L2 between steps"}
 
 
+def bwd_run(name, steps, warmup, sfu_peak):
+    """Kernel figures of the backward (ssm_scan_bwd: checkpoint pass, reverse walk, tile sums)
+    on a fixed-length workload's shape (inputs and dy drawn on the device).  Its SFU count is
+    twice the forward's D(N+2) per token (the forward exponentials are evaluated once in the
+    checkpoint pass and once more in the recomputation)."""
+    import torch
+    import selective_state_space_15_b200 as ssm
+    stream = torch.cuda.current_stream()
+    c = workloads.CONFIGS[name]
+    b, D, N, L = c["batch"], c["dim"], c["dstate"], c["seqlen"]
+    dt = torch.float32 if c["dtype"] == "f32" else torch.bfloat16
+    g = torch.Generator(device="cuda")
+    g.manual_seed(c["seed"])
+    mk = lambda *sh: torch.randn(*sh, generator=g, device="cuda", dtype=torch.float32).to(dt)  # noqa: E731
+    u, dl, z, B, C, dy = mk(b, D, L), mk(b, D, L), mk(b, D, L), mk(b, N, L), mk(b, N, L), mk(b, D, L)
+    A, Dsk, bias = (torch.from_numpy(x).cuda() for x in workloads.channel_params(np.random.default_rng(c["seed"]), D, N))
+    ms = time_kernel(lambda: ssm.scan_bwd(u, dl, B, C, A, dy, Dsk, bias, z, stream=stream), steps, warmup, stream)
+    exps = 2 * b * L * D * (N + 2)
+    return {"ms": round(ms, 4), "tokens_per_s": b * L / (ms * 1e-3), "sfu_frac": round(exps / (ms * 1e-3) / sfu_peak, 4),
+            "shape": f"batch {b}, D={D}, N={N}, L={L}, {c['dtype']}", "exps_counted": "2 D (N+2) per token",
+            "launches": "checkpoint forward + reverse walk + tile sums (+ 4 memsets)"}
+
+
+SSD_SHAPE = dict(batch=4, nheads=32, headdim=64, dstate=128, seqlen=4096, seed=910)
+
+
+def ssd_run(steps, warmup, tensor_peak):
+    """Kernel figures of the SSD chunked form on tcgen05 (ssm_ssd_fwd): 4 sequences x 32 heads x
+    64 channels (D = 2048), N = 128, L = 4096, bf16; against the dense fp16/bf16 tensor peak."""
+    import torch
+    import selective_state_space_15_b200 as ssm
+    stream = torch.cuda.current_stream()
+    c = SSD_SHAPE
+    inp = workloads.ssd_inputs(c["batch"], c["nheads"], c["headdim"], c["dstate"], c["seqlen"], seed=c["seed"])
+    bf = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)  # noqa: E731
+    x, B, C = bf(inp.x), bf(inp.B), bf(inp.C)
+    dt, A = torch.from_numpy(inp.dt).cuda(), torch.from_numpy(inp.A).cuda()
+    y = torch.empty_like(x)
+    hl = torch.empty(c["batch"], c["nheads"], c["headdim"], c["dstate"], device="cuda")
+    ms = time_kernel(lambda: ssm.ssd_fwd(x, dt, A, B, C, y=y, h_last=hl, stream=stream), steps, warmup, stream)
+    T, P, N = 128, c["headdim"], c["dstate"]
+    chunks = c["batch"] * c["nheads"] * ((c["seqlen"] + T - 1) // T)
+    flops = chunks * (2 * T * T * N + 3 * 2 * T * P * N)
+    return {"ms": round(ms, 4), "tokens_per_s": c["batch"] * c["seqlen"] / (ms * 1e-3),
+            "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "tensor_frac": round(flops / (ms * 1e-3) / 1e12 / tensor_peak, 4),
+            "shape": "4 sequences x 32 heads x 64 channels, N=128, L=4096, bf16 in/out, fp16 operands, fp32 accumulate",
+            "flops_counted": "per head and 128-step chunk: 2 T T N + 6 T P N (C B^T, masked scores x V, C' H^T, state)"}
+
+
 def secondary(steps, warmup, hbm_peak, sfu_peak):
     """Kernel-only figures for the small float32, long-sequence, pool-prefill and decode workloads (single GPU)."""
     out = {name: small_batch_run(name, steps, warmup, sfu_peak, hbm_peak) for name in ("tiny_f32", "batch_f32")}
@@ -431,7 +480,18 @@ def secondary(steps, warmup, hbm_peak, sfu_peak):
     out["varlen_zoh_bf16"] = varlen_zoh_run(max(3, steps // 4), warmup, sfu_peak)
     out["decode_bf16"] = decode_run(steps, warmup, hbm_peak)
     out["decode_loop_bf16"] = decode_loop_run(hbm_peak)
+    out["bwd_batch_f32"] = bwd_run("batch_f32", max(3, steps // 8), warmup, sfu_peak)
+    out["ssd_bf16"] = ssd_run(max(3, steps // 4), warmup, tensor_peak())
     return out
+
+
+def tensor_peak():
+    """Dense bf16 (= fp16) tensor peak, TFLOP/s: the measured burst figure, else the fallback."""
+    try:
+        with open(PEAKS_PATH) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        return 1590.0
 
 
 # ------------------------------------------------------------------------------ arms
@@ -643,6 +703,10 @@ def run_other(args, rank, world, local_rank):
     sfu_peak = N_SM * SFU_PER_CLK_PER_SM * sm_max * 1e6
     if args.workload == "decode_bf16":
         r = decode_run(args.steps, args.warmup, hbm_peak)
+    elif args.workload == "bwd_batch_f32":
+        r = bwd_run("batch_f32", args.steps, args.warmup, sfu_peak)
+    elif args.workload == "ssd_bf16":
+        r = ssd_run(args.steps, args.warmup, tensor_peak())
     elif args.workload in ("tiny_f32", "batch_f32"):
         r = small_batch_run(args.workload, args.steps, args.warmup, sfu_peak, hbm_peak)
     else:
@@ -660,7 +724,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-secondary", action="store_true", help="skip the long-sequence/decode figures")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "long_bf16", "long_n128_bf16", "decode_bf16", "tiny_f32", "batch_f32"],
+                    choices=[WORKLOAD, "long_bf16", "long_n128_bf16", "decode_bf16", "tiny_f32", "batch_f32",
+                             "bwd_batch_f32", "ssd_bf16"],
                     help="with --kernel-only: time another workload's kernel alone (for ncu captures)")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="with --kernel-only and a long workload: a shorter sequence (profiler captures)")

@@ -32,6 +32,11 @@
  *     happen before any launch: on error nothing is launched and outputs are untouched.
  *     Problems found by a kernel (e.g. an out-of-range slot id) are recorded in a device
  *     status word read by ssm_get_device_status.
+ *   - Host threads: every entry point may be called from several host threads at once, on
+ *     the same device or on different ones (one thread per GPU is the intended use).  The
+ *     only host state is a table of per-(kernel, device) launch facts, filled on first use
+ *     under a lock, and the lock-guarded no-allocation scratch (ssm_scan_fwd_noalloc).
+ *     Concurrent calls must not share a workspace or outputs.
  *   - Element strides are in elements; the time axis always has stride 1.  A stride of 0
  *     means "contiguous" (the natural value for the documented layout).
  *   - Inputs u, delta, z, B, C have the dtype `dtype`; y has it too unless y_fp32 is set

@@ -19,7 +19,7 @@
 // recompute), none a third time.
 //
 // Lanes: LPC = 4 lanes share a channel and split its states (NS = N / 4 each); a warp holds
-// 8 channels, a CTA four warps (32 channels).  Per block a lane evaluates the per-step terms
+// 8 channels, a CTA W warps (8 W channels; the host picks W so that there are enough units).  Per block a lane evaluates the per-step terms
 // (softplus, its derivative, the gate) for 2 of the 8 steps and hands them to the channel's
 // other lanes by shuffles; sums over the states (yraw, du, dDelta) are reduced across those 4
 // lanes.  The sums over channels (dB, dC) go through shared memory: every lane writes its
@@ -55,12 +55,12 @@ __device__ __forceinline__ float sigmoid_from_w(float x, float w) {
   return (x > 0.f ? 1.f : w) * r;
 }
 
-template <typename T, typename TG, int N, int TC>
+template <typename T, typename TG, int N, int TC, int W>
 struct BwdCfg {
   static constexpr int kLPC = 4;
   static constexpr int kNS = N / kLPC;
   static constexpr int kCPW = 32 / kLPC;  // 8 channels per warp
-  static constexpr int kWarps = 4;
+  static constexpr int kWarps = W;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kCT = kWarps * kCPW;
   static constexpr int kSub = 8 / kLPC;   // steps of an 8-step block a lane prepares: 2
@@ -84,9 +84,9 @@ struct BwdCfg {
   static_assert(kOffY % 16 == 0 && kOffBF % 16 == 0 && kOffPart % 16 == 0, "aligned buffers");
 };
 
-template <typename T, typename TG, int N, int TC, bool HAS_Z>
-__global__ void __launch_bounds__(128, 3) seq_bwd_kernel(const ScanArgs args, const BwdArgs bw) {
-  using Cfg = BwdCfg<T, TG, N, TC>;
+template <typename T, typename TG, int N, int TC, int W, bool HAS_Z>
+__global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs args, const BwdArgs bw) {
+  using Cfg = BwdCfg<T, TG, N, TC, W>;
   constexpr int LPC = Cfg::kLPC, NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT, NT = Cfg::kThreads;
   constexpr int XP = Cfg::kXP, SUB = Cfg::kSub;
   constexpr int V = Elem<T>::kVec;

@@ -414,11 +414,17 @@ void launch_update(const ssm::UpdateArgs &a, int G, bool has_z, bool zoh, dim3 b
 constexpr int kBwdTC16 = 32;  // chunk of the backward kernel for 16-bit inputs (64-byte rows)
 struct BwdPlan {
   int64_t nblk = 0, ntiles = 0, nunits = 0;
+  int warps = 4;  // warps per CTA (8 channels each)
   size_t off_ckpt = 0, off_part = 0, bytes = 0;
 };
+// Units are (sequence, tile of 8 W channels) walked serially from the end: W = 4 when that
+// still gives four units per SM, else 2, else 1 (more, narrower units for few channels).
+constexpr int64_t kBwdUnitsWanted = 4 * 148;
 bool make_bwd_plan(const ssm_scan_params *p, bool vec, BwdPlan &bp) {
   if (!vec || p->dstate != 16 || groups_of(p) != 1 || p->discretization != SSM_DISC_EULER) return false;
-  constexpr int64_t CT = 32;  // BwdCfg::kCT
+  const int64_t pairs = p->batch * p->dim;
+  bp.warps = pairs >= 32 * kBwdUnitsWanted ? 4 : (pairs >= 16 * kBwdUnitsWanted ? 2 : 1);
+  const int64_t CT = 8 * bp.warps;
   bp.nblk = (p->seqlen + 7) / 8;
   bp.ntiles = (p->dim + CT - 1) / CT;
   bp.nunits = p->batch * bp.ntiles;
@@ -460,20 +466,27 @@ ssm_status_t launch_bwd(ScanArgs a, const ssm::BwdArgs &bwa, const BwdPlan &bp, 
   }
   // 2. the backward walk
   {
-    constexpr int TC = sizeof(T) == 2 ? kBwdTC16 : 16;
-    using Cfg = ssm::BwdCfg<T, TG, N, TC>;
-    auto kern = ssm::seq_bwd_kernel<T, TG, N, TC, HAS_Z>;
-    LaunchInfo li;
-    if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
-      return SSM_ERR_CUDA;
     ScanArgs b = a;
     b.ntiles = int(bp.ntiles);
     b.nseq = int(p->batch);
     b.total_units = int(bp.nunits);
     b.ticket = reinterpret_cast<uint32_t *>(ws + 16);
-    const int64_t blocks = std::min<int64_t>(bp.nunits, int64_t(li.num_sms) * li.blocks_per_sm);
-    kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, st>>>(b, bwa);
-    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+    auto walk = [&](auto w_tag) -> ssm_status_t {
+      constexpr int W = decltype(w_tag)::value;
+      constexpr int TC = sizeof(T) == 2 ? kBwdTC16 : 16;
+      using Cfg = ssm::BwdCfg<T, TG, N, TC, W>;
+      auto kern = ssm::seq_bwd_kernel<T, TG, N, TC, W, HAS_Z>;
+      LaunchInfo li;
+      if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
+        return SSM_ERR_CUDA;
+      const int64_t blocks = std::min<int64_t>(bp.nunits, int64_t(li.num_sms) * li.blocks_per_sm);
+      kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, st>>>(b, bwa);
+      return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    };
+    const ssm_status_t ws_st = bp.warps == 4 ? walk(std::integral_constant<int, 4>{})
+                             : bp.warps == 2 ? walk(std::integral_constant<int, 2>{})
+                                             : walk(std::integral_constant<int, 1>{});
+    if (ws_st != SSM_OK) return ws_st;
   }
   // 3. dB, dC from the tiles' partial sums
   {

@@ -182,10 +182,11 @@ def test_backward_host_checks(lib):
     assert f(ctypes.byref(_params(dim=64, ngroups=2)), ctypes.byref(g), None, 0, None) == 2
     assert f(ctypes.byref(_params(x_dim_stride=130, seqlen=128)), ctypes.byref(g), None, 0, None) == 2
     assert f(ctypes.byref(p), ctypes.byref(g), None, 0, None) == 6                  # SSM_ERR_WORKSPACE
-    # workspace: checkpoints every 8 steps and per-32-channel-tile partial rows of dB and dC
+    # workspace: checkpoints every 8 steps and per-tile partial rows of dB and dC (64 channels of
+    # one sequence: 8-channel tiles, one warp each)
     need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(p))
     ckpt = 1 * (128 // 8) * 64 * 16 * 4
-    part = 2 * 1 * 2 * 16 * 128 * 4
+    part = 8 * 1 * 2 * 16 * 128 * 4
     assert ckpt + part <= need <= ckpt + part + 512
     assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(_params(dstate=32))) == 0
 
