@@ -423,10 +423,10 @@ def decode_loop_run(hbm_peak, loop_steps=100):
 
 
 def bwd_run(name, steps, warmup, sfu_peak):
-    """Kernel figures of the backward (ssm_scan_bwd: checkpoint pass, reverse walk, tile sums)
+    """Kernel figures of the backward (ssm_scan_bwd: segment pass, segment scan, reverse walk)
     on a fixed-length workload's shape (inputs and dy drawn on the device).  Its SFU count is
     twice the forward's D(N+2) per token (the forward exponentials are evaluated once in the
-    checkpoint pass and once more in the recomputation)."""
+    segment pass and once more in the walk's recomputation)."""
     import torch
     import selective_state_space_15_b200 as ssm
     stream = torch.cuda.current_stream()
@@ -442,7 +442,7 @@ def bwd_run(name, steps, warmup, sfu_peak):
     exps = 2 * b * L * D * (N + 2)
     return {"ms": round(ms, 4), "tokens_per_s": b * L / (ms * 1e-3), "sfu_frac": round(exps / (ms * 1e-3) / sfu_peak, 4),
             "shape": f"batch {b}, D={D}, N={N}, L={L}, {c['dtype']}", "exps_counted": "2 D (N+2) per token",
-            "launches": "checkpoint forward + reverse walk + tile sums (+ 4 memsets)"}
+            "launches": "segment pass + segment scan + reverse walk (+ 6 memsets)"}
 
 
 SSD_SHAPE = dict(batch=4, nheads=32, headdim=64, dstate=128, seqlen=4096, seed=910)

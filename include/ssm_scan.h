@@ -205,10 +205,15 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
  * Gradients of the fixed-length batch scan: the reverse-mode derivative of ssm_scan_fwd's
  * outputs y and h_last with respect to u, delta, z, B, C, A, Dskip, delta_bias and h0, for
  * training.  It follows the schedule of the "会议长序列建模…" page (ufo.work), §2.2 (strategy B:
- * keep checkpoints, recompute the rest) and its second article, §3.1 (chunk-level checkpoints):
- * a forward pass keeps only the state every few steps (in the workspace), then the sequence
- * is walked backwards, each short stretch recomputed from its checkpoint and the adjoint
- * recurrence dh_{t-1} = exp(Delta_t A) (dh_t + C_t dyraw_t) carried from the end.
+ * keep checkpoints, recompute the rest) and its second article, §3.1 (chunk-boundary states
+ * and the composition of chunk operators): the sequence is cut into time segments; a first
+ * pass keeps, per segment, its state every 8 steps from a zero start and its zero-start
+ * forward and adjoint operators (in the workspace); the operators are composed across the
+ * segments (the true state entering and adjoint leaving each); then every segment is walked
+ * backwards, each 8-step stretch recomputed from its checkpoint and the adjoint recurrence
+ * dh_{t-1} = exp(Delta_t A) (dh_t + C_t dyraw_t) carried from the segment's end.  dA, dDskip,
+ * ddelta_bias, dB and dC are sums formed with atomics, so their last bits may differ from
+ * call to call; du, ddelta, dz and dh0 are reproducible.
  *
  * `p` describes the forward problem as for ssm_scan_fwd (the same inputs; p->y and p->h_last
  * are not used and may be NULL).  Supported:
@@ -227,7 +232,7 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
  *   dDskip, ddelta_bias : [dim] float32, or NULL (not computed)
  *   dh0         : [batch][dim][dstate] float32, or NULL (not computed)
  * The workspace (ssm_scan_bwd_workspace_size bytes, 16-byte aligned) holds the checkpoints
- * and per-tile partial sums of dB and dC; its contents on entry do not matter.
+ * and the per-segment operators; its contents on entry do not matter.
  */
 typedef struct ssm_scan_grads {
   const void *dy;

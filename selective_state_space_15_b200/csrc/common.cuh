@@ -172,6 +172,21 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Plain arrive (no transaction bytes): completes the phase of a count-1 barrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// 1-D bulk copy shared -> global, tracked by bulk groups (no multicast).  Same alignment rules.
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store has finished reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until every committed bulk store has completed its global writes.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -224,10 +239,6 @@ struct ScanArgs {
   int nchains;       // nseq * ntiles
   int group;         // chunks per work unit
   int total_units;   // nchains * ceil(nchunks / group) (chunked kernel); units (lane-sequential kernel)
-  // checkpoint mode of the lane-sequential kernel (the backward's first pass): the state
-  // entering every 8-step block is stored to ckpt[b][block][dim][N]; y is not computed
-  float *ckpt;
-  int64_t ckpt_blocks;  // blocks per sequence: ceil(seqlen / 8)
 };
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {

@@ -1,11 +1,24 @@
-// Backward pass of the selective scan (gradients for training), lane-sequential.
+// Backward pass of the selective scan (gradients for training), in time segments.
 //
 // Schedule ("ufo.work" page, §2.2, strategy B: keep checkpoints, recompute the rest; its
-// second article, §3.1: chunk-level checkpoints).  A first launch (the lane-sequential
-// forward kernel in checkpoint mode) stores the state entering every 8-step block.  This
-// kernel then walks each (sequence, channel tile) from the end: for every 8-step block it
-// recomputes a_t = exp(Delta_t A) and h_t from the block's checkpoint, keeping them in
-// registers, and runs the adjoint recurrence backwards through the block:
+// second article, §3.1: chunk-boundary states and the composition of chunk operators).  The
+// sequence is cut into segments of seg_len steps so that every (sequence, segment, channel
+// tile) is a unit of its own and even one long sequence fills the GPU:
+//
+//  1. bwd_seg_kernel, per unit, in forward order from a zero state: the zero-start state hz
+//     entering every 8-step block (the block's checkpoint) and the sum of Delta from the
+//     segment start to the block (exp(A sum) is the block's decay from the segment start); at
+//     the segment end hz (the segment's forward operator applied to zero), the sum of Delta
+//     over the segment (its decay exp(A sum)) and the zero-start adjoint
+//         G = sum_t (prod_{k <= t} a_k) C_t dyraw_t,
+//     which the segment passes to the step before it when no adjoint enters from its end (with
+//     mu entering from the end it passes exp(A sum) mu + G).
+//  2. bwd_seg_scan_kernel, per (sequence, channel, state): the segment operators composed
+//     forwards from h0 (the true state entering each segment) and backwards from dh_last (the
+//     true adjoint entering each segment from its end).
+//  3. seq_bwd_kernel, per unit: walks the segment from its end.  For every 8-step block it
+//     recomputes a_t = exp(Delta_t A) and h_t from the block's state hz + exp(A sum) h_start,
+//     keeping them in registers, and runs the adjoint recurrence backwards through the block:
 //
 //   dyraw_t  = dy_t silu(z_t)                 dz_t = dy_t yraw_t silu'(z_t)
 //   dh      += dyraw_t C_t                    (y_t reads h_t)
@@ -14,23 +27,23 @@
 //   dDelta_t = sum_n (dh h_{t-1} a_t A + dh B_t u_t)      ddelta_t = dDelta_t sigmoid(delta_t + bias)
 //   dA      += dh h_{t-1} a_t Delta_t         dh *= a_t                   (on to h_{t-1})
 //
-// with yraw_t = sum_n C_t h_t + D u_t (the ungated output).  dh starts from dh_last and ends
-// as dh0.  Each exponential of the forward is evaluated twice in total (checkpoint pass and
-// recompute), none a third time.
+// with yraw_t = sum_n C_t h_t + D u_t (the ungated output).  dh starts from the adjoint that
+// enters the segment from its end and, in the first segment, ends as dh0.  Each forward
+// exponential is evaluated twice (segment pass, recompute), none a third time.
 //
 // Lanes: LPC = 4 lanes share a channel and split its states (NS = N / 4 each); a warp holds
-// 8 channels, a CTA W warps (8 W channels; the host picks W so that there are enough units).  Per block a lane evaluates the per-step terms
-// (softplus, its derivative, the gate) for 2 of the 8 steps and hands them to the channel's
-// other lanes by shuffles; sums over the states (yraw, du, dDelta) are reduced across those 4
-// lanes.  The sums over channels (dB, dC) go through shared memory: every lane writes its
-// per-state terms, each warp adds its 8 channels, the four warps meet in a per-chunk
-// accumulator, and the CTA writes one partial row per (tile, sequence, state) to the
-// workspace; a last kernel adds the tiles' partials.  dA, dDskip and dbias are summed in
-// registers and added to their outputs with atomics once per unit.
+// 8 channels, a CTA W warps.  Per block a lane evaluates the per-step terms (softplus, its
+// derivative, the gate) for 2 of the 8 steps and hands them to the channel's other lanes by
+// shuffles; sums over the states (yraw, du, dDelta) are reduced across those 4 lanes.  The
+// sums over channels (dB, dC) go through shared memory: every lane writes its per-state
+// terms, each warp adds its 8 channels, the warps meet in a per-chunk accumulator (shared
+// atomics), and the CTA adds the chunk's rows to dB and dC with global atomics (16-byte
+// vector atomics where the rows allow them).  dA, dDskip and dbias are summed in registers
+// and added with atomics once per unit.
 //
 // Staging is the forward's: TMA bulk copies of the u, delta, z, dy rows and the B, C rows of a
-// chunk (here in reverse chunk order), double-buffered, with B and C widened to float32 in a
-// [step][state] layout once per chunk.
+// chunk, double-buffered, with B and C widened to float32 in a [step][state] layout once per
+// chunk.  Segments are whole chunks.
 #pragma once
 
 #include "common.cuh"
@@ -43,9 +56,16 @@ struct BwdArgs {
   const float *dh_last;    // [batch][dim][N] or nullptr
   void *du, *ddelta, *dz;  // [batch][dim][seqlen], dtype TG
   float *dA, *dDskip, *dbias, *dh0;
-  const float *ckpt;       // [batch][ckpt_blocks][dim][N]: state entering each 8-step block
-  float *partials;         // [ntiles][batch][2][N][seqlen]: per-tile sums of dB (0) and dC (1)
-  int64_t ckpt_blocks;
+  float *dB, *dC;          // [batch][N][seqlen], zero on entry to the walk (summed by atomics)
+  float *ckpt;             // [batch][nblk][dim][N]: zero-start state of the segment entering each block
+  float *cumd;             // [batch][nblk][dim]: sum of Delta from the segment start to the block
+  float *seg_sum;          // [batch][nseg][dim]: sum of Delta over the segment
+  float *seg_h;            // [batch][nseg][dim][N]: zero-start final state; after the scan: state entering
+  float *seg_g;            // [batch][nseg][dim][N]: zero-start adjoint; after the scan: adjoint from the end
+  int64_t nblk;            // blocks per sequence: ceil(seqlen / 8)
+  int64_t seg_len;         // steps per segment (a multiple of the chunk)
+  int nseg;                // segments per sequence
+  int vec_dbc;             // dB, dC rows take 16-byte vector atomics
 };
 
 // sigmoid(x) from w = e^-|x| (which the softplus already has): 1/(1+w) for x > 0, w/(1+w) else.
@@ -55,8 +75,30 @@ __device__ __forceinline__ float sigmoid_from_w(float x, float w) {
   return (x > 0.f ? 1.f : w) * r;
 }
 
+// softplus(x) from one exponential (the forward kernels' softplus_fast) and, when asked for,
+// sigmoid(x), its derivative, from the same exponential
+template <bool kFast, bool kSig> __device__ __forceinline__ float softplus_sig(float x, float &sgm) {
+  if constexpr (kFast) {
+    const float w = ex2_approx(-fabsf(x) * kLog2e);
+    float q = fmaf(w, -0.00853909645229578f, 0.044089239090681076f);
+    q = fmaf(w, q, -0.10768117010593414f);
+    q = fmaf(w, q, 0.17745204269886017f);
+    q = fmaf(w, q, -0.24495449662208557f);
+    q = fmaf(w, q, 0.33275479078292847f);
+    q = fmaf(w, q, -0.4999740421772003f);
+    q = fmaf(w, q, 0.9999998211860657f);
+    if constexpr (kSig) sgm = sigmoid_from_w(x, w);
+    return fmaf(w, q, fmaxf(x, 0.f));
+  } else {
+    if constexpr (kSig) sgm = 1.f / (1.f + expf(-x));
+    return softplus_precise(x);
+  }
+}
+
 template <typename T, typename TG, int N, int TC, int W>
 struct BwdCfg {
+  static constexpr int kN = N;
+  static constexpr int kTC = TC;
   static constexpr int kLPC = 4;
   static constexpr int kNS = N / kLPC;
   static constexpr int kCPW = 32 / kLPC;  // 8 channels per warp
@@ -79,17 +121,286 @@ struct BwdCfg {
   static constexpr size_t kOffPart = kOffBF + 2 * kBFElems * sizeof(float);
   static constexpr size_t kOffAcc = kOffPart + kWarps * kPartElems * sizeof(float);
   static constexpr size_t kSmemBytes = kOffAcc + 2 * kAccElems * sizeof(float);
+  static constexpr size_t kSegSmemBytes = kOffPart;  // the segment pass needs the staging only
   static_assert(kNS % 4 == 0, "whole float4 groups of states per lane");
   static_assert(TC % 8 == 0 && (kXP * sizeof(T)) % 16 == 0 && (kXP * sizeof(TG)) % 16 == 0, "16-byte rows");
   static_assert(kOffY % 16 == 0 && kOffBF % 16 == 0 && kOffPart % 16 == 0, "aligned buffers");
 };
 
+// Where a unit's work lies: unit = (sequence s, segment, channel tile), tiles fastest.
+struct BwdUnit {
+  int tile, seg, s;
+  int64_t d0, t_lo, t_hi;
+  int c_lo, c_hi;  // chunks [c_lo, c_hi)
+};
+template <int TC, int CT>
+__device__ __forceinline__ BwdUnit bwd_unit(const ScanArgs &args, const BwdArgs &bw, int unit) {
+  BwdUnit w;
+  w.tile = unit % args.ntiles;
+  const int rest = unit / args.ntiles;
+  w.seg = rest % bw.nseg;
+  w.s = rest / bw.nseg;
+  w.d0 = int64_t(w.tile) * CT;
+  w.t_lo = int64_t(w.seg) * bw.seg_len;
+  w.t_hi = min64(args.seqlen, w.t_lo + bw.seg_len);
+  w.c_lo = int(w.t_lo / TC);
+  w.c_hi = int((w.t_hi + TC - 1) / TC);
+  return w;
+}
+
+// TMA staging of chunk cc: the u, delta (and z) rows and the dy rows of the tile and the B, C
+// rows of the chunk window, into buffer `buf`, completing on `bar`.
+template <typename Cfg, typename T, typename TG>
+__device__ __forceinline__ void bwd_stage(const ScanArgs &args, const BwdArgs &bw, T *xs0, TG *ys0, T *bcs0,
+                                          uint64_t *bar, int buf, int cc, int nx, int nvalid, int64_t d0,
+                                          int64_t xbase, int64_t bcbase) {
+  constexpr int CT = Cfg::kCT, NT = Cfg::kThreads, XP = Cfg::kXP, N = Cfg::kN, TC = Cfg::kTC;
+  constexpr int V = Elem<T>::kVec;
+  const int64_t seqlen_r = (args.seqlen + V - 1) / V * V;
+  const int64_t wstart = int64_t(cc) * TC;
+  const int64_t wend = min64(wstart + TC, seqlen_r);
+  const uint32_t rows_t = uint32_t((wend - wstart) * int64_t(sizeof(T)));
+  const uint32_t rows_g = uint32_t((wend - wstart) * int64_t(sizeof(TG)));
+  T *xd = xs0 + buf * Cfg::kXElems;
+  TG *yd = ys0 + buf * Cfg::kYElems;
+  T *bd = bcs0 + buf * Cfg::kBCElems;
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0)
+    mbar_arrive_expect_tx(bar, rows_t * uint32_t(nx * nvalid + 2 * N) + rows_g * uint32_t(nvalid));
+  for (int r = threadIdx.x; r < (nx + 1) * CT + 2 * N; r += NT) {
+    if (r < nx * CT) {
+      const int which = r / CT, c2 = r % CT;
+      if (c2 >= nvalid) continue;
+      const T *base = static_cast<const T *>(which == 0 ? args.u : (which == 1 ? args.delta : args.z));
+      bulk_g2s(xd + size_t(r) * XP, base + xbase + (d0 + c2) * args.x_dim_stride + wstart, rows_t, bar);
+    } else if (r < (nx + 1) * CT) {
+      const int c2 = r - nx * CT;
+      if (c2 >= nvalid) continue;
+      bulk_g2s(yd + size_t(c2) * XP, static_cast<const TG *>(bw.dy) + xbase + (d0 + c2) * args.x_dim_stride + wstart,
+               rows_g, bar);
+    } else {
+      const int r2 = r - (nx + 1) * CT, which = r2 / N, n = r2 % N;
+      const T *base = static_cast<const T *>(which == 0 ? args.B : args.C);
+      bulk_g2s(bd + size_t(r2) * TC, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, rows_t, bar);
+    }
+  }
+}
+
+// B and C of a staged chunk widened to float32, [step][state] (C at kCOff)
+template <typename Cfg, typename T>
+__device__ __forceinline__ void bwd_widen(const T *bs, float *bfw) {
+  constexpr int N = Cfg::kN, TC = Cfg::kTC;
+  for (int i = threadIdx.x; i < 2 * N * (TC / 8); i += Cfg::kThreads) {
+    const int row = i % (2 * N), blk = i / (2 * N);
+    float f[8];
+    load_sub<T, 8>(bs + size_t(row) * TC + blk * 8, f);
+    float *dst = bfw + (row >= N ? Cfg::kCOff : 0) + blk * 8 * N + row % N;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dst[j * N] = f[j];
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// 1. The segment pass.
+template <typename T, typename TG, int N, int TC, int W, bool HAS_Z>
+__global__ void __launch_bounds__(W * 32, 12 / W) bwd_seg_kernel(const ScanArgs args, const BwdArgs bw) {
+  using Cfg = BwdCfg<T, TG, N, TC, W>;
+  constexpr int LPC = Cfg::kLPC, NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT;
+  constexpr int XP = Cfg::kXP, SUB = Cfg::kSub;
+  constexpr bool kFast = Elem<T>::kFast;
+  constexpr int nx = HAS_Z ? 3 : 2;
+
+  extern __shared__ __align__(16) unsigned char smem[];
+  T *const xs0 = reinterpret_cast<T *>(smem);
+  TG *const ys0 = reinterpret_cast<TG *>(smem + Cfg::kOffY);
+  T *const bcs0 = reinterpret_cast<T *>(smem + Cfg::kOffBC);
+  float *const bf0 = reinterpret_cast<float *>(smem + Cfg::kOffBF);
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int unit_sh;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int g = lane % LPC, c = lane / LPC;
+  const int ch = warp * CPW + c;
+  const int lbase = lane - g;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  uint32_t gc = 0;
+
+  for (;;) {
+    if (threadIdx.x == 0) unit_sh = int(atomicAdd(args.ticket, 1u));
+    __syncthreads();
+    const int unit = unit_sh;
+    if (unit >= args.total_units) break;
+    const BwdUnit w = bwd_unit<TC, CT>(args, bw, unit);
+    const int nvalid = int(min64(CT, args.dim - w.d0));
+    const int64_t d = w.d0 + ch;
+    const bool ch_ok = d < args.dim;
+    const int64_t xbase = int64_t(w.s) * args.x_batch_stride;
+    const int64_t bcbase = int64_t(w.s) * args.bc_batch_stride;
+
+    float2 A2[NS / 2], hz[NS / 2], pp[NS / 2], gb[NS / 2];
+    float bias = 0.f, cd = 0.f;
+#pragma unroll
+    for (int p = 0; p < NS / 2; ++p) {
+      A2[p] = hz[p] = gb[p] = make_float2(0.f, 0.f);
+      pp[p] = make_float2(1.f, 1.f);
+    }
+    if (ch_ok) {
+      const float *Ar = args.A + d * N + g * NS;
+#pragma unroll
+      for (int p = 0; p < NS / 2; ++p) A2[p] = make_float2(Ar[2 * p] * kLog2e, Ar[2 * p + 1] * kLog2e);
+      bias = args.bias ? args.bias[d] : 0.f;
+    }
+
+    // one 8-step block, first step first
+    auto block = [&](auto masked_tag, const T *X, const TG *Y, const float *Bf, int64_t wstart, int sb) {
+      constexpr bool kMasked = decltype(masked_tag)::value;
+      const int k0 = sb * 8;
+      const int64_t gblk = (wstart + k0) / 8;
+      const int rel_hi = int(min64(w.t_hi - (wstart + k0), 8));
+      const int c0 = k0 + g * SUB;
+      float uv[SUB], dv[SUB], gv[SUB], dm[SUB], um[SUB], rm[SUB];
+      [[maybe_unused]] float zv[SUB];
+      load_sub<T, SUB>(X + size_t(ch) * XP + c0, uv);
+      load_sub<T, SUB>(X + size_t(CT + ch) * XP + c0, dv);
+      if constexpr (HAS_Z) load_sub<T, SUB>(X + size_t(2 * CT + ch) * XP + c0, zv);
+      load_sub<TG, SUB>(Y + size_t(ch) * XP + c0, gv);
+#pragma unroll
+      for (int j = 0; j < SUB; ++j) {
+        float unused;
+        const float dt = softplus_sig<kFast, false>(dv[j] + bias, unused);
+        float dyr = gv[j];
+        if constexpr (HAS_Z) dyr *= silu_t<kFast>(zv[j]);
+        const bool in = ch_ok && (!kMasked || g * SUB + j < rel_hi);  // stale rows stay out
+        dm[j] = in ? dt : 0.f;
+        um[j] = in ? dt * uv[j] : 0.f;
+        rm[j] = in ? dyr : 0.f;
+      }
+      float dl[8], dU[8], dr[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        dl[k] = __shfl_sync(0xffffffffu, dm[k % SUB], lbase + k / SUB);
+        dU[k] = __shfl_sync(0xffffffffu, um[k % SUB], lbase + k / SUB);
+        dr[k] = __shfl_sync(0xffffffffu, rm[k % SUB], lbase + k / SUB);
+      }
+      if (ch_ok) {
+        const int64_t bo = (int64_t(w.s) * bw.nblk + gblk) * args.dim + d;
+        float *ck = bw.ckpt + bo * N + g * NS;
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q)
+          reinterpret_cast<float4 *>(ck)[q] = make_float4(hz[2 * q].x, hz[2 * q].y, hz[2 * q + 1].x, hz[2 * q + 1].y);
+        if (g == 0) bw.cumd[bo] = cd;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int t = k0 + k;
+        const float2 dd = make_float2(dl[k], dl[k]), uu = make_float2(dU[k], dU[k]), rr = make_float2(dr[k], dr[k]);
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q) {
+          float4 b4 = reinterpret_cast<const float4 *>(Bf + t * N + g * NS)[q];
+          float4 c4 = reinterpret_cast<const float4 *>(Bf + Cfg::kCOff + t * N + g * NS)[q];
+          if constexpr (kMasked) {
+            if (k >= rel_hi) b4 = c4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int p = 2 * q + e;
+            const float2 bp = e ? make_float2(b4.z, b4.w) : make_float2(b4.x, b4.y);
+            const float2 cp = e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+            const float2 x = __fmul2_rn(dd, A2[p]);
+            const float2 a = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            hz[p] = __ffma2_rn(a, hz[p], __fmul2_rn(uu, bp));
+            pp[p] = __fmul2_rn(pp[p], a);
+            gb[p] = __ffma2_rn(pp[p], __fmul2_rn(rr, cp), gb[p]);
+          }
+        }
+        cd += dl[k];
+      }
+    };
+
+    if (w.c_hi > w.c_lo)
+      bwd_stage<Cfg>(args, bw, xs0, ys0, bcs0, &bars[gc & 1u], int(gc & 1u), w.c_lo, nx, nvalid, w.d0, xbase, bcbase);
+    for (int cc = w.c_lo; cc < w.c_hi; ++cc, ++gc) {
+      const int buf = int(gc & 1u);
+      const int64_t wstart = int64_t(cc) * TC;
+      const bool landed = mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
+      bwd_widen<Cfg>(bcs0 + buf * Cfg::kBCElems, bf0 + buf * Cfg::kBFElems);
+      // chunk cc widened; every warp is done with chunk cc-1's buffers
+      if (__syncthreads_or(!landed)) {
+        mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);  // no copy left writing shared memory
+        return;
+      }
+      if (cc + 1 < w.c_hi)
+        bwd_stage<Cfg>(args, bw, xs0, ys0, bcs0, &bars[buf ^ 1], buf ^ 1, cc + 1, nx, nvalid, w.d0, xbase, bcbase);
+      const T *X = xs0 + buf * Cfg::kXElems;
+      const TG *Y = ys0 + buf * Cfg::kYElems;
+      const float *Bf = bf0 + buf * Cfg::kBFElems;
+#pragma unroll 1
+      for (int sb = 0; sb < TC / 8; ++sb) {
+        if (wstart + sb * 8 >= w.t_hi) break;  // uniform
+        if (wstart + sb * 8 + 8 <= w.t_hi)
+          block(std::false_type{}, X, Y, Bf, wstart, sb);
+        else
+          block(std::true_type{}, X, Y, Bf, wstart, sb);
+      }
+    }
+    if (ch_ok) {
+      const int64_t o = (int64_t(w.s) * bw.nseg + w.seg) * args.dim + d;
+#pragma unroll
+      for (int q = 0; q < NS / 4; ++q) {
+        reinterpret_cast<float4 *>(bw.seg_h + o * N + g * NS)[q] =
+            make_float4(hz[2 * q].x, hz[2 * q].y, hz[2 * q + 1].x, hz[2 * q + 1].y);
+        reinterpret_cast<float4 *>(bw.seg_g + o * N + g * NS)[q] =
+            make_float4(gb[2 * q].x, gb[2 * q].y, gb[2 * q + 1].x, gb[2 * q + 1].y);
+      }
+      if (g == 0) bw.seg_sum[o] = cd;
+    }
+    __syncthreads();  // shared state of this unit is dead before the next unit overwrites it
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// 2. The segment scan: one thread per (sequence, channel, state).  Forwards, seg_h becomes the
+// state entering each segment (from h0); backwards, seg_g becomes the adjoint entering each
+// segment from its end (from dh_last).
+__global__ void __launch_bounds__(256) bwd_seg_scan_kernel(const float *A, const float *h0, const float *dh_last,
+                                                           const float *seg_sum, float *seg_h, float *seg_g,
+                                                           int64_t batch, int64_t dim, int N, int nseg) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= batch * dim * N) return;
+  const int64_t dn = e % (dim * N), s = e / (dim * N);
+  const int64_t d = dn / N, n = dn % N;
+  const float A2 = A[dn] * kLog2e;
+  float h = h0 ? h0[e] : 0.f;
+  for (int q = 0; q < nseg; ++q) {
+    const int64_t o = (s * nseg + q) * dim + d;
+    const float P = ex2_approx(A2 * seg_sum[o]);
+    const float gz = seg_h[o * N + n];
+    seg_h[o * N + n] = h;
+    h = fmaf(P, h, gz);
+  }
+  float mu = dh_last ? dh_last[e] : 0.f;
+  for (int q = nseg - 1; q >= 0; --q) {
+    const int64_t o = (s * nseg + q) * dim + d;
+    const float P = ex2_approx(A2 * seg_sum[o]);
+    const float gz = seg_g[o * N + n];
+    seg_g[o * N + n] = mu;
+    mu = fmaf(P, mu, gz);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// 3. The walk.
 template <typename T, typename TG, int N, int TC, int W, bool HAS_Z>
 __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs args, const BwdArgs bw) {
   using Cfg = BwdCfg<T, TG, N, TC, W>;
   constexpr int LPC = Cfg::kLPC, NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT, NT = Cfg::kThreads;
   constexpr int XP = Cfg::kXP, SUB = Cfg::kSub;
-  constexpr int V = Elem<T>::kVec;
   constexpr bool kFast = Elem<T>::kFast;
   constexpr int nx = HAS_Z ? 3 : 2;
 
@@ -108,7 +419,6 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
   const int ch = warp * CPW + c;
   const int lbase = lane - g;
   const int64_t L = args.seqlen;
-  const int64_t seqlen_r = (L + V - 1) / V * V;
   float *const part = part0 + size_t(warp) * Cfg::kPartElems;
 
   if (threadIdx.x == 0) {
@@ -125,79 +435,58 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
     __syncthreads();
     const int unit = unit_sh;
     if (unit >= args.total_units) break;
-    const int tile = unit % args.ntiles;
-    const int s = unit / args.ntiles;
-    const int64_t d0 = int64_t(tile) * CT;
+    const BwdUnit w = bwd_unit<TC, CT>(args, bw, unit);
+    const int s = w.s;
+    const int64_t d0 = w.d0;
     const int nvalid = int(min64(CT, args.dim - d0));
     const int64_t d = d0 + ch;
     const bool ch_ok = d < args.dim;
     const int64_t xbase = int64_t(s) * args.x_batch_stride;
     const int64_t bcbase = int64_t(s) * args.bc_batch_stride;
-    const int nchunks = L > 0 ? int((L + TC - 1) / TC) : 0;
+    const int64_t so = (int64_t(s) * bw.nseg + w.seg) * args.dim + d;  // this segment's row
 
-    float2 A2[NS / 2], An[NS / 2], dh[NS / 2], dAacc[NS / 2];
+    float2 A2[NS / 2], An[NS / 2], dh[NS / 2], dAacc[NS / 2], hs[NS / 2];
     float bias = 0.f, Dd = 0.f, dDacc = 0.f, dbacc = 0.f;
 #pragma unroll
     for (int p = 0; p < NS / 2; ++p) {
-      A2[p] = An[p] = dh[p] = dAacc[p] = make_float2(0.f, 0.f);
+      A2[p] = An[p] = dh[p] = dAacc[p] = hs[p] = make_float2(0.f, 0.f);
     }
     if (ch_ok) {
       const float *Ar = args.A + d * N + g * NS;
+      const float *mr = bw.seg_g + so * N + g * NS;  // the adjoint entering from the segment's end
+      const float *hr = bw.seg_h + so * N + g * NS;  // the state entering the segment
 #pragma unroll
       for (int p = 0; p < NS / 2; ++p) {
         An[p] = make_float2(Ar[2 * p], Ar[2 * p + 1]);
         A2[p] = make_float2(An[p].x * kLog2e, An[p].y * kLog2e);
-      }
-      if (bw.dh_last) {
-        const float *hr = bw.dh_last + (int64_t(s) * args.dim + d) * N + g * NS;
-#pragma unroll
-        for (int p = 0; p < NS / 2; ++p) dh[p] = make_float2(hr[2 * p], hr[2 * p + 1]);
+        dh[p] = make_float2(mr[2 * p], mr[2 * p + 1]);
+        hs[p] = make_float2(hr[2 * p], hr[2 * p + 1]);
       }
       bias = args.bias ? args.bias[d] : 0.f;
       Dd = args.Dskip ? args.Dskip[d] : 0.f;
     }
 
-    auto issue_chunk = [&](int buf, int cc) {
-      const int64_t wstart = int64_t(cc) * TC;
-      const int64_t wend = min64(wstart + TC, seqlen_r);
-      const uint32_t rows_t = uint32_t((wend - wstart) * int64_t(sizeof(T)));
-      const uint32_t rows_g = uint32_t((wend - wstart) * int64_t(sizeof(TG)));
-      T *xd = xs0 + buf * Cfg::kXElems;
-      TG *yd = ys0 + buf * Cfg::kYElems;
-      T *bd = bcs0 + buf * Cfg::kBCElems;
-      fence_proxy_async_smem();
-      if (threadIdx.x == 0)
-        mbar_arrive_expect_tx(&bars[buf], rows_t * uint32_t(nx * nvalid + 2 * N) + rows_g * uint32_t(nvalid));
-      for (int r = threadIdx.x; r < (nx + 1) * CT + 2 * N; r += NT) {
-        if (r < nx * CT) {
-          const int which = r / CT, c2 = r % CT;
-          if (c2 >= nvalid) continue;
-          const T *base = static_cast<const T *>(which == 0 ? args.u : (which == 1 ? args.delta : args.z));
-          bulk_g2s(xd + size_t(r) * XP, base + xbase + (d0 + c2) * args.x_dim_stride + wstart, rows_t, &bars[buf]);
-        } else if (r < (nx + 1) * CT) {
-          const int c2 = r - nx * CT;
-          if (c2 >= nvalid) continue;
-          bulk_g2s(yd + size_t(c2) * XP,
-                   static_cast<const TG *>(bw.dy) + xbase + (d0 + c2) * args.x_dim_stride + wstart, rows_g, &bars[buf]);
-        } else {
-          const int r2 = r - (nx + 1) * CT, which = r2 / N, n = r2 % N;
-          const T *base = static_cast<const T *>(which == 0 ? args.B : args.C);
-          bulk_g2s(bd + size_t(r2) * TC, base + bcbase + int64_t(n) * args.bc_state_stride + wstart, rows_t,
-                   &bars[buf]);
-        }
-      }
-    };
-
-    // the chunk accumulator `acc` (dB, dC summed over the CTA's channels) -> the tile's partial
-    // rows, then cleared for its next use
+    // the chunk accumulator `acc` (dB, dC summed over the CTA's channels) added to dB and dC,
+    // then cleared for its next use
     auto flush_acc = [&](int abuf, int cc) {
       float *acc = acc0 + abuf * Cfg::kAccElems;
       const int64_t wstart = int64_t(cc) * TC;
-      for (int i = threadIdx.x; i < 2 * N * TC; i += NT) {
-        const int row = i / TC, t = i % TC;  // row = which * N + n
-        if (wstart + t < L)
-          bw.partials[((int64_t(tile) * args.nseq + s) * 2 * N + row) * L + wstart + t] = acc[i];
-        acc[i] = 0.f;
+      for (int i = threadIdx.x; i < 2 * N * (TC / 4); i += NT) {
+        const int row = i / (TC / 4), t = (i % (TC / 4)) * 4;  // row = which * N + n
+        const int64_t gt = wstart + t;
+        float4 *src = reinterpret_cast<float4 *>(acc + row * TC + t);
+        const float4 v = *src;
+        *src = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (gt >= L) continue;
+        float *dst = (row >= N ? bw.dC : bw.dB) + (int64_t(s) * N + row % N) * L + gt;
+        if (bw.vec_dbc) {
+          atomicAdd(reinterpret_cast<float4 *>(dst), v);  // L % 4 == 0: the group lies inside the row
+        } else {
+          atomicAdd(dst, v.x);
+          if (gt + 1 < L) atomicAdd(dst + 1, v.y);
+          if (gt + 2 < L) atomicAdd(dst + 2, v.z);
+          if (gt + 3 < L) atomicAdd(dst + 3, v.w);
+        }
       }
     };
 
@@ -209,30 +498,16 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
       const int rel_hi = int(min64(L - (wstart + k0), 8));  // steps of the block inside the sequence
       // ---- this lane's SUB steps: softplus, its derivative, the gate
       const int c0 = k0 + g * SUB;
-      float uv[SUB], dv[SUB], zv[SUB], gv[SUB], dm[SUB], um[SUB], sg[SUB], zs[SUB], zd[SUB];
+      float uv[SUB], dv[SUB], gv[SUB], dm[SUB], um[SUB], sg[SUB];
+      [[maybe_unused]] float zv[SUB], zs[SUB], zd[SUB];
       load_sub<T, SUB>(X + size_t(ch) * XP + c0, uv);
       load_sub<T, SUB>(X + size_t(CT + ch) * XP + c0, dv);
       if constexpr (HAS_Z) load_sub<T, SUB>(X + size_t(2 * CT + ch) * XP + c0, zv);
       load_sub<TG, SUB>(Y + size_t(ch) * XP + c0, gv);
 #pragma unroll
       for (int j = 0; j < SUB; ++j) {
-        const float x = dv[j] + bias;
-        float dt, sgm;
-        if constexpr (kFast) {
-          const float w = ex2_approx(-fabsf(x) * kLog2e);
-          float q = fmaf(w, -0.00853909645229578f, 0.044089239090681076f);
-          q = fmaf(w, q, -0.10768117010593414f);
-          q = fmaf(w, q, 0.17745204269886017f);
-          q = fmaf(w, q, -0.24495449662208557f);
-          q = fmaf(w, q, 0.33275479078292847f);
-          q = fmaf(w, q, -0.4999740421772003f);
-          q = fmaf(w, q, 0.9999998211860657f);
-          dt = fmaf(w, q, fmaxf(x, 0.f));
-          sgm = sigmoid_from_w(x, w);
-        } else {
-          dt = softplus_precise(x);
-          sgm = 1.f / (1.f + expf(-x));
-        }
+        float sgm;
+        float dt = softplus_sig<kFast, true>(dv[j] + bias, sgm);
         float du = dt * uv[j], gy = gv[j];
         // a channel past the end of a ragged tile, or a step past the end of the sequence, takes
         // no part (its staged rows are stale; selects keep non-finite values out of the sums)
@@ -257,17 +532,26 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
         dl[k] = __shfl_sync(0xffffffffu, dm[k % SUB], lbase + k / SUB);
         dU[k] = __shfl_sync(0xffffffffu, um[k % SUB], lbase + k / SUB);
       }
-      // ---- recompute a_t and h_t over the block from its checkpoint
+      // ---- recompute a_t and h_t over the block from its state: the segment's zero-start
+      // state plus the state entering the segment, decayed to the block
       float2 hin[NS / 2];
 #pragma unroll
       for (int p = 0; p < NS / 2; ++p) hin[p] = make_float2(0.f, 0.f);
       if (ch_ok) {
-        const float *ck = bw.ckpt + ((int64_t(s) * bw.ckpt_blocks + gblk) * args.dim + d) * N + g * NS;
+        const int64_t bo = (int64_t(s) * bw.nblk + gblk) * args.dim + d;
+        const float *ck = bw.ckpt + bo * N + g * NS;
+        const float cdv = bw.cumd[bo];
+        const float2 cd2 = make_float2(cdv, cdv);
 #pragma unroll
         for (int q = 0; q < NS / 4; ++q) {
           const float4 v = reinterpret_cast<const float4 *>(ck)[q];
-          hin[2 * q] = make_float2(v.x, v.y);
-          hin[2 * q + 1] = make_float2(v.z, v.w);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int p = 2 * q + e;
+            const float2 x = __fmul2_rn(cd2, A2[p]);
+            const float2 dec = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            hin[p] = __ffma2_rn(dec, hs[p], e ? make_float2(v.z, v.w) : make_float2(v.x, v.y));
+          }
         }
       }
       float2 a[8][NS / 2], h[8][NS / 2];
@@ -436,32 +720,24 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
       __syncwarp();  // the warp's terms are consumed before the next block rewrites them
     };
 
-    // ------------------------------------------------------------- chunks, last first
-    if (nchunks > 0) issue_chunk(int(gc & 1u), nchunks - 1);
+    // ------------------------------------------------------------- the segment's chunks, last first
+    if (w.c_hi > w.c_lo)
+      bwd_stage<Cfg>(args, bw, xs0, ys0, bcs0, &bars[gc & 1u], int(gc & 1u), w.c_hi - 1, nx, nvalid, d0, xbase,
+                     bcbase);
     int prev_acc = -1;  // accumulator of the chunk done before this one (to be flushed)
-    for (int cc = nchunks - 1; cc >= 0; --cc, ++gc) {
+    for (int cc = w.c_hi - 1; cc >= w.c_lo; --cc, ++gc) {
       const int buf = int(gc & 1u);
       const int64_t wstart = int64_t(cc) * TC;
       const bool landed = mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
-      {
-        const T *bs = bcs0 + buf * Cfg::kBCElems;
-        float *bfw = bf0 + buf * Cfg::kBFElems;
-        for (int i = threadIdx.x; i < 2 * N * (TC / 8); i += NT) {
-          const int row = i % (2 * N), blk = i / (2 * N);
-          float f[8];
-          load_sub<T, 8>(bs + size_t(row) * TC + blk * 8, f);
-          float *dst = bfw + (row >= N ? Cfg::kCOff : 0) + blk * 8 * N + row % N;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) dst[j * N] = f[j];
-        }
-      }
+      bwd_widen<Cfg>(bcs0 + buf * Cfg::kBCElems, bf0 + buf * Cfg::kBFElems);
       // chunk cc widened; every warp is done with chunk cc+1 (its buffers and accumulator)
       if (__syncthreads_or(!landed)) {
         mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);  // no copy left writing shared memory
         return;
       }
       if (prev_acc >= 0) flush_acc(prev_acc, cc + 1);
-      if (cc > 0) issue_chunk(buf ^ 1, cc - 1);
+      if (cc > w.c_lo)
+        bwd_stage<Cfg>(args, bw, xs0, ys0, bcs0, &bars[buf ^ 1], buf ^ 1, cc - 1, nx, nvalid, d0, xbase, bcbase);
       const T *X = xs0 + buf * Cfg::kXElems;
       const TG *Y = ys0 + buf * Cfg::kYElems;
       const float *Bf = bf0 + buf * Cfg::kBFElems;
@@ -477,11 +753,11 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
       prev_acc = buf;
     }
     __syncthreads();
-    if (prev_acc >= 0) flush_acc(prev_acc, 0);
+    if (prev_acc >= 0) flush_acc(prev_acc, w.c_lo);
 
     // ------------------------------------------------------------- per-unit results
     if (ch_ok) {
-      if (bw.dh0) {
+      if (bw.dh0 && w.seg == 0) {
         float *hr = bw.dh0 + (int64_t(s) * args.dim + d) * N + g * NS;
 #pragma unroll
         for (int p = 0; p < NS / 2; ++p) {
@@ -506,22 +782,6 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
       if (bw.dbias) atomicAdd(bw.dbias + d, dbacc);
     }
     __syncthreads();  // shared state of this unit is dead before the next unit overwrites it
-  }
-}
-
-// dB, dC = the sum of the tiles' partial rows.  One thread per (sequence, which, state, step).
-__global__ void __launch_bounds__(256) bwd_reduce_tiles_kernel(const float *partials, float *dB, float *dC,
-                                                              int64_t ntiles, int64_t per_tile, int64_t per_which,
-                                                              int64_t L) {
-  // per_tile = batch * 2 * N * L (one tile's partials); element e of it = ((s * 2 + which) * N + n) * L + t
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < per_tile;
-       e += int64_t(gridDim.x) * blockDim.x) {
-    float sum = 0.f;
-    for (int64_t tl = 0; tl < ntiles; ++tl) sum += partials[tl * per_tile + e];
-    const int64_t row = e / L, t = e % L;          // row = (s * 2 + which) * N + n
-    const int64_t n = row % per_which, sw = row / per_which;
-    const int64_t s = sw / 2, which = sw % 2;
-    (which ? dC : dB)[(s * per_which + n) * L + t] = sum;
   }
 }
 

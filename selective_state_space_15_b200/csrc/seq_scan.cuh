@@ -116,16 +116,14 @@ template <typename TO, int SUB> __device__ __forceinline__ void store_sub(TO *p,
   }
 }
 
-// CKPT: checkpoint mode (fixed-length batches): the state entering every 8-step block is
-// stored to args.ckpt and nothing else is written (no y, no final state).
-template <typename T, typename TO, int N, int LPC, int TC, int W, bool HAS_Z, bool CKPT = false>
+template <typename T, typename TO, int N, int LPC, int TC, int W, bool HAS_Z>
 __global__ void __launch_bounds__(W * 32, (LPC == 1 ? 8 : 16) / W) seq_scan_kernel(const ScanArgs args) {
   using Cfg = SeqCfg<T, N, LPC, TC, W>;
   constexpr int NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT, NT = Cfg::kThreads, XP = Cfg::kXP;
   constexpr int SUB = Cfg::kSub;
   constexpr int V = Elem<T>::kVec;
   constexpr bool kFast = Elem<T>::kFast;
-  constexpr int nx = CKPT ? 2 : (HAS_Z ? 3 : 2);
+  constexpr int nx = HAS_Z ? 3 : 2;
 
   extern __shared__ __align__(16) unsigned char smem[];
   T *const xs0 = reinterpret_cast<T *>(smem);           // [2][3][CT][XP]
@@ -291,15 +289,6 @@ __global__ void __launch_bounds__(W * 32, (LPC == 1 ? 8 : 16) / W) seq_scan_kern
             dU[4 * q] = u4.x; dU[4 * q + 1] = u4.y; dU[4 * q + 2] = u4.z; dU[4 * q + 3] = u4.w;
           }
         }
-        if constexpr (CKPT) {
-          // the state entering this block (steps before the sequence start are identities)
-          const int64_t gblk = (wstart - w0) / 8 + blk;  // blocks past the sequence end are not stored
-          if (ch_ok && gblk < args.ckpt_blocks) {
-            float *ck = args.ckpt + ((int64_t(s) * args.ckpt_blocks + gblk) * args.dim + d) * N + g * NS;
-#pragma unroll
-            for (int n = 0; n < NS; n += 2) *reinterpret_cast<float2 *>(ck + n) = make_float2(h[n], h[n + 1]);
-          }
-        }
         // ---- the recurrence over the block's 8 steps for this lane's NS states, in step pairs
         float2 yp2[4];
 #pragma unroll
@@ -309,8 +298,7 @@ __global__ void __launch_bounds__(W * 32, (LPC == 1 ? 8 : 16) / W) seq_scan_kern
 #pragma unroll
           for (int n = 0; n < NS; ++n) {
             const float4 b4 = reinterpret_cast<const float4 *>(Bb + size_t(n) * BP + blk * 8)[q];
-            [[maybe_unused]] float4 c4;
-            if constexpr (!CKPT) c4 = reinterpret_cast<const float4 *>(Cb + size_t(n) * BP + blk * 8)[q];
+            const float4 c4 = reinterpret_cast<const float4 *>(Cb + size_t(n) * BP + blk * 8)[q];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int k2 = 2 * q + e;
@@ -326,13 +314,11 @@ __global__ void __launch_bounds__(W * 32, (LPC == 1 ? 8 : 16) / W) seq_scan_kern
               }
               const float h0v = fmaf(a.x, h[n], bb.x);
               h[n] = fmaf(a.y, h0v, bb.y);
-              if constexpr (!CKPT)
-                yp2[k2] = __ffma2_rn(e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y), make_float2(h0v, h[n]),
+              yp2[k2] = __ffma2_rn(e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y), make_float2(h0v, h[n]),
                                      yp2[k2]);
             }
           }
         }
-        if constexpr (CKPT) continue;
         float yp[8];
 #pragma unroll
         for (int k2 = 0; k2 < 4; ++k2) {
@@ -357,7 +343,8 @@ __global__ void __launch_bounds__(W * 32, (LPC == 1 ? 8 : 16) / W) seq_scan_kern
         // ---- skip term, gate, store this lane's SUB steps
         if (ch_ok) {
           const int c0 = blk * 8 + g * SUB;
-          float uv[SUB], zv[SUB], o[SUB];
+          float uv[SUB], o[SUB];
+          [[maybe_unused]] float zv[SUB];
           load_sub<T, SUB>(ru + c0, uv);
           if constexpr (HAS_Z) load_sub<T, SUB>(rz + c0, zv);
 #pragma unroll
@@ -445,7 +432,7 @@ __global__ void __launch_bounds__(W * 32, (LPC == 1 ? 8 : 16) / W) seq_scan_kern
     }
 
     // ------------------------------------------------------------- final state
-    if (!CKPT && args.h_last && srow >= 0 && ch_ok) {
+    if (args.h_last && srow >= 0 && ch_ok) {
       float *hr = args.h_last + (srow * args.dim + d) * N + g * NS;
 #pragma unroll
       for (int n = 0; n < NS; ++n) hr[n] = h[n];

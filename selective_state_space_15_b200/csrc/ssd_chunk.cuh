@@ -22,8 +22,10 @@
 // significant bits: the bf16 inputs are represented exactly, the computed operands (M, V, V',
 // C', H) are rounded once, and every sum is accumulated in float32.
 //
-// One CTA (four warps, 128 threads) per (sequence, head) walks the chunks in order.  Shared
-// memory: seven operand tiles (176 KB); tensor memory: 256 columns (G, Y, the state).
+// One CTA (eight warps: two threads per row of every tile) per (sequence, head) walks the
+// chunks in order.  Inputs are read with 16-byte loads along the time axis; the transposed
+// operands (C^T, B^T: rows t) are formed in shared memory from the row-major copies (rows n).
+// Shared memory: seven operand tiles (176 KB); tensor memory: 256 columns (G, Y, the state).
 #pragma once
 
 #include "common.cuh"
@@ -57,8 +59,9 @@ constexpr uint32_t kSsdOffM = kSsdOffBN + kSsdTile128;   // M [t][s]
 constexpr uint32_t kSsdOffV = kSsdOffM + kSsdTile128;    // V [p][s]
 constexpr uint32_t kSsdOffVS = kSsdOffV + kSsdTile64;    // V' [p][s]
 constexpr uint32_t kSsdOffH = kSsdOffVS + kSsdTile64;    // H [p][n]
-constexpr uint32_t kSsdOffCum = kSsdOffH + kSsdTile64;   // cum [128] float
-constexpr uint32_t kSsdSmemBytes = kSsdOffCum + kSsdT * 4 + 1024;  // + slack to align the base to 1024
+constexpr uint32_t kSsdOffCum = kSsdOffH + kSsdTile64;   // cum, dt, decay to the chunk end: 3 x [128] float
+constexpr uint32_t kSsdSmemBytes = kSsdOffCum + 3 * kSsdT * 4 + 1024;  // + slack to align the base to 1024
+constexpr int kSsdThreads = 256;
 
 // Write 8 float16 values (K-elements 8j .. 8j+7 of row r) into a K-major swizzled operand
 // whose K extent is split into 64-element tiles of `rows` rows each.
@@ -71,18 +74,41 @@ __device__ __forceinline__ void ssd_put8(unsigned char *tile, uint32_t rows, uin
   *reinterpret_cast<uint4 *>(tile + kb * rows * 128u + tc::sw128_offset(r, kk)) = *reinterpret_cast<uint4 *>(h);
 }
 
-__global__ void __launch_bounds__(128, 1) ssd_chunk_kernel(const SsdArgs args) {
+// The same for 8 float16 values already converted.
+__device__ __forceinline__ void ssd_put8h(unsigned char *tile, uint32_t rows, uint32_t r, uint32_t k0, uint4 v) {
+  const uint32_t kb = k0 >> 6, kk = k0 & 63u;
+  *reinterpret_cast<uint4 *>(tile + kb * rows * 128u + tc::sw128_offset(r, kk)) = v;
+}
+// Element (r, k) of such an operand.
+__device__ __forceinline__ uint16_t ssd_get(const unsigned char *tile, uint32_t rows, uint32_t r, uint32_t k) {
+  return *reinterpret_cast<const uint16_t *>(tile + (k >> 6) * rows * 128u + tc::sw128_offset(r, k & 63u));
+}
+// 8 consecutive bf16 values of a row (16-byte load; element-wise past the sequence end, zeros there).
+__device__ __forceinline__ void ssd_load8(const __nv_bfloat16 *row, int64_t t, int64_t L, float (&f)[8]) {
+  if (t + 8 <= L) {
+    unpack16<__nv_bfloat16>(*reinterpret_cast<const uint4 *>(row), f);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = t + i < L ? __bfloat162float(row[i]) : 0.f;
+  }
+}
+
+__global__ void __launch_bounds__(kSsdThreads, 1) ssd_chunk_kernel(const SsdArgs args) {
   constexpr int T = kSsdT, P = kSsdP, N = kSsdN;
   extern __shared__ unsigned char ssd_smem_raw[];
   // operand tiles start on a 1024-byte boundary (the swizzle atom)
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(ssd_smem_raw) + 1023) & ~uintptr_t(1023));
   float *cum = reinterpret_cast<float *>(smem + kSsdOffCum);
+  float *dts = cum + T;   // Delta of the chunk's steps (0 past the end)
+  float *wdec = dts + T;  // exp(cum_T - cum_s): decay from step s to the chunk end
+  unsigned char *tmp = smem + kSsdOffM;  // C [n][t] before the transpose; y [p][t] after the products
   __shared__ __align__(8) uint64_t bar_g, bar_y;
   __shared__ uint32_t tmem_slot;
   __shared__ float warp_sum[4];
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int r = tid & 127, hf = tid >> 7;           // tile row of this thread and its half of the row
   const int64_t bh = blockIdx.x;                 // (sequence, head)
   const int64_t b = bh / args.nheads, h = bh % args.nheads;
   const int64_t L = args.seqlen;
@@ -106,16 +132,17 @@ __global__ void __launch_bounds__(128, 1) ssd_chunk_kernel(const SsdArgs args) {
   tc::fence_after_sync();
   const uint32_t tmem = tmem_slot;
   const uint32_t t_G = tmem, t_Y = tmem + 128, t_H = tmem + 192;      // column bases
-  const uint32_t lane_base = uint32_t(warp * 32) << 16;               // this warp's lanes
+  const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;         // this warp's lanes (= rows r)
 
-  // the state: tensor memory [n][p] (thread n owns lane n), float32; h0 or zero
+  // the state: tensor memory [n][p] (lane n), float32; h0 or zero.  Thread (r, hf): lane r,
+  // columns [32 hf, 32 hf + 32)
   {
     float v[16];
 #pragma unroll
-    for (int c = 0; c < P / 16; ++c) {
+    for (int c = 2 * hf; c < 2 * hf + 2; ++c) {
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        v[i] = args.h0 ? args.h0[(bh * P + c * 16 + i) * N + tid] : 0.f;
+        v[i] = args.h0 ? args.h0[(bh * P + c * 16 + i) * N + r] : 0.f;
       tc::tmem_st16(t_H + lane_base + c * 16, v);
     }
     tc::tmem_wait_st();
@@ -131,83 +158,91 @@ __global__ void __launch_bounds__(128, 1) ssd_chunk_kernel(const SsdArgs args) {
 
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = int64_t(c) * T;
-    const int64_t tt = t0 + tid;                // this thread's step (row t of G and Y)
+    const int64_t tt = t0 + r;                  // the step of row r (of G, M, Y, C^T, B^T)
     const bool t_ok = tt < L;
-    // ---- prefix sum of Delta A over the chunk (steps past the end add 0)
-    float v = t_ok ? dtg[tt] * Ah : 0.f;
+    // ---- Delta, the prefix sum of Delta A over the chunk (steps past the end add 0), decays
+    if (tid < T) {
+      const float dtv = t_ok ? dtg[tt] : 0.f;
+      dts[r] = dtv;
+      float v = dtv * Ah;
 #pragma unroll
-    for (int off = 1; off < 32; off *= 2) {
-      const float o = __shfl_up_sync(0xffffffffu, v, off);
-      if (lane >= off) v += o;
+      for (int off = 1; off < 32; off *= 2) {
+        const float o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+      }
+      if (lane == 31) warp_sum[warp] = v;
+      cum[r] = v;  // the warp's part; the other warps' sums are added below
     }
-    if (lane == 31) warp_sum[warp] = v;
     __syncthreads();
-    for (int w = 0; w < warp; ++w) v += warp_sum[w];
-    cum[tid] = v;
+    if (tid < T) {
+      float v = cum[r];
+      for (int w = 0; w < warp; ++w) v += warp_sum[w];
+      cum[r] = v;
+    }
     __syncthreads();
-    const float cum_t = v, cum_T = cum[T - 1];
+    const float cum_t = cum[r], cum_T = cum[T - 1];
+    if (tid < T) wdec[r] = __expf(cum_T - cum_t);
 
-    // ---- operand tiles (thread tid: row t of C^T and B^T, row n of B, row p of V / V')
+    // ---- B [n][s] and C [n][t] (row n = r, half hf of the chunk), 16-byte loads
     {
-      float cv[8], bv[8];
-#pragma unroll 1
-      for (int n0 = 0; n0 < N; n0 += 8) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          cv[i] = t_ok ? __bfloat162float(Cg[(n0 + i) * L + tt]) : 0.f;
-          bv[i] = t_ok ? __bfloat162float(Bg[(n0 + i) * L + tt]) : 0.f;
-        }
-        ssd_put8(smem + kSsdOffCT, 128, tid, n0, cv);
-        ssd_put8(smem + kSsdOffBT, 128, tid, n0, bv);
-      }
-      // B [n][s]: row n = tid, 16-byte loads along the sequence
-      const __nv_bfloat16 *brow = Bg + int64_t(tid) * L + t0;
-#pragma unroll 1
-      for (int s0 = 0; s0 < T; s0 += 8) {
+      const __nv_bfloat16 *brow = Bg + int64_t(r) * L + t0, *crow = Cg + int64_t(r) * L + t0;
+#pragma unroll 2
+      for (int s0 = hf * 64; s0 < hf * 64 + 64; s0 += 8) {
         float f[8];
-        if (t0 + s0 + 8 <= L) {
-          unpack16<__nv_bfloat16>(*reinterpret_cast<const uint4 *>(brow + s0), f);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = t0 + s0 + i < L ? __bfloat162float(brow[s0 + i]) : 0.f;
-        }
-        ssd_put8(smem + kSsdOffBN, 128, tid, s0, f);
+        ssd_load8(brow + s0, t0 + s0, L, f);
+        ssd_put8(smem + kSsdOffBN, 128, r, s0, f);
+        ssd_load8(crow + s0, t0 + s0, L, f);
+        ssd_put8(tmp, 128, r, s0, f);
       }
-      // V [p][s] = x[p][s] Delta_s and V' = V exp(cum_T - cum_s): two threads per row p
-      const int p = tid >> 1, half = tid & 1;
+    }
+    __syncthreads();  // wdec, B and C in place
+    // ---- V [p][s] = x[p][s] Delta_s and V' = V exp(cum_T - cum_s): four threads per row p
+    {
+      const int p = tid >> 2, q = tid & 3;
       const __nv_bfloat16 *xrow = xg + int64_t(p) * L + t0;
-#pragma unroll 1
-      for (int s0 = half * 64; s0 < half * 64 + 64; s0 += 8) {
-        float f[8], fv[8], fs[8];
-        if (t0 + s0 + 8 <= L) {
-          unpack16<__nv_bfloat16>(*reinterpret_cast<const uint4 *>(xrow + s0), f);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = t0 + s0 + i < L ? __bfloat162float(xrow[s0 + i]) : 0.f;
-        }
+#pragma unroll 2
+      for (int s0 = q * 32; s0 < q * 32 + 32; s0 += 8) {
+        float f[8], fs[8];
+        ssd_load8(xrow + s0, t0 + s0, L, f);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int64_t ts = t0 + s0 + i;
-          const float d = ts < L ? dtg[ts] : 0.f;
-          fv[i] = f[i] * d;
-          fs[i] = fv[i] * __expf(cum_T - cum[s0 + i]);
+          f[i] *= dts[s0 + i];
+          fs[i] = f[i] * wdec[s0 + i];
         }
-        ssd_put8(smem + kSsdOffV, 64, p, s0, fv);
+        ssd_put8(smem + kSsdOffV, 64, p, s0, f);
         ssd_put8(smem + kSsdOffVS, 64, p, s0, fs);
       }
-      // H [p][n] from the state (thread n reads its tensor-memory lane: the P values of row n)
+    }
+    // ---- H [p][n] from the state (lane n = r holds row n; this thread's 32 columns p)
+    {
       float hv[16];
 #pragma unroll
-      for (int cb = 0; cb < P / 16; ++cb) {
+      for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
         tc::tmem_ld16(t_H + lane_base + cb * 16, hv);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const uint32_t pp = cb * 16 + i, kb = uint32_t(tid) >> 6, kk = uint32_t(tid) & 63u;
+          const uint32_t pp = cb * 16 + i, kb = uint32_t(r) >> 6, kk = uint32_t(r) & 63u;
           *reinterpret_cast<__half *>(smem + kSsdOffH + kb * 64u * 128u + tc::sw128_offset(pp, kk)) =
               __float2half_rn(hv[i]);
         }
       }
+    }
+    // ---- C^T [t][n] and B^T [s][n] from the row-major copies (row t = r, states of half hf)
+#pragma unroll 2
+    for (int n0 = hf * 64; n0 < hf * 64 + 64; n0 += 8) {
+      uint16_t cv[8], bv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cv[i] = ssd_get(tmp, 128, n0 + i, r);
+        bv[i] = ssd_get(smem + kSsdOffBN, 128, n0 + i, r);
+      }
+      ssd_put8h(smem + kSsdOffCT, 128, r, n0,
+                make_uint4(cv[0] | (uint32_t(cv[1]) << 16), cv[2] | (uint32_t(cv[3]) << 16),
+                           cv[4] | (uint32_t(cv[5]) << 16), cv[6] | (uint32_t(cv[7]) << 16)));
+      ssd_put8h(smem + kSsdOffBT, 128, r, n0,
+                make_uint4(bv[0] | (uint32_t(bv[1]) << 16), bv[2] | (uint32_t(bv[3]) << 16),
+                           bv[4] | (uint32_t(bv[5]) << 16), bv[6] | (uint32_t(bv[7]) << 16)));
     }
     tc::fence_async_smem();
     tc::fence_before_sync();
@@ -230,7 +265,7 @@ __global__ void __launch_bounds__(128, 1) ssd_chunk_kernel(const SsdArgs args) {
     // ---- M[t][s] = G exp(cum_t - cum_s) (s <= t), C' = C exp(cum_t), state *= exp(cum_T)
     {
 #pragma unroll 1
-      for (int s0 = 0; s0 < T; s0 += 16) {
+      for (int s0 = hf * 64; s0 < hf * 64 + 64; s0 += 16) {
         float g[16];
         tc::tmem_ld16(t_G + lane_base + s0, g);
         tc::tmem_wait_ld();
@@ -238,25 +273,24 @@ __global__ void __launch_bounds__(128, 1) ssd_chunk_kernel(const SsdArgs args) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int s = s0 + i;
-          const float m = s <= tid ? g[i] * __expf(cum_t - cum[s]) : 0.f;
+          const float m = s <= r ? g[i] * __expf(cum_t - cum[s]) : 0.f;
           if (i < 8) m0[i] = m; else m1[i - 8] = m;
         }
-        ssd_put8(smem + kSsdOffM, 128, tid, s0, m0);
-        ssd_put8(smem + kSsdOffM, 128, tid, s0 + 8, m1);
+        ssd_put8(smem + kSsdOffM, 128, r, s0, m0);
+        ssd_put8(smem + kSsdOffM, 128, r, s0 + 8, m1);
       }
-      const float e_t = __expf(cum_t);
-#pragma unroll 1
-      for (int n0 = 0; n0 < N; n0 += 8) {
+      const __half2 e_t = __float2half2_rn(__expf(cum_t));
+#pragma unroll 2
+      for (int n0 = hf * 64; n0 < hf * 64 + 64; n0 += 8) {
         const uint32_t kb = uint32_t(n0) >> 6;
-        unsigned char *q = smem + kSsdOffCT + kb * 128u * 128u + tc::sw128_offset(tid, n0 & 63);
-        __half2 *hq = reinterpret_cast<__half2 *>(q);
+        __half2 *hq = reinterpret_cast<__half2 *>(smem + kSsdOffCT + kb * 128u * 128u + tc::sw128_offset(r, n0 & 63));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) hq[i] = __hmul2(hq[i], __float2half2_rn(e_t));
+        for (int i = 0; i < 4; ++i) hq[i] = __hmul2(hq[i], e_t);
       }
       const float e_T = __expf(cum_T);
       float hv[16];
 #pragma unroll
-      for (int cb = 0; cb < P / 16; ++cb) {
+      for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
         tc::tmem_ld16(t_H + lane_base + cb * 16, hv);
         tc::tmem_wait_ld();
 #pragma unroll
@@ -295,26 +329,42 @@ __global__ void __launch_bounds__(128, 1) ssd_chunk_kernel(const SsdArgs args) {
     mbar_wait_bounded(&bar_y, uint32_t(c & 1));
     tc::fence_after_sync();
 
-    // ---- y[p][t] for this thread's step; the final state
+    // ---- y: row t = r, columns p of half hf, through a [p][t] bf16 tile (the products are
+    // done with M), then 16-byte stores of whole row pieces
     {
+      __nv_bfloat16 *ys = reinterpret_cast<__nv_bfloat16 *>(tmp);
       float yv[16];
 #pragma unroll
-      for (int cb = 0; cb < P / 16; ++cb) {
+      for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
         tc::tmem_ld16(t_Y + lane_base + cb * 16, yv);
         tc::tmem_wait_ld();
-        if (t_ok) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) args.y[(bh * P + cb * 16 + i) * L + tt] = __float2bfloat16_rn(yv[i]);
-        }
+        for (int i = 0; i < 16; ++i) ys[(cb * 16 + i) * T + r] = __float2bfloat16_rn(yv[i]);
       }
       if (c == nchunks - 1 && args.h_last) {
         float hv[16];
 #pragma unroll
-        for (int cb = 0; cb < P / 16; ++cb) {
+        for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
           tc::tmem_ld16(t_H + lane_base + cb * 16, hv);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) args.h_last[(bh * P + cb * 16 + i) * N + tid] = hv[i];
+          for (int i = 0; i < 16; ++i) args.h_last[(bh * P + cb * 16 + i) * N + r] = hv[i];
+        }
+      }
+      __syncthreads();
+      const int p = tid >> 2, q = tid & 3;
+      __nv_bfloat16 *yrow = args.y + (bh * P + p) * L + t0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s0 = q * 32 + j * 8;
+        const uint4 v = *reinterpret_cast<const uint4 *>(ys + p * T + s0);
+        if (t0 + s0 + 8 <= L) {
+          *reinterpret_cast<uint4 *>(yrow + s0) = v;
+        } else {
+          const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (t0 + s0 + i < L) yrow[s0 + i] = e[i];
         }
       }
     }

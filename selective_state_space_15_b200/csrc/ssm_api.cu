@@ -129,7 +129,7 @@ constexpr int kSeqWarps = SSM_SEQ_WARPS;
 constexpr int kSeqMaxCtasPerSm = SSM_SEQ_MAX_CTAS;
 // AUTO: measured on B200, the chunked kernel is the faster of the two on every workload here
 // (packed bf16 batch of 16 x 2048: 0.50 vs 0.53 ms), so AUTO takes it; the sequential kernel
-// is chosen explicitly (and runs the checkpoint pass of the backward).
+// is chosen explicitly.
 constexpr int64_t kSeqMinPairs = int64_t(1) << 62;
 bool seq_supported(const ssm_scan_params *p, bool vec) {
   return vec && (p->dstate == 16 || p->dstate == 32) && p->discretization == SSM_DISC_EULER;
@@ -382,16 +382,23 @@ ssm_status_t noalloc_scratch(void **out) {
   return SSM_OK;
 }
 
-// Decode launches: the N = 16 kernel (one warp per 32 channels, coalesced quads), else G
-// states per thread.
+// Decode launches: the N = 16 kernel (pool slices streamed by bulk copies), else G states per
+// thread.
 template <typename T, typename TO, bool ZOH>
-void launch_update_disc(const ssm::UpdateArgs &a, int G, bool has_z, dim3 blocks, cudaStream_t st) {
+ssm_status_t launch_update_disc(const ssm::UpdateArgs &a, int G, bool has_z, dim3 blocks, cudaStream_t st) {
   using namespace ssm;
   if (a.dstate == 16) {
-    const dim3 b16(unsigned((a.dim + kUpdateThreads - 1) / kUpdateThreads), blocks.y);
-    if (has_z) state_update16_kernel<T, TO, true, ZOH><<<b16, kUpdateThreads, 0, st>>>(a);
-    else state_update16_kernel<T, TO, false, ZOH><<<b16, kUpdateThreads, 0, st>>>(a);
-    return;
+    // one block per (channel group, residue class of requests): as many request classes as
+    // keep every resident block slot busy
+    auto kern = has_z ? state_update16_bulk_kernel<T, TO, true, ZOH> : state_update16_bulk_kernel<T, TO, false, ZOH>;
+    LaunchInfo li;
+    if (launch_info(reinterpret_cast<const void *>(kern), kUpdateThreads, kUpdBulkSmem, li) != SSM_OK)
+      return SSM_ERR_CUDA;
+    const int64_t ngrp = (a.dim + kUpdBulkCh - 1) / kUpdBulkCh;
+    const int64_t slots = int64_t(li.num_sms) * li.blocks_per_sm;
+    const int64_t nrb = std::min<int64_t>(std::max<int64_t>(1, std::min<int64_t>(a.R, slots / ngrp)), 65535);
+    kern<<<dim3(unsigned(ngrp), unsigned(nrb)), kUpdateThreads, kUpdBulkSmem, st>>>(a);
+    return SSM_OK;
   }
   auto go = [&](auto g_tag) {
     constexpr int GG = decltype(g_tag)::value;
@@ -401,102 +408,91 @@ void launch_update_disc(const ssm::UpdateArgs &a, int G, bool has_z, dim3 blocks
   if (G == 16) go(std::integral_constant<int, 16>{});
   else if (G == 8) go(std::integral_constant<int, 8>{});
   else go(std::integral_constant<int, 4>{});
+  return SSM_OK;
 }
 template <typename T, typename TO>
-void launch_update(const ssm::UpdateArgs &a, int G, bool has_z, bool zoh, dim3 blocks, cudaStream_t st) {
-  if (zoh) launch_update_disc<T, TO, true>(a, G, has_z, blocks, st);
-  else launch_update_disc<T, TO, false>(a, G, has_z, blocks, st);
+ssm_status_t launch_update(const ssm::UpdateArgs &a, int G, bool has_z, bool zoh, dim3 blocks, cudaStream_t st) {
+  return zoh ? launch_update_disc<T, TO, true>(a, G, has_z, blocks, st)
+             : launch_update_disc<T, TO, false>(a, G, has_z, blocks, st);
 }
 
 // ---- backward (ssm_scan_bwd) ----
-// Workspace: two unit tickets (16 bytes each), the checkpoints [batch][ceil(L/8)][dim][N] and
-// the per-tile partial sums of dB and dC [tiles][batch][2][N][L], all float32.
-constexpr int kBwdTC16 = 32;  // chunk of the backward kernel for 16-bit inputs (64-byte rows)
+// Units are (sequence, time segment, tile of 32 channels), segments whole chunks, at least
+// kBwdMinSegChunks chunks long and otherwise as long as still gives kBwdUnitsWanted units.
+// Workspace (float32 unless noted): two unit tickets (16 bytes each), the block checkpoints
+// [batch][nblk][dim][N], the per-block Delta sums [batch][nblk][dim], the per-segment Delta
+// sums [batch][nseg][dim] and the two per-segment state arrays [batch][nseg][dim][N].
+constexpr int kBwdTC16 = 32;  // chunk of the backward kernels for 16-bit inputs (64-byte rows)
+constexpr int kBwdWarps = 4;  // warps per CTA (8 channels each)
+constexpr int64_t kBwdUnitsWanted = 8 * 148;
+constexpr int64_t kBwdMinSegChunks = 4;
 struct BwdPlan {
-  int64_t nblk = 0, ntiles = 0, nunits = 0;
-  int warps = 4;  // warps per CTA (8 channels each)
-  size_t off_ckpt = 0, off_part = 0, bytes = 0;
+  int64_t nblk = 0, ntiles = 0, nseg = 0, seg_len = 0, nunits = 0;
+  size_t off_ckpt = 0, off_cumd = 0, off_ssum = 0, off_sh = 0, off_sg = 0, bytes = 0;
 };
-// Units are (sequence, tile of 8 W channels) walked serially from the end: W = 4 when that
-// still gives four units per SM, else 2, else 1 (more, narrower units for few channels).
-constexpr int64_t kBwdUnitsWanted = 4 * 148;
 bool make_bwd_plan(const ssm_scan_params *p, bool vec, BwdPlan &bp) {
   if (!vec || p->dstate != 16 || groups_of(p) != 1 || p->discretization != SSM_DISC_EULER) return false;
-  const int64_t pairs = p->batch * p->dim;
-  bp.warps = pairs >= 32 * kBwdUnitsWanted ? 4 : (pairs >= 16 * kBwdUnitsWanted ? 2 : 1);
-  const int64_t CT = 8 * bp.warps;
-  bp.nblk = (p->seqlen + 7) / 8;
+  const int64_t TC = p->dtype == SSM_F32 ? 16 : kBwdTC16;
+  const int64_t CT = 8 * kBwdWarps, L = p->seqlen, N = p->dstate;
+  bp.nblk = (L + 7) / 8;
   bp.ntiles = (p->dim + CT - 1) / CT;
-  bp.nunits = p->batch * bp.ntiles;
-  bp.off_ckpt = 32;
-  const size_t ckpt = size_t(p->batch) * bp.nblk * p->dim * p->dstate * sizeof(float);
-  bp.off_part = (bp.off_ckpt + ckpt + 255) / 256 * 256;
-  bp.bytes = bp.off_part + size_t(bp.ntiles) * p->batch * 2 * p->dstate * p->seqlen * sizeof(float);
+  const int64_t chunks = std::max<int64_t>(1, (L + TC - 1) / TC);
+  const int64_t rows = std::max<int64_t>(1, p->batch * bp.ntiles);
+  const int64_t want_seg = (kBwdUnitsWanted + rows - 1) / rows;  // segments per sequence wanted
+  const int64_t seg_chunks = std::max<int64_t>(kBwdMinSegChunks, chunks / std::max<int64_t>(1, want_seg));
+  bp.seg_len = seg_chunks * TC;
+  bp.nseg = std::max<int64_t>(1, (L + bp.seg_len - 1) / bp.seg_len);
+  bp.nunits = p->batch * bp.nseg * bp.ntiles;
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t f = sizeof(float), B = size_t(p->batch), D = size_t(p->dim);
+  bp.off_ckpt = 256;
+  bp.off_cumd = al(bp.off_ckpt + B * bp.nblk * D * N * f);
+  bp.off_ssum = al(bp.off_cumd + B * bp.nblk * D * f);
+  bp.off_sh = al(bp.off_ssum + B * bp.nseg * D * f);
+  bp.off_sg = al(bp.off_sh + B * bp.nseg * D * N * f);
+  bp.bytes = bp.off_sg + B * bp.nseg * D * N * f;
   return true;
 }
 
 template <typename T, typename TG, bool HAS_Z>
 ssm_status_t launch_bwd(ScanArgs a, const ssm::BwdArgs &bwa, const BwdPlan &bp, const ssm_scan_params *p,
-                        float *dB, float *dC, unsigned char *ws, cudaStream_t st) {
-  constexpr int N = 16;
-  // 1. checkpoints: the lane-sequential forward in checkpoint mode
+                        unsigned char *ws, cudaStream_t st) {
+  constexpr int N = 16, W = kBwdWarps;
+  constexpr int TC = sizeof(T) == 2 ? kBwdTC16 : 16;
+  using Cfg = ssm::BwdCfg<T, TG, N, TC, W>;
+  a.ntiles = int(bp.ntiles);
+  a.nseq = int(p->batch);
+  a.total_units = int(bp.nunits);
+  // 1. the segment pass
   {
-    constexpr int LPC = seq_lpc(N);
-    constexpr int TC = sizeof(T) == 2 ? 32 : 16;
-    using Cfg = ssm::SeqCfg<T, N, LPC, TC, kSeqWarps>;
-    auto kern = ssm::seq_scan_kernel<T, T, N, LPC, TC, kSeqWarps, false, true>;
+    auto kern = ssm::bwd_seg_kernel<T, TG, N, TC, W, HAS_Z>;
+    LaunchInfo li;
+    if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSegSmemBytes, li) != SSM_OK)
+      return SSM_ERR_CUDA;
+    ScanArgs f = a;
+    f.ticket = reinterpret_cast<uint32_t *>(ws);
+    const int64_t blocks = std::min<int64_t>(bp.nunits, int64_t(li.num_sms) * li.blocks_per_sm);
+    kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSegSmemBytes, st>>>(f, bwa);
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+  }
+  // 2. the segment scan
+  {
+    const int64_t n = p->batch * p->dim * N;
+    ssm::bwd_seg_scan_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(
+        p->A, p->h0, bwa.dh_last, bwa.seg_sum, bwa.seg_h, bwa.seg_g, p->batch, p->dim, N, int(bp.nseg));
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+  }
+  // 3. the walk
+  {
+    auto kern = ssm::seq_bwd_kernel<T, TG, N, TC, W, HAS_Z>;
     LaunchInfo li;
     if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
       return SSM_ERR_CUDA;
-    const int64_t ct = Cfg::kCT;
-    ScanArgs f = a;
-    f.ntiles = int((p->dim + ct - 1) / ct);
-    f.tiles_per_group = f.ntiles;
-    f.group_dim = p->dim;
-    f.nseq = int(p->batch);
-    f.total_units = int(p->batch * f.ntiles);
-    f.ticket = reinterpret_cast<uint32_t *>(ws);
-    f.ckpt = reinterpret_cast<float *>(ws + bp.off_ckpt);
-    f.ckpt_blocks = bp.nblk;
-    f.y = nullptr;
-    f.h_last = nullptr;
-    const int64_t blocks = std::min<int64_t>(f.total_units, int64_t(li.num_sms) * li.blocks_per_sm);
-    kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, st>>>(f);
-    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
-  }
-  // 2. the backward walk
-  {
     ScanArgs b = a;
-    b.ntiles = int(bp.ntiles);
-    b.nseq = int(p->batch);
-    b.total_units = int(bp.nunits);
     b.ticket = reinterpret_cast<uint32_t *>(ws + 16);
-    auto walk = [&](auto w_tag) -> ssm_status_t {
-      constexpr int W = decltype(w_tag)::value;
-      constexpr int TC = sizeof(T) == 2 ? kBwdTC16 : 16;
-      using Cfg = ssm::BwdCfg<T, TG, N, TC, W>;
-      auto kern = ssm::seq_bwd_kernel<T, TG, N, TC, W, HAS_Z>;
-      LaunchInfo li;
-      if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
-        return SSM_ERR_CUDA;
-      const int64_t blocks = std::min<int64_t>(bp.nunits, int64_t(li.num_sms) * li.blocks_per_sm);
-      kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, st>>>(b, bwa);
-      return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
-    };
-    const ssm_status_t ws_st = bp.warps == 4 ? walk(std::integral_constant<int, 4>{})
-                             : bp.warps == 2 ? walk(std::integral_constant<int, 2>{})
-                                             : walk(std::integral_constant<int, 1>{});
-    if (ws_st != SSM_OK) return ws_st;
-  }
-  // 3. dB, dC from the tiles' partial sums
-  {
-    const int64_t per_tile = p->batch * 2 * N * p->seqlen;
-    const int64_t blocks = std::min<int64_t>((per_tile + 255) / 256, 148 * 16);
-    if (blocks > 0) {
-      ssm::bwd_reduce_tiles_kernel<<<unsigned(blocks), 256, 0, st>>>(bwa.partials, dB, dC, bp.ntiles, per_tile, N,
-                                                                     p->seqlen);
-      if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
-    }
+    const int64_t blocks = std::min<int64_t>(bp.nunits, int64_t(li.num_sms) * li.blocks_per_sm);
+    kern<<<unsigned(blocks), Cfg::kThreads, Cfg::kSmemBytes, st>>>(b, bwa);
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
   }
   return SSM_OK;
 }
@@ -617,9 +613,11 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool has_z = p->z != nullptr, zoh = p->discretization == SSM_DISC_ZOH;
   using bf16 = __nv_bfloat16;
-  if (p->dtype == SSM_BF16 && !p->y_fp32) launch_update<bf16, bf16>(a, G, has_z, zoh, blocks, st);
-  else if (p->dtype == SSM_BF16) launch_update<bf16, float>(a, G, has_z, zoh, blocks, st);
-  else launch_update<float, float>(a, G, has_z, zoh, blocks, st);
+  ssm_status_t ls;
+  if (p->dtype == SSM_BF16 && !p->y_fp32) ls = launch_update<bf16, bf16>(a, G, has_z, zoh, blocks, st);
+  else if (p->dtype == SSM_BF16) ls = launch_update<bf16, float>(a, G, has_z, zoh, blocks, st);
+  else ls = launch_update<float, float>(a, G, has_z, zoh, blocks, st);
+  if (ls != SSM_OK) return ls;
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -654,25 +652,32 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params *p, const ssm_scan_grads *g, voi
     }
     return SSM_OK;
   }
+  const size_t nbc = size_t(p->batch) * p->dstate * p->seqlen * sizeof(float);
+  if (cudaMemsetAsync(g->dB, 0, nbc, cs) != cudaSuccess || cudaMemsetAsync(g->dC, 0, nbc, cs) != cudaSuccess)
+    return SSM_ERR_CUDA;
   ssm::BwdArgs bwa{};
   bwa.dy = g->dy; bwa.dh_last = g->dh_last;
   bwa.du = g->du; bwa.ddelta = g->ddelta; bwa.dz = g->dz;
   bwa.dA = g->dA; bwa.dDskip = p->Dskip ? g->dDskip : nullptr; bwa.dbias = p->delta_bias ? g->ddelta_bias : nullptr;
   bwa.dh0 = g->dh0;
-  bwa.ckpt = reinterpret_cast<const float *>(ws + bp.off_ckpt);
-  bwa.partials = reinterpret_cast<float *>(ws + bp.off_part);
-  bwa.ckpt_blocks = bp.nblk;
+  bwa.dB = g->dB; bwa.dC = g->dC;
+  bwa.ckpt = reinterpret_cast<float *>(ws + bp.off_ckpt);
+  bwa.cumd = reinterpret_cast<float *>(ws + bp.off_cumd);
+  bwa.seg_sum = reinterpret_cast<float *>(ws + bp.off_ssum);
+  bwa.seg_h = reinterpret_cast<float *>(ws + bp.off_sh);
+  bwa.seg_g = reinterpret_cast<float *>(ws + bp.off_sg);
+  bwa.nblk = bp.nblk;
+  bwa.seg_len = bp.seg_len;
+  bwa.nseg = int(bp.nseg);
+  bwa.vec_dbc = (aligned16(g->dB) && aligned16(g->dC) && p->seqlen % 4 == 0) ? 1 : 0;
   a.cu_seqlens = nullptr;
   using bf16 = __nv_bfloat16;
   const bool has_z = p->z != nullptr;
   if (p->dtype == SSM_BF16 && !p->y_fp32)
-    return has_z ? launch_bwd<bf16, bf16, true>(a, bwa, bp, p, g->dB, g->dC, ws, cs)
-                 : launch_bwd<bf16, bf16, false>(a, bwa, bp, p, g->dB, g->dC, ws, cs);
+    return has_z ? launch_bwd<bf16, bf16, true>(a, bwa, bp, p, ws, cs) : launch_bwd<bf16, bf16, false>(a, bwa, bp, p, ws, cs);
   if (p->dtype == SSM_BF16)
-    return has_z ? launch_bwd<bf16, float, true>(a, bwa, bp, p, g->dB, g->dC, ws, cs)
-                 : launch_bwd<bf16, float, false>(a, bwa, bp, p, g->dB, g->dC, ws, cs);
-  return has_z ? launch_bwd<float, float, true>(a, bwa, bp, p, g->dB, g->dC, ws, cs)
-               : launch_bwd<float, float, false>(a, bwa, bp, p, g->dB, g->dC, ws, cs);
+    return has_z ? launch_bwd<bf16, float, true>(a, bwa, bp, p, ws, cs) : launch_bwd<bf16, float, false>(a, bwa, bp, p, ws, cs);
+  return has_z ? launch_bwd<float, float, true>(a, bwa, bp, p, ws, cs) : launch_bwd<float, float, false>(a, bwa, bp, p, ws, cs);
 }
 
 ssm_status_t ssm_ssd_fwd(const ssm_ssd_params *p, ssm_stream_t stream) {
@@ -692,7 +697,7 @@ ssm_status_t ssm_ssd_fwd(const ssm_ssd_params *p, ssm_stream_t stream) {
     return SSM_OK;
   }
   LaunchInfo li;
-  if (launch_info(reinterpret_cast<const void *>(ssm::ssd_chunk_kernel), 128, ssm::kSsdSmemBytes, li) != SSM_OK)
+  if (launch_info(reinterpret_cast<const void *>(ssm::ssd_chunk_kernel), ssm::kSsdThreads, ssm::kSsdSmemBytes, li) != SSM_OK)
     return SSM_ERR_CUDA;
   ssm::SsdArgs a{};
   a.x = static_cast<const __nv_bfloat16 *>(p->x);
@@ -705,7 +710,7 @@ ssm_status_t ssm_ssd_fwd(const ssm_ssd_params *p, ssm_stream_t stream) {
   a.h_last = p->h_last;
   a.nheads = p->nheads;
   a.seqlen = p->seqlen;
-  ssm::ssd_chunk_kernel<<<unsigned(p->batch * p->nheads), 128, ssm::kSsdSmemBytes,
+  ssm::ssd_chunk_kernel<<<unsigned(p->batch * p->nheads), ssm::kSsdThreads, ssm::kSsdSmemBytes,
                           reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }

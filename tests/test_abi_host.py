@@ -182,12 +182,16 @@ def test_backward_host_checks(lib):
     assert f(ctypes.byref(_params(dim=64, ngroups=2)), ctypes.byref(g), None, 0, None) == 2
     assert f(ctypes.byref(_params(x_dim_stride=130, seqlen=128)), ctypes.byref(g), None, 0, None) == 2
     assert f(ctypes.byref(p), ctypes.byref(g), None, 0, None) == 6                  # SSM_ERR_WORKSPACE
-    # workspace: checkpoints every 8 steps and per-tile partial rows of dB and dC (64 channels of
-    # one sequence: 8-channel tiles, one warp each)
+    # workspace: the block checkpoints and block Delta sums (every 8 steps), and per segment its
+    # Delta sum and two state arrays; 128 steps of one sequence make a single segment
     need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(p))
-    ckpt = 1 * (128 // 8) * 64 * 16 * 4
-    part = 8 * 1 * 2 * 16 * 128 * 4
-    assert ckpt + part <= need <= ckpt + part + 512
+    ckpt, cumd = 1 * (128 // 8) * 64 * 16 * 4, 1 * (128 // 8) * 64 * 4
+    seg = 1 * 1 * 64 * 4 + 2 * (1 * 1 * 64 * 16 * 4)
+    assert ckpt + cumd + seg <= need <= ckpt + cumd + seg + 5 * 256
+    # a long sequence is cut into segments: the per-segment arrays grow with their number
+    long_need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(_params(seqlen=1 << 16)))
+    long_blocks = (1 << 16) // 8 * 64 * (16 + 1) * 4
+    assert long_need > long_blocks + seg
     assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(_params(dstate=32))) == 0
 
 

@@ -100,3 +100,36 @@ def test_bad_slot_is_skipped_and_reported():
     assert torch.all(y[1:] == 123.0)                                        # skipped rows untouched
     changed = (pool_t != before).any(dim=(1, 2)).cpu().numpy()
     assert changed.tolist() == [False, False, True, False, False, False, False, False]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_decode_many_requests_per_block_with_bad_slots(dtype):
+    """More requests than resident blocks per channel group (every block walks several
+    requests through its staging ring), a ragged last channel group (300 = 256 + 44) and bad
+    slot ids spread over the requests: good rows match the oracle, bad rows are skipped."""
+    prob = workloads.decode_problem(num_slots=800, dim=300, dstate=16, R=700, dtype=dtype, seed=9)
+    slots = prob.slot_ids.copy()
+    bad = np.arange(5, 700, 97)
+    slots[bad] = np.where(bad % 2 == 0, -1, 800 + bad)
+    pool_t = torch.from_numpy(prob.pool0).cuda()
+    slots_t = torch.from_numpy(slots).cuda()
+    A, D, bias = (torch.from_numpy(x).cuda() for x in (prob.A, prob.Dskip, prob.bias))
+    good = np.setdiff1d(np.arange(700), bad)
+    pool = prob.pool0.astype(np.float64)
+    pool_mag = np.abs(pool)
+    ssm.device_status()
+    for step in range(3):
+        x = workloads.decode_step_inputs(prob, step)
+        u, dl, z = (dev(x[k], dtype) for k in ("u", "delta", "z"))
+        B, C = dev(x["B"], dtype), dev(x["C"], dtype)
+        y = torch.full(u.shape, 7.0, device="cuda", dtype=u.dtype)
+        ssm.state_update(pool_t, slots_t, u, dl, B, C, A, D, bias, z, y=y)
+        assert ssm.device_status() == 4                                     # SSM_ERR_BAD_SLOT
+        ref = oracle.state_update(pool, slots[good], x["u"][good], x["delta"][good], x["B"][good], x["C"][good],
+                                  prob.A, prob.Dskip, prob.bias, x["z"][good], pool_mag=pool_mag)
+        check(f"y step {step}", host(y)[good], ref["y"], ref["y_mag"], TOL[dtype], dtype)
+        assert torch.all(y[torch.from_numpy(bad).cuda()] == 7.0)
+    got = host(pool_t)
+    check("pool", got[slots[good]], pool[slots[good]], pool_mag[slots[good]], TOL[dtype])
+    others = np.setdiff1d(np.arange(800), slots[good])
+    assert np.array_equal(pool_t.cpu().numpy()[others], prob.pool0[others])
