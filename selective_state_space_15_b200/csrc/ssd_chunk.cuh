@@ -74,23 +74,21 @@ __device__ __forceinline__ void ssd_put8(unsigned char *tile, uint32_t rows, uin
   *reinterpret_cast<uint4 *>(tile + kb * rows * 128u + tc::sw128_offset(r, kk)) = *reinterpret_cast<uint4 *>(h);
 }
 
-// The same for 8 float16 values already converted.
-__device__ __forceinline__ void ssd_put8h(unsigned char *tile, uint32_t rows, uint32_t r, uint32_t k0, uint4 v) {
-  const uint32_t kb = k0 >> 6, kk = k0 & 63u;
-  *reinterpret_cast<uint4 *>(tile + kb * rows * 128u + tc::sw128_offset(r, kk)) = v;
-}
-// Element (r, k) of such an operand.
-__device__ __forceinline__ uint16_t ssd_get(const unsigned char *tile, uint32_t rows, uint32_t r, uint32_t k) {
-  return *reinterpret_cast<const uint16_t *>(tile + (k >> 6) * rows * 128u + tc::sw128_offset(r, k & 63u));
-}
-// 8 consecutive bf16 values of a row (16-byte load; element-wise past the sequence end, zeros there).
-__device__ __forceinline__ void ssd_load8(const __nv_bfloat16 *row, int64_t t, int64_t L, float (&f)[8]) {
-  if (t + 8 <= L) {
-    unpack16<__nv_bfloat16>(*reinterpret_cast<const uint4 *>(row), f);
-  } else {
+// 8 float32 values as float16 at byte `off` of a tile (a 16-byte chunk of a swizzled row).
+__device__ __forceinline__ void ssd_st8(unsigned char *p, const float (&v)[8]) {
+  __half2 h[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = t + i < L ? __bfloat162float(row[i]) : 0.f;
-  }
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4 *>(p) = *reinterpret_cast<uint4 *>(h);
+}
+// 8 consecutive bf16 values of a row as they are stored (zeros past the sequence end).
+__device__ __forceinline__ uint4 ssd_raw8(const __nv_bfloat16 *row, int64_t t, int64_t L) {
+  if (t + 8 <= L) return *reinterpret_cast<const uint4 *>(row);
+  uint16_t e[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) e[i] = t + i < L ? reinterpret_cast<const uint16_t *>(row)[i] : uint16_t(0);
+  return make_uint4(e[0] | (uint32_t(e[1]) << 16), e[2] | (uint32_t(e[3]) << 16), e[4] | (uint32_t(e[5]) << 16),
+                    e[6] | (uint32_t(e[7]) << 16));
 }
 
 __global__ void __launch_bounds__(kSsdThreads, 1) ssd_chunk_kernel(const SsdArgs args) {
@@ -133,6 +131,16 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_chunk_kernel(const SsdArgs
   const uint32_t tmem = tmem_slot;
   const uint32_t t_G = tmem, t_Y = tmem + 128, t_H = tmem + 192;      // column bases
   const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;         // this warp's lanes (= rows r)
+  // Swizzled byte offsets (tc::sw128_offset) this thread uses every chunk: ro[j] = 16-byte chunk
+  // j of row r (rows r of B, C, C^T, B^T, M); element (n, r) of a [n][K] tile with n = 8m + i
+  // (column r read down the rows: the transposes, the H tile) lies at n * 128 + co[i].
+  uint32_t ro[8], co[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ro[j] = tc::sw128_offset(uint32_t(r), uint32_t(8 * j));
+    co[j] = tc::sw128_offset(uint32_t(j), uint32_t(r) & 63u) - uint32_t(j) * 128u;
+  }
+  const uint32_t rcol = (uint32_t(r) >> 6) * 128u * 128u;  // the 64-column tile of column r (128-row tiles)
 
   // the state: tensor memory [n][p] (lane n), float32; h0 or zero.  Thread (r, hf): lane r,
   // columns [32 hf, 32 hf + 32)
@@ -156,13 +164,33 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_chunk_kernel(const SsdArgs
   const uint32_t a_H = tc::smem_addr(smem + kSsdOffH);
   const int nchunks = int((L + T - 1) / T);
 
+  // The raw inputs of a chunk, in registers: B and C rows n = r (half hf of the chunk's steps),
+  // x row p = tid / 4 (a quarter), Delta of step r.  Loaded one chunk ahead, so that the global
+  // loads of chunk c + 1 are in flight while chunk c is computed.
+  uint4 rb[8], rc[8], rx[4];
+  float rdt = 0.f;
+  auto load_raw = [&](int cc) {
+    const int64_t t0 = int64_t(cc) * T;
+    const __nv_bfloat16 *brow = Bg + int64_t(r) * L + t0, *crow = Cg + int64_t(r) * L + t0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int s0 = hf * 64 + j * 8;
+      rb[j] = ssd_raw8(brow + s0, t0 + s0, L);
+      rc[j] = ssd_raw8(crow + s0, t0 + s0, L);
+    }
+    const int p = tid >> 2, q = tid & 3;
+    const __nv_bfloat16 *xrow = xg + int64_t(p) * L + t0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) rx[j] = ssd_raw8(xrow + q * 32 + j * 8, t0 + q * 32 + j * 8, L);
+    if (tid < T) rdt = t0 + r < L ? dtg[t0 + r] : 0.f;
+  };
+  load_raw(0);
+
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = int64_t(c) * T;
-    const int64_t tt = t0 + r;                  // the step of row r (of G, M, Y, C^T, B^T)
-    const bool t_ok = tt < L;
     // ---- Delta, the prefix sum of Delta A over the chunk (steps past the end add 0), decays
     if (tid < T) {
-      const float dtv = t_ok ? dtg[tt] : 0.f;
+      const float dtv = rdt;
       dts[r] = dtv;
       float v = dtv * Ah;
 #pragma unroll
@@ -183,36 +211,38 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_chunk_kernel(const SsdArgs
     const float cum_t = cum[r], cum_T = cum[T - 1];
     if (tid < T) wdec[r] = __expf(cum_T - cum_t);
 
-    // ---- B [n][s] and C [n][t] (row n = r, half hf of the chunk), 16-byte loads
-    {
-      const __nv_bfloat16 *brow = Bg + int64_t(r) * L + t0, *crow = Cg + int64_t(r) * L + t0;
-#pragma unroll 2
-      for (int s0 = hf * 64; s0 < hf * 64 + 64; s0 += 8) {
-        float f[8];
-        ssd_load8(brow + s0, t0 + s0, L, f);
-        ssd_put8(smem + kSsdOffBN, 128, r, s0, f);
-        ssd_load8(crow + s0, t0 + s0, L, f);
-        ssd_put8(tmp, 128, r, s0, f);
-      }
+    // ---- B [n][s] and C [n][t] (row n = r, half hf of the chunk) from the registers
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float f[8];
+      unpack16<__nv_bfloat16>(rb[j], f);
+      ssd_st8(smem + kSsdOffBN + hf * 128 * 128 + ro[j], f);
+      unpack16<__nv_bfloat16>(rc[j], f);
+      ssd_st8(tmp + hf * 128 * 128 + ro[j], f);
     }
     __syncthreads();  // wdec, B and C in place
     // ---- V [p][s] = x[p][s] Delta_s and V' = V exp(cum_T - cum_s): four threads per row p
     {
       const int p = tid >> 2, q = tid & 3;
-      const __nv_bfloat16 *xrow = xg + int64_t(p) * L + t0;
-#pragma unroll 2
-      for (int s0 = q * 32; s0 < q * 32 + 32; s0 += 8) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s0 = q * 32 + j * 8;
         float f[8], fs[8];
-        ssd_load8(xrow + s0, t0 + s0, L, f);
+        unpack16<__nv_bfloat16>(rx[j], f);
+        const float4 d0 = *reinterpret_cast<const float4 *>(dts + s0), d1 = *reinterpret_cast<const float4 *>(dts + s0 + 4);
+        const float4 w0 = *reinterpret_cast<const float4 *>(wdec + s0), w1 = *reinterpret_cast<const float4 *>(wdec + s0 + 4);
+        const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+        const float ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          f[i] *= dts[s0 + i];
-          fs[i] = f[i] * wdec[s0 + i];
+          f[i] *= dd[i];
+          fs[i] = f[i] * ww[i];
         }
         ssd_put8(smem + kSsdOffV, 64, p, s0, f);
         ssd_put8(smem + kSsdOffVS, 64, p, s0, fs);
       }
     }
+    if (c + 1 < nchunks) load_raw(c + 1);  // lands while this chunk is computed
     // ---- H [p][n] from the state (lane n = r holds row n; this thread's 32 columns p)
     {
       float hv[16];
@@ -220,29 +250,28 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_chunk_kernel(const SsdArgs
       for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
         tc::tmem_ld16(t_H + lane_base + cb * 16, hv);
         tc::tmem_wait_ld();
+        unsigned char *hcol = smem + kSsdOffH + (uint32_t(r) >> 6) * 64u * 128u + cb * 16 * 128;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint32_t pp = cb * 16 + i, kb = uint32_t(r) >> 6, kk = uint32_t(r) & 63u;
-          *reinterpret_cast<__half *>(smem + kSsdOffH + kb * 64u * 128u + tc::sw128_offset(pp, kk)) =
-              __float2half_rn(hv[i]);
-        }
+        for (int i = 0; i < 16; ++i) *reinterpret_cast<__half *>(hcol + i * 128 + co[i & 7]) = __float2half_rn(hv[i]);
       }
     }
     // ---- C^T [t][n] and B^T [s][n] from the row-major copies (row t = r, states of half hf)
-#pragma unroll 2
-    for (int n0 = hf * 64; n0 < hf * 64 + 64; n0 += 8) {
-      uint16_t cv[8], bv[8];
+    {
+      const unsigned char *ccol = tmp + rcol + hf * 64 * 128, *bcol = smem + kSsdOffBN + rcol + hf * 64 * 128;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        cv[i] = ssd_get(tmp, 128, n0 + i, r);
-        bv[i] = ssd_get(smem + kSsdOffBN, 128, n0 + i, r);
+      for (int m = 0; m < 8; ++m) {
+        uint32_t cw[4], bw[4];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          const uint32_t o0 = (8 * m + i) * 128 + co[i], o1 = (8 * m + i + 1) * 128 + co[i + 1];
+          cw[i / 2] = *reinterpret_cast<const uint16_t *>(ccol + o0) |
+                      (uint32_t(*reinterpret_cast<const uint16_t *>(ccol + o1)) << 16);
+          bw[i / 2] = *reinterpret_cast<const uint16_t *>(bcol + o0) |
+                      (uint32_t(*reinterpret_cast<const uint16_t *>(bcol + o1)) << 16);
+        }
+        *reinterpret_cast<uint4 *>(smem + kSsdOffCT + hf * 128 * 128 + ro[m]) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint4 *>(smem + kSsdOffBT + hf * 128 * 128 + ro[m]) = make_uint4(bw[0], bw[1], bw[2], bw[3]);
       }
-      ssd_put8h(smem + kSsdOffCT, 128, r, n0,
-                make_uint4(cv[0] | (uint32_t(cv[1]) << 16), cv[2] | (uint32_t(cv[3]) << 16),
-                           cv[4] | (uint32_t(cv[5]) << 16), cv[6] | (uint32_t(cv[7]) << 16)));
-      ssd_put8h(smem + kSsdOffBT, 128, r, n0,
-                make_uint4(bv[0] | (uint32_t(bv[1]) << 16), bv[2] | (uint32_t(bv[3]) << 16),
-                           bv[4] | (uint32_t(bv[5]) << 16), bv[6] | (uint32_t(bv[7]) << 16)));
     }
     tc::fence_async_smem();
     tc::fence_before_sync();
@@ -264,26 +293,36 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_chunk_kernel(const SsdArgs
 
     // ---- M[t][s] = G exp(cum_t - cum_s) (s <= t), C' = C exp(cum_t), state *= exp(cum_T)
     {
-#pragma unroll 1
-      for (int s0 = hf * 64; s0 < hf * 64 + 64; s0 += 16) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int s0 = hf * 64 + 16 * m;
         float g[16];
         tc::tmem_ld16(t_G + lane_base + s0, g);
         tc::tmem_wait_ld();
         float m0[8], m1[8];
+        if (s0 > r) {  // the block lies above the diagonal (s > t)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int s = s0 + i;
-          const float m = s <= r ? g[i] * __expf(cum_t - cum[s]) : 0.f;
-          if (i < 8) m0[i] = m; else m1[i - 8] = m;
+          for (int i = 0; i < 8; ++i) m0[i] = m1[i] = 0.f;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 c4 = *reinterpret_cast<const float4 *>(cum + s0 + 4 * q);
+            const float cs[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 4 * q + e;
+              const float v = s0 + i <= r ? g[i] * __expf(cum_t - cs[e]) : 0.f;
+              if (i < 8) m0[i] = v; else m1[i - 8] = v;
+            }
+          }
         }
-        ssd_put8(smem + kSsdOffM, 128, r, s0, m0);
-        ssd_put8(smem + kSsdOffM, 128, r, s0 + 8, m1);
+        ssd_st8(smem + kSsdOffM + hf * 128 * 128 + ro[2 * m], m0);
+        ssd_st8(smem + kSsdOffM + hf * 128 * 128 + ro[2 * m + 1], m1);
       }
       const __half2 e_t = __float2half2_rn(__expf(cum_t));
-#pragma unroll 2
-      for (int n0 = hf * 64; n0 < hf * 64 + 64; n0 += 8) {
-        const uint32_t kb = uint32_t(n0) >> 6;
-        __half2 *hq = reinterpret_cast<__half2 *>(smem + kSsdOffCT + kb * 128u * 128u + tc::sw128_offset(r, n0 & 63));
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        __half2 *hq = reinterpret_cast<__half2 *>(smem + kSsdOffCT + hf * 128 * 128 + ro[m]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) hq[i] = __hmul2(hq[i], e_t);
       }
