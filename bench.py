@@ -439,8 +439,11 @@ def bwd_run(name, steps, warmup, sfu_peak):
     u, dl, z, B, C, dy = mk(b, D, L), mk(b, D, L), mk(b, D, L), mk(b, N, L), mk(b, N, L), mk(b, D, L)
     A, Dsk, bias = (torch.from_numpy(x).cuda() for x in workloads.channel_params(np.random.default_rng(c["seed"]), D, N))
     ms = time_kernel(lambda: ssm.scan_bwd(u, dl, B, C, A, dy, Dsk, bias, z, stream=stream), steps, warmup, stream)
+    ms_zoh = time_kernel(lambda: ssm.scan_bwd(u, dl, B, C, A, dy, Dsk, bias, z, stream=stream, zoh=True), steps,
+                         warmup, stream)
     exps = 2 * b * L * D * (N + 2)
-    return {"ms": round(ms, 4), "tokens_per_s": b * L / (ms * 1e-3), "sfu_frac": round(exps / (ms * 1e-3) / sfu_peak, 4),
+    return {"ms": round(ms, 4), "ms_zoh": round(ms_zoh, 4), "tokens_per_s": b * L / (ms * 1e-3),
+            "sfu_frac": round(exps / (ms * 1e-3) / sfu_peak, 4),
             "shape": f"batch {b}, D={D}, N={N}, L={L}, {c['dtype']}", "exps_counted": "2 D (N+2) per token",
             "launches": "segment pass + segment scan + reverse walk (+ 6 memsets)"}
 

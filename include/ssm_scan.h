@@ -217,9 +217,11 @@ ssm_status_t ssm_state_update(float *pool, int64_t num_slots, const int32_t *slo
  *
  * `p` describes the forward problem as for ssm_scan_fwd (the same inputs; p->y and p->h_last
  * are not used and may be NULL).  Supported:
- * dstate 16, ngroups <= 1, the Euler input matrix (p->discretization = SSM_DISC_EULER), and
- * every tensor base and row stride 16-byte aligned (the forward's fast path; dy, du, ddelta and
- * dz included).  Other cases return SSM_ERR_UNSUPPORTED before anything runs.
+ * dstate 16, ngroups <= 1, either discretisation (Euler or the zero-order hold, whose input
+ * coefficient c = (exp(Delta A) - 1) / A has dc/dDelta = exp(Delta A) and
+ * dc/dA = (Delta exp(Delta A) - c) / A), and every tensor base and row stride 16-byte aligned
+ * (the forward's fast path; dy, du, ddelta and dz included).  Other cases return
+ * SSM_ERR_UNSUPPORTED before anything runs.
  *
  * Every gradient is overwritten (not accumulated into).  "The dtype of y" below is the input
  * dtype, or float32 when p->y_fp32 is set.

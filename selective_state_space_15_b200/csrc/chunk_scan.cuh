@@ -177,6 +177,9 @@ chunk_scan_kernel(const ScanArgs args) {
     __syncthreads();
   }
   uint32_t gc = 0;  // chunks staged by this CTA so far: selects buffer and barrier parity
+#ifdef SSM_TRACE_CTA
+  const unsigned long long trace_t0 = global_ns();
+#endif
 
   for (int iter = 0;; ++iter) {
     // ------------------------------------------------------------- pick a work unit
@@ -733,6 +736,9 @@ chunk_scan_kernel(const ScanArgs args) {
     }
     __syncthreads();  // shared state of this unit is dead before the next unit overwrites it
   }
+#ifdef SSM_TRACE_CTA
+  if (threadIdx.x == 0) trace_cta(trace_t0);
+#endif
 #undef SSM_GU
 #undef SSM_GDL
 #undef SSM_GZ

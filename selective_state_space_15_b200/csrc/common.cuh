@@ -202,6 +202,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 __device__ int g_status = 0;
 __device__ __forceinline__ void report_status(int code) { atomicCAS(&g_status, 0, code); }
 
+#ifdef SSM_TRACE_CTA
+// Diagnostic build only (-DSSM_TRACE_CTA): every CTA of a traced kernel appends (SM id, start,
+// end) in global-timer nanoseconds, read back with ssm_debug_read_trace.  Adds no work to the
+// traced kernel beyond two timer reads and one store per CTA.
+constexpr int kTraceMax = 65536;
+__device__ unsigned long long g_trace[kTraceMax][3];
+__device__ unsigned int g_trace_n = 0;
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void trace_cta(unsigned long long t0) {
+  unsigned int sm;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+  const unsigned int i = atomicAdd(&g_trace_n, 1u);
+  if (i < kTraceMax) {
+    g_trace[i][0] = sm;
+    g_trace[i][1] = t0;
+    g_trace[i][2] = global_ns();
+  }
+}
+#endif
+
 // Bounded wait for an mbarrier phase: every try_wait suspends for a hardware-defined time;
 // after kMaxTries failed tries the wait gives up, records SSM_ERR_TIMEOUT and returns false
 // so that the caller carries on (with unusable data) instead of hanging the GPU.

@@ -27,7 +27,10 @@
 //   dDelta_t = sum_n (dh h_{t-1} a_t A + dh B_t u_t)      ddelta_t = dDelta_t sigmoid(delta_t + bias)
 //   dA      += dh h_{t-1} a_t Delta_t         dh *= a_t                   (on to h_{t-1})
 //
-// with yraw_t = sum_n C_t h_t + D u_t (the ungated output).  dh starts from the adjoint that
+// with yraw_t = sum_n C_t h_t + D u_t (the ungated output).  With the zero-order hold the input
+// coefficient Delta becomes c = (a - 1) / A per state (zoh_coef2): dB_t += dh c u, du_t =
+// dyraw D + sum_n dh c B, dDelta_t = sum_n dh a (h_{t-1} A + B u) (dc/dDelta = a), and dA gains
+// dh B u dc/dA (zoh_dcdA2).  dh starts from the adjoint that
 // enters the segment from its end and, in the first segment, ends as dh0.  Each forward
 // exponential is evaluated twice (segment pass, recompute), none a third time.
 //
@@ -36,8 +39,8 @@
 // derivative, the gate) for 2 of the 8 steps and hands them to the channel's other lanes by
 // shuffles; sums over the states (yraw, du, dDelta) are reduced across those 4 lanes.  The
 // sums over channels (dB, dC) go through shared memory: every lane writes its per-state
-// terms, each warp adds its 8 channels, the warps meet in a per-chunk accumulator (shared
-// atomics), and the CTA adds the chunk's rows to dB and dC with global atomics (16-byte
+// terms of four steps at a time, each warp adds its 8 channels, the warps meet in a per-chunk
+// accumulator (shared atomics), and the CTA adds the chunk's rows to dB and dC with global atomics (16-byte
 // vector atomics where the rows allow them).  dA, dDskip and dbias are summed in registers
 // and added with atomics once per unit.
 //
@@ -95,6 +98,24 @@ template <bool kFast, bool kSig> __device__ __forceinline__ float softplus_sig(f
   }
 }
 
+// Zero-order hold: the derivative of the input coefficient c = (e^x - 1) / A (x = Delta A) with
+// respect to A, dc/dA = (Delta a - c) / A = Delta^2 psi(x), psi(x) = (x e^x - e^x + 1) / x^2.
+// Where |x| < 1/4 the difference cancels, so the series psi = sum_{k>=2} (k-1)/k! x^(k-2) =
+// 1/2 + x/3 + x^2/8 + x^3/30 + x^4/144 + x^5/840 is taken (truncation below |x|^6/5760 <
+// 1e-7 relative); elsewhere the direct form loses at most a few ulp to the cancellation.  As in
+// zoh_coef2 both branches are evaluated and selected (the unselected one may be inf/nan).
+// (The derivative with respect to Delta is dc/dDelta = a.)
+__device__ __forceinline__ float2 zoh_dcdA2(float2 dt, float2 x, float2 a, float2 c, float2 invA) {
+  float2 s = __ffma2_rn(x, make_float2(1.f / 840.f, 1.f / 840.f), make_float2(1.f / 144.f, 1.f / 144.f));
+  s = __ffma2_rn(x, s, make_float2(1.f / 30.f, 1.f / 30.f));
+  s = __ffma2_rn(x, s, make_float2(0.125f, 0.125f));
+  s = __ffma2_rn(x, s, make_float2(1.f / 3.f, 1.f / 3.f));
+  s = __ffma2_rn(x, s, make_float2(0.5f, 0.5f));
+  const float2 near = __fmul2_rn(__fmul2_rn(dt, dt), s);
+  const float2 far = __fmul2_rn(__ffma2_rn(dt, a, make_float2(-c.x, -c.y)), invA);
+  return make_float2(fabsf(x.x) < 0.25f ? near.x : far.x, fabsf(x.y) < 0.25f ? near.y : far.y);
+}
+
 template <typename T, typename TG, int N, int TC, int W>
 struct BwdCfg {
   static constexpr int kN = N;
@@ -112,8 +133,9 @@ struct BwdCfg {
   static constexpr size_t kBCElems = size_t(2) * N * TC;
   static constexpr int kCOff = TC * N + 16;
   static constexpr size_t kBFElems = size_t(2) * TC * N + 16;
-  // per warp: the per-state dB, dC terms of one 8-step block, [8][2][LPC][CPW] groups of NS
-  static constexpr size_t kPartElems = size_t(8) * 2 * kLPC * kCPW * kNS;
+  // per warp: the per-state dB, dC terms of half an 8-step block, [4][2][LPC][CPW] groups of NS
+  // (the two halves are added to the accumulator one after the other)
+  static constexpr size_t kPartElems = size_t(4) * 2 * kLPC * kCPW * kNS;
   static constexpr size_t kAccElems = size_t(2) * N * TC;     // [2: dB, dC][N][TC], per buffer
   static constexpr size_t kOffY = 2 * kXElems * sizeof(T);
   static constexpr size_t kOffBC = kOffY + 2 * kYElems * sizeof(TG);
@@ -202,7 +224,7 @@ __device__ __forceinline__ void bwd_widen(const T *bs, float *bfw) {
 
 // ---------------------------------------------------------------------------------------------
 // 1. The segment pass.
-template <typename T, typename TG, int N, int TC, int W, bool HAS_Z>
+template <typename T, typename TG, int N, int TC, int W, bool HAS_Z, bool ZOH>
 __global__ void __launch_bounds__(W * 32, 12 / W) bwd_seg_kernel(const ScanArgs args, const BwdArgs bw) {
   using Cfg = BwdCfg<T, TG, N, TC, W>;
   constexpr int LPC = Cfg::kLPC, NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT;
@@ -244,16 +266,21 @@ __global__ void __launch_bounds__(W * 32, 12 / W) bwd_seg_kernel(const ScanArgs 
     const int64_t bcbase = int64_t(w.s) * args.bc_batch_stride;
 
     float2 A2[NS / 2], hz[NS / 2], pp[NS / 2], gb[NS / 2];
+    [[maybe_unused]] float2 IA[NS / 2];  // 1/A (zero-order hold)
     float bias = 0.f, cd = 0.f;
 #pragma unroll
     for (int p = 0; p < NS / 2; ++p) {
       A2[p] = hz[p] = gb[p] = make_float2(0.f, 0.f);
       pp[p] = make_float2(1.f, 1.f);
+      if constexpr (ZOH) IA[p] = make_float2(0.f, 0.f);
     }
     if (ch_ok) {
       const float *Ar = args.A + d * N + g * NS;
 #pragma unroll
-      for (int p = 0; p < NS / 2; ++p) A2[p] = make_float2(Ar[2 * p] * kLog2e, Ar[2 * p + 1] * kLog2e);
+      for (int p = 0; p < NS / 2; ++p) {
+        A2[p] = make_float2(Ar[2 * p] * kLog2e, Ar[2 * p + 1] * kLog2e);
+        if constexpr (ZOH) IA[p] = make_float2(inv_or_zero(Ar[2 * p]), inv_or_zero(Ar[2 * p + 1]));
+      }
       bias = args.bias ? args.bias[d] : 0.f;
     }
 
@@ -278,7 +305,7 @@ __global__ void __launch_bounds__(W * 32, 12 / W) bwd_seg_kernel(const ScanArgs 
         if constexpr (HAS_Z) dyr *= silu_t<kFast>(zv[j]);
         const bool in = ch_ok && (!kMasked || g * SUB + j < rel_hi);  // stale rows stay out
         dm[j] = in ? dt : 0.f;
-        um[j] = in ? dt * uv[j] : 0.f;
+        um[j] = in ? (ZOH ? uv[j] : dt * uv[j]) : 0.f;  // the input's factor besides B: Delta u, or u
         rm[j] = in ? dyr : 0.f;
       }
       float dl[8], dU[8], dr[8];
@@ -314,7 +341,9 @@ __global__ void __launch_bounds__(W * 32, 12 / W) bwd_seg_kernel(const ScanArgs 
             const float2 cp = e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
             const float2 x = __fmul2_rn(dd, A2[p]);
             const float2 a = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            hz[p] = __ffma2_rn(a, hz[p], __fmul2_rn(uu, bp));
+            float2 q = uu;
+            if constexpr (ZOH) q = __fmul2_rn(uu, zoh_coef2(dd, __fmul2_rn(x, make_float2(kLn2, kLn2)), a, IA[p]));
+            hz[p] = __ffma2_rn(a, hz[p], __fmul2_rn(q, bp));
             pp[p] = __fmul2_rn(pp[p], a);
             gb[p] = __ffma2_rn(pp[p], __fmul2_rn(rr, cp), gb[p]);
           }
@@ -396,8 +425,11 @@ __global__ void __launch_bounds__(256) bwd_seg_scan_kernel(const float *A, const
 
 // ---------------------------------------------------------------------------------------------
 // 3. The walk.
-template <typename T, typename TG, int N, int TC, int W, bool HAS_Z>
-__global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs args, const BwdArgs bw) {
+#ifndef SSM_BWD_WARPS_PER_SM
+#define SSM_BWD_WARPS_PER_SM 12  // resident warps per SM the walk is compiled for (its register budget)
+#endif
+template <typename T, typename TG, int N, int TC, int W, bool HAS_Z, bool ZOH>
+__global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kernel(const ScanArgs args, const BwdArgs bw) {
   using Cfg = BwdCfg<T, TG, N, TC, W>;
   constexpr int LPC = Cfg::kLPC, NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT, NT = Cfg::kThreads;
   constexpr int XP = Cfg::kXP, SUB = Cfg::kSub;
@@ -446,10 +478,12 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
     const int64_t so = (int64_t(s) * bw.nseg + w.seg) * args.dim + d;  // this segment's row
 
     float2 A2[NS / 2], An[NS / 2], dh[NS / 2], dAacc[NS / 2], hs[NS / 2];
+    [[maybe_unused]] float2 IA[NS / 2];  // 1/A (zero-order hold)
     float bias = 0.f, Dd = 0.f, dDacc = 0.f, dbacc = 0.f;
 #pragma unroll
     for (int p = 0; p < NS / 2; ++p) {
       A2[p] = An[p] = dh[p] = dAacc[p] = hs[p] = make_float2(0.f, 0.f);
+      if constexpr (ZOH) IA[p] = make_float2(0.f, 0.f);
     }
     if (ch_ok) {
       const float *Ar = args.A + d * N + g * NS;
@@ -459,6 +493,7 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
       for (int p = 0; p < NS / 2; ++p) {
         An[p] = make_float2(Ar[2 * p], Ar[2 * p + 1]);
         A2[p] = make_float2(An[p].x * kLog2e, An[p].y * kLog2e);
+        if constexpr (ZOH) IA[p] = make_float2(inv_or_zero(An[p].x), inv_or_zero(An[p].y));
         dh[p] = make_float2(mr[2 * p], mr[2 * p + 1]);
         hs[p] = make_float2(hr[2 * p], hr[2 * p + 1]);
       }
@@ -490,6 +525,30 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
       }
     };
 
+    // dB, dC terms of four steps (chunk-local steps t0 .. t0 + 3, buffer slots 0..3): the warp's 8
+    // channels added up, then into the CTA's chunk accumulator
+    auto reduce_part = [&](float *acc, int t0) {
+      __syncwarp();
+      for (int o = lane; o < 4 * 2 * LPC * (NS / 4); o += 32) {
+        // output group o = ((kk * 2 + which) * LPC + gg) * (NS / 4) + q: 4 states of one step
+        const int q = o % (NS / 4), gg = (o / (NS / 4)) % LPC, which = (o / (NS / 4 * LPC)) % 2;
+        const int kk = o / (NS / 4 * LPC * 2);
+        const float *src = part + ((size_t(kk) * 2 + which) * LPC * CPW + size_t(gg) * CPW) * NS + q * 4;
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int cc = 0; cc < CPW; ++cc) {
+          const float4 v = *reinterpret_cast<const float4 *>(src + cc * NS);
+          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+        }
+        float *dst = acc + (size_t(which) * N + gg * NS + q * 4) * TC + t0 + kk;
+        atomicAdd(dst, sum.x);
+        atomicAdd(dst + TC, sum.y);
+        atomicAdd(dst + 2 * TC, sum.z);
+        atomicAdd(dst + 3 * TC, sum.w);
+      }
+      __syncwarp();  // the terms are consumed before the buffer is rewritten
+    };
+
     // one 8-step block, from the end of the block to its start
     auto block = [&](auto masked_tag, const T *X, const TG *Y, const float *Bf, float *acc, int64_t wstart, int sb) {
       constexpr bool kMasked = decltype(masked_tag)::value;
@@ -508,7 +567,7 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
       for (int j = 0; j < SUB; ++j) {
         float sgm;
         float dt = softplus_sig<kFast, true>(dv[j] + bias, sgm);
-        float du = dt * uv[j], gy = gv[j];
+        float du = ZOH ? uv[j] : dt * uv[j], gy = gv[j];  // the input's factor besides B: Delta u, or u
         // a channel past the end of a ragged tile, or a step past the end of the sequence, takes
         // no part (its staged rows are stale; selects keep non-finite values out of the sums)
         const bool in = ch_ok && (!kMasked || g * SUB + j < rel_hi);
@@ -575,7 +634,9 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
             const float2 cp = e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
             const float2 x = __fmul2_rn(dd, A2[p]);
             a[k][p] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            h[k][p] = __ffma2_rn(a[k][p], k ? h[k - 1][p] : hin[p], __fmul2_rn(uu, bp));
+            float2 q = uu;
+            if constexpr (ZOH) q = __fmul2_rn(uu, zoh_coef2(dd, __fmul2_rn(x, make_float2(kLn2, kLn2)), a[k][p], IA[p]));
+            h[k][p] = __ffma2_rn(a[k][p], k ? h[k - 1][p] : hin[p], __fmul2_rn(q, bp));
             acc2 = __ffma2_rn(cp, h[k][p], acc2);
           }
         }
@@ -615,16 +676,20 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
       float dr[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) dr[k] = __shfl_sync(0xffffffffu, dym[k % SUB], lbase + k / SUB);
-      // ---- the adjoint recurrence, last step first
+      // ---- the adjoint recurrence, last step first.  S1 = sum_n dh c B (c = Delta for Euler:
+      // the factor Delta is applied after the sum), S2 = sum_n dh h_{t-1} a A, and for the
+      // zero-order hold S3 = sum_n dh a B (dc/dDelta = a)
       float s1[8], s2[8];
+      [[maybe_unused]] float s3[8];
 #pragma unroll
       for (int k = 7; k >= 0; --k) {
         const int t = k0 + k;
         const float2 dd = make_float2(dl[k], dl[k]), uu = make_float2(dU[k], dU[k]);
         const float2 dyr = make_float2(dr[k], dr[k]);
         float2 S1 = make_float2(0.f, 0.f), S2 = make_float2(0.f, 0.f);
-        float *pb = part + ((size_t(k) * 2 + 0) * LPC * CPW + size_t(g) * CPW + c) * NS;  // dB terms
-        float *pc = part + ((size_t(k) * 2 + 1) * LPC * CPW + size_t(g) * CPW + c) * NS;  // dC terms
+        [[maybe_unused]] float2 S3 = make_float2(0.f, 0.f);
+        float *pb = part + ((size_t(k & 3) * 2 + 0) * LPC * CPW + size_t(g) * CPW + c) * NS;  // dB terms
+        float *pc = part + ((size_t(k & 3) * 2 + 1) * LPC * CPW + size_t(g) * CPW + c) * NS;  // dC terms
 #pragma unroll
         for (int q = 0; q < NS / 4; ++q) {
           float4 b4 = reinterpret_cast<const float4 *>(Bf + t * N + g * NS)[q];
@@ -640,11 +705,22 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
             const float2 cp = e ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
             dh[p] = __ffma2_rn(dyr, cp, dh[p]);                 // y_t reads h_t
             tc[e] = __fmul2_rn(dyr, h[k][p]);                    // dC_t term of this channel
-            tb[e] = __fmul2_rn(dh[p], uu);                       // dB_t term: dh Delta u
-            S1 = __ffma2_rn(dh[p], bp, S1);                      // sum_n dh B
             const float2 daa = __fmul2_rn(__fmul2_rn(dh[p], k ? h[k - 1][p] : hin[p]), a[k][p]);
             S2 = __ffma2_rn(daa, An[p], S2);                     // sum_n dh h_{t-1} a A
             dAacc[p] = __ffma2_rn(daa, dd, dAacc[p]);            // dA += dh h_{t-1} a Delta
+            if constexpr (ZOH) {
+              const float2 x = __fmul2_rn(__fmul2_rn(dd, A2[p]), make_float2(kLn2, kLn2));
+              const float2 cz = zoh_coef2(dd, x, a[k][p], IA[p]);
+              tb[e] = __fmul2_rn(dh[p], __fmul2_rn(cz, uu));     // dB_t term: dh c u
+              const float2 db = __fmul2_rn(dh[p], bp);
+              S1 = __ffma2_rn(db, cz, S1);                       // sum_n dh c B
+              S3 = __ffma2_rn(db, a[k][p], S3);                  // sum_n dh a B
+              // dA += dh B u dc/dA
+              dAacc[p] = __ffma2_rn(__fmul2_rn(db, uu), zoh_dcdA2(dd, x, a[k][p], cz, IA[p]), dAacc[p]);
+            } else {
+              tb[e] = __fmul2_rn(dh[p], uu);                     // dB_t term: dh Delta u
+              S1 = __ffma2_rn(dh[p], bp, S1);                    // sum_n dh B
+            }
             dh[p] = __fmul2_rn(dh[p], a[k][p]);                  // on to h_{t-1}
           }
           reinterpret_cast<float4 *>(pb)[q] = make_float4(tb[0].x, tb[0].y, tb[1].x, tb[1].y);
@@ -652,7 +728,10 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
         }
         s1[k] = S1.x + S1.y;
         s2[k] = S2.x + S2.y;
+        if constexpr (ZOH) s3[k] = S3.x + S3.y;
+        if (k == 4) reduce_part(acc, k0 + 4);  // steps 4..7 done: their terms leave the buffer
       }
+      reduce_part(acc, k0);
       // ---- sums over the channel's lanes of sum_n dh B and sum_n dh h a A, for this lane's steps
 #pragma unroll
       for (int lev = 0; (1 << lev) < LPC; ++lev) {
@@ -664,14 +743,23 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
           const float send2 = upper ? s2[j] : s2[half + j], keep2 = upper ? s2[half + j] : s2[j];
           s1[j] = keep1 + __shfl_xor_sync(0xffffffffu, send1, off);
           s2[j] = keep2 + __shfl_xor_sync(0xffffffffu, send2, off);
+          if constexpr (ZOH) {
+            const float send3 = upper ? s3[j] : s3[half + j], keep3 = upper ? s3[half + j] : s3[j];
+            s3[j] = keep3 + __shfl_xor_sync(0xffffffffu, send3, off);
+          }
         }
       }
       if (ch_ok) {
         float odu[SUB], odd[SUB];
 #pragma unroll
         for (int j = 0; j < SUB; ++j) {
-          odu[j] = fmaf(dym[j], Dd, dm[j] * s1[j]);              // du = dyraw D + Delta sum dh B
-          odd[j] = fmaf(uv[j], s1[j], s2[j]) * sg[j];            // (sum dh h a A + u sum dh B) sigmoid
+          if constexpr (ZOH) {
+            odu[j] = fmaf(dym[j], Dd, s1[j]);                    // du = dyraw D + sum dh c B
+            odd[j] = fmaf(uv[j], s3[j], s2[j]) * sg[j];          // (sum dh h a A + u sum dh a B) sigmoid
+          } else {
+            odu[j] = fmaf(dym[j], Dd, dm[j] * s1[j]);            // du = dyraw D + Delta sum dh B
+            odd[j] = fmaf(uv[j], s1[j], s2[j]) * sg[j];          // (sum dh h a A + u sum dh B) sigmoid
+          }
           if constexpr (kMasked) {
             const bool in = g * SUB + j < rel_hi;
             odd[j] = in ? odd[j] : 0.f;
@@ -698,26 +786,6 @@ __global__ void __launch_bounds__(W * 32, 12 / W) seq_bwd_kernel(const ScanArgs 
             }
         }
       }
-      // ---- dB, dC: add the warp's 8 channels, then into the CTA's chunk accumulator
-      __syncwarp();
-      for (int o = lane; o < 8 * 2 * LPC * (NS / 4); o += 32) {
-        // output group o = ((k * 2 + which) * LPC + gg) * (NS / 4) + q: 4 states of one step
-        const int q = o % (NS / 4), gg = (o / (NS / 4)) % LPC, which = (o / (NS / 4 * LPC)) % 2;
-        const int k = o / (NS / 4 * LPC * 2);
-        const float *src = part + ((size_t(k) * 2 + which) * LPC * CPW + size_t(gg) * CPW) * NS + q * 4;
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int cc = 0; cc < CPW; ++cc) {
-          const float4 v = *reinterpret_cast<const float4 *>(src + cc * NS);
-          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-        }
-        float *dst = acc + (size_t(which) * N + gg * NS + q * 4) * TC + k0 + k;
-        atomicAdd(dst, sum.x);
-        atomicAdd(dst + TC, sum.y);
-        atomicAdd(dst + 2 * TC, sum.z);
-        atomicAdd(dst + 3 * TC, sum.w);
-      }
-      __syncwarp();  // the warp's terms are consumed before the next block rewrites them
     };
 
     // ------------------------------------------------------------- the segment's chunks, last first

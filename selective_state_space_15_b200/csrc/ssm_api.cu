@@ -431,7 +431,7 @@ struct BwdPlan {
   size_t off_ckpt = 0, off_cumd = 0, off_ssum = 0, off_sh = 0, off_sg = 0, bytes = 0;
 };
 bool make_bwd_plan(const ssm_scan_params *p, bool vec, BwdPlan &bp) {
-  if (!vec || p->dstate != 16 || groups_of(p) != 1 || p->discretization != SSM_DISC_EULER) return false;
+  if (!vec || p->dstate != 16 || groups_of(p) != 1) return false;
   const int64_t TC = p->dtype == SSM_F32 ? 16 : kBwdTC16;
   const int64_t CT = 8 * kBwdWarps, L = p->seqlen, N = p->dstate;
   bp.nblk = (L + 7) / 8;
@@ -454,7 +454,9 @@ bool make_bwd_plan(const ssm_scan_params *p, bool vec, BwdPlan &bp) {
   return true;
 }
 
-template <typename T, typename TG, bool HAS_Z>
+template <typename X> struct TypeTag { using type = X; };
+
+template <typename T, typename TG, bool HAS_Z, bool ZOH>
 ssm_status_t launch_bwd(ScanArgs a, const ssm::BwdArgs &bwa, const BwdPlan &bp, const ssm_scan_params *p,
                         unsigned char *ws, cudaStream_t st) {
   constexpr int N = 16, W = kBwdWarps;
@@ -465,7 +467,7 @@ ssm_status_t launch_bwd(ScanArgs a, const ssm::BwdArgs &bwa, const BwdPlan &bp, 
   a.total_units = int(bp.nunits);
   // 1. the segment pass
   {
-    auto kern = ssm::bwd_seg_kernel<T, TG, N, TC, W, HAS_Z>;
+    auto kern = ssm::bwd_seg_kernel<T, TG, N, TC, W, HAS_Z, ZOH>;
     LaunchInfo li;
     if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSegSmemBytes, li) != SSM_OK)
       return SSM_ERR_CUDA;
@@ -484,7 +486,7 @@ ssm_status_t launch_bwd(ScanArgs a, const ssm::BwdArgs &bwa, const BwdPlan &bp, 
   }
   // 3. the walk
   {
-    auto kern = ssm::seq_bwd_kernel<T, TG, N, TC, W, HAS_Z>;
+    auto kern = ssm::seq_bwd_kernel<T, TG, N, TC, W, HAS_Z, ZOH>;
     LaunchInfo li;
     if (launch_info(reinterpret_cast<const void *>(kern), Cfg::kThreads, Cfg::kSmemBytes, li) != SSM_OK)
       return SSM_ERR_CUDA;
@@ -672,12 +674,17 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params *p, const ssm_scan_grads *g, voi
   bwa.vec_dbc = (aligned16(g->dB) && aligned16(g->dC) && p->seqlen % 4 == 0) ? 1 : 0;
   a.cu_seqlens = nullptr;
   using bf16 = __nv_bfloat16;
-  const bool has_z = p->z != nullptr;
-  if (p->dtype == SSM_BF16 && !p->y_fp32)
-    return has_z ? launch_bwd<bf16, bf16, true>(a, bwa, bp, p, ws, cs) : launch_bwd<bf16, bf16, false>(a, bwa, bp, p, ws, cs);
-  if (p->dtype == SSM_BF16)
-    return has_z ? launch_bwd<bf16, float, true>(a, bwa, bp, p, ws, cs) : launch_bwd<bf16, float, false>(a, bwa, bp, p, ws, cs);
-  return has_z ? launch_bwd<float, float, true>(a, bwa, bp, p, ws, cs) : launch_bwd<float, float, false>(a, bwa, bp, p, ws, cs);
+  const bool has_z = p->z != nullptr, zoh = p->discretization == SSM_DISC_ZOH;
+  auto go = [&](auto t_tag, auto tg_tag) -> ssm_status_t {
+    using T = typename decltype(t_tag)::type;
+    using TG = typename decltype(tg_tag)::type;
+    if (zoh)
+      return has_z ? launch_bwd<T, TG, true, true>(a, bwa, bp, p, ws, cs) : launch_bwd<T, TG, false, true>(a, bwa, bp, p, ws, cs);
+    return has_z ? launch_bwd<T, TG, true, false>(a, bwa, bp, p, ws, cs) : launch_bwd<T, TG, false, false>(a, bwa, bp, p, ws, cs);
+  };
+  if (p->dtype == SSM_BF16 && !p->y_fp32) return go(TypeTag<bf16>{}, TypeTag<bf16>{});
+  if (p->dtype == SSM_BF16) return go(TypeTag<bf16>{}, TypeTag<float>{});
+  return go(TypeTag<float>{}, TypeTag<float>{});
 }
 
 ssm_status_t ssm_ssd_fwd(const ssm_ssd_params *p, ssm_stream_t stream) {
@@ -714,6 +721,22 @@ ssm_status_t ssm_ssd_fwd(const ssm_ssd_params *p, ssm_stream_t stream) {
                           reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
+
+#ifdef SSM_TRACE_CTA
+// Diagnostic build only: copy the CTA trace of the chunked scan kernel (entries of SM id, start
+// and end in global-timer nanoseconds) to `host` and clear it; returns the entry count.
+int64_t ssm_debug_read_trace(unsigned long long *host, int64_t max_entries) {
+  unsigned int n = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpyFromSymbol(&n, ssm::g_trace_n, sizeof(n)) != cudaSuccess)
+    return -1;
+  const int64_t m = std::min<int64_t>(std::min<int64_t>(n, ssm::kTraceMax), max_entries);
+  if (m > 0 && cudaMemcpyFromSymbol(host, ssm::g_trace, size_t(m) * 3 * sizeof(unsigned long long)) != cudaSuccess)
+    return -1;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(ssm::g_trace_n, &zero, sizeof(zero)) != cudaSuccess) return -1;
+  return m;
+}
+#endif
 
 size_t ssm_scan_bwd_workspace_size(const ssm_scan_params *p) {
   ScanArgs a;

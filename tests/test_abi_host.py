@@ -178,7 +178,7 @@ def test_backward_host_checks(lib):
         setattr(g_noz, name, fake)
     assert f(ctypes.byref(pz), ctypes.byref(g_noz), None, 0, None) == 1            # z given, no dz
     assert f(ctypes.byref(_params(dstate=32)), ctypes.byref(g), None, 0, None) == 2
-    assert f(ctypes.byref(_params(discretization=ssm.DISC_ZOH)), ctypes.byref(g), None, 0, None) == 2
+    assert f(ctypes.byref(_params(discretization=ssm.DISC_ZOH)), ctypes.byref(g), None, 0, None) == 6  # supported
     assert f(ctypes.byref(_params(dim=64, ngroups=2)), ctypes.byref(g), None, 0, None) == 2
     assert f(ctypes.byref(_params(x_dim_stride=130, seqlen=128)), ctypes.byref(g), None, 0, None) == 2
     assert f(ctypes.byref(p), ctypes.byref(g), None, 0, None) == 6                  # SSM_ERR_WORKSPACE

@@ -54,7 +54,7 @@ def check_grads(got, ref, tol, grad_dtype, names=NAMES):
         assert e <= tol, f"{name}: row-normwise error {e:.3e} > {tol:.1e}"
 
 
-def run_bwd(inp, dtype, dy, grad_dtype=None, h0=None, dh_last=None, gate=True, to_host=True):
+def run_bwd(inp, dtype, dy, grad_dtype=None, h0=None, dh_last=None, gate=True, to_host=True, zoh=False):
     u, dl = dev(inp.u, dtype), dev(inp.delta, dtype)
     z = dev(inp.z, dtype) if gate else None
     B, C = dev(inp.B, dtype), dev(inp.C, dtype)
@@ -64,18 +64,18 @@ def run_bwd(inp, dtype, dy, grad_dtype=None, h0=None, dh_last=None, gate=True, t
     h0t = torch.from_numpy(h0).cuda() if h0 is not None else None
     dht = torch.from_numpy(dh_last).cuda() if dh_last is not None else None
     out = ssm.scan_bwd(u, dl, B, C, A, dyt, D, bias, z, h0t, dht,
-                       grad_dtype=torch.float32 if gdt == "f32" else None)
+                       grad_dtype=torch.float32 if gdt == "f32" else None, zoh=zoh)
     torch.cuda.synchronize()
     if not to_host:
         return out
     return {k: (host(v) if v is not None else None) for k, v in out.items()}
 
 
-def oracle_bwd(inp, dy, h0=None, dh_last=None, gate=True, channels=None):
+def oracle_bwd(inp, dy, h0=None, dh_last=None, gate=True, channels=None, zoh=False):
     sl = slice(None) if channels is None else channels
     r = oracle.scan_bwd(inp.u[:, sl], inp.delta[:, sl], inp.B, inp.C, inp.A[sl], dy[:, sl], inp.Dskip[sl],
                         inp.bias[sl], inp.z[:, sl] if gate else None, None if h0 is None else h0[:, sl],
-                        None if dh_last is None else dh_last[:, sl], nthreads=NTHREADS)
+                        None if dh_last is None else dh_last[:, sl], nthreads=NTHREADS, zoh=zoh)
     return r
 
 
@@ -84,6 +84,7 @@ def draw_dy(shape, dtype, seed):
     return workloads.round_to_bf16(x) if dtype == "bf16" else x
 
 
+@pytest.mark.parametrize("zoh", [False, True], ids=["euler", "zoh"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", [
     (1, 16, 16, 256),      # the tiny workload's shape
@@ -91,14 +92,30 @@ def draw_dy(shape, dtype, seed):
     (3, 33, 16, 8),        # one block
     (1, 64, 16, 1000),
 ])
-def test_bwd_small_full(shape, dtype):
+def test_bwd_small_full(shape, dtype, zoh):
     b, D, N, L = shape
     inp = workloads.batch_inputs(b, D, N, L, dtype, seed=800 + L + D, h0=True)
     dy = draw_dy((b, D, L), dtype, 801 + L)
     dh_last = np.random.default_rng(802).standard_normal((b, D, N)).astype(np.float32)
-    got = run_bwd(inp, dtype, dy, h0=inp.h0, dh_last=dh_last)
-    ref = oracle_bwd(inp, dy, h0=inp.h0, dh_last=dh_last)
+    got = run_bwd(inp, dtype, dy, h0=inp.h0, dh_last=dh_last, zoh=zoh)
+    ref = oracle_bwd(inp, dy, h0=inp.h0, dh_last=dh_last, zoh=zoh)
     check_grads(got, ref, TOL[dtype], dtype)
+
+
+def test_bwd_zoh_with_zero_and_positive_decays():
+    """Zero-order hold where A = 0 for some states (c = Delta, dc/dA = Delta^2 / 2 from the
+    series) and small |Delta A| everywhere else in a channel (the series side of both
+    coefficients), next to the usual decays."""
+    b, D, N, L = 1, 24, 16, 200
+    inp = workloads.batch_inputs(b, D, N, L, "f32", seed=870, h0=True)
+    A = inp.A.copy()
+    A[0:8, 0:4] = 0.0
+    A[8:16] *= 1e-3
+    inp.A = A
+    dy = draw_dy((b, D, L), "f32", 871)
+    got = run_bwd(inp, "f32", dy, h0=inp.h0, zoh=True)
+    ref = oracle_bwd(inp, dy, h0=inp.h0, zoh=True)
+    check_grads(got, ref, TOL["f32"], "f32")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -121,28 +138,30 @@ def test_bwd_bf16_inputs_float32_gradients_strict():
     check_grads(got, ref, TOL["bf16"], "f32")
 
 
-def test_bwd_batch_f32_workload():
+@pytest.mark.parametrize("zoh", [False, True], ids=["euler", "zoh"])
+def test_bwd_batch_f32_workload(zoh):
     """The float32 batch workload (batch 2, D=1536, N=16, L=2048), every gradient in full."""
     inp = workloads.config_inputs("batch_f32")
     b, D, L = inp.u.shape
     dy = draw_dy((b, D, L), "f32", 830)
-    got = run_bwd(inp, "f32", dy)
-    ref = oracle_bwd(inp, dy)
+    got = run_bwd(inp, "f32", dy, zoh=zoh)
+    ref = oracle_bwd(inp, dy, zoh=zoh)
     check_grads(got, ref, TOL["f32"], "f32")
 
 
-def test_bwd_long_workload_sampled():
+@pytest.mark.parametrize("zoh", [False, True], ids=["euler", "zoh"])
+def test_bwd_long_workload_sampled(zoh):
     """The long bf16 workload (1 x 2560 channels x 131072 steps) with dy nonzero on sampled
     channels only: the gradients then come from those channels alone (the others carry no
     adjoint), so the oracle run on the sample gives every gradient exactly -- dB and dC, which
     sum over channels, included.  The other channels' per-step gradients must be zero."""
     inp = workloads.config_inputs("long_bf16")
     b, D, L = inp.u.shape
-    ch = np.arange(9, D, 523)
+    ch = np.arange(9, D, 523) if not zoh else np.arange(301, D, 611)
     dy = np.zeros((b, D, L), dtype=np.float32)
     dy[:, ch] = draw_dy((b, len(ch), L), "bf16", 840)
-    got = run_bwd(inp, "bf16", dy, to_host=False)
-    ref = oracle_bwd(inp, dy, channels=ch)
+    got = run_bwd(inp, "bf16", dy, to_host=False, zoh=zoh)
+    ref = oracle_bwd(inp, dy, channels=ch, zoh=zoh)
     idx = torch.from_numpy(ch).cuda()
     sub = {k: host(v.index_select(1, idx) if k in ("du", "ddelta", "dz", "dh0") else
                    v.index_select(0, idx) if k in ("dA", "dDskip", "dbias") else v)
@@ -174,8 +193,42 @@ def test_bwd_rejections_and_workspace():
     g2.dy = dy.data_ptr()
     assert lib.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g2), None, 0, stream) == 1         # outputs missing
     pz = ssm.scan_params(u, dl, B, C, A, z=z, zoh=True)
-    assert lib.ssm_scan_bwd(ctypes.byref(pz), ctypes.byref(g), None, 0, stream) == 2         # zero-order hold
+    assert lib.ssm_scan_bwd(ctypes.byref(pz), ctypes.byref(g), None, 0, stream) == 6         # zero-order hold: supported
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     assert lib.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g), ctypes.c_void_p(ws.data_ptr()), need, stream) == 0
     torch.cuda.synchronize()
     assert ssm.device_status() == 0
+
+
+def test_bwd_padded_rows_ragged_length_through_the_abi():
+    """Rows padded to a 16-byte stride (304) around a length that is not a multiple of 4 (301):
+    the per-step gradients keep u's strides and must leave the padding alone, and dB, dC
+    ([b, N, L] contiguous: 1204-byte rows) take the scalar-atomic path of the channel sums."""
+    b, D, N, L, P = 2, 40, 16, 301, 304
+    inp = workloads.batch_inputs(b, D, N, L, "f32", seed=860, h0=True)
+    dy_h = draw_dy((b, D, L), "f32", 861)
+    view = lambda x: dev(x, "f32", pitch=P)[..., :L]  # noqa: E731  (NaN in the padding)
+    u, dl, z, B, C, dy = (view(x) for x in (inp.u, inp.delta, inp.z, inp.B, inp.C, dy_h))
+    A, Dk, bias, h0 = (torch.from_numpy(x).cuda() for x in (inp.A, inp.Dskip, inp.bias, inp.h0))
+    outs = {k: torch.full((b, D, P), float("nan"), device="cuda")[..., :L] for k in ("du", "ddelta", "dz")}
+    dB, dC = torch.empty(b, N, L, device="cuda"), torch.empty(b, N, L, device="cuda")
+    dA, dD, db = torch.empty(D, N, device="cuda"), torch.empty(D, device="cuda"), torch.empty(D, device="cuda")
+    dh0 = torch.empty(b, D, N, device="cuda")
+    p = ssm.scan_params(u, dl, B, C, A, Dk, bias, z, h0)
+    lib = ssm.load()
+    need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(p))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    g = ssm.ScanGrads()
+    g.dy, g.du, g.ddelta, g.dz = dy.data_ptr(), outs["du"].data_ptr(), outs["ddelta"].data_ptr(), outs["dz"].data_ptr()
+    g.dB, g.dC, g.dA, g.dDskip, g.ddelta_bias, g.dh0 = (t.data_ptr() for t in (dB, dC, dA, dD, db, dh0))
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g), ctypes.c_void_p(ws.data_ptr()), need, stream) == 0
+    torch.cuda.synchronize()
+    assert ssm.device_status() == 0
+    got = {"du": host(outs["du"]), "ddelta": host(outs["ddelta"]), "dz": host(outs["dz"]), "dB": host(dB),
+           "dC": host(dC), "dA": host(dA), "dDskip": host(dD), "dbias": host(db), "dh0": host(dh0)}
+    ref = oracle_bwd(inp, dy_h, h0=inp.h0)
+    check_grads(got, ref, TOL["f32"], "f32")
+    for k in ("du", "ddelta", "dz"):
+        pad = outs[k].as_strided((b, D, P - L), (D * P, P, 1), storage_offset=L)
+        assert torch.isnan(pad).all(), f"{k}: the kernel wrote into the row padding"
