@@ -67,9 +67,16 @@ struct ChunkCfg {
   static constexpr int kVec = Elem<T>::kVec;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kXPitch = kTC + kVec;  // u/delta/z row pitch (elements): +16 bytes
-  // B/C row pitch (elements).  With lane groups, the two groups of a quarter-warp read
-  // neighbouring states at the same steps: 16 bytes of padding put them in distinct banks.
-  static constexpr int kBCPitch = kTC + (kLG > 1 ? 16 / int(sizeof(T)) : 0);
+  // 16-bit B/C of the N=16 tiles with chunks of up to 128 steps are widened to float32 once
+  // per chunk (double-buffered [2][2][N][BFPitch]), so the state loop loads them without
+  // converting; their 16-bit copies then need a single staging buffer (a chunk's copy lands
+  // after the previous one was widened).
+  static constexpr bool kBF = sizeof(T) == 2 && N == 16 && NG == 1 && kTC <= 128;
+  // B/C row pitch (elements).  With lane groups, the groups of a quarter-warp read
+  // neighbouring states at the same steps: 16 bytes of padding put them in distinct banks
+  // (in the float32 copy when there is one, else in the 16-bit staging).
+  static constexpr int kBCPitch = kTC + ((kLG > 1 && !kBF) ? 16 / int(sizeof(T)) : 0);
+  static constexpr int kBFPitch = kTC + (kLG > 1 ? 4 : 0);
   // shared memory layout (bytes), staging double-buffered
   static constexpr size_t kXBytes = size_t(3) * kCT * kXPitch * sizeof(T);  // u, delta, z
   static constexpr size_t kBCBytes = size_t(2) * N * kBCPitch * sizeof(T);  // B, C
@@ -82,11 +89,11 @@ struct ChunkCfg {
   // channels hit distinct banks); with few groups each lane computes its own.
   static constexpr bool kSharedDelta = NG >= 4;
   static constexpr int kDPitch = kTC + 4;
-  // With two lane groups per warp each group evaluates Delta, Delta*u for half of a lane's
-  // steps and the halves meet in a per-warp buffer of float4: [2][KI/4][kXQ], one column per
-  // lane pair.  The row pitch kXQ (16 + 16/kVec float4) puts a half's writes from the two
-  // groups of a quarter-warp in distinct banks.
-  static constexpr bool kLaneDelta = !kSharedDelta && kLG == 2 && KI / kVec == 2;
+  // With lane groups each group evaluates Delta, Delta*u for 1/kLG of a lane's steps (a
+  // 16-byte vector or half of one) and the parts meet in a per-warp buffer of float4:
+  // [2][KI/4][kXQ], one column per lane of a group.  The row pitch kXQ (CPW SPW + 16/kVec
+  // float4) puts the writes of a quarter-warp's groups in distinct banks.
+  static constexpr bool kLaneDelta = !kSharedDelta && kLG > 1 && KI / kVec == 2 && (KI / kLG) % 4 == 0;
   static constexpr int kXQ = CPW * SPW + 16 / kVec;
   static constexpr size_t kDBytes = kSharedDelta ? size_t(2) * kCT * kDPitch * sizeof(float)
                                     : kLaneDelta ? size_t(kWarps) * 2 * (KI / 4) * kXQ * 16
@@ -94,13 +101,8 @@ struct ChunkCfg {
   static constexpr int kNP = N + 1;         // row pitch of the per-(channel, state) arrays
   static constexpr size_t kParamBytes =
       size_t(2) * kCT * kNP * sizeof(float) + size_t(2) * kCT * sizeof(float) + kMaxSortedSeqs * sizeof(int);
-  // 16-bit B/C of the wide N=16 tile are widened to float32 once per chunk (double-buffered
-  // [2][2][N][TC]), so the state loop loads them without converting; their 16-bit copies
-  // then need a single staging buffer (a chunk's copy lands after the previous one was
-  // widened).
-  static constexpr bool kBF = sizeof(T) == 2 && N == 16 && kLG == 1 && NG == 1;
   static constexpr size_t kBCAll = (kBF ? 1 : 2) * kBCBytes;  // 16-bit B/C staging
-  static constexpr size_t kBFBytes = kBF ? size_t(2) * 2 * N * kTC * sizeof(float) : 0;
+  static constexpr size_t kBFBytes = kBF ? size_t(2) * 2 * N * kBFPitch * sizeof(float) : 0;
   static constexpr size_t kSmemBytes = 2 * kXBytes + kBCAll + kYBytes + kDBytes + kBFBytes + kParamBytes;
   // 1/A per (channel, state) after the parameters, for the zero-order hold only
   static constexpr size_t kInvABytes = size_t(kCT) * kNP * sizeof(float);
@@ -109,7 +111,8 @@ struct ChunkCfg {
   static_assert(kLG == 1 || NG == 1, "states split either across warps or inside a warp");
   static_assert(N % (NG * kLG) == 0 && KI % (NG * kLG) == 0, "state / step split");
   static_assert(kXBytes % 16 == 0 && kBCBytes % 16 == 0, "16-byte aligned buffers");
-  static_assert(!kBF || kBCPitch == kTC, "widened B/C rows are unpadded");
+  static_assert(!kBF || kBCPitch == kTC, "the 16-bit staging of widened B/C rows is unpadded");
+  static_assert((kBFPitch * sizeof(float)) % 16 == 0, "16-byte float32 B/C rows");
 };
 
 template <typename T, typename TO, int N, int KI, int SPW, int CPW, int CW, int NG, bool HAS_Z, bool VEC,
@@ -134,8 +137,9 @@ chunk_scan_kernel(const ScanArgs args) {
   float *dls = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + Cfg::kBCAll + Cfg::kYBytes);  // [2][CT][DP]
   constexpr int DP = Cfg::kDPitch;
   float *const bcf = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + Cfg::kBCAll + Cfg::kYBytes +
-                                               Cfg::kDBytes);  // [2][2][N][TC] (kBF only)
-  constexpr size_t kBFElems = size_t(2) * N * TC;
+                                               Cfg::kDBytes);  // [2][2][N][BFP] (kBF only)
+  constexpr int BFP = Cfg::kBFPitch;
+  constexpr size_t kBFElems = size_t(2) * N * BFP;
   float *A2s = reinterpret_cast<float *>(smem + 2 * Cfg::kXBytes + Cfg::kBCAll + Cfg::kYBytes +
                                          Cfg::kDBytes + Cfg::kBFBytes);  // [CT][NP]
   float *carry_s = A2s + CT * NP;                                 // [CT][NP]
@@ -336,7 +340,7 @@ chunk_scan_kernel(const ScanArgs args) {
         T val = Elem<T>::from_f32(0.f);
         if (t < args.seqlen) val = base[bcbase + int64_t(n) * args.bc_state_stride + t];
         if constexpr (Cfg::kBF)
-          bcf[buf * kBFElems + size_t(row) * TC + j] = Elem<T>::to_f32(val);
+          bcf[buf * kBFElems + size_t(row) * BFP + j] = Elem<T>::to_f32(val);
         else
           bdst[size_t(row) * Cfg::kBCPitch + j] = val;
       }
@@ -354,26 +358,36 @@ chunk_scan_kernel(const ScanArgs args) {
 #pragma unroll
       for (int p = 0; p < KP; ++p) y[p] = make_float2(0.f, 0.f);
       if constexpr (Cfg::kLaneDelta) {
-        // this lane group evaluates vector lg of the lane's KI steps; the other group the rest
-        // float4 q of the lane pair's Delta (rows 0 .. KI/4-1) and Delta*u (rows KI/4 ..)
-        constexpr int XQ = Cfg::kXQ, Q = KI / 4;
+        // this lane group evaluates steps [lg SG, (lg + 1) SG) of the lane's KI steps, the other
+        // groups the rest; float4 q of the lane's Delta (rows 0 .. KI/4-1) and Delta*u (rows
+        // KI/4 ..) in column lr
+        constexpr int XQ = Cfg::kXQ, Q = KI / 4, SG = KI / LG;
+        static_assert(SG == V || (SG * 2 == V && sizeof(T) == 2), "a group's steps: a vector or half of one");
         float4 *xw = reinterpret_cast<float4 *>(dls) + size_t(warp) * 2 * Q * XQ + lr;
-        const T *ru = X + size_t(ch) * XP + tl0 + lg * V;
-        const T *rd = X + size_t(CT + ch) * XP + tl0 + lg * V;
+        const T *ru = X + size_t(ch) * XP + tl0 + lg * SG;
+        const T *rd = X + size_t(CT + ch) * XP + tl0 + lg * SG;
         const float bias = bias_s[ch];
-        float2 vu[V / 2], vd[V / 2];
-        unpack16x2<T>(*reinterpret_cast<const uint4 *>(ru), vu);
-        unpack16x2<T>(*reinterpret_cast<const uint4 *>(rd), vd);
+        float2 vu[SG / 2], vd[SG / 2];
+        if constexpr (SG == V) {
+          unpack16x2<T>(*reinterpret_cast<const uint4 *>(ru), vu);
+          unpack16x2<T>(*reinterpret_cast<const uint4 *>(rd), vd);
+        } else {  // four 16-bit values: 8 bytes
+          const uint2 wu = *reinterpret_cast<const uint2 *>(ru), wd = *reinterpret_cast<const uint2 *>(rd);
+          vu[0] = make_float2(__uint_as_float(wu.x << 16), __uint_as_float(wu.x & 0xffff0000u));
+          vu[1] = make_float2(__uint_as_float(wu.y << 16), __uint_as_float(wu.y & 0xffff0000u));
+          vd[0] = make_float2(__uint_as_float(wd.x << 16), __uint_as_float(wd.x & 0xffff0000u));
+          vd[1] = make_float2(__uint_as_float(wd.y << 16), __uint_as_float(wd.y & 0xffff0000u));
+        }
         __syncwarp();  // the previous chunk's reads of the buffer are done
 #pragma unroll
-        for (int e = 0; e < V / 2; e += 2) {
+        for (int e = 0; e < SG / 2; e += 2) {
           float4 l4, u4;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             float2 dt = make_float2(softplus_t<kFast>(vd[e + h].x + bias), softplus_t<kFast>(vd[e + h].y + bias));
             float2 uu;
             if constexpr (kMasked) {
-              const int i = tl0 + lg * V + 2 * (e + h);
+              const int i = tl0 + lg * SG + 2 * (e + h);
               dt.x = (i >= rel_lo && i < rel_hi) ? dt.x : 0.f;
               dt.y = (i + 1 >= rel_lo && i + 1 < rel_hi) ? dt.y : 0.f;
               uu = make_float2(dt.x != 0.f ? (ZOH ? vu[e + h].x : dt.x * vu[e + h].x) : 0.f,
@@ -387,11 +401,11 @@ chunk_scan_kernel(const ScanArgs args) {
               l4.z = dt.x; l4.w = dt.y; u4.z = uu.x; u4.w = uu.y;
             }
           }
-          const int q = lg * (V / 4) + e / 2;
+          const int q = lg * (SG / 4) + e / 2;
           xw[q * XQ] = l4;
           xw[(Q + q) * XQ] = u4;
         }
-        __syncwarp();  // both halves written
+        __syncwarp();  // every group's part written
         float2 ds = make_float2(0.f, 0.f);
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
@@ -481,8 +495,8 @@ chunk_scan_kernel(const ScanArgs args) {
         if constexpr (FWD && ZOH) IA2 = make_float2(invAs[ch * NP + n1], invAs[ch * NP + n1]);
         [[maybe_unused]] const T *rb = Bsm + size_t(n1) * Cfg::kBCPitch + tl0;
         [[maybe_unused]] const T *rc = Csm + size_t(n2) * Cfg::kBCPitch + tl0;
-        [[maybe_unused]] const float4 *rbf = reinterpret_cast<const float4 *>(Bf + size_t(n1) * TC + tl0);
-        [[maybe_unused]] const float4 *rcf = reinterpret_cast<const float4 *>(Bf + size_t(N + n2) * TC + tl0);
+        [[maybe_unused]] const float4 *rbf = reinterpret_cast<const float4 *>(Bf + size_t(n1) * BFP + tl0);
+        [[maybe_unused]] const float4 *rcf = reinterpret_cast<const float4 *>(Bf + size_t(N + n2) * BFP + tl0);
         // V/2 step pairs of float32 B (or C) from shared memory
         auto ldf = [](const float4 *q, float2 (&o)[V / 2]) {
 #pragma unroll
@@ -683,11 +697,12 @@ chunk_scan_kernel(const ScanArgs args) {
           // widen the chunk's 16-bit B/C (the single staging copy) into its float32 buffer
           float *dst = bcf + buf * kBFElems;
           for (int i = threadIdx.x; i < 2 * N * TC / V; i += NT) {
+            const int row = i / (TC / V), col = (i % (TC / V)) * V;
             float f[V];
-            unpack16<T>(*reinterpret_cast<const uint4 *>(bc0 + size_t(i) * V), f);
+            unpack16<T>(*reinterpret_cast<const uint4 *>(bc0 + size_t(row) * TC + col), f);
 #pragma unroll
             for (int k = 0; k < V / 4; ++k)
-              reinterpret_cast<float4 *>(dst + size_t(i) * V)[k] =
+              reinterpret_cast<float4 *>(dst + size_t(row) * BFP + col)[k] =
                   make_float4(f[4 * k], f[4 * k + 1], f[4 * k + 2], f[4 * k + 3]);
           }
         }

@@ -66,7 +66,16 @@ struct ShapeInfo {
 template <int N, bool NARROW, bool F32 = false> struct Shape;
 template <int N, bool NARROW> struct Shape<N, NARROW, true> : Shape<N, NARROW, false> {};
 template <> struct Shape<16, false> { static constexpr int KI = 16, SPW = 4, CPW = 8, CW = 4, NG = 1; };
-template <> struct Shape<16, true> { static constexpr int KI = 16, SPW = 16, CPW = 1, CW = 4, NG = 1; };
+// Narrow N=16 tile for 16-bit inputs: 16 segments x 2 lane groups (8 states each) of one channel
+// per warp, 256-step chunks, B/C converted in the state loop.  SSM_NARROW16_LG = 4 builds 8
+// segments x 4 lane groups (4 states each), 128-step chunks with B/C widened to float32 once per
+// chunk: measured 35 % slower on a 131072-step sequence of 2560 channels (4.43 vs 3.29 ms).
+#ifndef SSM_NARROW16_LG
+#define SSM_NARROW16_LG 2
+#endif
+template <> struct Shape<16, true> {
+  static constexpr int KI = 16, SPW = SSM_NARROW16_LG == 4 ? 8 : 16, CPW = 1, CW = 4, NG = 1;
+};
 template <> struct Shape<16, true, true> { static constexpr int KI = 8, SPW = 16, CPW = 1, CW = 4, NG = 1; };
 template <> struct Shape<32, false> { static constexpr int KI = 16, SPW = 8, CPW = 4, CW = 8, NG = 1; };
 template <> struct Shape<64, false> { static constexpr int KI = 8, SPW = 8, CPW = 4, CW = 8, NG = 1; };
