@@ -94,3 +94,24 @@ def test_ssd_host_rejections():
     assert lib.ssm_ssd_fwd(ctypes.byref(p), None) == 2                   # head dim 64 only
     p.headdim, p.seqlen = 64, 100
     assert lib.ssm_ssd_fwd(ctypes.byref(p), None) == 2                   # seqlen a multiple of 8
+
+
+@pytest.mark.parametrize("shape,h0", [
+    ((1, 2, 64, 128, 384), True),     # three chunks, initial state
+    ((2, 3, 64, 128, 200), False),    # ragged last chunk
+])
+def test_ssd_against_the_chunked_ssd_oracle(shape, h0):
+    """The kernel against oracle/ssd.py's fp64 chunked form (itself pinned against the scan
+    oracle on the CPU), with the same 128-step chunking: y within the bf16 budget of the
+    oracle's own output scale per head, h_last likewise."""
+    from oracle.ssd import ssd_chunked
+    b, H, P, N, L = shape
+    inp = workloads.ssd_inputs(b, H, P, N, L, seed=930 + L + H, h0=h0)
+    y, hl = run_ssd(inp)
+    for s in range(b):
+        ry, rh = ssd_chunked(inp.x[s], inp.dt[s], inp.A, inp.B[s], inp.C[s], 128,
+                             None if inp.h0 is None else inp.h0[s])
+        for h in range(H):
+            ey = np.max(np.abs(y[s, h] - ry[h])) / np.max(np.abs(ry[h]))
+            eh = np.max(np.abs(hl[s, h] - rh[h])) / np.max(np.abs(rh[h]))
+            assert ey <= TOL["bf16"] + 2.0 ** -8 and eh <= TOL["bf16"], (s, h, ey, eh)
