@@ -405,21 +405,51 @@ __global__ void __launch_bounds__(256) bwd_seg_scan_kernel(const float *A, const
   const int64_t dn = e % (dim * N), s = e / (dim * N);
   const int64_t d = dn / N, n = dn % N;
   const float A2 = A[dn] * kLog2e;
+  // Segments in batches of 8: a batch's loads are all issued before its results are written
+  // back in place, so they are in flight together (the values do not depend on h or mu).
+  constexpr int Q = 8;
+  float P[Q], gz[Q];
   float h = h0 ? h0[e] : 0.f;
-  for (int q = 0; q < nseg; ++q) {
-    const int64_t o = (s * nseg + q) * dim + d;
-    const float P = ex2_approx(A2 * seg_sum[o]);
-    const float gz = seg_h[o * N + n];
-    seg_h[o * N + n] = h;
-    h = fmaf(P, h, gz);
+  for (int q0 = 0; q0 < nseg; q0 += Q) {
+#pragma unroll
+    for (int i = 0; i < Q; ++i) {
+      const int q = q0 + i;
+      if (q < nseg) {
+        const int64_t o = (s * nseg + q) * dim + d;
+        P[i] = seg_sum[o];
+        gz[i] = seg_h[o * N + n];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < Q; ++i) {
+      const int q = q0 + i;
+      if (q < nseg) {
+        const int64_t o = (s * nseg + q) * dim + d;
+        seg_h[o * N + n] = h;
+        h = fmaf(ex2_approx(A2 * P[i]), h, gz[i]);
+      }
+    }
   }
   float mu = dh_last ? dh_last[e] : 0.f;
-  for (int q = nseg - 1; q >= 0; --q) {
-    const int64_t o = (s * nseg + q) * dim + d;
-    const float P = ex2_approx(A2 * seg_sum[o]);
-    const float gz = seg_g[o * N + n];
-    seg_g[o * N + n] = mu;
-    mu = fmaf(P, mu, gz);
+  for (int q0 = nseg - 1; q0 >= 0; q0 -= Q) {
+#pragma unroll
+    for (int i = 0; i < Q; ++i) {
+      const int q = q0 - i;
+      if (q >= 0) {
+        const int64_t o = (s * nseg + q) * dim + d;
+        P[i] = seg_sum[o];
+        gz[i] = seg_g[o * N + n];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < Q; ++i) {
+      const int q = q0 - i;
+      if (q >= 0) {
+        const int64_t o = (s * nseg + q) * dim + d;
+        seg_g[o * N + n] = mu;
+        mu = fmaf(ex2_approx(A2 * P[i]), mu, gz[i]);
+      }
+    }
   }
 }
 
