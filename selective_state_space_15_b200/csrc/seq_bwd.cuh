@@ -38,11 +38,11 @@
 // 8 channels, a CTA W warps.  Per block a lane evaluates the per-step terms (softplus, its
 // derivative, the gate) for 2 of the 8 steps and hands them to the channel's other lanes by
 // shuffles; sums over the states (yraw, du, dDelta) are reduced across those 4 lanes.  The
-// sums over channels (dB, dC) go through shared memory: every lane writes its per-state
-// terms of four steps at a time, each warp adds its 8 channels, the warps meet in a per-chunk
-// accumulator (shared atomics), and the CTA adds the chunk's rows to dB and dC with global atomics (16-byte
-// vector atomics where the rows allow them).  dA, dDskip and dbias are summed in registers
-// and added with atomics once per unit.
+// sums over channels (dB, dC) go through a per-warp buffer in shared memory: every lane writes
+// its per-state terms of four steps at a time, then lane (which, n) of the warp adds the warp's
+// 8 channels for those four steps and adds them to dB or dC with one 16-byte vector atomic in
+// global memory (scalar atomics where the rows do not allow it).  dA, dDskip and dbias are
+// summed in registers and added with atomics once per unit.
 //
 // Staging is the forward's: TMA bulk copies of the u, delta, z, dy rows and the B, C rows of a
 // chunk, double-buffered, with B and C widened to float32 in a [step][state] layout once per
@@ -133,18 +133,19 @@ struct BwdCfg {
   static constexpr size_t kBCElems = size_t(2) * N * TC;
   static constexpr int kCOff = TC * N + 16;
   static constexpr size_t kBFElems = size_t(2) * TC * N + 16;
-  // per warp: the per-state dB, dC terms of half an 8-step block, [4][2][LPC][CPW] groups of NS
-  // (the two halves are added to the accumulator one after the other)
-  static constexpr size_t kPartElems = size_t(4) * 2 * kLPC * kCPW * kNS;
-  static constexpr size_t kAccElems = size_t(2) * N * TC;     // [2: dB, dC][N][TC], per buffer
+  // per warp: the per-state dB, dC terms of half an 8-step block, [4 steps][CPW channels][2 N]
+  // (the two halves of a block leave the buffer one after the other); in a channel's row of 2 N
+  // words dB's terms come first for even channels and dC's first for odd ones, so that both the
+  // lanes' 16-byte writes and the per-(which, n) column reads are free of bank conflicts
+  static constexpr size_t kPartElems = size_t(4) * kCPW * 2 * N;
   static constexpr size_t kOffY = 2 * kXElems * sizeof(T);
   static constexpr size_t kOffBC = kOffY + 2 * kYElems * sizeof(TG);
   static constexpr size_t kOffBF = (kOffBC + 2 * kBCElems * sizeof(T) + 15) / 16 * 16;
   static constexpr size_t kOffPart = kOffBF + 2 * kBFElems * sizeof(float);
-  static constexpr size_t kOffAcc = kOffPart + kWarps * kPartElems * sizeof(float);
-  static constexpr size_t kSmemBytes = kOffAcc + 2 * kAccElems * sizeof(float);
+  static constexpr size_t kSmemBytes = kOffPart + kWarps * kPartElems * sizeof(float);
   static constexpr size_t kSegSmemBytes = kOffPart;  // the segment pass needs the staging only
   static_assert(kNS % 4 == 0, "whole float4 groups of states per lane");
+  static_assert(2 * N == 32, "one (which, state) pair per lane in the dB/dC reduction");
   static_assert(TC % 8 == 0 && (kXP * sizeof(T)) % 16 == 0 && (kXP * sizeof(TG)) % 16 == 0, "16-byte rows");
   static_assert(kOffY % 16 == 0 && kOffBF % 16 == 0 && kOffPart % 16 == 0, "aligned buffers");
 };
@@ -472,7 +473,6 @@ __global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kern
   T *const bcs0 = reinterpret_cast<T *>(smem + Cfg::kOffBC);                    // [2][2][N][TC]
   float *const bf0 = reinterpret_cast<float *>(smem + Cfg::kOffBF);             // [2][kBFElems]
   float *const part0 = reinterpret_cast<float *>(smem + Cfg::kOffPart);         // [W][kPartElems]
-  float *const acc0 = reinterpret_cast<float *>(smem + Cfg::kOffAcc);           // [2][2][N][TC]
   __shared__ __align__(8) uint64_t bars[2];
   __shared__ int unit_sh;
 
@@ -488,7 +488,6 @@ __global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kern
     mbar_init(&bars[1], 1);
     mbar_init_fence();
   }
-  for (int i = threadIdx.x; i < int(2 * Cfg::kAccElems); i += NT) acc0[i] = 0.f;
   __syncthreads();
   uint32_t gc = 0;
 
@@ -531,56 +530,36 @@ __global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kern
       Dd = args.Dskip ? args.Dskip[d] : 0.f;
     }
 
-    // the chunk accumulator `acc` (dB, dC summed over the CTA's channels) added to dB and dC,
-    // then cleared for its next use
-    auto flush_acc = [&](int abuf, int cc) {
-      float *acc = acc0 + abuf * Cfg::kAccElems;
-      const int64_t wstart = int64_t(cc) * TC;
-      for (int i = threadIdx.x; i < 2 * N * (TC / 4); i += NT) {
-        const int row = i / (TC / 4), t = (i % (TC / 4)) * 4;  // row = which * N + n
-        const int64_t gt = wstart + t;
-        float4 *src = reinterpret_cast<float4 *>(acc + row * TC + t);
-        const float4 v = *src;
-        *src = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (gt >= L) continue;
-        float *dst = (row >= N ? bw.dC : bw.dB) + (int64_t(s) * N + row % N) * L + gt;
-        if (bw.vec_dbc) {
-          atomicAdd(reinterpret_cast<float4 *>(dst), v);  // L % 4 == 0: the group lies inside the row
-        } else {
-          atomicAdd(dst, v.x);
-          if (gt + 1 < L) atomicAdd(dst + 1, v.y);
-          if (gt + 2 < L) atomicAdd(dst + 2, v.z);
-          if (gt + 3 < L) atomicAdd(dst + 3, v.w);
-        }
-      }
-    };
-
-    // dB, dC terms of four steps (chunk-local steps t0 .. t0 + 3, buffer slots 0..3): the warp's 8
-    // channels added up, then into the CTA's chunk accumulator
-    auto reduce_part = [&](float *acc, int t0) {
+    // dB, dC terms of four steps (chunk-local steps t0 .. t0 + 3, buffer slots 0..3): lane
+    // (which, n) adds up the warp's 8 channels for the four steps and adds them to dB or dC
+    auto reduce_part = [&](int64_t wstart, int t0) {
       __syncwarp();
-      for (int o = lane; o < 4 * 2 * LPC * (NS / 4); o += 32) {
-        // output group o = ((kk * 2 + which) * LPC + gg) * (NS / 4) + q: 4 states of one step
-        const int q = o % (NS / 4), gg = (o / (NS / 4)) % LPC, which = (o / (NS / 4 * LPC)) % 2;
-        const int kk = o / (NS / 4 * LPC * 2);
-        const float *src = part + ((size_t(kk) * 2 + which) * LPC * CPW + size_t(gg) * CPW) * NS + q * 4;
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int which = lane / N, n = lane % N;
+      float v[4];
 #pragma unroll
-        for (int cc = 0; cc < CPW; ++cc) {
-          const float4 v = *reinterpret_cast<const float4 *>(src + cc * NS);
-          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-        }
-        float *dst = acc + (size_t(which) * N + gg * NS + q * 4) * TC + t0 + kk;
-        atomicAdd(dst, sum.x);
-        atomicAdd(dst + TC, sum.y);
-        atomicAdd(dst + 2 * TC, sum.z);
-        atomicAdd(dst + 3 * TC, sum.w);
+      for (int kk = 0; kk < 4; ++kk) {
+        float sum = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < CPW; ++cc)
+          sum += part[(size_t(kk) * CPW + cc) * (2 * N) + (which ^ (cc & 1)) * N + n];
+        v[kk] = sum;
       }
       __syncwarp();  // the terms are consumed before the buffer is rewritten
+      const int64_t gt = wstart + t0;
+      if (gt < L) {
+        float *dst = (which ? bw.dC : bw.dB) + (int64_t(s) * N + n) * L + gt;
+        if (bw.vec_dbc) {
+          atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(v[0], v[1], v[2], v[3]));  // L % 4 == 0
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            if (gt + kk < L) atomicAdd(dst + kk, v[kk]);
+        }
+      }
     };
 
     // one 8-step block, from the end of the block to its start
-    auto block = [&](auto masked_tag, const T *X, const TG *Y, const float *Bf, float *acc, int64_t wstart, int sb) {
+    auto block = [&](auto masked_tag, const T *X, const TG *Y, const float *Bf, int64_t wstart, int sb) {
       constexpr bool kMasked = decltype(masked_tag)::value;
       const int k0 = sb * 8;                      // chunk-local first step of the block
       const int64_t gblk = (wstart + k0) / 8;     // block index in the sequence
@@ -718,8 +697,9 @@ __global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kern
         const float2 dyr = make_float2(dr[k], dr[k]);
         float2 S1 = make_float2(0.f, 0.f), S2 = make_float2(0.f, 0.f);
         [[maybe_unused]] float2 S3 = make_float2(0.f, 0.f);
-        float *pb = part + ((size_t(k & 3) * 2 + 0) * LPC * CPW + size_t(g) * CPW + c) * NS;  // dB terms
-        float *pc = part + ((size_t(k & 3) * 2 + 1) * LPC * CPW + size_t(g) * CPW + c) * NS;  // dC terms
+        float *prow = part + (size_t(k & 3) * CPW + c) * (2 * N) + g * NS;
+        float *pb = prow + (c & 1) * N;        // dB terms
+        float *pc = prow + (1 - (c & 1)) * N;  // dC terms
 #pragma unroll
         for (int q = 0; q < NS / 4; ++q) {
           float4 b4 = reinterpret_cast<const float4 *>(Bf + t * N + g * NS)[q];
@@ -759,9 +739,9 @@ __global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kern
         s1[k] = S1.x + S1.y;
         s2[k] = S2.x + S2.y;
         if constexpr (ZOH) s3[k] = S3.x + S3.y;
-        if (k == 4) reduce_part(acc, k0 + 4);  // steps 4..7 done: their terms leave the buffer
+        if (k == 4) reduce_part(wstart, k0 + 4);  // steps 4..7 done: their terms leave the buffer
       }
-      reduce_part(acc, k0);
+      reduce_part(wstart, k0);
       // ---- sums over the channel's lanes of sum_n dh B and sum_n dh h a A, for this lane's steps
 #pragma unroll
       for (int lev = 0; (1 << lev) < LPC; ++lev) {
@@ -822,36 +802,30 @@ __global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kern
     if (w.c_hi > w.c_lo)
       bwd_stage<Cfg>(args, bw, xs0, ys0, bcs0, &bars[gc & 1u], int(gc & 1u), w.c_hi - 1, nx, nvalid, d0, xbase,
                      bcbase);
-    int prev_acc = -1;  // accumulator of the chunk done before this one (to be flushed)
     for (int cc = w.c_hi - 1; cc >= w.c_lo; --cc, ++gc) {
       const int buf = int(gc & 1u);
       const int64_t wstart = int64_t(cc) * TC;
       const bool landed = mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);
       bwd_widen<Cfg>(bcs0 + buf * Cfg::kBCElems, bf0 + buf * Cfg::kBFElems);
-      // chunk cc widened; every warp is done with chunk cc+1 (its buffers and accumulator)
+      // chunk cc widened; every warp is done with chunk cc+1's buffers
       if (__syncthreads_or(!landed)) {
         mbar_wait_bounded(&bars[buf], (gc >> 1) & 1u);  // no copy left writing shared memory
         return;
       }
-      if (prev_acc >= 0) flush_acc(prev_acc, cc + 1);
       if (cc > w.c_lo)
         bwd_stage<Cfg>(args, bw, xs0, ys0, bcs0, &bars[buf ^ 1], buf ^ 1, cc - 1, nx, nvalid, d0, xbase, bcbase);
       const T *X = xs0 + buf * Cfg::kXElems;
       const TG *Y = ys0 + buf * Cfg::kYElems;
       const float *Bf = bf0 + buf * Cfg::kBFElems;
-      float *acc = acc0 + buf * Cfg::kAccElems;
 #pragma unroll 1
       for (int sb = TC / 8 - 1; sb >= 0; --sb) {
         if (wstart + sb * 8 >= L) continue;  // a block wholly past the end (uniform)
         if (wstart + sb * 8 + 8 <= L)
-          block(std::false_type{}, X, Y, Bf, acc, wstart, sb);
+          block(std::false_type{}, X, Y, Bf, wstart, sb);
         else
-          block(std::true_type{}, X, Y, Bf, acc, wstart, sb);
+          block(std::true_type{}, X, Y, Bf, wstart, sb);
       }
-      prev_acc = buf;
     }
-    __syncthreads();
-    if (prev_acc >= 0) flush_acc(prev_acc, w.c_lo);
 
     // ------------------------------------------------------------- per-unit results
     if (ch_ok) {
