@@ -505,6 +505,23 @@ __global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kern
     const int64_t xbase = int64_t(s) * args.x_batch_stride;
     const int64_t bcbase = int64_t(s) * args.bc_batch_stride;
     const int64_t so = (int64_t(s) * bw.nseg + w.seg) * args.dim + d;  // this segment's row
+    // The checkpoint (zero-start state entering a block) and the sum of Delta from the segment
+    // start to the block, for the block the walk takes next: blocks are taken last first, one
+    // after the other, and each block's values are loaded while the block before it is walked.
+    float4 ckn[NS / 4];
+    float cdn = 0.f;
+#pragma unroll
+    for (int q = 0; q < NS / 4; ++q) ckn[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int64_t blk_lo = w.t_lo / 8;  // the segment's first block (segments are whole chunks)
+    auto load_ckpt = [&](int64_t gb) {
+      if (ch_ok && gb >= blk_lo) {
+        const int64_t bo = (int64_t(s) * bw.nblk + gb) * args.dim + d;
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q) ckn[q] = reinterpret_cast<const float4 *>(bw.ckpt + bo * N + g * NS)[q];
+        cdn = bw.cumd[bo];
+      }
+    };
+    if (w.t_hi > w.t_lo) load_ckpt((w.t_hi - 1) / 8);  // the segment's last block comes first
 
     float2 A2[NS / 2], An[NS / 2], dh[NS / 2], dAacc[NS / 2], hs[NS / 2];
     [[maybe_unused]] float2 IA[NS / 2];  // 1/A (zero-order hold)
@@ -605,14 +622,16 @@ __global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kern
       float2 hin[NS / 2];
 #pragma unroll
       for (int p = 0; p < NS / 2; ++p) hin[p] = make_float2(0.f, 0.f);
+      float4 ckv[NS / 4];
+#pragma unroll
+      for (int q = 0; q < NS / 4; ++q) ckv[q] = ckn[q];
+      const float cdv = cdn;
+      load_ckpt(gblk - 1);  // in flight while this block is walked
       if (ch_ok) {
-        const int64_t bo = (int64_t(s) * bw.nblk + gblk) * args.dim + d;
-        const float *ck = bw.ckpt + bo * N + g * NS;
-        const float cdv = bw.cumd[bo];
         const float2 cd2 = make_float2(cdv, cdv);
 #pragma unroll
         for (int q = 0; q < NS / 4; ++q) {
-          const float4 v = reinterpret_cast<const float4 *>(ck)[q];
+          const float4 v = ckv[q];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int p = 2 * q + e;
