@@ -225,8 +225,11 @@ __device__ __forceinline__ void bwd_widen(const T *bs, float *bfw) {
 
 // ---------------------------------------------------------------------------------------------
 // 1. The segment pass.
+#ifndef SSM_BWD_SEG_WARPS_PER_SM
+#define SSM_BWD_SEG_WARPS_PER_SM 20  // resident warps per SM the segment pass is compiled for (96 registers)
+#endif
 template <typename T, typename TG, int N, int TC, int W, bool HAS_Z, bool ZOH>
-__global__ void __launch_bounds__(W * 32, 12 / W) bwd_seg_kernel(const ScanArgs args, const BwdArgs bw) {
+__global__ void __launch_bounds__(W * 32, SSM_BWD_SEG_WARPS_PER_SM / W) bwd_seg_kernel(const ScanArgs args, const BwdArgs bw) {
   using Cfg = BwdCfg<T, TG, N, TC, W>;
   constexpr int LPC = Cfg::kLPC, NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT;
   constexpr int XP = Cfg::kXP, SUB = Cfg::kSub;
