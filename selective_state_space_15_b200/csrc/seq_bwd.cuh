@@ -462,8 +462,12 @@ __global__ void __launch_bounds__(256) bwd_seg_scan_kernel(const float *A, const
 #ifndef SSM_BWD_WARPS_PER_SM
 #define SSM_BWD_WARPS_PER_SM 12  // resident warps per SM the walk is compiled for (its register budget)
 #endif
+#ifndef SSM_BWD_ZOH_WARPS_PER_SM
+#define SSM_BWD_ZOH_WARPS_PER_SM 8  // the same for the zero-order-hold walk (no spills at 8)
+#endif
 template <typename T, typename TG, int N, int TC, int W, bool HAS_Z, bool ZOH>
-__global__ void __launch_bounds__(W * 32, SSM_BWD_WARPS_PER_SM / W) seq_bwd_kernel(const ScanArgs args, const BwdArgs bw) {
+__global__ void __launch_bounds__(W * 32, (ZOH ? SSM_BWD_ZOH_WARPS_PER_SM : SSM_BWD_WARPS_PER_SM) / W)
+    seq_bwd_kernel(const ScanArgs args, const BwdArgs bw) {
   using Cfg = BwdCfg<T, TG, N, TC, W>;
   constexpr int LPC = Cfg::kLPC, NS = Cfg::kNS, CPW = Cfg::kCPW, CT = Cfg::kCT, NT = Cfg::kThreads;
   constexpr int XP = Cfg::kXP, SUB = Cfg::kSub;
