@@ -432,6 +432,10 @@ ssm_status_t launch_update(const ssm::UpdateArgs &a, int G, bool has_z, bool zoh
 // [batch][nblk][dim][N], the per-block Delta sums [batch][nblk][dim], the per-segment Delta
 // sums [batch][nseg][dim] and the two per-segment state arrays [batch][nseg][dim][N].
 constexpr int kBwdTC16 = 32;  // chunk of the backward kernels for 16-bit inputs (64-byte rows)
+#ifndef SSM_BWD_TC_F32
+#define SSM_BWD_TC_F32 32
+#endif
+constexpr int kBwdTC32 = SSM_BWD_TC_F32;  // the same for float32 inputs (128-byte rows; 72 KB, 3 CTAs per SM)
 constexpr int kBwdWarps = 4;  // warps per CTA (8 channels each)
 constexpr int64_t kBwdUnitsWanted = 8 * 148;
 constexpr int64_t kBwdMinSegChunks = 4;
@@ -441,7 +445,7 @@ struct BwdPlan {
 };
 bool make_bwd_plan(const ssm_scan_params *p, bool vec, BwdPlan &bp) {
   if (!vec || p->dstate != 16 || groups_of(p) != 1) return false;
-  const int64_t TC = p->dtype == SSM_F32 ? 16 : kBwdTC16;
+  const int64_t TC = p->dtype == SSM_F32 ? kBwdTC32 : kBwdTC16;
   const int64_t CT = 8 * kBwdWarps, L = p->seqlen, N = p->dstate;
   bp.nblk = (L + 7) / 8;
   bp.ntiles = (p->dim + CT - 1) / CT;
@@ -469,7 +473,7 @@ template <typename T, typename TG, bool HAS_Z, bool ZOH>
 ssm_status_t launch_bwd(ScanArgs a, const ssm::BwdArgs &bwa, const BwdPlan &bp, const ssm_scan_params *p,
                         unsigned char *ws, cudaStream_t st) {
   constexpr int N = 16, W = kBwdWarps;
-  constexpr int TC = sizeof(T) == 2 ? kBwdTC16 : 16;
+  constexpr int TC = sizeof(T) == 2 ? kBwdTC16 : kBwdTC32;
   using Cfg = ssm::BwdCfg<T, TG, N, TC, W>;
   a.ntiles = int(bp.ntiles);
   a.nseq = int(p->batch);
