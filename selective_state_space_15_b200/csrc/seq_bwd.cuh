@@ -133,11 +133,12 @@ struct BwdCfg {
   static constexpr size_t kBCElems = size_t(2) * N * TC;
   static constexpr int kCOff = TC * N + 16;
   static constexpr size_t kBFElems = size_t(2) * TC * N + 16;
-  // per warp: the per-state dB, dC terms of half an 8-step block, [4 steps][CPW channels][2 N]
-  // (the two halves of a block leave the buffer one after the other); in a channel's row of 2 N
-  // words dB's terms come first for even channels and dC's first for odd ones, so that both the
-  // lanes' 16-byte writes and the per-(which, n) column reads are free of bank conflicts
-  static constexpr size_t kPartElems = size_t(4) * kCPW * 2 * N;
+  // per warp: the per-state dB, dC terms of half an 8-step block, [2 step pairs][CPW channels]
+  // [2 N states][2 steps] (the two halves of a block leave the buffer one after the other); in a
+  // channel's row dB's terms come first for even channels and dC's first for odd ones, and odd
+  // channels swap the two 16-byte halves of every 32-byte group, so that both the lanes' 16-byte
+  // writes and the per-(which, n) float2 column reads are free of bank conflicts
+  static constexpr size_t kPartElems = size_t(2) * kCPW * 2 * N * 2;
   static constexpr size_t kOffY = 2 * kXElems * sizeof(T);
   static constexpr size_t kOffBC = kOffY + 2 * kYElems * sizeof(TG);
   static constexpr size_t kOffBF = (kOffBC + 2 * kBCElems * sizeof(T) + 15) / 16 * 16;
@@ -145,7 +146,7 @@ struct BwdCfg {
   static constexpr size_t kSmemBytes = kOffPart + kWarps * kPartElems * sizeof(float);
   static constexpr size_t kSegSmemBytes = kOffPart;  // the segment pass needs the staging only
   static_assert(kNS % 4 == 0, "whole float4 groups of states per lane");
-  static_assert(2 * N == 32, "one (which, state) pair per lane in the dB/dC reduction");
+  static_assert(2 * N == 32 && kNS == 4, "one (which, state) pair per lane in the dB/dC reduction");
   static_assert(TC % 8 == 0 && (kXP * sizeof(T)) % 16 == 0 && (kXP * sizeof(TG)) % 16 == 0, "16-byte rows");
   static_assert(kOffY % 16 == 0 && kOffBF % 16 == 0 && kOffPart % 16 == 0, "aligned buffers");
 };
@@ -561,12 +562,15 @@ __global__ void __launch_bounds__(W * 32, (ZOH ? SSM_BWD_ZOH_WARPS_PER_SM : SSM_
       const int which = lane / N, n = lane % N;
       float v[4];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        float sum = 0.f;
+      for (int kp = 0; kp < 2; ++kp) {  // steps t0 + 2 kp and t0 + 2 kp + 1
+        float2 sum = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int cc = 0; cc < CPW; ++cc)
-          sum += part[(size_t(kk) * CPW + cc) * (2 * N) + (which ^ (cc & 1)) * N + n];
-        v[kk] = sum;
+        for (int cc = 0; cc < CPW; ++cc) {
+          const int word = ((((which ^ (cc & 1)) * N) + n) * 2) ^ ((cc & 1) << 2);
+          sum = __fadd2_rn(sum, *reinterpret_cast<const float2 *>(part + (size_t(kp) * CPW + cc) * (4 * N) + word));
+        }
+        v[2 * kp] = sum.x;
+        v[2 * kp + 1] = sum.y;
       }
       __syncwarp();  // the terms are consumed before the buffer is rewritten
       const int64_t gt = wstart + t0;
@@ -716,6 +720,7 @@ __global__ void __launch_bounds__(W * 32, (ZOH ? SSM_BWD_ZOH_WARPS_PER_SM : SSM_
       // zero-order hold S3 = sum_n dh a B (dc/dDelta = a)
       float s1[8], s2[8];
       [[maybe_unused]] float s3[8];
+      float2 hb[2], hc[2];  // dB, dC terms of the odd step, written with the even step below it
 #pragma unroll
       for (int k = 7; k >= 0; --k) {
         const int t = k0 + k;
@@ -723,9 +728,6 @@ __global__ void __launch_bounds__(W * 32, (ZOH ? SSM_BWD_ZOH_WARPS_PER_SM : SSM_
         const float2 dyr = make_float2(dr[k], dr[k]);
         float2 S1 = make_float2(0.f, 0.f), S2 = make_float2(0.f, 0.f);
         [[maybe_unused]] float2 S3 = make_float2(0.f, 0.f);
-        float *prow = part + (size_t(k & 3) * CPW + c) * (2 * N) + g * NS;
-        float *pb = prow + (c & 1) * N;        // dB terms
-        float *pc = prow + (1 - (c & 1)) * N;  // dC terms
 #pragma unroll
         for (int q = 0; q < NS / 4; ++q) {
           float4 b4 = reinterpret_cast<const float4 *>(Bf + t * N + g * NS)[q];
@@ -759,8 +761,22 @@ __global__ void __launch_bounds__(W * 32, (ZOH ? SSM_BWD_ZOH_WARPS_PER_SM : SSM_
             }
             dh[p] = __fmul2_rn(dh[p], a[k][p]);                  // on to h_{t-1}
           }
-          reinterpret_cast<float4 *>(pb)[q] = make_float4(tb[0].x, tb[0].y, tb[1].x, tb[1].y);
-          reinterpret_cast<float4 *>(pc)[q] = make_float4(tc[0].x, tc[0].y, tc[1].x, tc[1].y);
+          if (k & 1) {
+            hb[0] = tb[0];
+            hb[1] = tb[1];
+            hc[0] = tc[0];
+            hc[1] = tc[1];
+          } else {
+            // steps k and k + 1 of the lane's four states as (step k, step k + 1) pairs
+            float *prow = part + (size_t((k & 3) >> 1) * CPW + c) * (4 * N);
+            const int sw = (c & 1) * 4;
+            float *pb = prow + ((c & 1) * N + g * NS) * 2;        // dB terms
+            float *pc = prow + ((1 - (c & 1)) * N + g * NS) * 2;  // dC terms
+            *reinterpret_cast<float4 *>(pb + sw) = make_float4(tb[0].x, hb[0].x, tb[0].y, hb[0].y);
+            *reinterpret_cast<float4 *>(pb + 4 - sw) = make_float4(tb[1].x, hb[1].x, tb[1].y, hb[1].y);
+            *reinterpret_cast<float4 *>(pc + sw) = make_float4(tc[0].x, hc[0].x, tc[0].y, hc[0].y);
+            *reinterpret_cast<float4 *>(pc + 4 - sw) = make_float4(tc[1].x, hc[1].x, tc[1].y, hc[1].y);
+          }
         }
         s1[k] = S1.x + S1.y;
         s2[k] = S2.x + S2.y;
