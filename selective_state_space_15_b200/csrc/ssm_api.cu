@@ -437,8 +437,14 @@ constexpr int kBwdTC16 = 32;  // chunk of the backward kernels for 16-bit inputs
 #endif
 constexpr int kBwdTC32 = SSM_BWD_TC_F32;  // the same for float32 inputs (128-byte rows; 72 KB, 3 CTAs per SM)
 constexpr int kBwdWarps = 4;  // warps per CTA (8 channels each)
-constexpr int64_t kBwdUnitsWanted = 8 * 148;
-constexpr int64_t kBwdMinSegChunks = 4;
+#ifndef SSM_BWD_UNITS_PER_SM
+#define SSM_BWD_UNITS_PER_SM 32  // backward units wanted per SM: long sequences cut into more segments balance better
+#endif
+#ifndef SSM_BWD_MIN_SEG_CHUNKS
+#define SSM_BWD_MIN_SEG_CHUNKS 4
+#endif
+constexpr int64_t kBwdUnitsWanted = SSM_BWD_UNITS_PER_SM * 148;
+constexpr int64_t kBwdMinSegChunks = SSM_BWD_MIN_SEG_CHUNKS;
 struct BwdPlan {
   int64_t nblk = 0, ntiles = 0, nseg = 0, seg_len = 0, nunits = 0;
   size_t off_ckpt = 0, off_cumd = 0, off_ssum = 0, off_sh = 0, off_sg = 0, bytes = 0;
